@@ -1,0 +1,527 @@
+#!/usr/bin/env python
+"""Throughput of the DSA forward pass (indexer -> top-k -> sparse MLA attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one whole forward pass over one batch of synthetic input of the chosen
+workload, with inputs resident in HBM.  Prints ONE JSON line (rank 0).
+
+  value      tokens/s over all ranks (query rows processed / max-over-ranks device time)
+  e2e        same metric through the public API with pinned host buffers; the H2D copy
+             of the step's inputs and the D2H copy of its outputs are inside the timing
+  roofline   the dominant kernel: algorithmic FLOPs (or bytes) per launch / its mean
+             CUDA-event duration, against the measured peak in MEASURED_PEAKS.json
+  stages     the same for every kernel of the step
+  workloads  the other workloads the metric names (decode at 128K context; 128K prefill
+             in 4096-query chunks), measured the same way with fewer steps
+  cpu_baseline  the fp64 oracle on a bounded sample of the headline workload, host cores
+
+Multi-GPU (torchrun): every rank runs its own independent problem (weak scaling, no
+collective on the data path); a barrier and CUDA synchronisation bracket the timed
+region and the slowest rank's time is used.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dsa_inputs import WORKLOADS, make_inputs, make_key_side, make_query_side  # noqa: E402
+
+METRIC = "DSA tokens/s (prefill 32K/128K, decode@128K ctx); % of FP8 peak / HBM roofline"
+HEADLINE = "prefill_32k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------------ setup
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-extra", action="store_true", help="skip the supplementary workloads")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if (args.impl == "ours" and torch.cuda.is_available()) else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, local, world
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"dsa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------ work model
+
+def work_model(wl, Lq=None, q_offset=None):
+    """Algorithmic work of one forward over queries [q_offset, q_offset+Lq) (per batch), x B."""
+    Lq = wl.Lq if Lq is None else Lq
+    q0 = wl.q_offset if q_offset is None else q_offset
+    first, last = q0 + 1, q0 + Lq
+    causal = (first + last) * Lq // 2 * wl.B
+    t = np.arange(q0, q0 + Lq, dtype=np.int64)
+    selected = int(np.minimum(wl.k, t + 1).sum()) * wl.B
+    rows = wl.B * Lq
+    return {
+        "rows": rows,
+        "causal_pairs": causal,
+        "selected_pairs": selected,
+        # indexer: one FP8 dot of width d_I per (pair, head); bytes: keys + scales read, scores written
+        "indexer_flops": 2.0 * causal * wl.H_I * wl.d_I,
+        "indexer_bytes": wl.B * (q0 + Lq) * (wl.d_I + 4) + rows * wl.H_I * (wl.d_I + 2) + causal * 4.0,
+        # top-k: causal scores read once, indices written
+        "topk_bytes": causal * 4.0 + rows * wl.k * 4.0,
+        # attention: S = q.c (d_qk) and O = p.v (d_v) per (selected pair, head)
+        "attn_flops": 2.0 * selected * wl.H * (wl.D + wl.Dv),
+        "attn_bytes": selected * wl.D * 2.0 + rows * wl.H * (wl.D + wl.Dv) * 2.0,
+    }
+
+
+# ------------------------------------------------------------------------------------ our arm
+
+class Runner:
+    """Inputs resident on the device, outputs and workspace preallocated."""
+
+    def __init__(self, wl, seed, device="cuda"):
+        import sparse_attention_19_b200 as dsa
+        self.dsa = dsa
+        self.wl = wl
+        self.device = device
+        chunk = wl.chunk if wl.chunk else wl.Lq
+        self.chunks = []
+        keys = make_key_side(wl, device, seed)
+        self.keys = keys
+        n_chunks = wl.Lq // chunk
+        for c in range(n_chunks):
+            if wl.chunk:
+                qs = make_query_side(wl, device, seed, chunk_index=c, Lq=chunk)
+                q_offset = wl.q_offset + c * chunk
+            else:
+                qs = make_query_side(wl, device, seed)
+                q_offset = wl.q_offset
+            self.chunks.append((q_offset, qs))
+        self.chunk_len = chunk
+        B, H, Dv, k = wl.B, wl.H, wl.Dv, wl.k
+        self.indices = torch.empty(B, wl.Lq, k, dtype=torch.int32, device=device)
+        self.out = torch.empty(B, wl.Lq, H, Dv, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(B, wl.Lq, H, dtype=torch.float32, device=device)
+        ws = 0
+        for q_offset, _ in self.chunks:
+            ws = max(ws, dsa.workspace_size(dsa.OP_FORWARD, B, chunk, q_offset + chunk, k, H, Dv))
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+        self.launches_per_call = 3 + (1 if dsa.workspace_size(dsa.OP_SPARSE_ATTN, B, chunk, wl.Lk, k, H, Dv) else 0)
+        self.work = [work_model(wl, chunk, q0) for q0, _ in self.chunks]
+
+    def step(self, stream, events=None):
+        wl, c = self.wl, self.chunk_len
+        for n, (q_offset, qs) in enumerate(self.chunks):
+            Lk = q_offset + c
+            sl = slice(n * c, (n + 1) * c) if wl.chunk else slice(None)
+            k_I = self.keys["k_I"][:, :Lk] if wl.chunk else self.keys["k_I"]
+            k_scale = self.keys["k_scale"][:, :Lk] if wl.chunk else self.keys["k_scale"]
+            kv = self.keys["kv"][:, :Lk] if wl.chunk else self.keys["kv"]
+            if wl.chunk:   # a chunk's key side is a prefix of the whole sequence (contiguous when B == 1)
+                assert wl.B == 1
+            self.dsa.forward(qs["q_I"], qs["q_scale"], qs["w"], k_I.contiguous() if wl.B > 1 else k_I,
+                             k_scale, qs["q"], kv, wl.k, wl.Dv, wl.scale, q_offset,
+                             indices=self.indices[:, sl], out=self.out[:, sl], lse=self.lse[:, sl],
+                             workspace=self.ws, stream=stream,
+                             stage_events=None if events is None else events[n])
+
+    def totals(self):
+        tot = {}
+        for w in self.work:
+            for k, v in w.items():
+                tot[k] = tot.get(k, 0) + v
+        return tot
+
+
+def time_runner(runner, steps, warmup, world, sample_clocks, local):
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        runner.step(stream)
+    torch.cuda.synchronize()
+    nchunks = len(runner.chunks)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nchunks)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local) if sample_clocks else None
+    if sampler:
+        sampler.__enter__()
+        time.sleep(0.3)
+    start.record(stream)
+    for s in range(steps):
+        runner.step(stream, ev[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.__exit__()
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    stage_ms = [0.0, 0.0, 0.0]
+    for s in range(steps):
+        for c in range(nchunks):
+            e = ev[s][c]
+            for i in range(3):
+                stage_ms[i] += e[i].elapsed_time(e[i + 1])
+    stage_ms = [x / steps for x in stage_ms]
+    return total_ms / steps, stage_ms, (sampler.summary() if sampler else None)
+
+
+def roofline_stages(wl, runner, stage_ms, peaks, peak_src):
+    tot = runner.totals()
+    fp8_burst = 2.0 * peaks["bf16_tflops"]
+    fp8_sust = 2.0 * peaks["bf16_tflops_sustained"]
+    decode = wl.Lq == 1
+    calls = len(runner.chunks)
+    out = {}
+    # indexer: FP8 contraction for prefill; streams the key cache for decode
+    if decode:
+        out["indexer"] = dict(bound="hbm", achieved=tot["indexer_bytes"] / (stage_ms[0] * 1e-3) / 1e9,
+                              peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["indexer_bytes"] / calls)
+    else:
+        out["indexer"] = dict(bound="tensor", achieved=tot["indexer_flops"] / (stage_ms[0] * 1e-3) / 1e12,
+                              peak=fp8_sust, unit="TFLOP/s", algorithmic=tot["indexer_flops"] / calls,
+                              peak_note=f"fp8 = 2 x {peak_src} sustained bf16 (nominal fp8:bf16 ratio)")
+    out["topk"] = dict(bound="hbm", achieved=tot["topk_bytes"] / (stage_ms[1] * 1e-3) / 1e9,
+                       peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["topk_bytes"] / calls)
+    if decode:
+        out["sparse_attn"] = dict(bound="hbm", achieved=tot["attn_bytes"] / (stage_ms[2] * 1e-3) / 1e9,
+                                  peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["attn_bytes"] / calls,
+                                  tflops=tot["attn_flops"] / (stage_ms[2] * 1e-3) / 1e12)
+    else:
+        out["sparse_attn"] = dict(bound="tensor", achieved=tot["attn_flops"] / (stage_ms[2] * 1e-3) / 1e12,
+                                  peak=peaks["bf16_tflops_sustained"], unit="TFLOP/s",
+                                  algorithmic=tot["attn_flops"] / calls)
+    for name, ms in zip(("indexer", "topk", "sparse_attn"), stage_ms):
+        d = out[name]
+        d["ms_per_step"] = ms
+        d["frac"] = d["achieved"] / d["peak"]
+        d["launches_per_step"] = calls
+    total = sum(stage_ms)
+    for name, ms in zip(("indexer", "topk", "sparse_attn"), stage_ms):
+        out[name]["share"] = ms / total if total > 0 else None
+    return out
+
+
+def traffic_from_profiles(kernel_name, workload):
+    """ncu DRAM bytes per launch recorded under profiles/ for this kernel + workload, if current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(path))
+        return d.get(workload, {}).get(kernel_name)
+    except Exception:
+        return None
+
+
+def measure_e2e(wl, runner, steps, warmup, world):
+    """Public API with pinned host buffers: H2D inputs + forward + D2H outputs each step."""
+    stream = torch.cuda.current_stream()
+    host_in = []
+    for q_offset, qs in runner.chunks:
+        host_in.append({k: v.cpu().pin_memory() for k, v in qs.items()})
+    host_keys = {k: v.cpu().pin_memory() for k, v in runner.keys.items()}
+    h_idx = torch.empty(runner.indices.shape, dtype=torch.int32).pin_memory()
+    h_out = torch.empty(runner.out.shape, dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty(runner.lse.shape, dtype=torch.float32).pin_memory()
+    bi = sum(v.numel() * v.element_size() for v in host_keys.values())
+    bi += sum(v.numel() * v.element_size() for d in host_in for v in d.values())
+    bo = sum(t.numel() * t.element_size() for t in (h_idx, h_out, h_lse))
+
+    def one():
+        for k, v in host_keys.items():
+            runner.keys[k].copy_(v, non_blocking=True)
+        for (q_offset, qs), hd in zip(runner.chunks, host_in):
+            for k, v in hd.items():
+                qs[k].copy_(v, non_blocking=True)
+        runner.step(stream)
+        h_idx.copy_(runner.indices, non_blocking=True)
+        h_out.copy_(runner.out, non_blocking=True)
+        h_lse.copy_(runner.lse, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world)
+    return ms, bi, bo
+
+
+# ------------------------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(wl, inp_dev_or_host, n_rows, seed=0):
+    """Time the oracle on n_rows rows spread evenly over the workload (one chunk for chunked)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    total = wl.B * wl.Lq
+    rows = np.unique(np.linspace(0, total - 1, n_rows).astype(np.int64))
+    r = oracle.rows_from_inputs(inp_dev_or_host, rows, wl.Lq, wl.q_offset)
+    b_used = np.unique(r["row_b"])
+    keys = {
+        "k_I": inp_dev_or_host["k_I"][torch.as_tensor(b_used)].cpu().numpy(),
+        "k_scale": inp_dev_or_host["k_scale"][torch.as_tensor(b_used)].cpu().numpy(),
+        "kv": inp_dev_or_host["kv"][torch.as_tensor(b_used)].cpu().view(torch.int16).numpy().view(np.uint16),
+    }
+    row_b = np.searchsorted(b_used, r["row_b"])
+    t0 = time.perf_counter()
+    oracle.dsa_forward(row_b, r["row_t"], r["q_I"], r["q_scale"], r["w"], keys["k_I"], keys["k_scale"], r["q"],
+                       keys["kv"], wl.k, wl.scale, wl.Dv)
+    return len(rows), time.perf_counter() - t0
+
+
+def cpu_baseline(wl, inp, budget_s=15.0):
+    import oracle
+    cores = oracle.num_threads()
+    n0 = max(cores, 4)
+    n, dt = oracle_sample(wl, inp, n0)
+    n_target = int(min(4 * n0 * 64, max(n, n * budget_s / max(dt, 1e-3))))
+    if n_target > n * 1.5:
+        n, dt = oracle_sample(wl, inp, n_target, seed=1)
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} query rows spread evenly over the {wl.name} workload "
+                      f"(all of their indexer pairs, top-k and attention), {dt:.1f} s on {cores} threads"}
+
+
+def _oracle_inputs(wl, seed):
+    """Inputs for the oracle arm: generated on the GPU when there is one (only the
+    sampled rows and the key side are copied to the host), else on the host."""
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_key_side(wl, dev, seed)
+    if wl.chunk:   # the last chunk's queries stand for the workload
+        c = wl.Lq // wl.chunk - 1
+        inp.update(make_query_side(wl, dev, seed, chunk_index=c, Lq=wl.chunk))
+        return inp, wl.with_(Lq=wl.chunk, q_offset=c * wl.chunk)
+    inp.update(make_query_side(wl, dev, seed))
+    return inp, wl
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm (host cores), rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    wl = WORKLOADS[args.workload]
+    inp, wl_eff = _oracle_inputs(wl, args.seed)
+    cores = oracle.num_threads()
+    n_rows = max(2 * cores, 8)
+    for _ in range(args.warmup):
+        oracle_sample(wl_eff, inp, max(cores // 2, 1))
+    total_rows, total_s = 0, 0.0
+    for s in range(args.steps):
+        n, dt = oracle_sample(wl_eff, inp, n_rows, seed=s)
+        total_rows += n
+        total_s += dt
+    value = total_rows / total_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, "host cores (fp64 oracle)"),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {n_rows} query rows spread evenly over {wl_eff.name} "
+                                   f"(Lq={wl_eff.Lq}, q_offset={wl_eff.q_offset})"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl, l2_note):
+    return {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "q_offset": wl.q_offset,
+            "chunk": wl.chunk or None, "k": wl.k, "H_I": wl.H_I, "d_I": wl.d_I, "H": wl.H, "d_qk": wl.D,
+            "d_v": wl.Dv, "indexer": "fp8 e4m3, per-token fp32 scales", "attention": "bf16, fp32 accumulate",
+            "l2": l2_note, "parallelism": "independent problem per GPU"}
+
+
+# ------------------------------------------------------------------------------------ main
+
+def main():
+    args = parse()
+    rank, local, world = dist_init(args)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    import sparse_attention_19_b200 as dsa
+    peaks, peak_src = load_peaks()
+    wl = WORKLOADS[args.workload]
+    runner = Runner(wl, seed=args.seed + rank)
+    ms, stage_ms, clocks = time_runner(runner, args.steps, args.warmup, world, rank == 0, local)
+    ms_max = max_over_ranks(ms, world)
+    tot = runner.totals()
+    tokens = tot["rows"] * world
+    value = tokens / (ms_max * 1e-3)
+    stages = roofline_stages(wl, runner, stage_ms, peaks, peak_src)
+    dom = max(stages, key=lambda n: stages[n]["ms_per_step"])
+    d = stages[dom]
+    kernel_names = {"indexer": "indexer_kernel", "topk": "topk_kernel", "sparse_attn": "sparse_attn_kernel"}
+    roof = {"kernel": kernel_names[dom], "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
+            "unit": d["unit"], "frac": d["frac"],
+            "traffic": traffic_from_profiles(kernel_names[dom], wl.name),
+            "per_launch_algorithmic": d["algorithmic"], "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8+bf16 (fp32 accumulate)", "data": "synthetic",
+        "config": config_of(wl, "inputs larger than L2 (q alone is %.1f GB)" % (
+            wl.B * wl.Lq * wl.H * wl.D * 2 / 1e9)),
+        "roofline": roof,
+        "stages": {k: {kk: (round(vv, 6) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                   for k, v in stages.items()},
+        "gpu_launches": runner.launches_per_call * len(runner.chunks) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        q_offset0, qs0 = runner.chunks[-1]
+        inp = dict(runner.keys, **qs0)
+        wl_cpu = wl.with_(Lq=runner.chunk_len, q_offset=q_offset0) if wl.chunk else wl
+        line["cpu_baseline"] = cpu_baseline(wl_cpu, inp)
+    if not args.no_e2e:
+        e_ms, bi, bo = measure_e2e(wl, runner, max(2, min(args.steps, 5)), 1, world)
+        line["e2e"] = {"value": tokens / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
+                       "d2h_bytes_per_step": bo, "ms_per_step": e_ms}
+    extra = {}
+    if not args.no_extra:
+        for name in ("decode_128k", "prefill_128k"):
+            if name == wl.name:
+                continue
+            del runner
+            torch.cuda.empty_cache()
+            w2 = WORKLOADS[name]
+            runner = Runner(w2, seed=args.seed + rank)
+            steps2 = max(3, args.steps // (4 if w2.chunk else 1))
+            ms2, st2, _ = time_runner(runner, steps2, 2, world, False, local)
+            ms2 = max_over_ranks(ms2, world)
+            t2 = runner.totals()
+            s2 = roofline_stages(w2, runner, st2, peaks, peak_src)
+            extra[name] = {"value": t2["rows"] * world / (ms2 * 1e-3), "unit": "tokens/s", "ms_per_step": ms2,
+                           "steps": steps2, "warmup": 2,
+                           "stages": {k: {kk: (round(vv, 6) if isinstance(vv, float) else vv)
+                                          for kk, vv in v.items()} for k, v in s2.items()}}
+        del runner
+        torch.cuda.empty_cache()
+        line["workloads"] = extra
+    assert dsa.device_status() == 0, "a device-side wait gave up during the run"
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

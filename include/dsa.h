@@ -1,0 +1,168 @@
+/*
+ * dsa.h -- C ABI of the DeepSeek Sparse Attention (DSA) forward pass on one
+ * NVIDIA B200 (sm_100a).  Exported by libdsa.so.
+ *
+ * What it computes (DeepSeek-V3.2 technical-report summary, ai.flicky.cc,
+ * section "DSA: внимание только к важному"):
+ *
+ *   lightning indexer ("Молниеносный индексатор", equation for I_{t,s}):
+ *       I[t,s] = sum_{j<H_I} w[t,j] * ReLU(q_I[t,j] . k_I[s])        for s <= t
+ *     with q_I and k_I in FP8 e4m3, each token carrying one positive fp32
+ *     scale (q_I[t,j] = e4m3 * q_scale[t], k_I[s] = e4m3 * k_scale[s]);
+ *   top-k selection and attention ("Отбор и основное внимание", equation for u_t):
+ *       u_t = Attn(h_t, { c_s : I[t,s] in Top-k(I[t,:]) }),   k = 2048,
+ *     MLA in MQA form: one latent KV row c_s (width d_qk) is shared by all H
+ *     query heads; its leading d_v columns are the value.
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer is caller-owned DEVICE memory, row-major and contiguous,
+ *     16-byte aligned.  The library never allocates, frees or synchronises;
+ *     it only enqueues kernels on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).
+ *   - Query i of batch b sits at sequence position t = q_offset + i and sees
+ *     keys 0..t.  Keys 0..Lk-1 exist; q_offset + Lq <= Lk is required.
+ *     Decode is Lq = 1, q_offset = Lk - 1; a prefill chunk is
+ *     q_offset = chunk start, Lk = q_offset + Lq.
+ *   - Argument and shape errors return before anything is enqueued.  A launch
+ *     failure returns DSA_ERR_CUDA.  Faults inside a kernel show up at the
+ *     caller's next synchronisation.  Kernels never trap: a device-side wait
+ *     that exceeds its limit is recorded and reported by dsa_device_status().
+ *   - Supported shapes: (H_I, d_I) in {(4, 64), (64, 128)};
+ *     (H, d_qk, d_v) in {(16, 192, 128), (128, 576, 512)}; 1 <= k <= 2048;
+ *     Lk < 2^31 / 16 per batch.  Anything else returns DSA_ERR_UNSUPPORTED.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1, /* NULL pointer, negative size, misaligned pointer, q_offset+Lq > Lk */
+    DSA_ERR_UNSUPPORTED = 2, /* a shape outside the supported set */
+    DSA_ERR_WORKSPACE = 3,   /* workspace smaller than dsa_workspace_size() */
+    DSA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    DSA_ERR_TIMEOUT = 5      /* a device-side wait gave up (see dsa_device_status) */
+} dsa_status;
+
+/* Inputs of the lightning indexer (equation for I_{t,s}). */
+typedef struct {
+    int B, Lq, Lk, q_offset;
+    int H_I, d_I;            /* indexer heads and head width */
+    const void *q_I;         /* e4m3 codes [B, Lq, H_I, d_I] */
+    const float *q_scale;    /* fp32 [B, Lq], > 0; NULL means 1.0 */
+    const void *w;           /* bf16 [B, Lq, H_I] */
+    const void *k_I;         /* e4m3 codes [B, Lk, d_I] */
+    const float *k_scale;    /* fp32 [B, Lk], > 0; NULL means 1.0 */
+} dsa_indexer_args;
+
+/* Inputs of the MQA / MLA-absorbed attention (equation for u_t). */
+typedef struct {
+    int H, d_qk, d_v;        /* query heads, latent row width, value width (d_v <= d_qk) */
+    float scale;             /* softmax scale applied to q . c_s */
+    const void *q;           /* bf16 [B, Lq, H, d_qk] */
+    const void *kv;          /* bf16 [B, Lk, d_qk]: latent rows c_s; value = leading d_v columns */
+} dsa_attn_args;
+
+/* Which entry point dsa_workspace_size() is asked about. */
+typedef enum {
+    DSA_OP_TOPK = 0,
+    DSA_OP_SPARSE_ATTN = 1,
+    DSA_OP_FORWARD = 2
+} dsa_op;
+
+/*
+ * Indexer scores, equation for I_{t,s}.
+ *   scores: fp32 [B, Lq, Lk]; scores[b,i,s] = I[q_offset+i, s] for s <= q_offset+i,
+ *   and -INFINITY for s > q_offset+i.
+ * Accumulation is fp32 over exact FP8 products; the per-token scales are
+ * applied after the head sum (they are positive, so they commute with ReLU).
+ */
+dsa_status dsa_indexer_scores(const dsa_indexer_args *args, float *scores, void *stream);
+
+/*
+ * Top-k selection over indexer scores ("Отбор и основное внимание": the k
+ * positions with the largest I[t,:]).
+ *   scores:  fp32 [B, Lq, Lk] (only entries s <= q_offset+i are read);
+ *   indices: int32 [B, Lq, k].  Row (b,i) receives the m = min(k, q_offset+i+1)
+ *            positions with the largest scores, ties to the smaller position,
+ *            -0.0 equal to +0.0, written in ascending position order in slots
+ *            0..m-1; slots m..k-1 receive -1.
+ *   workspace: may be NULL when dsa_workspace_size(DSA_OP_TOPK, ...) is 0.
+ */
+dsa_status dsa_topk(const float *scores, int B, int Lq, int Lk, int q_offset, int k,
+                    int32_t *indices, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Sparse MQA attention over the selected latent rows (equation for u_t).
+ *   indices: int32 [B, Lq, k]; entries outside [0, Lk) are skipped.
+ *   out:     bf16 [B, Lq, H, d_v];  out[b,i,h,:] = sum_s p_s kv[b,s,:d_v],
+ *            p = softmax over the selected s of scale * q[b,i,h,:] . kv[b,s,:].
+ *   lse:     fp32 [B, Lq, H] or NULL; natural-log log-sum-exp of the logits
+ *            (-INFINITY and out = 0 for a row with no valid entry).
+ * Rows with B*Lq small are split over the k entries across CTAs and merged
+ * (split-k); the workspace holds the partial results.
+ */
+dsa_status dsa_sparse_attn(const dsa_attn_args *args, int B, int Lq, int Lk,
+                           const int32_t *indices, int k, void *out, float *lse,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The whole forward pass: indexer -> top-k -> sparse attention.
+ * `iargs` and `aargs` describe the same B, Lq, Lk, q_offset.
+ *   indices: int32 [B, Lq, k] (as dsa_topk); out: bf16 [B, Lq, H, d_v];
+ *   lse: fp32 [B, Lq, H] or NULL.
+ * The workspace holds the indexer scores of the call ([B, Lq, Lk] fp32) and
+ * the split-k partials.
+ */
+dsa_status dsa_forward(const dsa_indexer_args *iargs, const dsa_attn_args *aargs, int k,
+                       int32_t *indices, void *out, float *lse,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * dsa_forward with stage timing: when `stage_events` is not NULL it points to
+ * four cudaEvent_t handles (created by the caller) that are recorded on
+ * `stream` before the indexer, after the indexer, after the top-k and after the
+ * attention (including its split-k merge).  Everything else is dsa_forward.
+ */
+dsa_status dsa_forward_timed(const dsa_indexer_args *iargs, const dsa_attn_args *aargs, int k,
+                             int32_t *indices, void *out, float *lse,
+                             void *workspace, size_t workspace_bytes, void *stream,
+                             void *const *stage_events);
+
+/* Bytes of device workspace the entry point `op` needs for these sizes (0 = none). */
+size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_v);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *dsa_status_string(dsa_status status);
+
+/*
+ * Device-side status of this library on the current device: reads (and, when
+ * `clear` is non-zero, resets) the word the kernels write when a bounded wait
+ * gives up.  Synchronises the device.  Returns DSA_OK or DSA_ERR_TIMEOUT
+ * (DSA_ERR_CUDA if the read itself fails).
+ */
+dsa_status dsa_device_status(int clear);
+
+/*
+ * Self-test of the failure path: launches one CTA that waits, with a limit of
+ * about `spin_limit` polls, on a barrier that nothing will ever complete, and
+ * returns DSA_ERR_TIMEOUT after synchronising if (and only if) the wait gave
+ * up and the kernel returned normally.  Clears the device status first and
+ * afterwards.  No fault, trap or hang is involved.
+ */
+dsa_status dsa_selftest_wait_timeout(uint32_t spin_limit, void *stream);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,355 @@
+// dsa_api.cu -- the C ABI of libdsa.so (declared in include/dsa.h): argument
+// checks, TMA descriptor set-up, workspace layout and kernel dispatch for the
+// DeepSeek Sparse Attention forward pass.  Every step of the computation runs in
+// the kernels of indexer.cu, topk.cu and sparse_attn.cu; this file only checks,
+// describes and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "dsa_internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+__device__ uint32_t g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxK = 2048;
+constexpr int kAttnTile = 128;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem_bytes`-byte elements, box [box_rows, box_cols].
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t rows,
+               uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+dsa_status check_indexer(const dsa_indexer_args* a) {
+  if (!a || !a->q_I || !a->w || !a->k_I) return DSA_ERR_INVALID_ARG;
+  if (a->B <= 0 || a->Lq <= 0 || a->Lk <= 0 || a->q_offset < 0) return DSA_ERR_INVALID_ARG;
+  if ((long long)a->q_offset + a->Lq > a->Lk) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(a->q_I) || !aligned16(a->k_I) || !aligned16(a->w)) return DSA_ERR_INVALID_ARG;
+  if (a->q_scale && !aligned16(a->q_scale)) return DSA_ERR_INVALID_ARG;
+  if (a->k_scale && !aligned16(a->k_scale)) return DSA_ERR_INVALID_ARG;
+  const bool shape_ok = (a->H_I == 64 && a->d_I == 128) || (a->H_I == 4 && a->d_I == 64);
+  if (!shape_ok) return DSA_ERR_UNSUPPORTED;
+  if ((long long)a->B * a->Lk >= (1LL << 31) || (long long)a->B * a->Lq * a->H_I >= (1LL << 31))
+    return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status check_attn(const dsa_attn_args* a, int B, int Lq, int Lk) {
+  if (!a || !a->q || !a->kv) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || Lq <= 0 || Lk <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->kv)) return DSA_ERR_INVALID_ARG;
+  if (!(a->scale > 0.f) || !std::isfinite(a->scale)) return DSA_ERR_INVALID_ARG;
+  const bool shape_ok = (a->H == 128 && a->d_qk == 576 && a->d_v == 512) ||
+                        (a->H == 16 && a->d_qk == 192 && a->d_v == 128);
+  if (!shape_ok) return DSA_ERR_UNSUPPORTED;
+  if ((long long)B * Lk >= (1LL << 31) || (long long)B * Lq * 128 >= (1LL << 31)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+// Split-k factor for the attention: enough (row, split) units to cover the SM
+// pairs several times over; 1 for prefill-sized batches.
+int attn_splits(int rows, int n_tiles) {
+  const int pairs = sm_count() / 2;
+  int s = 1;
+  while (s < n_tiles && (long long)rows * s < 4LL * pairs) s *= 2;
+  return s < n_tiles ? s : n_tiles;
+}
+
+size_t attn_ws_bytes(int B, int Lq, int k, int H, int d_v) {
+  const int n_tiles = (k + kAttnTile - 1) / kAttnTile;
+  const int rows = B * Lq;
+  const int splits = attn_splits(rows, n_tiles);
+  if (splits <= 1) return 0;
+  const size_t per = (size_t)rows * splits * H;
+  return per * (size_t)d_v * 4 + per * 4 + 256;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper, cudaStream_t st) {
+  IndexerParams p{};
+  p.B = a->B; p.Lq = a->Lq; p.Lk = a->Lk; p.q_offset = a->q_offset;
+  p.H_I = a->H_I; p.d_I = a->d_I;
+  if (a->H_I == 64) {
+    p.qb = a->Lq >= 4 ? 4 : a->Lq;
+  } else {
+    const int r4 = (a->Lq + 3) / 4 * 4;
+    p.qb = r4 < 64 ? r4 : 64;
+  }
+  p.nsub = (a->Lq > p.qb) ? 2 : 1;
+  p.queries_per_unit = p.qb * p.nsub;
+  p.n_qblocks = (a->Lq + p.queries_per_unit - 1) / p.queries_per_unit;
+  const int sms = sm_count();
+  const long long base_units = (long long)p.n_qblocks * a->B;
+  const int max_tiles = (a->q_offset + a->Lq - 1) / 128 + 1;
+  int kch = 1;
+  if (base_units < 4LL * sms) {
+    kch = (int)((4LL * sms + base_units - 1) / base_units);
+    const int cap = (max_tiles + 7) / 8;           // keep at least ~8 key tiles per unit
+    if (kch > cap) kch = cap;
+    if (kch < 1) kch = 1;
+  }
+  p.kchunks = kch;
+  p.n_units = (int)(base_units * kch);
+  p.fill_upper = fill_upper ? 1 : 0;
+  p.q_scale = a->q_scale;
+  p.w = reinterpret_cast<const __nv_bfloat16*>(a->w);
+  p.k_scale = a->k_scale;
+  p.scores = scores;
+
+  const CUtensorMapSwizzle swz = (a->d_I == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap tq, tk;
+  if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->q_I, (uint64_t)a->B * a->Lq * a->H_I, a->d_I,
+                 a->d_I, (uint32_t)(p.qb * a->H_I), swz))
+    return DSA_ERR_CUDA;
+  if (!make_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 128,
+                 swz))
+    return DSA_ERR_CUDA;
+  const int grid = p.n_units < sms ? p.n_units : sms;
+  return launch_indexer(p, tq, tk, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, int k, int32_t* idx,
+                    cudaStream_t st) {
+  TopkParams p{};
+  p.scores = scores; p.B = B; p.Lq = Lq; p.Lk = Lk; p.q_offset = q_offset; p.k = k; p.indices = idx;
+  const long long nmax = (long long)q_offset + Lq < Lk ? (long long)q_offset + Lq : Lk;
+  if (nmax <= 32768) {
+    p.cache_cap = (int)round_up((size_t)nmax, 4);
+    p.cand_cap = 4096;
+  } else {
+    p.cache_cap = 0;
+    p.cand_cap = 16384;
+  }
+  return launch_topk(p, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status run_attn(const dsa_attn_args* a, int B, int Lq, int Lk, int q_offset, bool compact,
+                    const int32_t* idx, int k, void* out, float* lse, void* ws, size_t ws_bytes,
+                    cudaStream_t st) {
+  AttnParams p{};
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = a->H; p.k = k;
+  p.n_tiles = (k + kAttnTile - 1) / kAttnTile;
+  const int rows = B * Lq;
+  p.splits = attn_splits(rows, p.n_tiles);
+  p.tiles_per_split = (p.n_tiles + p.splits - 1) / p.splits;
+  p.n_units = rows * p.splits;
+  p.compact = compact ? 1 : 0;
+  p.q_offset = q_offset;
+  p.scale_log2 = a->scale * 1.4426950408889634f;
+  p.indices = idx;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  if (p.splits > 1) {
+    const size_t need = attn_ws_bytes(B, Lq, k, a->H, a->d_v);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return DSA_ERR_WORKSPACE;
+    const size_t per = (size_t)rows * p.splits * a->H;
+    p.part_o = reinterpret_cast<float*>(ws);
+    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + round_up(per * a->d_v * 4, 256));
+  }
+  CUtensorMap tq, tkv;
+  if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->q, (uint64_t)rows * a->H, a->d_qk, 64, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  if (!make_tmap(&tkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->kv, (uint64_t)B * Lk, a->d_qk, 64, 1,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  const int pairs = sm_count() / 2;
+  const int grid = p.n_units < pairs ? p.n_units : pairs;
+  if (launch_sparse_attn(p, a->d_qk, a->d_v, tq, tkv, grid, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (p.splits > 1 && launch_attn_combine(p, a->d_v, st) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+__global__ void wait_selftest_kernel(uint32_t limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t a = smem_u32(&bar);
+    bool done = false;
+    for (uint32_t i = 0; i < limit && !done; ++i) done = mbar_try_wait(a, 0);
+    if (!done) atomicExch(&g_device_error, DEV_ERR_TIMEOUT);
+    mbar_arrive(&bar);          // complete the phase so the barrier is left idle
+  }
+}
+
+}  // namespace
+
+cudaError_t read_device_error(uint32_t* value, bool clear) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  if (clear) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
+  }
+  return e;
+}
+
+cudaError_t launch_wait_selftest(uint32_t spin_limit, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(spin_limit);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+dsa_status dsa_indexer_scores(const dsa_indexer_args* args, float* scores, void* stream) {
+  dsa_status s = check_indexer(args);
+  if (s != DSA_OK) return s;
+  if (!scores || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  return run_indexer(args, scores, true, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_topk(const float* scores, int B, int Lq, int Lk, int q_offset, int k, int32_t* indices,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!scores || !indices || B <= 0 || Lq <= 0 || Lk <= 0 || q_offset < 0) return DSA_ERR_INVALID_ARG;
+  if ((long long)q_offset + Lq > Lk) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(indices)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+  if ((long long)B * Lq >= (1LL << 31)) return DSA_ERR_UNSUPPORTED;
+  return run_topk(scores, B, Lq, Lk, q_offset, k, indices, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_attn(const dsa_attn_args* args, int B, int Lq, int Lk, const int32_t* indices, int k,
+                           void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status s = check_attn(args, B, Lq, Lk);
+  if (s != DSA_OK) return s;
+  if (!indices || !out || !aligned16(indices) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (lse && !aligned16(lse)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+  return run_attn(args, B, Lq, Lk, 0, false, indices, k, out, lse, workspace, workspace_bytes,
+                  static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_v) {
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || k < 1 || k > kMaxK || H <= 0 || d_v <= 0) return 0;
+  switch (op) {
+    case DSA_OP_TOPK:
+      return 0;
+    case DSA_OP_SPARSE_ATTN:
+      return attn_ws_bytes(B, Lq, k, H, d_v);
+    case DSA_OP_FORWARD:
+      return round_up((size_t)B * Lq * (size_t)Lk * 4, 256) + attn_ws_bytes(B, Lq, k, H, d_v);
+  }
+  return 0;
+}
+
+dsa_status dsa_forward_timed(const dsa_indexer_args* iargs, const dsa_attn_args* aargs, int k, int32_t* indices,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream,
+                             void* const* stage_events) {
+  dsa_status s = check_indexer(iargs);
+  if (s != DSA_OK) return s;
+  s = check_attn(aargs, iargs->B, iargs->Lq, iargs->Lk);
+  if (s != DSA_OK) return s;
+  if (!indices || !out || !aligned16(indices) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (lse && !aligned16(lse)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+  const size_t need = dsa_workspace_size(DSA_OP_FORWARD, iargs->B, iargs->Lq, iargs->Lk, k, aargs->H, aargs->d_v);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> bool {
+    return !stage_events || cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
+  };
+  float* scores = static_cast<float*>(workspace);
+  const size_t score_bytes = round_up((size_t)iargs->B * iargs->Lq * (size_t)iargs->Lk * 4, 256);
+  char* attn_ws = static_cast<char*>(workspace) + score_bytes;
+  const size_t attn_ws_size = workspace_bytes - score_bytes;
+  if (!mark(0)) return DSA_ERR_CUDA;
+  s = run_indexer(iargs, scores, false, st);
+  if (s != DSA_OK) return s;
+  if (!mark(1)) return DSA_ERR_CUDA;
+  s = run_topk(scores, iargs->B, iargs->Lq, iargs->Lk, iargs->q_offset, k, indices, st);
+  if (s != DSA_OK) return s;
+  if (!mark(2)) return DSA_ERR_CUDA;
+  s = run_attn(aargs, iargs->B, iargs->Lq, iargs->Lk, iargs->q_offset, true, indices, k, out, lse, attn_ws,
+               attn_ws_size, st);
+  if (s != DSA_OK) return s;
+  if (!mark(3)) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status dsa_forward(const dsa_indexer_args* iargs, const dsa_attn_args* aargs, int k, int32_t* indices,
+                       void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return dsa_forward_timed(iargs, aargs, k, indices, out, lse, workspace, workspace_bytes, stream, nullptr);
+}
+
+const char* dsa_status_string(dsa_status status) {
+  switch (status) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG: invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED: shape outside the supported set";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE: workspace too small";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA: CUDA call or kernel launch failed";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT: a device-side wait gave up";
+  }
+  return "DSA_ERR_UNKNOWN";
+}
+
+dsa_status dsa_device_status(int clear) {
+  uint32_t v = 0;
+  if (read_device_error(&v, clear != 0) != cudaSuccess) return DSA_ERR_CUDA;
+  return v == DEV_ERR_NONE ? DSA_OK : DSA_ERR_TIMEOUT;
+}
+
+dsa_status dsa_selftest_wait_timeout(uint32_t spin_limit, void* stream) {
+  uint32_t v = 0;
+  if (read_device_error(&v, true) != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_wait_selftest(spin_limit, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (read_device_error(&v, true) != cudaSuccess) return DSA_ERR_CUDA;
+  return v == DEV_ERR_TIMEOUT ? DSA_ERR_TIMEOUT : DSA_OK;
+}
+
+int dsa_version(void) { return 100; }
+
+}  // extern "C"

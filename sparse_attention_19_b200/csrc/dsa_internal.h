@@ -1,0 +1,69 @@
+// dsa_internal.h -- parameter blocks and launchers shared by the kernels and the
+// C-ABI layer of libdsa.so.  Not part of the public interface (include/dsa.h is).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace dsa {
+
+// ---------------------------------------------------------------- indexer
+struct IndexerParams {
+  int B, Lq, Lk, q_offset;
+  int H_I, d_I;
+  int qb;                 // queries per MMA (N = qb * H_I <= 256)
+  int nsub;               // query sub-blocks resident per unit
+  int queries_per_unit;   // qb * nsub
+  int n_qblocks;          // ceil(Lq / queries_per_unit)
+  int kchunks;            // key-tile ranges per query block (>1 splits long rows across CTAs)
+  int n_units;            // n_qblocks * B * kchunks
+  int fill_upper;         // write -inf for s > t (full-matrix output)
+  const float* q_scale;   // [B, Lq] or null
+  const __nv_bfloat16* w; // [B, Lq, H_I]
+  const float* k_scale;   // [B, Lk] or null
+  float* scores;          // [B, Lq, Lk]
+};
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats);
+cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                           int grid, cudaStream_t stream);
+
+// ---------------------------------------------------------------- top-k
+struct TopkParams {
+  const float* scores;    // [B, Lq, Lk]
+  int B, Lq, Lk, q_offset, k;
+  int32_t* indices;       // [B, Lq, k]
+  int cache_cap;          // row elements cached in shared memory (0 = stream from global)
+  int cand_cap;           // candidate (key, position) pairs held in shared memory
+};
+size_t topk_smem_bytes(int cache_cap, int cand_cap);
+cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- sparse attention
+struct AttnParams {
+  int B, Lq, Lk, H, k;
+  int n_tiles;            // ceil(k / 128)
+  int splits;             // key-tile ranges per query (split-k); 1 = direct output
+  int tiles_per_split;
+  int n_units;            // B * Lq * splits
+  int compact;            // indices are valid-first (top-k output): skip all-padding tiles
+  int q_offset;           // only used when compact
+  float scale_log2;       // softmax scale * log2(e)
+  const int32_t* indices; // [B, Lq, k]
+  __nv_bfloat16* out;     // [B, Lq, H, d_v] (splits == 1)
+  float* lse;             // [B, Lq, H] or null (splits == 1)
+  float* part_o;          // [B*Lq, splits, H, d_v] fp32 (splits > 1)
+  float* part_lse;        // [B*Lq, splits, H] fp32 (splits > 1)
+};
+size_t attn_smem_bytes(int d_qk, int d_v);
+cudaError_t launch_sparse_attn(const AttnParams& p, int d_qk, int d_v, const CUtensorMap& tq,
+                               const CUtensorMap& tkv, int grid_clusters, cudaStream_t stream);
+cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t stream);
+
+// ---------------------------------------------------------------- misc
+cudaError_t read_device_error(uint32_t* value, bool clear);
+cudaError_t launch_wait_selftest(uint32_t spin_limit, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,313 @@
+// indexer.cu -- the lightning indexer on sm_100a tensor cores.
+//
+// Computes I[t,s] = q_scale[t] * k_scale[s] * sum_{j<H_I} w[t,j] * ReLU(q8[t,j] . k8[s])
+// (DeepSeek-V3.2 technical-report summary, "Молниеносный индексатор", equation for
+// I_{t,s}; FP8 per its third bullet).  The per-token scales are positive, so they
+// factor out of the ReLU and are applied after the head sum.
+//
+// Mapping.  One tcgen05.mma (kind::f8f6f4, fp32 accumulate in TMEM) multiplies a
+// tile of 128 keys (M, the A operand, K-major: one key row of d_I e4m3 bytes) by
+// QB queries x H_I heads (N = QB*H_I <= 256, the B operand).  With keys on the M
+// axis, TMEM lane = key and the H_I columns of one query sit in that lane, so the
+// ReLU, the weighting and the head sum are a per-thread loop in the epilogue with
+// no cross-thread reduction.  Each CTA keeps NSUB query sub-blocks resident in
+// shared memory and streams key tiles through a TMA ring; two TMEM accumulators
+// let the epilogue of one sub-block overlap the MMA of the next.
+//
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
+// warps 2..5 epilogue (warp w reads TMEM lanes 32*(w%4) .. +31).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "dsa_internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kKeysPerTile = 128;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+
+struct IndexerSmem {
+  // Barriers and small per-unit data first; big tiles follow at a 1024-byte boundary.
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t final_bar;
+  uint64_t epi_bar;          // rendezvous of the 4 epilogue warps
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct UnitInfo {
+  int b, i0, kt0, kt1;  // batch, first query, key-tile range [kt0, kt1)
+};
+
+__device__ __forceinline__ UnitInfo decode_unit(const IndexerParams& p, int u) {
+  // Longest work first: query blocks are visited from the last one down.
+  const int per_block = p.B * p.kchunks;
+  const int qblk = p.n_qblocks - 1 - u / per_block;
+  const int rem = u % per_block;
+  const int b = rem / p.kchunks;
+  const int kc = rem % p.kchunks;
+  UnitInfo info;
+  info.b = b;
+  info.i0 = qblk * p.queries_per_unit;
+  const int i_last = min(p.Lq, info.i0 + p.queries_per_unit) - 1;
+  const int t_last = p.q_offset + i_last;                       // <= Lk - 1
+  const int ntiles = t_last / kKeysPerTile + 1;
+  const int per_chunk = (ntiles + p.kchunks - 1) / p.kchunks;
+  info.kt0 = min(ntiles, kc * per_chunk);
+  info.kt1 = min(ntiles, (kc + 1) * per_chunk);
+  return info;
+}
+
+template <int H_I, int D_I>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+               const IndexerParams p) {
+  static_assert(D_I == 64 || D_I == 128, "d_I");
+  constexpr uint32_t kRowBytes = D_I;                  // one e4m3 row
+  constexpr uint32_t kLayout = (D_I == 128) ? LAYOUT_SW128 : LAYOUT_SW64;
+  constexpr uint32_t kAtomBytes = 8 * kRowBytes;       // 8-row swizzle atom
+  constexpr int kKSteps = D_I / 32;                    // MMA K = 32 bytes of e4m3
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  IndexerSmem& S = *reinterpret_cast<IndexerSmem*>(smem_raw);
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* tiles = smem_raw + (((raw_addr + (uint32_t)sizeof(IndexerSmem) + 1023u) & ~1023u) - raw_addr);
+  const int N = p.qb * H_I;                            // MMA N (queries x heads)
+  const int QU = p.queries_per_unit;                   // = qb * nsub
+  uint8_t* q_smem = tiles;                             // nsub * N rows
+  uint8_t* k_smem = tiles + (size_t)p.nsub * N * kRowBytes;
+  float* w_smem = reinterpret_cast<float*>(k_smem + (size_t)kStages * kKeysPerTile * kRowBytes);
+  float* sq_smem = w_smem + QU * H_I;
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  volatile uint32_t* abort_flag = &S.abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&S.q_full, 1);
+    mbar_init(&S.q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.k_full[s], 1);
+      mbar_init(&S.k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&S.acc_full[s], 1);
+      mbar_init(&S.acc_empty[s], 4);
+    }
+    mbar_init(&S.final_bar, 1);
+    mbar_init(&S.epi_bar, 4);
+    S.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = S.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      uint32_t q_phase = 0, kstage = 0, kphase = 0;
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const UnitInfo U = decode_unit(p, u);
+        if (!mbar_wait(&S.q_empty, q_phase ^ 1, abort_flag)) break;
+        q_phase ^= 1;
+        mbar_arrive_expect_tx(&S.q_full, (uint32_t)(p.nsub * N) * kRowBytes);
+        for (int sb = 0; sb < p.nsub; ++sb) {
+          const int row = ((U.b * p.Lq) + U.i0 + sb * p.qb) * H_I;
+          tma_load_2d(q_smem + (size_t)sb * N * kRowBytes, &tmap_q, &S.q_full, 0, row);
+        }
+        bool ok = true;
+        for (int kt = U.kt0; kt < U.kt1; ++kt) {
+          if (!mbar_wait(&S.k_empty[kstage], kphase ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&S.k_full[kstage], kKeysPerTile * kRowBytes);
+          tma_load_2d(k_smem + (size_t)kstage * kKeysPerTile * kRowBytes, &tmap_k, &S.k_full[kstage],
+                      0, U.b * p.Lk + kt * kKeysPerTile);
+          if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc = make_idesc(0, 0, 128, (uint32_t)N, 0, 0);  // e4m3 x e4m3 -> f32
+      uint32_t q_phase = 0, kstage = 0, kphase = 0, seq = 0;
+      const uint32_t q_base = smem_u32(q_smem), k_base = smem_u32(k_smem);
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const UnitInfo U = decode_unit(p, u);
+        if (!mbar_wait(&S.q_full, q_phase, abort_flag)) break;
+        q_phase ^= 1;
+        tc_fence_after();
+        bool ok = true;
+        for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
+          if (!mbar_wait(&S.k_full[kstage], kphase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = k_base + kstage * kKeysPerTile * kRowBytes;
+          for (int sb = 0; sb < p.nsub; ++sb) {
+            const uint32_t slot = seq & 1u, use = seq >> 1;
+            if (!mbar_wait(&S.acc_empty[slot], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + slot * (uint32_t)N;
+            const uint32_t b_addr = q_base + (uint32_t)(sb * N) * kRowBytes;
+#pragma unroll
+            for (int ks = 0; ks < kKSteps; ++ks) {
+              const uint64_t ad = make_smem_desc(a_addr + ks * 32, 16, kAtomBytes, kLayout);
+              const uint64_t bd = make_smem_desc(b_addr + ks * 32, 16, kAtomBytes, kLayout);
+              mma_f8_ss(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(&S.acc_full[slot]);
+            ++seq;
+          }
+          mma_commit(&S.k_empty[kstage]);
+          if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
+        }
+        mma_commit(&S.q_empty);
+        if (!ok) break;
+      }
+      // Every MMA issued here completes before the TMEM is released.
+      mma_commit(&S.final_bar);
+      mbar_wait(&S.final_bar, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t quarter = warp & 3u;              // TMEM lane quarter this warp may read
+    const uint32_t row = quarter * 32 + lane;        // key row within the tile
+    const int et = threadIdx.x - 64;                 // 0..127
+    uint32_t seq = 0, epi_phase = 0;
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      const UnitInfo U = decode_unit(p, u);
+      if (!warps_rendezvous(&S.epi_bar, epi_phase, abort_flag)) break;   // previous unit done with w/sq
+      for (int x = et; x < QU * H_I; x += 128) {
+        const int qq = x / H_I, j = x % H_I;
+        const int i = U.i0 + qq;
+        float wv = 0.f;
+        if (i < p.Lq) wv = __bfloat162float(p.w[((size_t)U.b * p.Lq + i) * H_I + j]);
+        w_smem[x] = wv;
+      }
+      for (int x = et; x < QU; x += 128) {
+        const int i = U.i0 + x;
+        sq_smem[x] = (i < p.Lq) ? (p.q_scale ? p.q_scale[(size_t)U.b * p.Lq + i] : 1.f) : 0.f;
+      }
+      if (!warps_rendezvous(&S.epi_bar, epi_phase, abort_flag)) break;
+      bool ok = true;
+      for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
+        const int s = kt * kKeysPerTile + (int)row;
+        const float sk = (s < p.Lk) ? (p.k_scale ? p.k_scale[(size_t)U.b * p.Lk + s] : 1.f) : 0.f;
+        for (int sb = 0; sb < p.nsub; ++sb) {
+          const uint32_t slot = seq & 1u, use = seq >> 1;
+          if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t t_base = tmem_base + ((quarter * 32u) << 16) + slot * (uint32_t)N;
+          // Each query owns H_I consecutive columns; walk them 32 at a time.
+          for (int q0 = 0; q0 < p.qb; q0 += (H_I >= 32 ? 1 : 32 / H_I)) {
+            uint32_t v[32];
+            float acc[(H_I >= 32) ? 1 : 32 / H_I];
+            constexpr int QPC = (H_I >= 32) ? 1 : 32 / H_I;   // queries per 32 columns
+            constexpr int CPQ = (H_I >= 32) ? H_I / 32 : 1;   // 32-column chunks per query
+#pragma unroll
+            for (int a = 0; a < QPC; ++a) acc[a] = 0.f;
+            const float* wq = w_smem + (size_t)(sb * p.qb + q0) * H_I;
+#pragma unroll
+            for (int c = 0; c < CPQ; ++c) {
+              tmem_ld32(t_base + (uint32_t)(q0 * H_I + c * 32), v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int a = (H_I >= 32) ? 0 : e / H_I;
+                const float x = __uint_as_float(v[e]);
+                acc[a] = fmaf(wq[c * 32 + e], fmaxf(x, 0.f), acc[a]);
+              }
+            }
+#pragma unroll
+            for (int a = 0; a < QPC; ++a) {
+              const int qq = sb * p.qb + q0 + a;
+              const int i = U.i0 + qq;
+              if (i < p.Lq && s < p.Lk) {
+                const int t = p.q_offset + i;
+                float* dst = p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s;
+                if (s <= t)
+                  __stcs(dst, acc[a] * sq_smem[qq] * sk);
+                else if (p.fill_upper)
+                  __stcs(dst, -INFINITY);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.acc_empty[slot]);
+          ++seq;
+        }
+      }
+      if (!ok) break;
+      // Full-matrix output: positions beyond this unit's causal tiles are -inf.
+      if (p.fill_upper && p.kchunks == 1) {
+        const int nt_all = (p.Lk + kKeysPerTile - 1) / kKeysPerTile;
+        for (int kt = U.kt1; kt < nt_all; ++kt) {
+          const int s = kt * kKeysPerTile + (int)row;
+          if (s >= p.Lk) continue;
+          for (int qq = 0; qq < QU; ++qq) {
+            const int i = U.i0 + qq;
+            if (i < p.Lq)
+              __stcs(p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s, -INFINITY);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <int H_I, int D_I>
+cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                             int grid, cudaStream_t stream) {
+  const size_t smem = indexer_smem_bytes(p.nsub * p.qb * H_I, D_I, p.queries_per_unit * H_I,
+                                         p.queries_per_unit);
+  auto kern = indexer_kernel<H_I, D_I>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats) {
+  size_t b = sizeof(IndexerSmem) + 1024;                       // barriers + alignment slack
+  b += (size_t)q_rows * d_I;                                   // resident query block
+  b += (size_t)kStages * kKeysPerTile * d_I;                   // key ring
+  b += (size_t)(w_floats + sq_floats) * sizeof(float);
+  // At least ~116 KB so that one CTA (and its 512 TMEM columns) owns each SM.
+  return b < 118784 ? 118784 : b;
+}
+
+cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                           int grid, cudaStream_t stream) {
+  if (p.H_I == 64 && p.d_I == 128) return launch_indexer_t<64, 128>(p, tq, tk, grid, stream);
+  if (p.H_I == 4 && p.d_I == 64) return launch_indexer_t<4, 64>(p, tq, tk, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dsa

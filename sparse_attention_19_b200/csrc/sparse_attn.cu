@@ -1,0 +1,571 @@
+// sparse_attn.cu -- sparse MQA / MLA-absorbed attention over the selected latent rows.
+//
+// For query row r (batch b, position t) and head h, over the selected positions s:
+//   z_s = scale * q[r,h,:] . kv[b,s,:]        (all d_qk columns: latent + rope)
+//   out[r,h,:] = sum_s softmax(z)_s * kv[b,s,:d_v]
+// (DeepSeek-V3.2 technical-report summary, "Отбор и основное внимание", equation
+// for u_t: attention only over the top-k latent entries c_s; MLA in MQA mode, one
+// KV row serves every query head.)
+//
+// Mapping onto a pair of SMs (a 2-CTA cluster, tcgen05 .cta_group::2):
+//   * Each CTA owns 64 of the 128 query heads; its Q rows (64 x d_qk bf16) stay in
+//     shared memory for the whole query.  MMA M = 128 heads across the pair.
+//   * Keys come in tiles of 128 selected positions.  S = Q K^T is one pair-MMA
+//     chain with N = 128 keys: each CTA gathers 64 of the tile's key rows, in
+//     64-column chunks (TMA tile::gather4, 128-byte swizzle), streamed through a
+//     ring.  S lands in TMEM as 64 columns per CTA (lanes 0-63: keys 0-63,
+//     lanes 64-127: keys 64-127 of the tile, for that CTA's 64 heads).
+//   * Four softmax warps per CTA turn S into P (bf16, in shared memory, the A
+//     operand of the next MMA) with an online softmax whose reference maximum
+//     only moves when a new maximum exceeds it by 2^8 (the accumulator is then
+//     rescaled in TMEM); the two lanes that hold one head's two key halves swap
+//     their maxima through shared memory.
+//   * O += P V is a pair-MMA with N = 256 value columns per instruction; V is
+//     the same gathered rows read as an MN-major operand, each CTA holding 128
+//     value columns of all 128 keys.  O for 64 heads x 512 columns fits in 256
+//     TMEM columns per CTA (the pair layout puts half of N in lanes 64-127), so
+//     S double-buffers beside it.
+//   * The leader CTA (rank 0) issues every MMA; both CTAs' TMA loads complete on
+//     the leader's barriers, and MMA completion is multicast to both CTAs.
+// Warp roles (192 threads per CTA): warps 0-3 softmax/epilogue (TMEM lane quarter
+// = warp), warp 4 TMA producer, warp 5 TMEM owner + MMA issuer (leader only).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "dsa_internal.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kTileKeys = 128;       // keys per tile (pair)
+constexpr int kHalfKeys = 64;        // keys per CTA in S
+constexpr int kKStages = 4;          // K-chunk ring depth
+constexpr int kVStages = 2;          // V ring depth
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kPlane64 = 64 * 128;    // 64 rows x 128 B  (Q plane, K stage, P plane)
+constexpr uint32_t kPlane128 = 128 * 128;  // 128 rows x 128 B (V plane)
+constexpr uint32_t kTmemS = 0;             // S buffers: columns [0, 128)
+constexpr uint32_t kTmemO = 128;           // O: columns [128, 128 + d_v/2)
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnBarriers {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t o_full, o_empty, pv_done, final_bar;
+  uint64_t xbar;             // rendezvous of the 4 softmax warps (max / sum exchange)
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+  float red_max[2][128];
+  float red_sum[128];
+};
+
+template <int DV>
+struct VShape {
+  static constexpr int kNpv = DV >= 256 ? DV / 256 : 1;   // PV instructions per tile
+  static constexpr int kN = DV >= 256 ? 256 : DV;         // N of one PV instruction
+  static constexpr int kPlanes = kN / 128;                // 64-column planes per CTA per instruction
+  static constexpr uint32_t kStageBytes = kPlanes * kPlane128;
+};
+
+struct Unit {
+  int row, b, t, j0, j1, split;
+};
+
+__device__ __forceinline__ Unit decode_unit(const AttnParams& p, int u) {
+  Unit U;
+  const int n_rows = p.B * p.Lq;
+  U.row = n_rows - 1 - u / p.splits;       // longest rows first (top-k output is valid-first)
+  U.split = u % p.splits;
+  U.b = U.row / p.Lq;
+  U.t = p.q_offset + U.row % p.Lq;
+  int nt = p.n_tiles;
+  if (p.compact) {
+    const int nvalid = min(p.k, U.t + 1);
+    nt = (nvalid + kTileKeys - 1) / kTileKeys;
+  }
+  U.j0 = min(nt, U.split * p.tiles_per_split);
+  U.j1 = min(nt, (U.split + 1) * p.tiles_per_split);
+  return U;
+}
+
+__device__ __forceinline__ int kv_row(const AttnParams& p, int b, int row, int pos) {
+  int s = -1;
+  if (pos < p.k) s = __ldg(p.indices + (size_t)row * p.k + pos);
+  if (s < 0 || s >= p.Lk) s = 0;            // padding: any valid row, masked in softmax
+  return b * p.Lk + s;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <int NC, int DV>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
+                   const AttnParams p) {
+  using VS = VShape<DV>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  AttnBarriers& S = *reinterpret_cast<AttnBarriers*>(smem_raw);
+  // 1024-byte aligned operand area (the 128-byte swizzle is address based).
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t area_off = ((raw_addr + sizeof(AttnBarriers) + 1023u) & ~1023u) - raw_addr;
+  uint8_t* area = smem_raw + area_off;
+  uint8_t* q_sm = area;                                             // NC planes
+  uint8_t* k_sm = q_sm + NC * kPlane64;                             // kKStages planes
+  uint8_t* v_sm = k_sm + kKStages * kPlane64;                       // kVStages x kPlanes planes
+  uint8_t* p_sm = v_sm + kVStages * VS::kStageBytes;                // 2 buffers x 2 planes
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int cluster_id = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
+  volatile uint32_t* abort_flag = &S.abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&S.q_full, 1);
+    mbar_init(&S.q_empty, 1);
+    for (int i = 0; i < kKStages; ++i) { mbar_init(&S.k_full[i], 1); mbar_init(&S.k_empty[i], 1); }
+    for (int i = 0; i < kVStages; ++i) { mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_empty[i], 8);   // 4 softmax warps x 2 CTAs
+      mbar_init(&S.p_full[i], 8);
+      mbar_init(&S.p_empty[i], 1);
+    }
+    mbar_init(&S.o_full, 1);
+    mbar_init(&S.o_empty, 8);
+    mbar_init(&S.pv_done, 1);
+    mbar_init(&S.final_bar, 1);
+    mbar_init(&S.xbar, 4);
+    S.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc_pair(&S.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = S.tmem_base;
+  const uint16_t kBoth = 0x3;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ producer
+    uint32_t q_use = 0, kc = 0, vc = 0;
+    const uint32_t q_full_l = mapa_shared(smem_u32(&S.q_full), 0);
+    bool ok = true;
+    if (lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
+    for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
+      const Unit U = decode_unit(p, u);
+      if (U.j0 >= U.j1) continue;
+      // Q: this CTA's 64 heads, NC planes of 64 columns.
+      if (lane == 0) {
+        ok = mbar_wait(&S.q_empty, (q_use & 1u) ^ 1u, abort_flag);
+        if (ok) {
+          if (leader) mbar_arrive_expect_tx(&S.q_full, 2u * NC * kPlane64);
+          const int qrow = U.row * p.H + (int)rank * 64;
+          for (int c = 0; c < NC; ++c) tma_load_2d_pair(q_sm + c * kPlane64, &tmap_q, q_full_l, c * 64, qrow);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++q_use;
+      // K chunks of tile j, then V of tile j-1 (the order the MMA consumes them).
+      auto load_k = [&](int j) -> bool {
+        // lanes 0..15: 4 keys each of this CTA's 64 keys
+        int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+        if (lane < 16) {
+          const int base = j * kTileKeys + (int)rank * kHalfKeys + (int)lane * 4;
+          r0 = kv_row(p, U.b, U.row, base + 0);
+          r1 = kv_row(p, U.b, U.row, base + 1);
+          r2 = kv_row(p, U.b, U.row, base + 2);
+          r3 = kv_row(p, U.b, U.row, base + 3);
+        }
+        for (int c = 0; c < NC; ++c) {
+          const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
+          bool w_ok = true;
+          if (lane == 0) {
+            w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
+            if (w_ok && leader) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
+          }
+          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+          if (!w_ok) return false;
+          const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
+          if (lane < 16)
+            tma_gather4_pair(k_sm + st * kPlane64 + lane * 512, &tmap_kv, full_l, c * 64, r0, r1, r2, r3);
+          ++kc;
+        }
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        // lanes 0..31: 4 keys each of all 128 keys of the tile
+        const int base = j * kTileKeys + (int)lane * 4;
+        const int r0 = kv_row(p, U.b, U.row, base + 0);
+        const int r1 = kv_row(p, U.b, U.row, base + 1);
+        const int r2 = kv_row(p, U.b, U.row, base + 2);
+        const int r3 = kv_row(p, U.b, U.row, base + 3);
+        for (int h = 0; h < VS::kNpv; ++h) {
+          const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+          bool w_ok = true;
+          if (lane == 0) {
+            w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
+            if (w_ok && leader) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
+          }
+          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+          if (!w_ok) return false;
+          const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
+          for (int pl = 0; pl < VS::kPlanes; ++pl) {
+            const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
+            tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane128 + lane * 512, &tmap_kv, full_l,
+                             col, r0, r1, r2, r3);
+          }
+          ++vc;
+        }
+        return true;
+      };
+      for (int j = U.j0; j < U.j1 && ok; ++j) {
+        ok = load_k(j);
+        if (ok && j > U.j0) ok = load_v(j - 1);
+      }
+      if (ok) ok = load_v(U.j1 - 1);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (leader && elect_one()) {
+      constexpr uint32_t idesc_s = make_idesc(1, 1, 128, kTileKeys, 0, 0);       // bf16, K-major x K-major
+      constexpr uint32_t idesc_pv = make_idesc(1, 1, 128, VS::kN, 0, 1);         // P K-major, V MN-major
+      const uint32_t q_base = smem_u32(q_sm), k_base = smem_u32(k_sm);
+      const uint32_t v_base = smem_u32(v_sm), p_base = smem_u32(p_sm);
+      uint32_t q_use = 0, kc = 0, vc = 0, sc = 0, pc = 0, oc = 0;
+      bool ok = true;
+      auto issue_s = [&](bool last_of_unit) -> bool {
+        const uint32_t sb = sc & 1u;
+        if (!mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag, true)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem_base + kTmemS + sb * kHalfKeys;
+        for (int c = 0; c < NC; ++c) {
+          const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
+          if (!mbar_wait(&S.k_full[st], ph, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_smem_desc(q_base + c * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
+            const uint64_t bd = make_smem_desc(k_base + st * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
+            mma_bf16_ss_pair(d, ad, bd, idesc_s, (c | kk) ? 1u : 0u);
+          }
+          mma_commit_pair_mc(&S.k_empty[st], kBoth);
+          ++kc;
+        }
+        mma_commit_pair_mc(&S.s_full[sb], kBoth);
+        if (last_of_unit) mma_commit_pair_mc(&S.q_empty, kBoth);
+        ++sc;
+        return true;
+      };
+      auto issue_pv = [&](bool first_of_unit, bool last_of_unit) -> bool {
+        const uint32_t pb = pc & 1u;
+        if (!mbar_wait(&S.p_full[pb], (pc >> 1) & 1u, abort_flag, true)) return false;
+        if (first_of_unit && !mbar_wait(&S.o_empty, (oc & 1u) ^ 1u, abort_flag, true)) return false;
+        tc_fence_after();
+        for (int h = 0; h < VS::kNpv; ++h) {
+          const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+          if (!mbar_wait(&S.v_full[st], ph, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t d = tmem_base + kTmemO + h * (VS::kN / 2);
+#pragma unroll
+          for (int kk = 0; kk < kTileKeys / 16; ++kk) {
+            const uint64_t ad = make_smem_desc(p_base + pb * 2 * kPlane64 + (kk >> 2) * kPlane64 + (kk & 3) * 32,
+                                               16, 1024, LAYOUT_SW128);
+            const uint64_t bd = make_smem_desc(v_base + st * VS::kStageBytes + kk * 2048, kPlane128, 1024,
+                                               LAYOUT_SW128);
+            mma_bf16_ss_pair(d, ad, bd, idesc_pv, (first_of_unit && kk == 0) ? 0u : 1u);
+          }
+          mma_commit_pair_mc(&S.v_empty[st], kBoth);
+          ++vc;
+        }
+        mma_commit_pair_mc(&S.p_empty[pb], kBoth);
+        mma_commit_pair_mc(&S.pv_done, kBoth);
+        if (last_of_unit) { mma_commit_pair_mc(&S.o_full, kBoth); ++oc; }
+        ++pc;
+        return true;
+      };
+      for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
+        const Unit U = decode_unit(p, u);
+        if (U.j0 >= U.j1) continue;
+        ok = mbar_wait(&S.q_full, q_use & 1u, abort_flag);
+        ++q_use;
+        tc_fence_after();
+        for (int j = U.j0; j < U.j1 && ok; ++j) {
+          ok = issue_s(j == U.j1 - 1);
+          if (ok && j > U.j0) ok = issue_pv(j - 1 == U.j0, false);
+        }
+        if (ok) ok = issue_pv(U.j1 - 1 == U.j0, true);
+      }
+      // Wait until every MMA this thread issued has completed before teardown.
+      mma_commit(&S.final_bar);
+      mbar_wait(&S.final_bar, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const uint32_t l = warp * 32 + lane;          // TMEM lane = (key half, head)
+    const uint32_t h = l & 63u;                   // head within this CTA
+    const uint32_t half = l >> 6;                 // which 64 keys of the tile this lane holds
+    const int head = (int)rank * 64 + (int)h;
+    const uint32_t lane_addr = (warp * 32u) << 16;
+    uint32_t sc = 0, pc = 0, oc = 0, xph = 0;
+    bool ok = true;
+    for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
+      const Unit U = decode_unit(p, u);
+      if (U.j0 >= U.j1) {
+        // An empty split: no keys.  Partial result is (O = 0, lse = -inf).
+        if (p.splits > 1 && half == 0 && head < p.H) {
+          const size_t prow = ((size_t)U.row * p.splits + U.split) * p.H + head;
+          p.part_lse[prow] = -INFINITY;
+          float4* o4 = reinterpret_cast<float4*>(p.part_o + prow * DV);
+          for (int x = 0; x < DV / 4; ++x) o4[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        continue;
+      }
+      float m = -INFINITY, lsum = 0.f;
+      for (int j = U.j0; j < U.j1 && ok; ++j) {
+        const uint32_t sb = sc & 1u;
+        ok = mbar_wait_warp(&S.s_full[sb], (sc >> 1) & 1u, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sv[64];
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+          tmem_ld32(tmem_base + lane_addr + kTmemS + sb * kHalfKeys, lo);
+          tmem_ld32(tmem_base + lane_addr + kTmemS + sb * kHalfKeys + 32, hi);
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
+        ++sc;
+        // Scale into log2 units and mask padding / out-of-range positions.
+        const int kbase = j * kTileKeys + (int)half * kHalfKeys;
+        const int32_t* irow = p.indices + (size_t)U.row * p.k;
+        float x[64];
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int pos = kbase + c;
+          const int s = (pos < p.k) ? __ldg(irow + pos) : -1;
+          const bool valid = (s >= 0) && (s < p.Lk);
+          x[c] = valid ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, x[c]);
+        }
+        const uint32_t rb = sc & 1u;
+        S.red_max[rb][l] = tmax;
+        ok = warps_rendezvous(&S.xbar, xph, abort_flag);
+        if (!ok) break;
+        tmax = fmaxf(tmax, S.red_max[rb][l ^ 64u]);
+        const float m_new = fmaxf(m, tmax);
+        const bool first = (j == U.j0);
+        if (first) {
+          m = m_new;
+        } else {
+          const bool need = m_new > m + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            // PV of the previous tile must be complete before O is touched.
+            ok = mbar_wait_warp(&S.pv_done, (pc - 1u) & 1u, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const float alpha = need ? exp2f(m - m_new) : 1.f;
+            for (int c0 = 0; c0 < VS::kNpv * (VS::kN / 2); c0 += 32) {
+              uint32_t ov[32];
+              tmem_ld32(tmem_base + lane_addr + kTmemO + c0, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              tmem_st32(tmem_base + lane_addr + kTmemO + c0, ov);
+            }
+            tmem_st_wait();
+            if (need) { lsum *= alpha; m = m_new; }
+          }
+        }
+        const float m_use = (m == -INFINITY) ? 0.f : m;
+        // P buffer reuse: PV two tiles back must be done.
+        const uint32_t pb = pc & 1u;
+        if (pc >= 2) {
+          ok = mbar_wait_warp(&S.p_empty[pb], ((pc >> 1) & 1u) ^ 1u, abort_flag);
+          if (!ok) break;
+        }
+        uint8_t* prow = p_sm + pb * 2 * kPlane64 + half * kPlane64 + (h >> 3) * 1024 + (h & 7) * 128;
+        float psum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = exp2f(x[c * 8 + 2 * e] - m_use);
+            const float p1 = exp2f(x[c * 8 + 2 * e + 1] - m_use);
+            const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+            const float2 back = __bfloat1622float2(v2);
+            psum += back.x + back.y;
+            w4[e] = *reinterpret_cast<const uint32_t*>(&v2);
+          }
+          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        lsum += psum;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.p_full[pb]), 0));
+        ++pc;
+      }
+      if (!ok) break;
+      // ---- epilogue of the unit
+      ok = mbar_wait_warp(&S.o_full, oc & 1u, abort_flag);
+      ++oc;
+      if (!ok) break;
+      tc_fence_after();
+      S.red_sum[l] = lsum;
+      ok = warps_rendezvous(&S.xbar, xph, abort_flag);
+      if (!ok) break;
+      const float total = lsum + S.red_sum[l ^ 64u];
+      ok = warps_rendezvous(&S.xbar, xph, abort_flag);   // red_sum may be rewritten next unit
+      if (!ok) break;
+      const float inv = total > 0.f ? 1.f / total : 0.f;
+      const float lse_v = total > 0.f ? (m + log2f(total)) * kLn2 : -INFINITY;
+      const bool write = head < p.H;
+      for (int hi = 0; hi < VS::kNpv; ++hi) {
+        for (int c0 = 0; c0 < VS::kN / 2; c0 += 32) {
+          uint32_t ov[32];
+          tmem_ld32(tmem_base + lane_addr + kTmemO + hi * (VS::kN / 2) + c0, ov);
+          tmem_ld_wait();
+          const int dv0 = hi * VS::kN + (int)half * (VS::kN / 2) + c0;
+          if (!write) continue;
+          if (p.splits == 1) {
+            __nv_bfloat16* dst = p.out + ((size_t)U.row * p.H + head) * DV + dv0;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(ov[e + 0]) * inv, __uint_as_float(ov[e + 1]) * inv);
+              w.y = pack_bf16(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+              w.z = pack_bf16(__uint_as_float(ov[e + 4]) * inv, __uint_as_float(ov[e + 5]) * inv);
+              w.w = pack_bf16(__uint_as_float(ov[e + 6]) * inv, __uint_as_float(ov[e + 7]) * inv);
+              *reinterpret_cast<uint4*>(dst + e) = w;
+            }
+          } else {
+            float* dst = p.part_o + (((size_t)U.row * p.splits + U.split) * p.H + head) * DV + dv0;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + e) =
+                  make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
+                              __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+          }
+        }
+      }
+      if (write && half == 0) {
+        if (p.splits == 1) {
+          if (p.lse) p.lse[(size_t)U.row * p.H + head] = lse_v;
+        } else {
+          p.part_lse[((size_t)U.row * p.splits + U.split) * p.H + head] = lse_v;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.o_empty), 0));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+// Merge split-k partials: lse = log sum_i exp(lse_i); out = sum_i exp(lse_i - lse) o_i.
+template <int DV>
+__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
+  const int warps = blockDim.x / 32;
+  const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int n = p.B * p.Lq * p.H;
+  if (gw >= n) return;
+  const int row = gw / p.H, head = gw % p.H;
+  float mx = -INFINITY;
+  for (int sp = 0; sp < p.splits; ++sp)
+    mx = fmaxf(mx, p.part_lse[((size_t)row * p.splits + sp) * p.H + head]);
+  float wsum = 0.f;
+  float acc[DV / 32];
+#pragma unroll
+  for (int e = 0; e < DV / 32; ++e) acc[e] = 0.f;
+  if (mx > -INFINITY) {
+    for (int sp = 0; sp < p.splits; ++sp) {
+      const size_t prow = ((size_t)row * p.splits + sp) * p.H + head;
+      const float wgt = expf(p.part_lse[prow] - mx);
+      wsum += wgt;
+      const float* src = p.part_o + prow * DV;
+#pragma unroll
+      for (int e = 0; e < DV / 32; ++e) acc[e] = fmaf(wgt, src[e * 32 + lane], acc[e]);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  __nv_bfloat16* dst = p.out + ((size_t)row * p.H + head) * DV;
+#pragma unroll
+  for (int e = 0; e < DV / 32; ++e) dst[e * 32 + lane] = __float2bfloat16_rn(acc[e] * inv);
+  if (lane == 0 && p.lse) p.lse[(size_t)row * p.H + head] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
+}
+
+template <int NC, int DV>
+cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkv, int grid_clusters,
+                     cudaStream_t stream) {
+  const size_t smem = attn_smem_bytes(NC * 64, DV);
+  auto kern = sparse_attn_kernel<NC, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid_clusters * 2, kThreads, smem, stream>>>(tq, tkv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attn_smem_bytes(int d_qk, int d_v) {
+  const int nc = d_qk / 64;
+  const int n = d_v >= 256 ? 256 : d_v;
+  const size_t v_stage = (size_t)(n / 128) * kPlane128;
+  size_t b = sizeof(AttnBarriers) + 1024;          // barriers + alignment slack
+  b += (size_t)nc * kPlane64;                      // Q
+  b += (size_t)kKStages * kPlane64;                // K ring
+  b += (size_t)kVStages * v_stage;                 // V ring
+  b += 4 * (size_t)kPlane64;                       // P double buffer
+  return b;
+}
+
+cudaError_t launch_sparse_attn(const AttnParams& p, int d_qk, int d_v, const CUtensorMap& tq,
+                               const CUtensorMap& tkv, int grid_clusters, cudaStream_t stream) {
+  if (d_qk == 576 && d_v == 512) return launch_t<9, 512>(p, tq, tkv, grid_clusters, stream);
+  if (d_qk == 192 && d_v == 128) return launch_t<3, 128>(p, tq, tkv, grid_clusters, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t stream) {
+  const int n = p.B * p.Lq * p.H;
+  const int grid = (n + 3) / 4;
+  if (d_v == 512) attn_combine_kernel<512><<<grid, 128, 0, stream>>>(p);
+  else if (d_v == 128) attn_combine_kernel<128><<<grid, 128, 0, stream>>>(p);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

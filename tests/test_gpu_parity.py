@@ -1,0 +1,272 @@
+"""CUDA path vs the fp64 oracle, through the C ABI, on seeded synthetic inputs.
+
+Stage tests feed each entry point inputs whose oracle answer is known (oracle
+scores into dsa_topk, oracle index sets into dsa_sparse_attn), so every stage is
+judged on its own; forward tests run the whole pass at the workload sizes and
+compare sampled rows."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_19_b200 as dsa
+from dsa_inputs import WORKLOADS, make_inputs, make_key_side, make_query_side
+import parity as P
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    dsa.lib()
+    yield
+    assert dsa.device_status() == 0
+
+
+def to_dev(d):
+    return {k: v.to(DEV) for k, v in d.items()}
+
+
+# ------------------------------------------------------------------ indexer
+
+def _indexer_case(wl, seed, rows=None):
+    inp = to_dev(make_inputs(wl, "cpu", seed))
+    scores = dsa.indexer_scores(inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], wl.q_offset)
+    torch.cuda.synchronize()
+    n = wl.B * wl.Lq
+    rows = np.arange(n) if rows is None else np.asarray(rows)
+    r = oracle.rows_from_inputs(inp, rows, wl.Lq, wl.q_offset)
+    keys = oracle.keys_from_inputs(inp)
+    ora = oracle.indexer_scores(r["row_b"], r["row_t"], r["q_I"], r["q_scale"], r["w"], keys["k_I"], keys["k_scale"])
+    gpu = scores.reshape(n, wl.Lk)[torch.as_tensor(rows, device=DEV)].double().cpu().numpy()
+    return gpu, ora, r
+
+
+def test_indexer_integer_config_is_exact():
+    wl = WORKLOADS["tiny"]
+    gpu, ora, r = _indexer_case(wl, 0)
+    assert np.array_equal(np.isneginf(gpu), np.isneginf(ora))     # -inf exactly above the diagonal
+    fin = np.isfinite(ora)
+    assert np.array_equal(gpu[fin], ora[fin])
+
+
+def test_indexer_fp8_scaled_ragged_sizes():
+    # prefill distributions (per-token scales, salient keys), sizes off every tile multiple
+    wl = WORKLOADS["prefill_32k"].with_(Lq=700, Lk=700)
+    rows = np.r_[0:9, 120:136, 300:310, 690:700]
+    gpu, ora, r = _indexer_case(wl, 1, rows)
+    assert np.all(np.isneginf(gpu[np.isneginf(ora)]))
+    P.check_scores(gpu, ora, r["row_t"])
+
+
+def test_indexer_query_offset_chunk():
+    wl = WORKLOADS["prefill_8k"].with_(Lq=200, Lk=1000, q_offset=800)
+    rows = np.r_[0:5, 97:103, 195:200]
+    gpu, ora, r = _indexer_case(wl, 2, rows)
+    P.check_scores(gpu, ora, r["row_t"])
+
+
+def test_indexer_decode_batches_split_keys():
+    wl = WORKLOADS["decode_128k"].with_(B=3, Lk=20001, q_offset=20000)
+    gpu, ora, r = _indexer_case(wl, 3)
+    P.check_scores(gpu, ora, r["row_t"])
+
+
+# ------------------------------------------------------------------ top-k
+
+def _topk_case(scores_f32, q_offset, k, exact=True):
+    """scores_f32: torch fp32 [B, Lq, Lk] on the device."""
+    B, Lq, Lk = scores_f32.shape
+    idx = dsa.topk(scores_f32, k, q_offset)
+    torch.cuda.synchronize()
+    sc = scores_f32.double().cpu().numpy().reshape(B * Lq, Lk)
+    row_t = q_offset + np.arange(B * Lq) % Lq
+    exp = oracle.topk(sc, row_t, k)
+    got = idx.cpu().numpy().reshape(B * Lq, k)
+    assert np.array_equal(got, exp)
+    return got
+
+
+def test_topk_on_oracle_scores_integer_config():
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl, "cpu", 0)
+    r = oracle.rows_from_inputs(inp, np.arange(wl.Lq), wl.Lq, 0)
+    keys = oracle.keys_from_inputs(inp)
+    sc = oracle.indexer_scores(r["row_b"], r["row_t"], r["q_I"], r["q_scale"], r["w"], keys["k_I"], keys["k_scale"])
+    s32 = torch.from_numpy(sc.astype(np.float32)).reshape(1, wl.Lq, wl.Lk).to(DEV)
+    _topk_case(s32, 0, wl.k)
+
+
+def test_topk_rounded_scores_with_ties_and_offset():
+    g = torch.Generator().manual_seed(11)
+    s = torch.round(torch.randn(2, 37, 5000, generator=g) * 10) / 10        # heavy ties
+    _topk_case(s.to(DEV), 4963, 2048)
+
+
+def test_topk_long_rows_streamed_from_global():
+    g = torch.Generator().manual_seed(12)
+    s = torch.randn(2, 1, 140000, generator=g)
+    s[0, 0, 1000:1100] = 0.0
+    s[0, 0, 1100:1200] = -0.0
+    _topk_case(s.to(DEV), 139999, 2048)
+
+
+def test_topk_edge_cases():
+    # all-equal rows select the first k positions; +-0 are equal; short rows take everything
+    s = torch.full((1, 4, 3000), 2.5)
+    s[0, 1] = 0.0
+    s[0, 1, ::2] = -0.0
+    s[0, 2] = torch.arange(3000, dtype=torch.float32) % 7
+    got = _topk_case(s.to(DEV), 2996, 1000)
+    assert list(got[0]) == list(range(1000))
+    assert list(got[1]) == list(range(1000))
+    short = torch.randn(1, 5, 64)
+    got = _topk_case(short.to(DEV), 0, 16)
+    assert list(got[0][:1]) == [0] and np.all(got[0][1:] == -1)
+
+
+def test_topk_boundary_bin_larger_than_candidate_buffer():
+    # 30000 identical values straddle the threshold: the candidate list overflows
+    # and the digit passes fall back to scanning the row.
+    s = torch.randn(1, 2, 33000)
+    s[:, :, 1000:31000] = 1.0
+    s[:, 1, 31000:] = 5.0
+    _topk_case(s.to(DEV), 32998, 2048)
+
+
+# ------------------------------------------------------------------ sparse attention
+
+def _attn_case(B, Lq, Lk, k, H, D, Dv, idx_np, seed, q_offset_for_oracle=0):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Lq, H, D, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, Lk, D, generator=g).to(torch.bfloat16)
+    idx = torch.from_numpy(idx_np.astype(np.int32)).reshape(B, Lq, k)
+    out, lse = dsa.sparse_attn(q.to(DEV), kv.to(DEV), idx.to(DEV), Dv, 1.0 / math.sqrt(192.0))
+    torch.cuda.synchronize()
+    rows = np.arange(B * Lq)
+    ora_idx = idx_np.reshape(B * Lq, k).copy()
+    ora_idx[(ora_idx < 0) | (ora_idx >= Lk)] = -1
+    oo, ol = oracle.sparse_attn(rows // Lq, P.bf16_bits(q).reshape(B * Lq, H, D), P.bf16_bits(kv), ora_idx,
+                                1.0 / math.sqrt(192.0), Dv)
+    err = P.check_attention(out.reshape(B * Lq, H, Dv), lse.reshape(B * Lq, H), oo, ol)
+    return out, lse, err
+
+
+def _compact_indices(rng, B, Lq, Lk, k, q_offset):
+    idx = np.full((B * Lq, k), -1, np.int64)
+    for r in range(B * Lq):
+        t = q_offset + r % Lq
+        m = min(k, t + 1)
+        idx[r, :m] = np.sort(rng.choice(t + 1, size=m, replace=False))
+    return idx
+
+
+def test_attention_tiny_shape_all_rows():
+    wl = WORKLOADS["tiny"]
+    rng = np.random.default_rng(5)
+    idx = _compact_indices(rng, 1, 300, 1024, wl.k, 724)
+    _attn_case(1, 300, 1024, wl.k, wl.H, wl.D, wl.Dv, idx, 5)
+
+
+def test_attention_mla_shape_padding_and_gaps():
+    rng = np.random.default_rng(6)
+    B, Lq, Lk, k = 1, 24, 3000, 2048
+    idx = _compact_indices(rng, B, Lq, Lk, k, 2980)
+    idx[3, 100:400] = -1                # holes in the middle of a row
+    idx[4, ::3] = Lk + 5                # out-of-range entries are skipped
+    idx[5, :] = -1
+    idx[5, 777] = 42                    # a single selected key
+    idx[6, :1500] = -1                  # only the tail of the row is valid
+    out, lse, _ = _attn_case(B, Lq, Lk, k, 128, 576, 512, idx, 6)
+
+
+def test_attention_row_without_valid_entries():
+    idx = np.full((1, 2, 256), -1, np.int64)
+    idx[0, 1, :5] = [1, 2, 3, 4, 5]
+    out, lse, _ = _attn_case(1, 2, 64, 256, 128, 576, 512, idx, 7)
+    assert torch.all(out[0, 0] == 0) and torch.all(torch.isneginf(lse[0, 0]))
+
+
+def test_attention_decode_split_k():
+    rng = np.random.default_rng(8)
+    B, Lk, k = 6, 5000, 2048
+    idx = np.stack([np.sort(rng.choice(Lk, size=k, replace=False)) for _ in range(B)])
+    _attn_case(B, 1, Lk, k, 128, 576, 512, idx, 8)
+
+
+# ------------------------------------------------------------------ whole forward
+
+def _forward(inp, wl, q_offset=None, Lq=None):
+    q_offset = wl.q_offset if q_offset is None else q_offset
+    idx, out, lse = dsa.forward(inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], inp["q"],
+                                inp["kv"], wl.k, wl.Dv, wl.scale, q_offset)
+    torch.cuda.synchronize()
+    return idx, out, lse
+
+
+def _check_forward_rows(inp, wl, idx, out, lse, rows, Lq, q_offset, exact_idx=False):
+    res, keys = P.oracle_forward_rows(inp, rows, Lq, q_offset, wl.k, wl.scale, wl.Dv)
+    sel = torch.as_tensor(rows, device=DEV)
+    gi = idx.reshape(-1, wl.k)[sel].cpu().numpy()
+    swaps = P.check_index_sets(gi, res["scores"], res["row_t"], wl.k, exact=exact_idx)
+    # attention judged on the GPU's own index set
+    oo, ol = oracle.sparse_attn(res["row_b"], res["q"], keys["kv"], gi, wl.scale, wl.Dv)
+    go = out.reshape(-1, wl.H, wl.Dv)[sel]
+    gl = lse.reshape(-1, wl.H)[sel]
+    err = P.check_attention(go, gl, oo, ol)
+    return swaps, err
+
+
+def test_forward_tiny_all_rows_exact_indices():
+    wl = WORKLOADS["tiny"]
+    inp = to_dev(make_inputs(wl, "cpu", 0))
+    idx, out, lse = _forward(inp, wl)
+    _check_forward_rows(inp, wl, idx, out, lse, np.arange(wl.Lq), wl.Lq, 0, exact_idx=True)
+
+
+def test_forward_prefill_8k_sampled_rows():
+    wl = WORKLOADS["prefill_8k"]
+    inp = make_inputs(wl, DEV, 0)
+    idx, out, lse = _forward(inp, wl)
+    rows = np.r_[0, 1, 2, 127, 128, 1000, 2046, 2047, 2048, 2049, 4095, 5000, 8190, 8191]
+    _check_forward_rows(inp, wl, idx, out, lse, rows, wl.Lq, 0)
+
+
+def test_forward_decode_128k_sampled_sequences():
+    wl = WORKLOADS["decode_128k"]
+    inp = make_key_side(wl, DEV, 0)
+    inp.update(make_query_side(wl, DEV, 0))
+    idx, out, lse = _forward(inp, wl)
+    _check_forward_rows(inp, wl, idx, out, lse, np.array([0, 17, 40, 63]), 1, wl.q_offset)
+
+
+def test_forward_prefill_32k_sampled_rows():
+    wl = WORKLOADS["prefill_32k"]
+    inp = make_inputs(wl, DEV, 0)
+    idx, out, lse = _forward(inp, wl)
+    rows = np.r_[0, 5, 2047, 2048, 9000, 16384, 30000, 32766, 32767]
+    _check_forward_rows(inp, wl, idx, out, lse, rows, wl.Lq, 0)
+
+
+def test_forward_prefill_128k_last_chunk_sampled_rows():
+    wl = WORKLOADS["prefill_128k"]
+    keys = make_key_side(wl, DEV, 0)
+    c = wl.Lq // wl.chunk - 1
+    q_offset = c * wl.chunk
+    qs = make_query_side(wl, DEV, 0, chunk_index=c, Lq=wl.chunk)
+    inp = dict(keys, **qs)
+    cw = wl.with_(Lq=wl.chunk, q_offset=q_offset)
+    idx, out, lse = _forward(inp, cw)
+    _check_forward_rows(inp, cw, idx, out, lse, np.array([0, 2048, 4095]), cw.Lq, q_offset)
+
+
+def test_wait_timeout_is_reported_not_trapped():
+    assert dsa.selftest_wait_timeout(1 << 14) == 5
+    assert dsa.device_status() == 0
+    x = torch.ones(4, device=DEV)
+    assert float(x.sum()) == 4.0          # the context is still usable
