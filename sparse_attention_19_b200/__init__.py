@@ -220,6 +220,9 @@ def forward(q_I, q_scale, w, k_I, k_scale, q, kv, k, d_v, scale, q_offset=0, ind
     if stage_events is not None:
         if len(stage_events) != 4:
             raise ValueError("stage_events needs four events")
+        for e in stage_events:          # torch creates the CUDA event on first use
+            if not e.cuda_event:
+                e.record(stream if stream is not None else torch.cuda.current_stream())
         ev = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
     _check(lib().dsa_forward_timed(ctypes.byref(ia), ctypes.byref(aa), int(k), _ptr(indices), _ptr(out), _ptr(lse),
                                    _ptr(workspace), nbytes, _stream(stream), ev), "dsa_forward")

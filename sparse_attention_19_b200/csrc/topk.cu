@@ -34,7 +34,9 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-struct TopkShared {
+// 16-byte multiple, so the row cache and the 8-byte candidate pairs that follow
+// it in dynamic shared memory stay aligned.
+struct alignas(16) TopkShared {
   uint32_t hist[2048];
   uint32_t warp_tot[kWarps];
   uint32_t bin, above, ncand;
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
   uint32_t* cache = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
-  uint2* cand = reinterpret_cast<uint2*>(cache + p.cache_cap);
+  uint2* cand = reinterpret_cast<uint2*>(cache + (p.cache_cap + 3) / 4 * 4);
 
   const int row = blockIdx.x;                       // b * Lq + i
   const int i = row % p.Lq;
@@ -197,7 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
 }  // namespace
 
 size_t topk_smem_bytes(int cache_cap, int cand_cap) {
-  return sizeof(TopkShared) + (size_t)cache_cap * 4 + (size_t)cand_cap * 8;
+  static_assert(sizeof(TopkShared) % 16 == 0, "candidate pairs must stay 8-byte aligned");
+  return sizeof(TopkShared) + (size_t)((cache_cap + 3) / 4 * 4) * 4 + (size_t)cand_cap * 8;
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream) {
