@@ -26,7 +26,7 @@ struct IndexerParams {
   const float* k_scale;   // [B, Lk] or null
   float* scores;          // [B, Lq, Lk]
 };
-size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats);
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages);
 cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                            int grid, cudaStream_t stream);
 

@@ -30,14 +30,14 @@ namespace dsa {
 namespace {
 
 constexpr int kKeysPerTile = 128;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 8;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 
 struct IndexerSmem {
   // Barriers and small per-unit data first; big tiles follow at a 1024-byte boundary.
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t k_full[kMaxStages], k_empty[kMaxStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t final_bar;
   uint64_t epi_bar;          // rendezvous of the 4 epilogue warps
@@ -68,7 +68,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const IndexerParams& p, int u) {
   return info;
 }
 
-template <int H_I, int D_I>
+template <int H_I, int D_I, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                const IndexerParams p) {
@@ -280,12 +280,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   }
 }
 
-template <int H_I, int D_I>
+template <int H_I, int D_I, int kStages>
 cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              int grid, cudaStream_t stream) {
   const size_t smem = indexer_smem_bytes(p.nsub * p.qb * H_I, D_I, p.queries_per_unit * H_I,
-                                         p.queries_per_unit);
-  auto kern = indexer_kernel<H_I, D_I>;
+                                         p.queries_per_unit, kStages);
+  auto kern = indexer_kernel<H_I, D_I, kStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
@@ -294,10 +294,10 @@ cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, cons
 
 }  // namespace
 
-size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats) {
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages) {
   size_t b = sizeof(IndexerSmem) + 1024;                       // barriers + alignment slack
   b += (size_t)q_rows * d_I;                                   // resident query block
-  b += (size_t)kStages * kKeysPerTile * d_I;                   // key ring
+  b += (size_t)stages * kKeysPerTile * d_I;                    // key ring
   b += (size_t)(w_floats + sq_floats) * sizeof(float);
   // At least ~116 KB so that one CTA (and its 512 TMEM columns) owns each SM.
   return b < 118784 ? 118784 : b;
@@ -305,8 +305,12 @@ size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats) {
 
 cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                            int grid, cudaStream_t stream) {
-  if (p.H_I == 64 && p.d_I == 128) return launch_indexer_t<64, 128>(p, tq, tk, grid, stream);
-  if (p.H_I == 4 && p.d_I == 64) return launch_indexer_t<4, 64>(p, tq, tk, grid, stream);
+  // A small resident query block (decode) leaves room for a deeper key ring.
+  const bool deep = p.nsub * p.qb * p.H_I <= 128;
+  if (p.H_I == 64 && p.d_I == 128)
+    return deep ? launch_indexer_t<64, 128, 8>(p, tq, tk, grid, stream)
+                : launch_indexer_t<64, 128, 4>(p, tq, tk, grid, stream);
+  if (p.H_I == 4 && p.d_I == 64) return launch_indexer_t<4, 64, 4>(p, tq, tk, grid, stream);
   return cudaErrorInvalidValue;
 }
 

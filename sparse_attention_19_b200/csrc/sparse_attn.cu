@@ -43,25 +43,27 @@ namespace dsa {
 namespace {
 
 constexpr int kTileKeys = 128;       // keys per tile (pair)
-constexpr int kHalfKeys = 64;        // keys per CTA in S
-constexpr int kKStages = 4;          // K-chunk ring depth
-constexpr int kVStages = 2;          // V ring depth
-constexpr int kThreads = 192;
+constexpr int kHalfKeys = 64;        // keys per CTA in S, and keys per V stage
+constexpr int kKStages = 6;          // K-chunk ring depth (8 KB stages)
+constexpr int kVStages = 4;          // V ring depth (64 keys x this CTA's value planes)
+constexpr int kMaxIdx = 2048;        // selected positions per row (staged in shared memory)
+constexpr int kThreads = 224;        // 7 warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kPlane64 = 64 * 128;    // 64 rows x 128 B  (Q plane, K stage, P plane)
-constexpr uint32_t kPlane128 = 128 * 128;  // 128 rows x 128 B (V plane)
+constexpr uint32_t kPlane64 = 64 * 128;    // 64 rows x 128 B  (Q plane, K stage, V plane, P plane)
 constexpr uint32_t kTmemS = 0;             // S buffers: columns [0, 128)
 constexpr uint32_t kTmemO = 128;           // O: columns [128, 128 + d_v/2)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMaxChunks = 9;
 
 struct AttnBarriers {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[kMaxChunks], q_empty[kMaxChunks];
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
-  uint64_t o_full, o_empty, pv_done, final_bar;
+  uint64_t p_full, p_empty;
+  uint64_t o_full, o_empty, final_bar;
+  uint64_t idx_full[2], idx_empty[2];
   uint64_t xbar;             // rendezvous of the 4 softmax warps (max / sum exchange)
   uint32_t tmem_base;
   uint32_t abort_flag;
@@ -74,7 +76,7 @@ struct VShape {
   static constexpr int kNpv = DV >= 256 ? DV / 256 : 1;   // PV instructions per tile
   static constexpr int kN = DV >= 256 ? 256 : DV;         // N of one PV instruction
   static constexpr int kPlanes = kN / 128;                // 64-column planes per CTA per instruction
-  static constexpr uint32_t kStageBytes = kPlanes * kPlane128;
+  static constexpr uint32_t kStageBytes = kPlanes * kPlane64;   // 64 keys x planes
 };
 
 struct Unit {
@@ -98,16 +100,16 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams& p, int u) {
   return U;
 }
 
-__device__ __forceinline__ int kv_row(const AttnParams& p, int b, int row, int pos) {
-  int s = -1;
-  if (pos < p.k) s = __ldg(p.indices + (size_t)row * p.k + pos);
-  if (s < 0 || s >= p.Lk) s = 0;            // padding: any valid row, masked in softmax
-  return b * p.Lk + s;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Row of kv (in the [B*Lk, d_qk] view) for a staged index; padding and out-of-range
+// entries gather row b*Lk (a valid row) and are masked in the softmax.
+__device__ __forceinline__ int gather_row(const int32_t* idx, int pos, int b, int Lk) {
+  const int s = idx[pos];
+  return b * Lk + ((s >= 0 && s < Lk) ? s : 0);
 }
 
 template <int NC, int DV>
@@ -115,6 +117,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
                    const AttnParams p) {
   using VS = VShape<DV>;
+  static_assert(NC <= kMaxChunks, "d_qk");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   AttnBarriers& S = *reinterpret_cast<AttnBarriers*>(smem_raw);
   // 1024-byte aligned operand area (the 128-byte swizzle is address based).
@@ -124,7 +127,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   uint8_t* q_sm = area;                                             // NC planes
   uint8_t* k_sm = q_sm + NC * kPlane64;                             // kKStages planes
   uint8_t* v_sm = k_sm + kKStages * kPlane64;                       // kVStages x kPlanes planes
-  uint8_t* p_sm = v_sm + kVStages * VS::kStageBytes;                // 2 buffers x 2 planes
+  uint8_t* p_sm = v_sm + kVStages * VS::kStageBytes;                // 2 planes (keys 0-63, 64-127)
+  int32_t* idx_sm = reinterpret_cast<int32_t*>(p_sm + 2 * kPlane64);  // 2 x kMaxIdx
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -133,21 +137,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const int cluster_id = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
   volatile uint32_t* abort_flag = &S.abort_flag;
+  const int idx_span = p.n_tiles * kTileKeys;                       // staged positions per row
 
   if (threadIdx.x == 0) {
-    mbar_init(&S.q_full, 1);
-    mbar_init(&S.q_empty, 1);
+    for (int i = 0; i < kMaxChunks; ++i) { mbar_init(&S.q_full[i], 1); mbar_init(&S.q_empty[i], 1); }
     for (int i = 0; i < kKStages; ++i) { mbar_init(&S.k_full[i], 1); mbar_init(&S.k_empty[i], 1); }
     for (int i = 0; i < kVStages; ++i) { mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_empty[i], 8);   // 4 softmax warps x 2 CTAs
-      mbar_init(&S.p_full[i], 8);
-      mbar_init(&S.p_empty[i], 1);
+      mbar_init(&S.s_empty[i], 8);     // 4 softmax warps x 2 CTAs
+      mbar_init(&S.idx_full[i], 1);
+      mbar_init(&S.idx_empty[i], 6);   // 4 softmax warps + 2 producer warps
     }
+    mbar_init(&S.p_full, 8);
+    mbar_init(&S.p_empty, 1);
     mbar_init(&S.o_full, 1);
     mbar_init(&S.o_empty, 8);
-    mbar_init(&S.pv_done, 1);
     mbar_init(&S.final_bar, 1);
     mbar_init(&S.xbar, 4);
     S.abort_flag = 0;
@@ -165,35 +170,48 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const uint16_t kBoth = 0x3;
 
   if (warp == 4) {
-    // ------------------------------------------------------------------ producer
-    uint32_t q_use = 0, kc = 0, vc = 0;
-    const uint32_t q_full_l = mapa_shared(smem_u32(&S.q_full), 0);
+    // ------------------------------------------------------------------ K producer
+    // Per unit: stage the row's indices, load this CTA's Q planes (each plane as
+    // soon as the previous unit's last S has finished with it), then gather this
+    // CTA's 64 keys of every tile, chunk by chunk.
+    uint32_t ucount = 0, kc = 0;
     bool ok = true;
     if (lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
     for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
       const Unit U = decode_unit(p, u);
       if (U.j0 >= U.j1) continue;
-      // Q: this CTA's 64 heads, NC planes of 64 columns.
+      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+      // Q planes
       if (lane == 0) {
-        ok = mbar_wait(&S.q_empty, (q_use & 1u) ^ 1u, abort_flag);
-        if (ok) {
-          if (leader) mbar_arrive_expect_tx(&S.q_full, 2u * NC * kPlane64);
-          const int qrow = U.row * p.H + (int)rank * 64;
-          for (int c = 0; c < NC; ++c) tma_load_2d_pair(q_sm + c * kPlane64, &tmap_q, q_full_l, c * 64, qrow);
+        const int qrow = U.row * p.H + (int)rank * 64;
+        for (int c = 0; c < NC && ok; ++c) {
+          ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
+          if (!ok) break;
+          if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane64);
+          tma_load_2d_pair(q_sm + c * kPlane64, &tmap_q, mapa_shared(smem_u32(&S.q_full[c]), 0), c * 64, qrow);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++q_use;
-      // K chunks of tile j, then V of tile j-1 (the order the MMA consumes them).
-      auto load_k = [&](int j) -> bool {
-        // lanes 0..15: 4 keys each of this CTA's 64 keys
+      if (!ok) break;
+      // indices of the row -> shared memory (buffer ib, free once unit ucount-2 is done)
+      ok = mbar_wait_warp(&S.idx_empty[ib], uph ^ 1u, abort_flag);
+      if (!ok) break;
+      {
+        int32_t* dst = idx_sm + ib * kMaxIdx;
+        const int32_t* src = p.indices + (size_t)U.row * p.k;
+        for (int x = (int)lane; x < idx_span; x += 32) dst[x] = (x < p.k) ? __ldg(src + x) : -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.idx_full[ib]);
+      }
+      const int32_t* idx = idx_sm + ib * kMaxIdx;
+      for (int j = U.j0; j < U.j1 && ok; ++j) {
         int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
         if (lane < 16) {
           const int base = j * kTileKeys + (int)rank * kHalfKeys + (int)lane * 4;
-          r0 = kv_row(p, U.b, U.row, base + 0);
-          r1 = kv_row(p, U.b, U.row, base + 1);
-          r2 = kv_row(p, U.b, U.row, base + 2);
-          r3 = kv_row(p, U.b, U.row, base + 3);
+          r0 = gather_row(idx, base + 0, U.b, p.Lk);
+          r1 = gather_row(idx, base + 1, U.b, p.Lk);
+          r2 = gather_row(idx, base + 2, U.b, p.Lk);
+          r3 = gather_row(idx, base + 3, U.b, p.Lk);
         }
         for (int c = 0; c < NC; ++c) {
           const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
@@ -203,45 +221,60 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             if (w_ok && leader) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
           }
           w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-          if (!w_ok) return false;
+          if (!w_ok) { ok = false; break; }
           const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
           if (lane < 16)
             tma_gather4_pair(k_sm + st * kPlane64 + lane * 512, &tmap_kv, full_l, c * 64, r0, r1, r2, r3);
           ++kc;
         }
-        return true;
-      };
-      auto load_v = [&](int j) -> bool {
-        // lanes 0..31: 4 keys each of all 128 keys of the tile
-        const int base = j * kTileKeys + (int)lane * 4;
-        const int r0 = kv_row(p, U.b, U.row, base + 0);
-        const int r1 = kv_row(p, U.b, U.row, base + 1);
-        const int r2 = kv_row(p, U.b, U.row, base + 2);
-        const int r3 = kv_row(p, U.b, U.row, base + 3);
-        for (int h = 0; h < VS::kNpv; ++h) {
-          const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
-          bool w_ok = true;
-          if (lane == 0) {
-            w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
-            if (w_ok && leader) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
-          }
-          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-          if (!w_ok) return false;
-          const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
-          for (int pl = 0; pl < VS::kPlanes; ++pl) {
-            const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
-            tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane128 + lane * 512, &tmap_kv, full_l,
-                             col, r0, r1, r2, r3);
-          }
-          ++vc;
-        }
-        return true;
-      };
-      for (int j = U.j0; j < U.j1 && ok; ++j) {
-        ok = load_k(j);
-        if (ok && j > U.j0) ok = load_v(j - 1);
       }
-      if (ok) ok = load_v(U.j1 - 1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+      ++ucount;
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ V producer
+    // For every tile: all 128 keys x this CTA's value columns, 64 keys per stage.
+    uint32_t ucount = 0, vc = 0;
+    bool ok = true;
+    for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
+      const Unit U = decode_unit(p, u);
+      if (U.j0 >= U.j1) continue;
+      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
+      if (!ok) break;
+      const int32_t* idx = idx_sm + ib * kMaxIdx;
+      const int pl = (int)lane / 16;                  // value plane this lane fills
+      const int g = (int)lane % 16;                   // 4-key group within the stage
+      for (int j = U.j0; j < U.j1 && ok; ++j) {
+        for (int kh = 0; kh < 2 && ok; ++kh) {
+          const int base = j * kTileKeys + kh * kHalfKeys + g * 4;
+          const int r0 = gather_row(idx, base + 0, U.b, p.Lk);
+          const int r1 = gather_row(idx, base + 1, U.b, p.Lk);
+          const int r2 = gather_row(idx, base + 2, U.b, p.Lk);
+          const int r3 = gather_row(idx, base + 3, U.b, p.Lk);
+          for (int h = 0; h < VS::kNpv; ++h) {
+            const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+            bool w_ok = true;
+            if (lane == 0) {
+              w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
+              if (w_ok && leader) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
+            }
+            w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+            if (!w_ok) { ok = false; break; }
+            const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
+            if (pl < VS::kPlanes) {
+              const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
+              tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + g * 512, &tmap_kv, full_l, col,
+                               r0, r1, r2, r3);
+            }
+            ++vc;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+      ++ucount;
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ MMA issuer
@@ -250,14 +283,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       constexpr uint32_t idesc_pv = make_idesc(1, 1, 128, VS::kN, 0, 1);         // P K-major, V MN-major
       const uint32_t q_base = smem_u32(q_sm), k_base = smem_u32(k_sm);
       const uint32_t v_base = smem_u32(v_sm), p_base = smem_u32(p_sm);
-      uint32_t q_use = 0, kc = 0, vc = 0, sc = 0, pc = 0, oc = 0;
+      uint32_t ucount = 0, kc = 0, vc = 0, sc = 0, pc = 0, oc = 0;
       bool ok = true;
-      auto issue_s = [&](bool last_of_unit) -> bool {
+      auto issue_s = [&](bool first_of_unit, bool last_of_unit) -> bool {
         const uint32_t sb = sc & 1u;
         if (!mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag, true)) return false;
         tc_fence_after();
         const uint32_t d = tmem_base + kTmemS + sb * kHalfKeys;
         for (int c = 0; c < NC; ++c) {
+          if (first_of_unit && !mbar_wait(&S.q_full[c], ucount & 1u, abort_flag)) return false;
           const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
           if (!mbar_wait(&S.k_full[st], ph, abort_flag)) return false;
           tc_fence_after();
@@ -268,36 +302,35 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             mma_bf16_ss_pair(d, ad, bd, idesc_s, (c | kk) ? 1u : 0u);
           }
           mma_commit_pair_mc(&S.k_empty[st], kBoth);
+          if (last_of_unit) mma_commit_pair_mc(&S.q_empty[c], kBoth);   // Q plane c free for the next unit
           ++kc;
         }
         mma_commit_pair_mc(&S.s_full[sb], kBoth);
-        if (last_of_unit) mma_commit_pair_mc(&S.q_empty, kBoth);
         ++sc;
         return true;
       };
       auto issue_pv = [&](bool first_of_unit, bool last_of_unit) -> bool {
-        const uint32_t pb = pc & 1u;
-        if (!mbar_wait(&S.p_full[pb], (pc >> 1) & 1u, abort_flag, true)) return false;
+        if (!mbar_wait(&S.p_full, pc & 1u, abort_flag, true)) return false;
         if (first_of_unit && !mbar_wait(&S.o_empty, (oc & 1u) ^ 1u, abort_flag, true)) return false;
         tc_fence_after();
-        for (int h = 0; h < VS::kNpv; ++h) {
-          const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
-          if (!mbar_wait(&S.v_full[st], ph, abort_flag)) return false;
-          tc_fence_after();
-          const uint32_t d = tmem_base + kTmemO + h * (VS::kN / 2);
+        for (int kh = 0; kh < 2; ++kh) {
+          for (int h = 0; h < VS::kNpv; ++h) {
+            const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+            if (!mbar_wait(&S.v_full[st], ph, abort_flag)) return false;
+            tc_fence_after();
+            const uint32_t d = tmem_base + kTmemO + h * (VS::kN / 2);
 #pragma unroll
-          for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-            const uint64_t ad = make_smem_desc(p_base + pb * 2 * kPlane64 + (kk >> 2) * kPlane64 + (kk & 3) * 32,
-                                               16, 1024, LAYOUT_SW128);
-            const uint64_t bd = make_smem_desc(v_base + st * VS::kStageBytes + kk * 2048, kPlane128, 1024,
-                                               LAYOUT_SW128);
-            mma_bf16_ss_pair(d, ad, bd, idesc_pv, (first_of_unit && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < kHalfKeys / 16; ++kk) {
+              const uint64_t ad = make_smem_desc(p_base + kh * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
+              const uint64_t bd = make_smem_desc(v_base + st * VS::kStageBytes + kk * 2048, kPlane64, 1024,
+                                                 LAYOUT_SW128);
+              mma_bf16_ss_pair(d, ad, bd, idesc_pv, (first_of_unit && kh == 0 && kk == 0) ? 0u : 1u);
+            }
+            mma_commit_pair_mc(&S.v_empty[st], kBoth);
+            ++vc;
           }
-          mma_commit_pair_mc(&S.v_empty[st], kBoth);
-          ++vc;
         }
-        mma_commit_pair_mc(&S.p_empty[pb], kBoth);
-        mma_commit_pair_mc(&S.pv_done, kBoth);
+        mma_commit_pair_mc(&S.p_empty, kBoth);
         if (last_of_unit) { mma_commit_pair_mc(&S.o_full, kBoth); ++oc; }
         ++pc;
         return true;
@@ -305,14 +338,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
         const Unit U = decode_unit(p, u);
         if (U.j0 >= U.j1) continue;
-        ok = mbar_wait(&S.q_full, q_use & 1u, abort_flag);
-        ++q_use;
-        tc_fence_after();
         for (int j = U.j0; j < U.j1 && ok; ++j) {
-          ok = issue_s(j == U.j1 - 1);
+          ok = issue_s(j == U.j0, j == U.j1 - 1);
           if (ok && j > U.j0) ok = issue_pv(j - 1 == U.j0, false);
         }
         if (ok) ok = issue_pv(U.j1 - 1 == U.j0, true);
+        ++ucount;
       }
       // Wait until every MMA this thread issued has completed before teardown.
       mma_commit(&S.final_bar);
@@ -325,7 +356,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     const uint32_t half = l >> 6;                 // which 64 keys of the tile this lane holds
     const int head = (int)rank * 64 + (int)h;
     const uint32_t lane_addr = (warp * 32u) << 16;
-    uint32_t sc = 0, pc = 0, oc = 0, xph = 0;
+    uint32_t ucount = 0, sc = 0, pc = 0, oc = 0, xph = 0;
     bool ok = true;
     for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
       const Unit U = decode_unit(p, u);
@@ -339,6 +370,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         }
         continue;
       }
+      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
+      if (!ok) break;
+      const int32_t* idx = idx_sm + ib * kMaxIdx;
       float m = -INFINITY, lsum = 0.f;
       for (int j = U.j0; j < U.j1 && ok; ++j) {
         const uint32_t sb = sc & 1u;
@@ -359,13 +394,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         ++sc;
         // Scale into log2 units and mask padding / out-of-range positions.
         const int kbase = j * kTileKeys + (int)half * kHalfKeys;
-        const int32_t* irow = p.indices + (size_t)U.row * p.k;
         float x[64];
         float tmax = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          const int pos = kbase + c;
-          const int s = (pos < p.k) ? __ldg(irow + pos) : -1;
+          const int s = idx[kbase + c];
           const bool valid = (s >= 0) && (s < p.Lk);
           x[c] = valid ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
           tmax = fmaxf(tmax, x[c]);
@@ -377,59 +410,55 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         tmax = fmaxf(tmax, S.red_max[rb][l ^ 64u]);
         const float m_new = fmaxf(m, tmax);
         const bool first = (j == U.j0);
-        if (first) {
-          m = m_new;
-        } else {
-          const bool need = m_new > m + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, need)) {
-            // PV of the previous tile must be complete before O is touched.
-            ok = mbar_wait_warp(&S.pv_done, (pc - 1u) & 1u, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            const float alpha = need ? exp2f(m - m_new) : 1.f;
-            for (int c0 = 0; c0 < VS::kNpv * (VS::kN / 2); c0 += 32) {
-              uint32_t ov[32];
-              tmem_ld32(tmem_base + lane_addr + kTmemO + c0, ov);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-              tmem_st32(tmem_base + lane_addr + kTmemO + c0, ov);
-            }
-            tmem_st_wait();
-            if (need) { lsum *= alpha; m = m_new; }
-          }
-        }
-        const float m_use = (m == -INFINITY) ? 0.f : m;
-        // P buffer reuse: PV two tiles back must be done.
-        const uint32_t pb = pc & 1u;
-        if (pc >= 2) {
-          ok = mbar_wait_warp(&S.p_empty[pb], ((pc >> 1) & 1u) ^ 1u, abort_flag);
-          if (!ok) break;
-        }
-        uint8_t* prow = p_sm + pb * 2 * kPlane64 + half * kPlane64 + (h >> 3) * 1024 + (h & 7) * 128;
+        const bool need = first || (m_new > m + kRescaleThreshold);
+        const float m_ref = need ? m_new : m;
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        // probabilities in bf16 (the sum uses the rounded values, matching what P.V sees)
+        uint32_t pw[32];
         float psum = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = exp2f(x[c * 8 + 2 * e] - m_use);
-            const float p1 = exp2f(x[c * 8 + 2 * e + 1] - m_use);
-            const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-            const float2 back = __bfloat1622float2(v2);
-            psum += back.x + back.y;
-            w4[e] = *reinterpret_cast<const uint32_t*>(&v2);
-          }
-          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int e = 0; e < 32; ++e) {
+          const __nv_bfloat162 v2 = __floats2bfloat162_rn(exp2f(x[2 * e] - m_use), exp2f(x[2 * e + 1] - m_use));
+          const float2 back = __bfloat1622float2(v2);
+          psum += back.x + back.y;
+          pw[e] = *reinterpret_cast<const uint32_t*>(&v2);
         }
+        // The single P buffer (and O) are free once the previous tile's P.V is done.
+        if (pc >= 1) {
+          ok = mbar_wait_warp(&S.p_empty, (pc - 1u) & 1u, abort_flag);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        if (!first && __any_sync(0xffffffffu, need)) {
+          const float alpha = need ? exp2f(m - m_new) : 1.f;
+          for (int c0 = 0; c0 < VS::kNpv * (VS::kN / 2); c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tmem_base + lane_addr + kTmemO + c0, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tmem_base + lane_addr + kTmemO + c0, ov);
+          }
+          tmem_st_wait();
+          if (need) lsum *= alpha;
+        }
+        if (need) m = m_new;
         lsum += psum;
+        uint8_t* prow = p_sm + half * kPlane64 + (h >> 3) * 1024 + (h & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) =
+              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.p_full[pb]), 0));
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.p_full), 0));
         ++pc;
       }
       if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+      ++ucount;
       // ---- epilogue of the unit
       ok = mbar_wait_warp(&S.o_full, oc & 1u, abort_flag);
       ++oc;
@@ -543,12 +572,13 @@ cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorM
 size_t attn_smem_bytes(int d_qk, int d_v) {
   const int nc = d_qk / 64;
   const int n = d_v >= 256 ? 256 : d_v;
-  const size_t v_stage = (size_t)(n / 128) * kPlane128;
+  const size_t v_stage = (size_t)(n / 128) * kPlane64;
   size_t b = sizeof(AttnBarriers) + 1024;          // barriers + alignment slack
   b += (size_t)nc * kPlane64;                      // Q
   b += (size_t)kKStages * kPlane64;                // K ring
   b += (size_t)kVStages * v_stage;                 // V ring
-  b += 4 * (size_t)kPlane64;                       // P double buffer
+  b += 2 * (size_t)kPlane64;                       // P (keys 0-63, 64-127)
+  b += 2 * (size_t)kMaxIdx * sizeof(int32_t);      // staged indices, two units
   return b;
 }
 
