@@ -12,7 +12,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/dsa.h"
+#include "dsa.h"
 #include "dsa_internal.h"
 #include "ptx.cuh"
 
@@ -142,8 +142,8 @@ dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper
   if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->q_I, (uint64_t)a->B * a->Lq * a->H_I, a->d_I,
                  a->d_I, (uint32_t)(p.qb * a->H_I), swz))
     return DSA_ERR_CUDA;
-  if (!make_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 128,
-                 swz))
+  if (!make_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 32,
+                 swz))                                     // key tiles arrive as four 32-row boxes
     return DSA_ERR_CUDA;
   const int grid = p.n_units < sms ? p.n_units : sms;
   return launch_indexer(p, tq, tk, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

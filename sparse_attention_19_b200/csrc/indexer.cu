@@ -14,8 +14,8 @@
 // shared memory and streams key tiles through a TMA ring; two TMEM accumulators
 // let the epilogue of one sub-block overlap the MMA of the next.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
-// warps 2..5 epilogue (warp w reads TMEM lanes 32*(w%4) .. +31).
+// Warp roles (288 threads): warps 0..3 epilogue (warp w reads TMEM lanes 32w .. 32w+31),
+// warp 4 TMEM owner + MMA issuer, warps 5..8 TMA loaders.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -31,7 +31,10 @@ namespace {
 
 constexpr int kKeysPerTile = 128;
 constexpr int kMaxStages = 8;
-constexpr int kThreads = 192;
+constexpr int kThreads = 288;        // warps 0-3 epilogue, 4 MMA, 5-8 loaders
+constexpr int kLoaders = 4;          // TMA requests from one warp are served in order, so each
+                                     // key tile is loaded as four 32-row boxes from four warps
+constexpr int kLoaderWarp0 = 5;
 constexpr int kTmemCols = 512;
 
 struct IndexerSmem {
@@ -109,7 +112,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 4) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -118,33 +121,37 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp >= kLoaderWarp0) {
+    // ------------------------------------------------------------ TMA loaders
+    // Loader 0 also loads the query block; every loader fills rows [32*pw, 32*pw+32)
+    // of each key stage.
+    const int pw = (int)warp - kLoaderWarp0;
     if (elect_one()) {
-      prefetch_tmap(&tmap_q);
-      prefetch_tmap(&tmap_k);
+      if (pw == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_k); }
       uint32_t q_phase = 0, kstage = 0, kphase = 0;
       for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
         const UnitInfo U = decode_unit(p, u);
-        if (!mbar_wait(&S.q_empty, q_phase ^ 1, abort_flag)) break;
-        q_phase ^= 1;
-        mbar_arrive_expect_tx(&S.q_full, (uint32_t)(p.nsub * N) * kRowBytes);
-        for (int sb = 0; sb < p.nsub; ++sb) {
-          const int row = ((U.b * p.Lq) + U.i0 + sb * p.qb) * H_I;
-          tma_load_2d(q_smem + (size_t)sb * N * kRowBytes, &tmap_q, &S.q_full, 0, row);
+        if (pw == 0) {
+          if (!mbar_wait(&S.q_empty, q_phase ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&S.q_full, (uint32_t)(p.nsub * N) * kRowBytes);
+          for (int sb = 0; sb < p.nsub; ++sb) {
+            const int row = ((U.b * p.Lq) + U.i0 + sb * p.qb) * H_I;
+            tma_load_2d(q_smem + (size_t)sb * N * kRowBytes, &tmap_q, &S.q_full, 0, row);
+          }
         }
+        q_phase ^= 1;
         bool ok = true;
         for (int kt = U.kt0; kt < U.kt1; ++kt) {
           if (!mbar_wait(&S.k_empty[kstage], kphase ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&S.k_full[kstage], kKeysPerTile * kRowBytes);
-          tma_load_2d(k_smem + (size_t)kstage * kKeysPerTile * kRowBytes, &tmap_k, &S.k_full[kstage],
-                      0, U.b * p.Lk + kt * kKeysPerTile);
+          if (pw == 0) mbar_arrive_expect_tx(&S.k_full[kstage], kKeysPerTile * kRowBytes);
+          tma_load_2d(k_smem + (size_t)kstage * kKeysPerTile * kRowBytes + pw * 32 * kRowBytes, &tmap_k,
+                      &S.k_full[kstage], 0, U.b * p.Lk + kt * kKeysPerTile + pw * 32);
           if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
         }
         if (!ok) break;
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       const uint32_t idesc = make_idesc(0, 0, 128, (uint32_t)N, 0, 0);  // e4m3 x e4m3 -> f32
@@ -187,9 +194,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t quarter = warp & 3u;              // TMEM lane quarter this warp may read
+    const uint32_t quarter = warp;                   // TMEM lane quarter this warp may read
     const uint32_t row = quarter * 32 + lane;        // key row within the tile
-    const int et = threadIdx.x - 64;                 // 0..127
+    const int et = threadIdx.x;                      // 0..127
     uint32_t seq = 0, epi_phase = 0;
     for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
       const UnitInfo U = decode_unit(p, u);
@@ -207,9 +214,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       }
       if (!warps_rendezvous(&S.epi_bar, epi_phase, abort_flag)) break;
       bool ok = true;
+      // The key scale of the next tile is loaded one iteration ahead, so its
+      // memory latency overlaps the current tile's epilogue.
+      auto key_scale = [&](int kt) -> float {
+        const int s = kt * kKeysPerTile + (int)row;
+        if (kt >= U.kt1 || s >= p.Lk) return 0.f;
+        return p.k_scale ? __ldg(p.k_scale + (size_t)U.b * p.Lk + s) : 1.f;
+      };
+      float sk_next = key_scale(U.kt0);
       for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
         const int s = kt * kKeysPerTile + (int)row;
-        const float sk = (s < p.Lk) ? (p.k_scale ? p.k_scale[(size_t)U.b * p.Lk + s] : 1.f) : 0.f;
+        const float sk = sk_next;
+        sk_next = key_scale(kt + 1);
         for (int sb = 0; sb < p.nsub; ++sb) {
           const uint32_t slot = seq & 1u, use = seq >> 1;
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
@@ -274,7 +290,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 4) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }

@@ -47,7 +47,10 @@ constexpr int kHalfKeys = 64;        // keys per CTA in S, and keys per V stage
 constexpr int kKStages = 6;          // K-chunk ring depth (8 KB stages)
 constexpr int kVStages = 4;          // V ring depth (64 keys x this CTA's value planes)
 constexpr int kMaxIdx = 2048;        // selected positions per row (staged in shared memory)
-constexpr int kThreads = 224;        // 7 warps
+constexpr int kThreads = 512;        // 16 warps: 4 softmax, 1 MMA, 11 loaders
+constexpr int kPool = 11;            // loader warps (TMA gathers from one warp are processed in order,
+                                     // so the gather rate grows with the number of issuing warps)
+constexpr int kPoolWarp0 = 5;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPlane64 = 64 * 128;    // 64 rows x 128 B  (Q plane, K stage, V plane, P plane)
 constexpr uint32_t kTmemS = 0;             // S buffers: columns [0, 128)
@@ -147,7 +150,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_empty[i], 8);     // 4 softmax warps x 2 CTAs
       mbar_init(&S.idx_full[i], 1);
-      mbar_init(&S.idx_empty[i], 6);   // 4 softmax warps + 2 producer warps
+      mbar_init(&S.idx_empty[i], 4 + kPool);   // 4 softmax warps + the loader warps
     }
     mbar_init(&S.p_full, 8);
     mbar_init(&S.p_empty, 1);
@@ -158,7 +161,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 4) {
     tmem_alloc_pair(&S.tmem_base, kTmemCols);
     tmem_relinquish_pair();
   }
@@ -169,22 +172,33 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const uint32_t tmem_base = S.tmem_base;
   const uint16_t kBoth = 0x3;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ K producer
-    // Per unit: stage the row's indices, load this CTA's Q planes (each plane as
-    // soon as the previous unit's last S has finished with it), then gather this
-    // CTA's 64 keys of every tile, chunk by chunk.
-    uint32_t ucount = 0, kc = 0;
+  if (warp >= kPoolWarp0) {
+    // ------------------------------------------------------------------ loader pool
+    // Every loader warp walks the same sequence of stages -- per unit the Q
+    // planes, then for each tile its NC key chunks (this CTA's 64 keys) followed
+    // by the value stages of the previous tile -- and issues its share of each
+    // stage's 4-row gathers (groups g = pw, pw + kPool, ...).
+    const int pw = (int)warp - kPoolWarp0;
+    uint32_t ucount = 0, kc = 0, vc = 0;
     bool ok = true;
-    if (lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
+    if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
+    // wait for a ring slot (lane 0 polls; the result is shared with the warp)
+    auto slot_free = [&](uint64_t* empty, uint32_t parity, uint64_t* full, uint32_t bytes) -> bool {
+      bool w_ok = true;
+      if (lane == 0) {
+        w_ok = mbar_wait(empty, parity, abort_flag);
+        if (w_ok && leader && pw == 0) mbar_arrive_expect_tx(full, bytes);
+      }
+      return __shfl_sync(0xffffffffu, w_ok, 0);
+    };
     for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
       const Unit U = decode_unit(p, u);
       if (U.j0 >= U.j1) continue;
       const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
-      // Q planes
+      // Q planes (plane c from loader warp c % kPool)
       if (lane == 0) {
         const int qrow = U.row * p.H + (int)rank * 64;
-        for (int c = 0; c < NC && ok; ++c) {
+        for (int c = pw; c < NC && ok; c += kPool) {
           ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
           if (!ok) break;
           if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane64);
@@ -193,90 +207,64 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      // indices of the row -> shared memory (buffer ib, free once unit ucount-2 is done)
-      ok = mbar_wait_warp(&S.idx_empty[ib], uph ^ 1u, abort_flag);
-      if (!ok) break;
-      {
+      // the last loader warp stages the row's indices (buffer ib, free once unit ucount-2 is done)
+      if (pw == kPool - 1) {
+        ok = mbar_wait_warp(&S.idx_empty[ib], uph ^ 1u, abort_flag);
+        if (!ok) break;
         int32_t* dst = idx_sm + ib * kMaxIdx;
         const int32_t* src = p.indices + (size_t)U.row * p.k;
         for (int x = (int)lane; x < idx_span; x += 32) dst[x] = (x < p.k) ? __ldg(src + x) : -1;
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.idx_full[ib]);
       }
-      const int32_t* idx = idx_sm + ib * kMaxIdx;
-      for (int j = U.j0; j < U.j1 && ok; ++j) {
-        int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
-        if (lane < 16) {
-          const int base = j * kTileKeys + (int)rank * kHalfKeys + (int)lane * 4;
-          r0 = gather_row(idx, base + 0, U.b, p.Lk);
-          r1 = gather_row(idx, base + 1, U.b, p.Lk);
-          r2 = gather_row(idx, base + 2, U.b, p.Lk);
-          r3 = gather_row(idx, base + 3, U.b, p.Lk);
-        }
-        for (int c = 0; c < NC; ++c) {
-          const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
-          bool w_ok = true;
-          if (lane == 0) {
-            w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
-            if (w_ok && leader) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
-          }
-          w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-          if (!w_ok) { ok = false; break; }
-          const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
-          if (lane < 16)
-            tma_gather4_pair(k_sm + st * kPlane64 + lane * 512, &tmap_kv, full_l, c * 64, r0, r1, r2, r3);
-          ++kc;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
-      ++ucount;
-    }
-  } else if (warp == 6) {
-    // ------------------------------------------------------------------ V producer
-    // For every tile: all 128 keys x this CTA's value columns, 64 keys per stage.
-    uint32_t ucount = 0, vc = 0;
-    bool ok = true;
-    for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
-      const Unit U = decode_unit(p, u);
-      if (U.j0 >= U.j1) continue;
-      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
       const int32_t* idx = idx_sm + ib * kMaxIdx;
-      const int pl = (int)lane / 16;                  // value plane this lane fills
-      const int g = (int)lane % 16;                   // 4-key group within the stage
-      for (int j = U.j0; j < U.j1 && ok; ++j) {
-        for (int kh = 0; kh < 2 && ok; ++kh) {
-          const int base = j * kTileKeys + kh * kHalfKeys + g * 4;
-          const int r0 = gather_row(idx, base + 0, U.b, p.Lk);
-          const int r1 = gather_row(idx, base + 1, U.b, p.Lk);
-          const int r2 = gather_row(idx, base + 2, U.b, p.Lk);
-          const int r3 = gather_row(idx, base + 3, U.b, p.Lk);
+      auto load_k = [&](int j) -> bool {
+        for (int c = 0; c < NC; ++c) {
+          const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
+          if (!slot_free(&S.k_empty[st], ph ^ 1u, &S.k_full[st], 2u * kPlane64)) return false;
+          const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
+          const int g = pw + kPool * (int)lane;                 // 4-key group of this lane
+          if (g < kHalfKeys / 4) {
+            const int base = j * kTileKeys + (int)rank * kHalfKeys + g * 4;
+            tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
+                             gather_row(idx, base + 0, U.b, p.Lk), gather_row(idx, base + 1, U.b, p.Lk),
+                             gather_row(idx, base + 2, U.b, p.Lk), gather_row(idx, base + 3, U.b, p.Lk));
+          }
+          ++kc;
+        }
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        for (int kh = 0; kh < 2; ++kh) {
           for (int h = 0; h < VS::kNpv; ++h) {
             const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
-            bool w_ok = true;
-            if (lane == 0) {
-              w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
-              if (w_ok && leader) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
-            }
-            w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-            if (!w_ok) { ok = false; break; }
+            if (!slot_free(&S.v_empty[st], ph ^ 1u, &S.v_full[st], 2u * VS::kStageBytes)) return false;
             const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
-            if (pl < VS::kPlanes) {
+            for (int g = pw + kPool * (int)lane; g < 16 * VS::kPlanes; g += 32 * kPool) {
+              const int pl = g / 16, kg = g % 16;
+              const int base = j * kTileKeys + kh * kHalfKeys + kg * 4;
               const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
-              tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + g * 512, &tmap_kv, full_l, col,
-                               r0, r1, r2, r3);
+              tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
+                               gather_row(idx, base + 0, U.b, p.Lk), gather_row(idx, base + 1, U.b, p.Lk),
+                               gather_row(idx, base + 2, U.b, p.Lk), gather_row(idx, base + 3, U.b, p.Lk));
             }
             ++vc;
           }
         }
+        return true;
+      };
+      for (int j = U.j0; j < U.j1 && ok; ++j) {
+        ok = load_k(j);
+        if (ok && j > U.j0) ok = load_v(j - 1);
       }
+      if (ok) ok = load_v(U.j1 - 1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
       ++ucount;
     }
-  } else if (warp == 5) {
+  } else if (warp == 4) {
     // ------------------------------------------------------------------ MMA issuer
     if (leader && elect_one()) {
       constexpr uint32_t idesc_s = make_idesc(1, 1, 128, kTileKeys, 0, 0);       // bf16, K-major x K-major
@@ -380,28 +368,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         ok = mbar_wait_warp(&S.s_full[sb], (sc >> 1) & 1u, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        uint32_t sv[64];
-        {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-          tmem_ld32(tmem_base + lane_addr + kTmemS + sb * kHalfKeys, lo);
-          tmem_ld32(tmem_base + lane_addr + kTmemS + sb * kHalfKeys + 32, hi);
-          tmem_ld_wait();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
-        ++sc;
-        // Scale into log2 units and mask padding / out-of-range positions.
+        // Two passes over this lane's 64 logits in TMEM (32 at a time, to stay within
+        // the register budget of a 512-thread CTA): the row maximum, then the
+        // probabilities, packed to bf16 pairs.
         const int kbase = j * kTileKeys + (int)half * kHalfKeys;
-        float x[64];
+        const uint32_t s_addr = tmem_base + lane_addr + kTmemS + sb * kHalfKeys;
         float tmax = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int s = idx[kbase + c];
-          const bool valid = (s >= 0) && (s < p.Lk);
-          x[c] = valid ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, x[c]);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t v[32];
+          tmem_ld32(s_addr + hh * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int s = idx[kbase + hh * 32 + c];
+            if (s >= 0 && s < p.Lk) tmax = fmaxf(tmax, __uint_as_float(v[c]) * p.scale_log2);
+          }
         }
         const uint32_t rb = sc & 1u;
         S.red_max[rb][l] = tmax;
@@ -413,16 +395,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         const bool need = first || (m_new > m + kRescaleThreshold);
         const float m_ref = need ? m_new : m;
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // probabilities in bf16 (the sum uses the rounded values, matching what P.V sees)
-        uint32_t pw[32];
-        float psum = 0.f;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const __nv_bfloat162 v2 = __floats2bfloat162_rn(exp2f(x[2 * e] - m_use), exp2f(x[2 * e + 1] - m_use));
-          const float2 back = __bfloat1622float2(v2);
-          psum += back.x + back.y;
-          pw[e] = *reinterpret_cast<const uint32_t*>(&v2);
-        }
         // The single P buffer (and O) are free once the previous tile's P.V is done.
         if (pc >= 1) {
           ok = mbar_wait_warp(&S.p_empty, (pc - 1u) & 1u, abort_flag);
@@ -443,12 +415,37 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           if (need) lsum *= alpha;
         }
         if (need) m = m_new;
-        lsum += psum;
+        // probabilities in bf16, straight into P (the sum uses the rounded values, as P.V sees them)
         uint8_t* prow = p_sm + half * kPlane64 + (h >> 3) * 1024 + (h & 7) * 128;
+        float psum = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) =
-              make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t v[32];
+          tmem_ld32(s_addr + hh * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c0 = q4 * 8 + 2 * e, c1 = c0 + 1;
+              const int s0 = idx[kbase + hh * 32 + c0], s1 = idx[kbase + hh * 32 + c1];
+              const float x0 = (s0 >= 0 && s0 < p.Lk) ? __uint_as_float(v[c0]) * p.scale_log2 - m_use : -INFINITY;
+              const float x1 = (s1 >= 0 && s1 < p.Lk) ? __uint_as_float(v[c1]) * p.scale_log2 - m_use : -INFINITY;
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(exp2f(x0), exp2f(x1));
+              const float2 back = __bfloat1622float2(v2);
+              psum += back.x + back.y;
+              w4[e] = *reinterpret_cast<const uint32_t*>(&v2);
+            }
+            const int c = hh * 4 + q4;                      // 16-byte chunk within the 128-byte row
+            *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+        lsum += psum;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
+        ++sc;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -517,7 +514,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   tc_fence_before();
   __syncthreads();
   cluster_sync();
-  if (warp == 5) {
+  if (warp == 4) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
