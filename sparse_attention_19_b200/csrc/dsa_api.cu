@@ -211,7 +211,7 @@ __global__ void wait_selftest_kernel(uint32_t limit) {
   if (threadIdx.x == 0) {
     const uint32_t a = smem_u32(&bar);
     bool done = false;
-    for (uint32_t i = 0; i < limit && !done; ++i) done = mbar_try_wait(a, 0);
+    for (uint32_t i = 0; i < limit && !done; ++i) done = mbar_test_wait(a, 0);
     if (!done) atomicExch(&g_device_error, DEV_ERR_TIMEOUT);
     mbar_arrive(&bar);          // complete the phase so the barrier is left idle
   }

@@ -41,7 +41,7 @@ struct IndexerSmem {
   // Barriers and small per-unit data first; big tiles follow at a 1024-byte boundary.
   uint64_t q_full, q_empty;
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t acc_full[8], acc_empty[8];     // TMEM accumulators: 512 / N of them (at most 8)
   uint64_t final_bar;
   uint64_t epi_bar;          // rendezvous of the 4 epilogue warps
   uint32_t tmem_base;
@@ -86,6 +86,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* tiles = smem_raw + (((raw_addr + (uint32_t)sizeof(IndexerSmem) + 1023u) & ~1023u) - raw_addr);
   const int N = p.qb * H_I;                            // MMA N (queries x heads)
+  const uint32_t nslot = min(8, kTmemCols / N);        // accumulators in flight (more when N is small)
   const int QU = p.queries_per_unit;                   // = qb * nsub
   uint8_t* q_smem = tiles;                             // nsub * N rows
   uint8_t* k_smem = tiles + (size_t)p.nsub * N * kRowBytes;
@@ -103,7 +104,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       mbar_init(&S.k_full[s], 1);
       mbar_init(&S.k_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 8; ++s) {
       mbar_init(&S.acc_full[s], 1);
       mbar_init(&S.acc_empty[s], 4);
     }
@@ -168,7 +169,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           tc_fence_after();
           const uint32_t a_addr = k_base + kstage * kKeysPerTile * kRowBytes;
           for (int sb = 0; sb < p.nsub; ++sb) {
-            const uint32_t slot = seq & 1u, use = seq >> 1;
+            const uint32_t slot = seq % nslot, use = seq / nslot;
             if (!mbar_wait(&S.acc_empty[slot], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + slot * (uint32_t)N;
@@ -227,39 +228,32 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const float sk = sk_next;
         sk_next = key_scale(kt + 1);
         for (int sb = 0; sb < p.nsub; ++sb) {
-          const uint32_t slot = seq & 1u, use = seq >> 1;
+          const uint32_t slot = seq % nslot, use = seq / nslot;
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t t_base = tmem_base + ((quarter * 32u) << 16) + slot * (uint32_t)N;
-          // Each query owns H_I consecutive columns; walk them 32 at a time.
-          for (int q0 = 0; q0 < p.qb; q0 += (H_I >= 32 ? 1 : 32 / H_I)) {
-            uint32_t v[32];
-            float acc[(H_I >= 32) ? 1 : 32 / H_I];
-            constexpr int QPC = (H_I >= 32) ? 1 : 32 / H_I;   // queries per 32 columns
-            constexpr int CPQ = (H_I >= 32) ? H_I / 32 : 1;   // 32-column chunks per query
+          // 64 columns per TMEM round trip (two loads, one wait); each query owns H_I columns.
+          constexpr int QPG = (H_I >= 64) ? 1 : 64 / H_I;      // queries per 64-column group
+          for (int g0 = 0; g0 < N; g0 += 64) {
+            uint32_t v[64];
+            tmem_ld32(t_base + (uint32_t)g0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+            tmem_ld32(t_base + (uint32_t)g0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+            tmem_ld_wait();
 #pragma unroll
-            for (int a = 0; a < QPC; ++a) acc[a] = 0.f;
-            const float* wq = w_smem + (size_t)(sb * p.qb + q0) * H_I;
+            for (int a = 0; a < QPG; ++a) {
+              const int qi = g0 / H_I + a;                    // query within the sub-block
+              const float* wq = w_smem + (size_t)(sb * p.qb + qi) * H_I;
+              float acc = 0.f;
 #pragma unroll
-            for (int c = 0; c < CPQ; ++c) {
-              tmem_ld32(t_base + (uint32_t)(q0 * H_I + c * 32), v);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int a = (H_I >= 32) ? 0 : e / H_I;
-                const float x = __uint_as_float(v[e]);
-                acc[a] = fmaf(wq[c * 32 + e], fmaxf(x, 0.f), acc[a]);
-              }
-            }
-#pragma unroll
-            for (int a = 0; a < QPC; ++a) {
-              const int qq = sb * p.qb + q0 + a;
+              for (int e = 0; e < (H_I >= 64 ? 64 : H_I); ++e)
+                acc = fmaf(wq[e], fmaxf(__uint_as_float(v[a * (H_I >= 64 ? 64 : H_I) + e]), 0.f), acc);
+              const int qq = sb * p.qb + qi;
               const int i = U.i0 + qq;
               if (i < p.Lq && s < p.Lk) {
                 const int t = p.q_offset + i;
                 float* dst = p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s;
                 if (s <= t)
-                  __stcs(dst, acc[a] * sq_smem[qq] * sk);
+                  __stcs(dst, acc * sq_smem[qq] * sk);
                 else if (p.fill_upper)
                   __stcs(dst, -INFINITY);
               }

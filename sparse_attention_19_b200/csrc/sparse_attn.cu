@@ -26,9 +26,21 @@
 //     TMEM columns per CTA (the pair layout puts half of N in lanes 64-127), so
 //     S double-buffers beside it.
 //   * The leader CTA (rank 0) issues every MMA; both CTAs' TMA loads complete on
-//     the leader's barriers, and MMA completion is multicast to both CTAs.
-// Warp roles (192 threads per CTA): warps 0-3 softmax/epilogue (TMEM lane quarter
-// = warp), warp 4 TMA producer, warp 5 TMEM owner + MMA issuer (leader only).
+//     the leader's barriers, and MMA completion is multicast to both CTAs.  The
+//     softmax warps of both CTAs signal the leader's barriers directly (after a
+//     fence.proxy.async for the P tile they wrote).  P is double-buffered, so the
+//     softmax of tile j+1 overlaps the P.V of tile j.
+//   * The MMA issuer never blocks on one operand while another is ready: it polls
+//     its barriers and issues P.V(j) as soon as P(j) is written, between the key
+//     chunks of S(j+1).
+//   * Loads: TMA requests from one warp are served in order, so the gather rate
+//     grows with the number of issuing warps.  Key chunks come from 5 warps and
+//     value stages from 5 others (each group walks its own ring, so a value slot
+//     that is still in use never holds back the next tile's keys); one more warp
+//     stages each unit's selected positions one unit ahead.
+// Warp roles (512 threads per CTA): warps 0-3 softmax/epilogue (TMEM lane quarter
+// = warp), warp 4 TMEM owner + MMA issuer (leader), warp 5 index staging, warps
+// 6-10 key loaders, warps 11-15 value loaders.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -45,12 +57,17 @@ namespace {
 constexpr int kTileKeys = 128;       // keys per tile (pair)
 constexpr int kHalfKeys = 64;        // keys per CTA in S, and keys per V stage
 constexpr int kKStages = 6;          // K-chunk ring depth (8 KB stages)
-constexpr int kVStages = 4;          // V ring depth (64 keys x this CTA's value planes)
-constexpr int kMaxIdx = 2048;        // selected positions per row (staged in shared memory)
-constexpr int kThreads = 512;        // 16 warps: 4 softmax, 1 MMA, 11 loaders
-constexpr int kPool = 11;            // loader warps (TMA gathers from one warp are processed in order,
-                                     // so the gather rate grows with the number of issuing warps)
-constexpr int kPoolWarp0 = 5;
+constexpr int kVStages = 3;          // V ring depth (64 keys x this CTA's value planes)
+constexpr int kPBufs = 2;            // P buffers (2 planes each: keys 0-63, 64-127)
+constexpr int kMaxIdx = 2048;        // selected positions per unit (staged in shared memory)
+constexpr int kMmaWarp = 4;
+constexpr int kStageWarp = 5;
+constexpr int kKWarp0 = 6;           // key-chunk loaders
+constexpr int kKWarps = 5;
+constexpr int kVWarp0 = kKWarp0 + kKWarps;   // value-stage loaders
+constexpr int kVWarps = 5;
+constexpr int kThreads = 32 * (kVWarp0 + kVWarps);   // 512 (4 warps per SM sub-partition: 128 registers)
+constexpr int kStageBatch = 16;      // index loads in flight per lane while staging
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPlane64 = 64 * 128;    // 64 rows x 128 B  (Q plane, K stage, V plane, P plane)
 constexpr uint32_t kTmemS = 0;             // S buffers: columns [0, 128)
@@ -58,15 +75,17 @@ constexpr uint32_t kTmemO = 128;           // O: columns [128, 128 + d_v/2)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxChunks = 9;
+constexpr uint32_t kIdleCheck = 1024;      // idle polls of the MMA issuer between clock reads
 
 struct AttnBarriers {
   uint64_t q_full[kMaxChunks], q_empty[kMaxChunks];
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full, p_empty;
+  uint64_t p_full[kPBufs], p_empty[kPBufs];
   uint64_t o_full, o_empty, final_bar;
   uint64_t idx_full[2], idx_empty[2];
+  uint32_t valid_mask[2][kMaxIdx / 32];   // per 32 staged positions: bit set = valid entry
   uint64_t xbar;             // rendezvous of the 4 softmax warps (max / sum exchange)
   uint32_t tmem_base;
   uint32_t abort_flag;
@@ -82,6 +101,7 @@ struct VShape {
   static constexpr uint32_t kStageBytes = kPlanes * kPlane64;   // 64 keys x planes
 };
 
+// A unit is one query row's key-tile range [j0, j1) (the whole row without split-k).
 struct Unit {
   int row, b, t, j0, j1, split;
 };
@@ -103,16 +123,25 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams& p, int u) {
   return U;
 }
 
+// First unit at or after u (stepping by the cluster count) that has key tiles;
+// returns p.n_units when there is none.
+__device__ __forceinline__ int next_unit(const AttnParams& p, int u, int step, Unit& U) {
+  for (; u < p.n_units; u += step) {
+    U = decode_unit(p, u);
+    if (U.j0 < U.j1) return u;
+  }
+  return p.n_units;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Row of kv (in the [B*Lk, d_qk] view) for a staged index; padding and out-of-range
-// entries gather row b*Lk (a valid row) and are masked in the softmax.
-__device__ __forceinline__ int gather_row(const int32_t* idx, int pos, int b, int Lk) {
-  const int s = idx[pos];
-  return b * Lk + ((s >= 0 && s < Lk) ? s : 0);
+// Row of kv (in the [B*Lk, d_qk] view) for a staged position; padding and
+// out-of-range entries were staged as row b*Lk (a valid row), masked in the softmax.
+__device__ __forceinline__ int gather_row(const int32_t* rows, int pos) {
+  return rows[pos] & 0x7fffffff;
 }
 
 template <int NC, int DV>
@@ -130,8 +159,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   uint8_t* q_sm = area;                                             // NC planes
   uint8_t* k_sm = q_sm + NC * kPlane64;                             // kKStages planes
   uint8_t* v_sm = k_sm + kKStages * kPlane64;                       // kVStages x kPlanes planes
-  uint8_t* p_sm = v_sm + kVStages * VS::kStageBytes;                // 2 planes (keys 0-63, 64-127)
-  int32_t* idx_sm = reinterpret_cast<int32_t*>(p_sm + 2 * kPlane64);  // 2 x kMaxIdx
+  uint8_t* p_sm = v_sm + kVStages * VS::kStageBytes;                // kPBufs x 2 planes
+  int32_t* idx_sm = reinterpret_cast<int32_t*>(p_sm + kPBufs * 2 * kPlane64);  // 2 x kMaxIdx
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -140,20 +169,21 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const int cluster_id = blockIdx.x >> 1;
   const int n_clusters = gridDim.x >> 1;
   volatile uint32_t* abort_flag = &S.abort_flag;
-  const int idx_span = p.n_tiles * kTileKeys;                       // staged positions per row
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxChunks; ++i) { mbar_init(&S.q_full[i], 1); mbar_init(&S.q_empty[i], 1); }
     for (int i = 0; i < kKStages; ++i) { mbar_init(&S.k_full[i], 1); mbar_init(&S.k_empty[i], 1); }
     for (int i = 0; i < kVStages; ++i) { mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); }
+    for (int i = 0; i < kPBufs; ++i) {
+      mbar_init(&S.p_full[i], 8);      // 4 softmax warps x 2 CTAs
+      mbar_init(&S.p_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_empty[i], 8);     // 4 softmax warps x 2 CTAs
       mbar_init(&S.idx_full[i], 1);
-      mbar_init(&S.idx_empty[i], 4 + kPool);   // 4 softmax warps + the loader warps
+      mbar_init(&S.idx_empty[i], 4 + kKWarps + kVWarps);   // softmax warps + loader warps
     }
-    mbar_init(&S.p_full, 8);
-    mbar_init(&S.p_empty, 1);
     mbar_init(&S.o_full, 1);
     mbar_init(&S.o_empty, 8);
     mbar_init(&S.final_bar, 1);
@@ -161,7 +191,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc_pair(&S.tmem_base, kTmemCols);
     tmem_relinquish_pair();
   }
@@ -172,33 +202,60 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const uint32_t tmem_base = S.tmem_base;
   const uint16_t kBoth = 0x3;
 
-  if (warp >= kPoolWarp0) {
-    // ------------------------------------------------------------------ loader pool
-    // Every loader warp walks the same sequence of stages -- per unit the Q
-    // planes, then for each tile its NC key chunks (this CTA's 64 keys) followed
-    // by the value stages of the previous tile -- and issues its share of each
-    // stage's 4-row gathers (groups g = pw, pw + kPool, ...).
-    const int pw = (int)warp - kPoolWarp0;
-    uint32_t ucount = 0, kc = 0, vc = 0;
+  if (warp == kStageWarp) {
+    // ------------------------------------------------------------------ index staging
+    // Each unit's selected positions [j0*128, j1*128) are staged (buffer ucount % 2)
+    // as the kv row to gather -- batch offset applied, bit 31 set for padding and
+    // out-of-range entries, which gather row b*Lk and are masked -- plus one
+    // validity ballot per 32 positions for the softmax.  The buffer is free again
+    // once the loaders and the softmax warps are done with the unit two back.
+    uint32_t ucount = 0;
+    Unit U;
+    for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units;
+         u = next_unit(p, u + n_clusters, n_clusters, U)) {
+      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+      if (!mbar_wait_warp(&S.idx_empty[ib], uph ^ 1u, abort_flag)) break;
+      int32_t* dst = idx_sm + ib * kMaxIdx;
+      uint32_t* vmask = S.valid_mask[ib];
+      const int x_begin = U.j0 * kTileKeys, span = (U.j1 - U.j0) * kTileKeys;
+      const int32_t* src = p.indices + (size_t)U.row * p.k;
+      for (int y0 = 0; y0 < span; y0 += 32 * kStageBatch) {
+        int sidx[kStageBatch];
+#pragma unroll
+        for (int e = 0; e < kStageBatch; ++e) {
+          const int y = y0 + e * 32 + (int)lane, x = x_begin + y;
+          sidx[e] = (y < span && x < p.k) ? __ldg(src + x) : -1;
+        }
+#pragma unroll
+        for (int e = 0; e < kStageBatch; ++e) {
+          const int y = y0 + e * 32 + (int)lane;
+          const bool valid = (sidx[e] >= 0) && (sidx[e] < p.Lk);
+          const int row = U.b * p.Lk + (valid ? sidx[e] : 0);
+          if (y < span) dst[y] = valid ? row : (int)((uint32_t)row | 0x80000000u);
+          const uint32_t bal = __ballot_sync(0xffffffffu, valid);
+          if (lane == 0 && y0 + e * 32 < span) vmask[(y0 + e * 32) / 32] = bal;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.idx_full[ib]);
+      ++ucount;
+    }
+  } else if (warp >= kKWarp0 && warp < kVWarp0) {
+    // ------------------------------------------------------------------ key loaders
+    // Per unit: the Q planes (plane c from warp c % kKWarps), then for each tile
+    // its NC key chunks (this CTA's 64 keys x 64 columns); each warp issues its
+    // share of a chunk's 4-row gathers (groups g = pw, pw + kKWarps, ...).
+    const int pw = (int)warp - kKWarp0;
+    uint32_t ucount = 0, kc = 0;
     bool ok = true;
     if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
-    // wait for a ring slot (lane 0 polls; the result is shared with the warp)
-    auto slot_free = [&](uint64_t* empty, uint32_t parity, uint64_t* full, uint32_t bytes) -> bool {
-      bool w_ok = true;
-      if (lane == 0) {
-        w_ok = mbar_wait(empty, parity, abort_flag);
-        if (w_ok && leader && pw == 0) mbar_arrive_expect_tx(full, bytes);
-      }
-      return __shfl_sync(0xffffffffu, w_ok, 0);
-    };
-    for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
-      const Unit U = decode_unit(p, u);
-      if (U.j0 >= U.j1) continue;
+    Unit U;
+    for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
+         u = next_unit(p, u + n_clusters, n_clusters, U)) {
       const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
-      // Q planes (plane c from loader warp c % kPool)
       if (lane == 0) {
         const int qrow = U.row * p.H + (int)rank * 64;
-        for (int c = pw; c < NC && ok; c += kPool) {
+        for (int c = pw; c < NC && ok; c += kKWarps) {
           ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
           if (!ok) break;
           if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane64);
@@ -207,131 +264,193 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      // the last loader warp stages the row's indices (buffer ib, free once unit ucount-2 is done)
-      if (pw == kPool - 1) {
-        ok = mbar_wait_warp(&S.idx_empty[ib], uph ^ 1u, abort_flag);
-        if (!ok) break;
-        int32_t* dst = idx_sm + ib * kMaxIdx;
-        const int32_t* src = p.indices + (size_t)U.row * p.k;
-        for (int x = (int)lane; x < idx_span; x += 32) dst[x] = (x < p.k) ? __ldg(src + x) : -1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.idx_full[ib]);
-      }
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
       const int32_t* idx = idx_sm + ib * kMaxIdx;
-      auto load_k = [&](int j) -> bool {
+      for (int j = U.j0; j < U.j1 && ok; ++j) {
         for (int c = 0; c < NC; ++c) {
           const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
-          if (!slot_free(&S.k_empty[st], ph ^ 1u, &S.k_full[st], 2u * kPlane64)) return false;
+          bool w_ok = true;
+          if (lane == 0) {
+            w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
+            if (w_ok && leader && pw == 0) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
+          }
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
           const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
-          const int g = pw + kPool * (int)lane;                 // 4-key group of this lane
+          const int g = pw + kKWarps * (int)lane;                 // 4-key group of this lane
           if (g < kHalfKeys / 4) {
-            const int base = j * kTileKeys + (int)rank * kHalfKeys + g * 4;
+            const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
             tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
-                             gather_row(idx, base + 0, U.b, p.Lk), gather_row(idx, base + 1, U.b, p.Lk),
-                             gather_row(idx, base + 2, U.b, p.Lk), gather_row(idx, base + 3, U.b, p.Lk));
+                             gather_row(idx, base + 0), gather_row(idx, base + 1),
+                             gather_row(idx, base + 2), gather_row(idx, base + 3));
           }
           ++kc;
         }
-        return true;
-      };
-      auto load_v = [&](int j) -> bool {
-        for (int kh = 0; kh < 2; ++kh) {
-          for (int h = 0; h < VS::kNpv; ++h) {
-            const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
-            if (!slot_free(&S.v_empty[st], ph ^ 1u, &S.v_full[st], 2u * VS::kStageBytes)) return false;
-            const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
-            for (int g = pw + kPool * (int)lane; g < 16 * VS::kPlanes; g += 32 * kPool) {
-              const int pl = g / 16, kg = g % 16;
-              const int base = j * kTileKeys + kh * kHalfKeys + kg * 4;
-              const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
-              tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
-                               gather_row(idx, base + 0, U.b, p.Lk), gather_row(idx, base + 1, U.b, p.Lk),
-                               gather_row(idx, base + 2, U.b, p.Lk), gather_row(idx, base + 3, U.b, p.Lk));
-            }
-            ++vc;
-          }
-        }
-        return true;
-      };
-      for (int j = U.j0; j < U.j1 && ok; ++j) {
-        ok = load_k(j);
-        if (ok && j > U.j0) ok = load_v(j - 1);
       }
-      if (ok) ok = load_v(U.j1 - 1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
       ++ucount;
     }
-  } else if (warp == 4) {
+  } else if (warp >= kVWarp0) {
+    // ------------------------------------------------------------------ value loaders
+    // Per tile, 2 x kNpv stages: 64 keys (kh) x this CTA's kN/2 columns of value
+    // block h, i.e. all 128 keys of the tile across the two key halves.
+    const int pw = (int)warp - kVWarp0;
+    uint32_t ucount = 0, vc = 0;
+    bool ok = true;
+    Unit U;
+    for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
+         u = next_unit(p, u + n_clusters, n_clusters, U)) {
+      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
+      if (!ok) break;
+      const int32_t* idx = idx_sm + ib * kMaxIdx;
+      for (int j = U.j0; j < U.j1 && ok; ++j) {
+        for (int kh = 0; kh < 2 && ok; ++kh) {
+          for (int h = 0; h < VS::kNpv; ++h) {
+            const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+            bool w_ok = true;
+            if (lane == 0) {
+              w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
+              if (w_ok && leader && pw == 0) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
+            }
+            if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+            const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
+            for (int g = pw + kVWarps * (int)lane; g < 16 * VS::kPlanes; g += 32 * kVWarps) {
+              const int pl = g / 16, kg = g % 16;
+              const int base = (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4;
+              const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
+              tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
+                               gather_row(idx, base + 0), gather_row(idx, base + 1),
+                               gather_row(idx, base + 2), gather_row(idx, base + 3));
+            }
+            ++vc;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+      ++ucount;
+    }
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    if (leader && elect_one()) {
+    // Two cursors over this cluster's tiles: S = Q K^T (one key chunk at a time)
+    // and O += P V (one value stage at a time).  Each poll issues whatever is
+    // ready, P.V first, so neither waits behind the other's operands.
+    const bool issuer = leader && elect_one();
+    if (issuer) {
       constexpr uint32_t idesc_s = make_idesc(1, 1, 128, kTileKeys, 0, 0);       // bf16, K-major x K-major
       constexpr uint32_t idesc_pv = make_idesc(1, 1, 128, VS::kN, 0, 1);         // P K-major, V MN-major
       const uint32_t q_base = smem_u32(q_sm), k_base = smem_u32(k_sm);
       const uint32_t v_base = smem_u32(v_sm), p_base = smem_u32(p_sm);
-      uint32_t ucount = 0, kc = 0, vc = 0, sc = 0, pc = 0, oc = 0;
-      bool ok = true;
-      auto issue_s = [&](bool first_of_unit, bool last_of_unit) -> bool {
-        const uint32_t sb = sc & 1u;
-        if (!mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag, true)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem_base + kTmemS + sb * kHalfKeys;
-        for (int c = 0; c < NC; ++c) {
-          if (first_of_unit && !mbar_wait(&S.q_full[c], ucount & 1u, abort_flag)) return false;
-          const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
-          if (!mbar_wait(&S.k_full[st], ph, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = make_smem_desc(q_base + c * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
-            const uint64_t bd = make_smem_desc(k_base + st * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
-            mma_bf16_ss_pair(d, ad, bd, idesc_s, (c | kk) ? 1u : 0u);
-          }
-          mma_commit_pair_mc(&S.k_empty[st], kBoth);
-          if (last_of_unit) mma_commit_pair_mc(&S.q_empty[c], kBoth);   // Q plane c free for the next unit
-          ++kc;
-        }
-        mma_commit_pair_mc(&S.s_full[sb], kBoth);
-        ++sc;
-        return true;
-      };
-      auto issue_pv = [&](bool first_of_unit, bool last_of_unit) -> bool {
-        if (!mbar_wait(&S.p_full, pc & 1u, abort_flag, true)) return false;
-        if (first_of_unit && !mbar_wait(&S.o_empty, (oc & 1u) ^ 1u, abort_flag, true)) return false;
-        tc_fence_after();
-        for (int kh = 0; kh < 2; ++kh) {
-          for (int h = 0; h < VS::kNpv; ++h) {
-            const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
-            if (!mbar_wait(&S.v_full[st], ph, abort_flag)) return false;
+      // S cursor: unit s_u (its ordinal s_uc), tile s_j, next chunk s_c
+      Unit sU, pU;
+      int s_u = next_unit(p, cluster_id, n_clusters, sU);
+      int s_j = sU.j0, s_c = 0;
+      uint32_t s_uc = 0;
+      bool s_buf = false;                       // S buffer of the current tile acquired
+      // P.V cursor: unit p_u, tile p_j, next value stage p_st
+      int p_u = s_u;
+      pU = sU;
+      int p_j = pU.j0, p_st = 0;
+      bool p_go = false;                        // P of the current tile is ready
+      uint32_t kc = 0, vc = 0, sc = 0, pc = 0, oc = 0;
+      uint32_t idle = 0;
+      uint64_t idle_t0 = 0;
+      while (p_u < p.n_units) {
+        bool progress = false;
+        // ---- O += P V
+        if (!p_go) {
+          const bool first = (p_j == pU.j0);
+          if (mbar_test_wait_cluster(smem_u32(&S.p_full[pc & 1u]), (pc >> 1) & 1u) &&
+              (!first || mbar_test_wait_cluster(smem_u32(&S.o_empty), (oc & 1u) ^ 1u))) {
+            p_go = true;
             tc_fence_after();
+          }
+        }
+        if (p_go) {
+          const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+          if (mbar_test_wait(smem_u32(&S.v_full[st]), ph)) {
+            tc_fence_after();
+            const int kh = p_st / VS::kNpv, h = p_st % VS::kNpv;
+            const bool first = (p_j == pU.j0);
             const uint32_t d = tmem_base + kTmemO + h * (VS::kN / 2);
+            const uint32_t pb = p_base + (pc & 1u) * 2 * kPlane64 + kh * kPlane64;
 #pragma unroll
             for (int kk = 0; kk < kHalfKeys / 16; ++kk) {
-              const uint64_t ad = make_smem_desc(p_base + kh * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
+              const uint64_t ad = make_smem_desc(pb + kk * 32, 16, 1024, LAYOUT_SW128);
               const uint64_t bd = make_smem_desc(v_base + st * VS::kStageBytes + kk * 2048, kPlane64, 1024,
                                                  LAYOUT_SW128);
-              mma_bf16_ss_pair(d, ad, bd, idesc_pv, (first_of_unit && kh == 0 && kk == 0) ? 0u : 1u);
+              mma_bf16_ss_pair(d, ad, bd, idesc_pv, (first && kh == 0 && kk == 0) ? 0u : 1u);
             }
             mma_commit_pair_mc(&S.v_empty[st], kBoth);
             ++vc;
+            progress = true;
+            if (++p_st == 2 * VS::kNpv) {
+              mma_commit_pair_mc(&S.p_empty[pc & 1u], kBoth);
+              if (p_j == pU.j1 - 1) { mma_commit_pair_mc(&S.o_full, kBoth); ++oc; }
+              ++pc;
+              p_st = 0;
+              p_go = false;
+              if (++p_j == pU.j1) {
+                p_u = next_unit(p, p_u + n_clusters, n_clusters, pU);
+                p_j = pU.j0;
+              }
+            }
           }
         }
-        mma_commit_pair_mc(&S.p_empty, kBoth);
-        if (last_of_unit) { mma_commit_pair_mc(&S.o_full, kBoth); ++oc; }
-        ++pc;
-        return true;
-      };
-      for (int u = cluster_id; u < p.n_units && ok; u += n_clusters) {
-        const Unit U = decode_unit(p, u);
-        if (U.j0 >= U.j1) continue;
-        for (int j = U.j0; j < U.j1 && ok; ++j) {
-          ok = issue_s(j == U.j0, j == U.j1 - 1);
-          if (ok && j > U.j0) ok = issue_pv(j - 1 == U.j0, false);
+        // ---- S = Q K^T
+        if (s_u < p.n_units) {
+          const uint32_t sb = sc & 1u;
+          if (!s_buf && mbar_test_wait_cluster(smem_u32(&S.s_empty[sb]), ((sc >> 1) & 1u) ^ 1u)) {
+            s_buf = true;
+            tc_fence_after();
+          }
+          if (s_buf) {
+            const bool first = (s_j == sU.j0);
+            const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
+            if ((!first || mbar_test_wait(smem_u32(&S.q_full[s_c]), s_uc & 1u)) &&
+                mbar_test_wait(smem_u32(&S.k_full[st]), ph)) {
+              tc_fence_after();
+              const uint32_t d = tmem_base + kTmemS + sb * kHalfKeys;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = make_smem_desc(q_base + s_c * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
+                const uint64_t bd = make_smem_desc(k_base + st * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
+                mma_bf16_ss_pair(d, ad, bd, idesc_s, (s_c | kk) ? 1u : 0u);
+              }
+              mma_commit_pair_mc(&S.k_empty[st], kBoth);
+              if (s_j == sU.j1 - 1) mma_commit_pair_mc(&S.q_empty[s_c], kBoth);   // Q plane free for the next unit
+              ++kc;
+              progress = true;
+              if (++s_c == NC) {
+                mma_commit_pair_mc(&S.s_full[sb], kBoth);
+                ++sc;
+                s_c = 0;
+                s_buf = false;
+                if (++s_j == sU.j1) {
+                  ++s_uc;
+                  s_u = next_unit(p, s_u + n_clusters, n_clusters, sU);
+                  s_j = sU.j0;
+                }
+              }
+            }
+          }
         }
-        if (ok) ok = issue_pv(U.j1 - 1 == U.j0, true);
-        ++ucount;
+        // ---- bounded idling
+        if (progress) {
+          idle = 0;
+        } else if ((++idle % kIdleCheck) == 0) {
+          if (*abort_flag) break;
+          const uint64_t now = global_timer_ns();
+          if (idle == kIdleCheck) {
+            idle_t0 = now;
+          } else if (now - idle_t0 > kWaitLimitNs) {
+            atomicExch(&g_device_error, DEV_ERR_TIMEOUT);
+            *abort_flag = 1u;
+            break;
+          }
+        }
       }
       // Wait until every MMA this thread issued has completed before teardown.
       mma_commit(&S.final_bar);
@@ -361,7 +480,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
-      const int32_t* idx = idx_sm + ib * kMaxIdx;
       float m = -INFINITY, lsum = 0.f;
       for (int j = U.j0; j < U.j1 && ok; ++j) {
         const uint32_t sb = sc & 1u;
@@ -369,22 +487,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         if (!ok) break;
         tc_fence_after();
         // Two passes over this lane's 64 logits in TMEM (32 at a time, to stay within
-        // the register budget of a 512-thread CTA): the row maximum, then the
-        // probabilities, packed to bf16 pairs.
-        const int kbase = j * kTileKeys + (int)half * kHalfKeys;
+        // the register budget): the row maximum, then the probabilities, packed to
+        // bf16 pairs.
         const uint32_t s_addr = tmem_base + lane_addr + kTmemS + sb * kHalfKeys;
-        float tmax = -INFINITY;
+        const uint32_t* vm = &S.valid_mask[ib][((j - U.j0) * kTileKeys + (int)half * kHalfKeys) / 32];
+        const uint32_t vmask0 = vm[0], vmask1 = vm[1];
+        float smax = -INFINITY;                       // maximum of the raw logits (scale > 0)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t v[32];
           tmem_ld32(s_addr + hh * 32, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int s = idx[kbase + hh * 32 + c];
-            if (s >= 0 && s < p.Lk) tmax = fmaxf(tmax, __uint_as_float(v[c]) * p.scale_log2);
-          }
+          for (int c = 0; c < 32; ++c)
+            if ((((hh == 0) ? vmask0 : vmask1) >> c) & 1u) smax = fmaxf(smax, __uint_as_float(v[c]));
         }
+        float tmax = smax * p.scale_log2;
         const uint32_t rb = sc & 1u;
         S.red_max[rb][l] = tmax;
         ok = warps_rendezvous(&S.xbar, xph, abort_flag);
@@ -395,13 +513,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         const bool need = first || (m_new > m + kRescaleThreshold);
         const float m_ref = need ? m_new : m;
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // The single P buffer (and O) are free once the previous tile's P.V is done.
-        if (pc >= 1) {
-          ok = mbar_wait_warp(&S.p_empty, (pc - 1u) & 1u, abort_flag);
-          if (!ok) break;
-        }
+        // P buffer pc % 2 is free once the P.V two tiles back is done.
+        const uint32_t pbuf = pc & 1u;
+        ok = mbar_wait_warp(&S.p_empty[pbuf], ((pc >> 1) & 1u) ^ 1u, abort_flag);
+        if (!ok) break;
         tc_fence_after();
         if (!first && __any_sync(0xffffffffu, need)) {
+          // Rescaling O needs the previous tile's P.V to be complete.
+          ok = mbar_wait_warp(&S.p_empty[pbuf ^ 1u], ((pc - 1u) >> 1) & 1u, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
           const float alpha = need ? exp2f(m - m_new) : 1.f;
           for (int c0 = 0; c0 < VS::kNpv * (VS::kN / 2); c0 += 32) {
             uint32_t ov[32];
@@ -416,9 +537,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         }
         if (need) m = m_new;
         // probabilities in bf16, straight into P (the sum uses the rounded values, as P.V sees them)
-        uint8_t* prow = p_sm + half * kPlane64 + (h >> 3) * 1024 + (h & 7) * 128;
+        uint8_t* prow = p_sm + (pbuf * 2 + half) * kPlane64 + (h >> 3) * 1024 + (h & 7) * 128;
         float psum = 0.f;
-#pragma unroll
+#pragma unroll 1   // one 32-column half at a time keeps the live registers low
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t v[32];
           tmem_ld32(s_addr + hh * 32, v);
@@ -429,9 +550,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int c0 = q4 * 8 + 2 * e, c1 = c0 + 1;
-              const int s0 = idx[kbase + hh * 32 + c0], s1 = idx[kbase + hh * 32 + c1];
-              const float x0 = (s0 >= 0 && s0 < p.Lk) ? __uint_as_float(v[c0]) * p.scale_log2 - m_use : -INFINITY;
-              const float x1 = (s1 >= 0 && s1 < p.Lk) ? __uint_as_float(v[c1]) * p.scale_log2 - m_use : -INFINITY;
+              const uint32_t vmh = (hh == 0) ? vmask0 : vmask1;
+              const float x0 = ((vmh >> c0) & 1u) ? fmaf(__uint_as_float(v[c0]), p.scale_log2, -m_use) : -INFINITY;
+              const float x1 = ((vmh >> c1) & 1u) ? fmaf(__uint_as_float(v[c1]), p.scale_log2, -m_use) : -INFINITY;
               const __nv_bfloat162 v2 = __floats2bfloat162_rn(exp2f(x0), exp2f(x1));
               const float2 back = __bfloat1622float2(v2);
               psum += back.x + back.y;
@@ -444,12 +565,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         lsum += psum;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
+        if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
         ++sc;
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.p_full), 0));
+        if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.p_full[pbuf]), 0));
         ++pc;
       }
       if (!ok) break;
@@ -507,14 +628,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&S.o_empty), 0));
+      if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.o_empty), 0));
     }
   }
 
   tc_fence_before();
   __syncthreads();
   cluster_sync();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
@@ -574,7 +695,7 @@ size_t attn_smem_bytes(int d_qk, int d_v) {
   b += (size_t)nc * kPlane64;                      // Q
   b += (size_t)kKStages * kPlane64;                // K ring
   b += (size_t)kVStages * v_stage;                 // V ring
-  b += 2 * (size_t)kPlane64;                       // P (keys 0-63, 64-127)
+  b += (size_t)kPBufs * 2 * kPlane64;              // P buffers (keys 0-63, 64-127 each)
   b += 2 * (size_t)kMaxIdx * sizeof(int32_t);      // staged indices, two units
   return b;
 }
