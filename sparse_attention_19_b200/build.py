@@ -23,7 +23,6 @@ INCLUDE = os.path.join(ROOT, "include")
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
-    "-rdc=true",
     "-Xcompiler", "-fPIC,-O2",
     "--expt-relaxed-constexpr",
     "-Xptxas", "-warn-spills",

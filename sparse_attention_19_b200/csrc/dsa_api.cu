@@ -18,8 +18,6 @@
 
 namespace dsa {
 
-__device__ uint32_t g_device_error = 0;
-
 namespace {
 
 constexpr int kMaxK = 2048;
@@ -222,13 +220,14 @@ __global__ void wait_selftest_kernel(uint32_t limit) {
 cudaError_t read_device_error(uint32_t* value, bool clear) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return e;
-  e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(uint32_t));
-  if (e != cudaSuccess) return e;
-  if (clear) {
-    const uint32_t zero = 0;
-    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
-  }
-  return e;
+  // Every unit's word holds DEV_ERR_NONE or the one code a failed wait records.
+  uint32_t words[4] = {0, 0, 0, 0};
+  if ((e = read_unit_error(&words[0], clear)) != cudaSuccess) return e;
+  if ((e = read_indexer_error(&words[1], clear)) != cudaSuccess) return e;
+  if ((e = read_topk_error(&words[2], clear)) != cudaSuccess) return e;
+  if ((e = read_attn_error(&words[3], clear)) != cudaSuccess) return e;
+  *value = words[0] | words[1] | words[2] | words[3];
+  return cudaSuccess;
 }
 
 cudaError_t launch_wait_selftest(uint32_t spin_limit, cudaStream_t stream) {

@@ -63,6 +63,10 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int d_qk, int d_v, const CUt
 cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t stream);
 
 // ---------------------------------------------------------------- misc
+// Error words of the kernel units (one per translation unit), and their union.
+cudaError_t read_indexer_error(uint32_t* value, bool clear);
+cudaError_t read_topk_error(uint32_t* value, bool clear);
+cudaError_t read_attn_error(uint32_t* value, bool clear);
 cudaError_t read_device_error(uint32_t* value, bool clear);
 cudaError_t launch_wait_selftest(uint32_t spin_limit, cudaStream_t stream);
 

@@ -324,4 +324,6 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
   return cudaErrorInvalidValue;
 }
 
+cudaError_t read_indexer_error(uint32_t* value, bool clear) { return read_unit_error(value, clear); }
+
 }  // namespace dsa

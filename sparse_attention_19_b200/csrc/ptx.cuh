@@ -11,12 +11,25 @@ namespace dsa {
 // ---------------------------------------------------------------- error word
 // Kernels never trap.  A wait that runs past its limit records a code in this
 // device word and makes its CTA wind down; the host reads it back after the
-// stream is synchronised.
+// stream is synchronised.  Each translation unit has its own copy (internal
+// linkage: the units are compiled whole-program, so that ptxas can give each
+// setmaxnreg region its own register budget) and reads it with
+// read_unit_error(), which the unit exports under its own name.
 enum : uint32_t {
   DEV_ERR_NONE = 0,
   DEV_ERR_TIMEOUT = 1,
 };
-extern __device__ uint32_t g_device_error;
+static __device__ uint32_t g_device_error = 0;
+
+// Reads (and optionally clears) this translation unit's error word.
+static inline cudaError_t read_unit_error(uint32_t* value, bool clear) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(uint32_t));
+  if (e == cudaSuccess && clear && *value != DEV_ERR_NONE) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
+  }
+  return e;
+}
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // a wait gives up after ~4 s
 
@@ -181,6 +194,19 @@ __device__ __forceinline__ bool warps_rendezvous(uint64_t* bar, uint32_t& phase,
   const bool ok = mbar_wait_warp(bar, phase, abort_flag);
   phase ^= 1u;
   return ok;
+}
+
+// ---------------------------------------------------------------- register split
+// Per-warpgroup register budget (all 4 warps of a warpgroup execute the same one).
+// The increases of a CTA must fit within what its decreases release from the
+// registers it was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------- fences

@@ -30,17 +30,18 @@
 //     softmax warps of both CTAs signal the leader's barriers directly (after a
 //     fence.proxy.async for the P tile they wrote).  P is double-buffered, so the
 //     softmax of tile j+1 overlaps the P.V of tile j.
-//   * The MMA issuer never blocks on one operand while another is ready: it polls
-//     its barriers and issues P.V(j) as soon as P(j) is written, between the key
-//     chunks of S(j+1).
+//   * S = Q K^T and O += P V are issued by two threads (warps 4 and 5 of the
+//     leader): at these shapes one thread's issue rate, not the tensor core, would
+//     bound the MMAs, and P.V(j) then never waits behind the key chunks of S(j+1).
 //   * Loads: TMA requests from one warp are served in order, so the gather rate
-//     grows with the number of issuing warps.  Key chunks come from 5 warps and
-//     value stages from 5 others (each group walks its own ring, so a value slot
-//     that is still in use never holds back the next tile's keys); one more warp
-//     stages each unit's selected positions one unit ahead.
-// Warp roles (512 threads per CTA): warps 0-3 softmax/epilogue (TMEM lane quarter
-// = warp), warp 4 TMEM owner + MMA issuer (leader), warp 5 index staging, warps
-// 6-10 key loaders, warps 11-15 value loaders.
+//     grows with the number of issuing warps.  Key chunks come from 9 warps and
+//     value stages from 9 others (each group walks its own ring, so a value slot
+//     that is still in use never holds back the next tile's keys); the value
+//     loaders also stage each unit's selected positions, one unit ahead.
+// Warp roles (768 threads per CTA): warps 0-3 softmax/epilogue (TMEM lane quarter
+// = warp), warp 4 TMEM owner + S issuer (leader), warp 5 P.V issuer (leader),
+// warps 6-14 key loaders, warps 15-23 value loaders + index staging.  The softmax
+// warpgroup holds 112 registers per thread, the others 72 (setmaxnreg).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -60,14 +61,27 @@ constexpr int kKStages = 6;          // K-chunk ring depth (8 KB stages)
 constexpr int kVStages = 3;          // V ring depth (64 keys x this CTA's value planes)
 constexpr int kPBufs = 2;            // P buffers (2 planes each: keys 0-63, 64-127)
 constexpr int kMaxIdx = 2048;        // selected positions per unit (staged in shared memory)
-constexpr int kMmaWarp = 4;
-constexpr int kStageWarp = 5;
+constexpr int kMmaWarp = 4;           // TMEM owner + S issuer
+constexpr int kPvWarp = 5;            // P.V issuer
+// Loaders own ring slots: kKWarpsPerSlot warps fill every key chunk that lands
+// in their slot (so a warp waits only on its own slot, and the chunks of
+// different slots are issued in parallel); likewise for the value stages.
+constexpr int kKWarpsPerSlot = 2;
+constexpr int kVWarpsPerSlot = 2;
 constexpr int kKWarp0 = 6;           // key-chunk loaders
-constexpr int kKWarps = 5;
+constexpr int kKWarps = kKStages * kKWarpsPerSlot;
 constexpr int kVWarp0 = kKWarp0 + kKWarps;   // value-stage loaders
-constexpr int kVWarps = 5;
-constexpr int kThreads = 32 * (kVWarp0 + kVWarps);   // 512 (4 warps per SM sub-partition: 128 registers)
-constexpr int kStageBatch = 16;      // index loads in flight per lane while staging
+constexpr int kVWarps = kVStages * kVWarpsPerSlot;
+constexpr int kThreads = 32 * (kVWarp0 + kVWarps);   // 768
+constexpr int kStageBatch = 8;       // index words in flight per warp while staging
+// Register split: the CTA launches with 80 registers per thread (6 warps per SM
+// sub-partition); the softmax warpgroup then takes 112 and the other warpgroups
+// (MMA issuers, loaders) keep 72.
+constexpr uint32_t kRegsLaunch = 80;
+constexpr uint32_t kRegsSoftmax = 112;
+constexpr uint32_t kRegsOther = 72;
+static_assert(128 * kRegsSoftmax + (kThreads - 128) * kRegsOther <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPlane64 = 64 * 128;    // 64 rows x 128 B  (Q plane, K stage, V plane, P plane)
 constexpr uint32_t kTmemS = 0;             // S buffers: columns [0, 128)
@@ -75,7 +89,6 @@ constexpr uint32_t kTmemO = 128;           // O: columns [128, 128 + d_v/2)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxChunks = 9;
-constexpr uint32_t kIdleCheck = 1024;      // idle polls of the MMA issuer between clock reads
 
 struct AttnBarriers {
   uint64_t q_full[kMaxChunks], q_empty[kMaxChunks];
@@ -83,7 +96,7 @@ struct AttnBarriers {
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[kPBufs], p_empty[kPBufs];
-  uint64_t o_full, o_empty, final_bar;
+  uint64_t o_full, o_empty, final_s, final_pv;
   uint64_t idx_full[2], idx_empty[2];
   uint32_t valid_mask[2][kMaxIdx / 32];   // per 32 staged positions: bit set = valid entry
   uint64_t xbar;             // rendezvous of the 4 softmax warps (max / sum exchange)
@@ -181,12 +194,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_empty[i], 8);     // 4 softmax warps x 2 CTAs
-      mbar_init(&S.idx_full[i], 1);
+      mbar_init(&S.idx_full[i], kVWarps);   // the value loaders stage the indices
       mbar_init(&S.idx_empty[i], 4 + kKWarps + kVWarps);   // softmax warps + loader warps
     }
     mbar_init(&S.o_full, 1);
     mbar_init(&S.o_empty, 8);
-    mbar_init(&S.final_bar, 1);
+    mbar_init(&S.final_s, 1);
+    mbar_init(&S.final_pv, 1);
     mbar_init(&S.xbar, 4);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -202,261 +216,245 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const uint32_t tmem_base = S.tmem_base;
   const uint16_t kBoth = 0x3;
 
-  if (warp == kStageWarp) {
-    // ------------------------------------------------------------------ index staging
-    // Each unit's selected positions [j0*128, j1*128) are staged (buffer ucount % 2)
-    // as the kv row to gather -- batch offset applied, bit 31 set for padding and
-    // out-of-range entries, which gather row b*Lk and are masked -- plus one
-    // validity ballot per 32 positions for the softmax.  The buffer is free again
-    // once the loaders and the softmax warps are done with the unit two back.
-    uint32_t ucount = 0;
-    Unit U;
-    for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units;
-         u = next_unit(p, u + n_clusters, n_clusters, U)) {
-      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
-      if (!mbar_wait_warp(&S.idx_empty[ib], uph ^ 1u, abort_flag)) break;
-      int32_t* dst = idx_sm + ib * kMaxIdx;
-      uint32_t* vmask = S.valid_mask[ib];
-      const int x_begin = U.j0 * kTileKeys, span = (U.j1 - U.j0) * kTileKeys;
-      const int32_t* src = p.indices + (size_t)U.row * p.k;
-      for (int y0 = 0; y0 < span; y0 += 32 * kStageBatch) {
-        int sidx[kStageBatch];
-#pragma unroll
-        for (int e = 0; e < kStageBatch; ++e) {
-          const int y = y0 + e * 32 + (int)lane, x = x_begin + y;
-          sidx[e] = (y < span && x < p.k) ? __ldg(src + x) : -1;
-        }
-#pragma unroll
-        for (int e = 0; e < kStageBatch; ++e) {
-          const int y = y0 + e * 32 + (int)lane;
-          const bool valid = (sidx[e] >= 0) && (sidx[e] < p.Lk);
-          const int row = U.b * p.Lk + (valid ? sidx[e] : 0);
-          if (y < span) dst[y] = valid ? row : (int)((uint32_t)row | 0x80000000u);
-          const uint32_t bal = __ballot_sync(0xffffffffu, valid);
-          if (lane == 0 && y0 + e * 32 < span) vmask[(y0 + e * 32) / 32] = bal;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.idx_full[ib]);
-      ++ucount;
-    }
-  } else if (warp >= kKWarp0 && warp < kVWarp0) {
-    // ------------------------------------------------------------------ key loaders
-    // Per unit: the Q planes (plane c from warp c % kKWarps), then for each tile
-    // its NC key chunks (this CTA's 64 keys x 64 columns); each warp issues its
-    // share of a chunk's 4-row gathers (groups g = pw, pw + kKWarps, ...).
-    const int pw = (int)warp - kKWarp0;
-    uint32_t ucount = 0, kc = 0;
-    bool ok = true;
-    if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
-    Unit U;
-    for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
-         u = next_unit(p, u + n_clusters, n_clusters, U)) {
-      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
-      if (lane == 0) {
-        const int qrow = U.row * p.H + (int)rank * 64;
-        for (int c = pw; c < NC && ok; c += kKWarps) {
-          ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
-          if (!ok) break;
-          if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane64);
-          tma_load_2d_pair(q_sm + c * kPlane64, &tmap_q, mapa_shared(smem_u32(&S.q_full[c]), 0), c * 64, qrow);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
-      if (!ok) break;
-      const int32_t* idx = idx_sm + ib * kMaxIdx;
-      for (int j = U.j0; j < U.j1 && ok; ++j) {
-        for (int c = 0; c < NC; ++c) {
-          const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
-          bool w_ok = true;
-          if (lane == 0) {
-            w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
-            if (w_ok && leader && pw == 0) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
+  if (warp >= 4) {
+    regs_decrease<kRegsOther>();
+    if (warp >= kKWarp0 && warp < kVWarp0) {
+      // ------------------------------------------------------------------ key loaders
+      // Per unit: the Q planes (plane c from warp c % kKWarps), then for each tile
+      // its NC key chunks (this CTA's 64 keys x 64 columns).  Chunk kc goes to
+      // ring slot kc % kKStages; the warps that own that slot each issue their
+      // share of its 16 four-row gathers.
+      constexpr int kGroupsPerWarp = (kHalfKeys / 4) / kKWarpsPerSlot;
+      const int pw = (int)warp - kKWarp0;
+      const uint32_t my_slot = (uint32_t)(pw / kKWarpsPerSlot);
+      const int part = pw % kKWarpsPerSlot;
+      uint32_t ucount = 0, kc = 0;
+      bool ok = true;
+      if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
+      Unit U;
+      for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
+           u = next_unit(p, u + n_clusters, n_clusters, U)) {
+        const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+        if (lane == 0) {
+          const int qrow = U.row * p.H + (int)rank * 64;
+          for (int c = pw; c < NC && ok; c += kKWarps) {
+            ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
+            if (!ok) break;
+            if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane64);
+            tma_load_2d_pair(q_sm + c * kPlane64, &tmap_q, mapa_shared(smem_u32(&S.q_full[c]), 0), c * 64, qrow);
           }
-          if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-          const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
-          const int g = pw + kKWarps * (int)lane;                 // 4-key group of this lane
-          if (g < kHalfKeys / 4) {
-            const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
-            tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
-                             gather_row(idx, base + 0), gather_row(idx, base + 1),
-                             gather_row(idx, base + 2), gather_row(idx, base + 3));
-          }
-          ++kc;
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
-      ++ucount;
-    }
-  } else if (warp >= kVWarp0) {
-    // ------------------------------------------------------------------ value loaders
-    // Per tile, 2 x kNpv stages: 64 keys (kh) x this CTA's kN/2 columns of value
-    // block h, i.e. all 128 keys of the tile across the two key halves.
-    const int pw = (int)warp - kVWarp0;
-    uint32_t ucount = 0, vc = 0;
-    bool ok = true;
-    Unit U;
-    for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
-         u = next_unit(p, u + n_clusters, n_clusters, U)) {
-      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
-      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
-      if (!ok) break;
-      const int32_t* idx = idx_sm + ib * kMaxIdx;
-      for (int j = U.j0; j < U.j1 && ok; ++j) {
-        for (int kh = 0; kh < 2 && ok; ++kh) {
-          for (int h = 0; h < VS::kNpv; ++h) {
-            const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
+        if (!ok) break;
+        const int32_t* idx = idx_sm + ib * kMaxIdx;
+        for (int j = U.j0; j < U.j1 && ok; ++j) {
+          for (int c = 0; c < NC; ++c, ++kc) {
+            const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
+            if (st != my_slot) continue;
             bool w_ok = true;
             if (lane == 0) {
-              w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
-              if (w_ok && leader && pw == 0) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
+              w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
+              if (w_ok && leader && part == 0) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
             }
             if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-            const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
-            for (int g = pw + kVWarps * (int)lane; g < 16 * VS::kPlanes; g += 32 * kVWarps) {
-              const int pl = g / 16, kg = g % 16;
-              const int base = (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4;
-              const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
-              tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
+            const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
+            if ((int)lane < kGroupsPerWarp) {
+              const int g = part * kGroupsPerWarp + (int)lane;      // 4-key group of this lane
+              const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
+              tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
                                gather_row(idx, base + 0), gather_row(idx, base + 1),
                                gather_row(idx, base + 2), gather_row(idx, base + 3));
             }
-            ++vc;
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+        ++ucount;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
-      ++ucount;
-    }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    // Two cursors over this cluster's tiles: S = Q K^T (one key chunk at a time)
-    // and O += P V (one value stage at a time).  Each poll issues whatever is
-    // ready, P.V first, so neither waits behind the other's operands.
-    const bool issuer = leader && elect_one();
-    if (issuer) {
-      constexpr uint32_t idesc_s = make_idesc(1, 1, 128, kTileKeys, 0, 0);       // bf16, K-major x K-major
-      constexpr uint32_t idesc_pv = make_idesc(1, 1, 128, VS::kN, 0, 1);         // P K-major, V MN-major
-      const uint32_t q_base = smem_u32(q_sm), k_base = smem_u32(k_sm);
-      const uint32_t v_base = smem_u32(v_sm), p_base = smem_u32(p_sm);
-      // S cursor: unit s_u (its ordinal s_uc), tile s_j, next chunk s_c
-      Unit sU, pU;
-      int s_u = next_unit(p, cluster_id, n_clusters, sU);
-      int s_j = sU.j0, s_c = 0;
-      uint32_t s_uc = 0;
-      bool s_buf = false;                       // S buffer of the current tile acquired
-      // P.V cursor: unit p_u, tile p_j, next value stage p_st
-      int p_u = s_u;
-      pU = sU;
-      int p_j = pU.j0, p_st = 0;
-      bool p_go = false;                        // P of the current tile is ready
-      uint32_t kc = 0, vc = 0, sc = 0, pc = 0, oc = 0;
-      uint32_t idle = 0;
-      uint64_t idle_t0 = 0;
-      while (p_u < p.n_units) {
-        bool progress = false;
-        // ---- O += P V
-        if (!p_go) {
-          const bool first = (p_j == pU.j0);
-          if (mbar_test_wait_cluster(smem_u32(&S.p_full[pc & 1u]), (pc >> 1) & 1u) &&
-              (!first || mbar_test_wait_cluster(smem_u32(&S.o_empty), (oc & 1u) ^ 1u))) {
-            p_go = true;
-            tc_fence_after();
+    } else if (warp >= kVWarp0) {
+      // ------------------------------------------------------------------ value loaders
+      // Index staging: the value loaders also stage each unit's selected positions
+      // [j0*128, j1*128) into buffer (unit ordinal % 2), one unit ahead, as the kv
+      // row to gather -- batch offset applied, bit 31 set for padding and
+      // out-of-range entries, which gather row b*Lk and are masked -- plus one
+      // validity ballot per 32 positions for the softmax.  Warp pw stages the
+      // 32-position words pw, pw + kVWarps, ...  A buffer is free again once the
+      // loaders and the softmax warps are done with the unit two back.
+      // Value stages: per tile, 2 x kNpv stages of 64 keys (kh) x this CTA's kN/2
+      // columns of value block h, i.e. all 128 keys of the tile across the two halves.
+      constexpr int kGroupsPerWarp = 16 * VS::kPlanes / kVWarpsPerSlot;
+      const int pw = (int)warp - kVWarp0;
+      const uint32_t my_slot = (uint32_t)(pw / kVWarpsPerSlot);
+      const int part = pw % kVWarpsPerSlot;
+      uint32_t ucount = 0, vc = 0;
+      bool ok = true;
+      auto stage = [&](const Unit& V, uint32_t buf) {
+        int32_t* dst = idx_sm + buf * kMaxIdx;
+        uint32_t* vmask = S.valid_mask[buf];
+        const int x_begin = V.j0 * kTileKeys, nwords = (V.j1 - V.j0) * (kTileKeys / 32);
+        const int32_t* src = p.indices + (size_t)V.row * p.k;
+        for (int w0 = pw; w0 < nwords; w0 += kVWarps * kStageBatch) {
+          int sidx[kStageBatch];
+#pragma unroll
+          for (int e = 0; e < kStageBatch; ++e) {
+            const int w = w0 + e * kVWarps, x = x_begin + w * 32 + (int)lane;
+            sidx[e] = (w < nwords && x < p.k) ? __ldg(src + x) : -1;
+          }
+#pragma unroll
+          for (int e = 0; e < kStageBatch; ++e) {
+            const int w = w0 + e * kVWarps;
+            if (w >= nwords) break;                       // warp-uniform
+            const bool valid = (sidx[e] >= 0) && (sidx[e] < p.Lk);
+            const int row = V.b * p.Lk + (valid ? sidx[e] : 0);
+            dst[w * 32 + (int)lane] = valid ? row : (int)((uint32_t)row | 0x80000000u);
+            const uint32_t bal = __ballot_sync(0xffffffffu, valid);
+            if (lane == 0) vmask[w] = bal;
           }
         }
-        if (p_go) {
-          const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
-          if (mbar_test_wait(smem_u32(&S.v_full[st]), ph)) {
-            tc_fence_after();
-            const int kh = p_st / VS::kNpv, h = p_st % VS::kNpv;
-            const bool first = (p_j == pU.j0);
-            const uint32_t d = tmem_base + kTmemO + h * (VS::kN / 2);
-            const uint32_t pb = p_base + (pc & 1u) * 2 * kPlane64 + kh * kPlane64;
-#pragma unroll
-            for (int kk = 0; kk < kHalfKeys / 16; ++kk) {
-              const uint64_t ad = make_smem_desc(pb + kk * 32, 16, 1024, LAYOUT_SW128);
-              const uint64_t bd = make_smem_desc(v_base + st * VS::kStageBytes + kk * 2048, kPlane64, 1024,
-                                                 LAYOUT_SW128);
-              mma_bf16_ss_pair(d, ad, bd, idesc_pv, (first && kh == 0 && kk == 0) ? 0u : 1u);
-            }
-            mma_commit_pair_mc(&S.v_empty[st], kBoth);
-            ++vc;
-            progress = true;
-            if (++p_st == 2 * VS::kNpv) {
-              mma_commit_pair_mc(&S.p_empty[pc & 1u], kBoth);
-              if (p_j == pU.j1 - 1) { mma_commit_pair_mc(&S.o_full, kBoth); ++oc; }
-              ++pc;
-              p_st = 0;
-              p_go = false;
-              if (++p_j == pU.j1) {
-                p_u = next_unit(p, p_u + n_clusters, n_clusters, pU);
-                p_j = pU.j0;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.idx_full[buf]);
+      };
+      Unit U, Un;
+      int u = next_unit(p, cluster_id, n_clusters, U);
+      if (u < p.n_units) stage(U, 0);                    // buffer 0 starts free
+      while (u < p.n_units && ok) {
+        const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+        const int un = next_unit(p, u + n_clusters, n_clusters, Un);
+        if (un < p.n_units) {
+          const uint32_t nb = (ucount + 1) & 1u, nph = ((ucount + 1) >> 1) & 1u;
+          ok = mbar_wait_warp(&S.idx_empty[nb], nph ^ 1u, abort_flag);
+          if (!ok) break;
+          stage(Un, nb);
+        }
+        ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
+        if (!ok) break;
+        const int32_t* idx = idx_sm + ib * kMaxIdx;
+        for (int j = U.j0; j < U.j1 && ok; ++j) {
+          for (int kh = 0; kh < 2 && ok; ++kh) {
+            for (int h = 0; h < VS::kNpv; ++h, ++vc) {
+              const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+              if (st != my_slot) continue;
+              bool w_ok = true;
+              if (lane == 0) {
+                w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
+                if (w_ok && leader && part == 0) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
+              }
+              if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+              const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
+              if ((int)lane < kGroupsPerWarp) {
+                const int g = part * kGroupsPerWarp + (int)lane;
+                const int pl = g / 16, kg = g % 16;
+                const int base = (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4;
+                const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
+                tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
+                                 gather_row(idx, base + 0), gather_row(idx, base + 1),
+                                 gather_row(idx, base + 2), gather_row(idx, base + 3));
               }
             }
           }
         }
-        // ---- S = Q K^T
-        if (s_u < p.n_units) {
-          const uint32_t sb = sc & 1u;
-          if (!s_buf && mbar_test_wait_cluster(smem_u32(&S.s_empty[sb]), ((sc >> 1) & 1u) ^ 1u)) {
-            s_buf = true;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+        ++ucount;
+        u = un;
+        U = Un;
+      }
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------------ S issuer
+      // S = Q K^T for each tile into TMEM buffer (tile ordinal % 2), one key chunk
+      // (4 MMAs of K = 16) per ring stage.  S and P.V come from two threads so that
+      // the single-thread issue rate bounds neither.
+      if (leader && elect_one()) {
+        constexpr uint32_t idesc_s = make_idesc(1, 1, 128, kTileKeys, 0, 0);       // bf16, K-major x K-major
+        const uint64_t q_desc = make_smem_desc(smem_u32(q_sm), 16, 1024, LAYOUT_SW128);
+        const uint64_t k_desc = make_smem_desc(smem_u32(k_sm), 16, 1024, LAYOUT_SW128);
+        uint32_t ucount = 0, kc = 0, sc = 0;
+        bool ok = true;
+        Unit U;
+        for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
+             u = next_unit(p, u + n_clusters, n_clusters, U)) {
+          for (int j = U.j0; j < U.j1 && ok; ++j) {
+            const uint32_t sb = sc & 1u;
+            ok = mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag, true);
+            if (!ok) break;
             tc_fence_after();
-          }
-          if (s_buf) {
-            const bool first = (s_j == sU.j0);
-            const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
-            if ((!first || mbar_test_wait(smem_u32(&S.q_full[s_c]), s_uc & 1u)) &&
-                mbar_test_wait(smem_u32(&S.k_full[st]), ph)) {
+            const uint32_t d = tmem_base + kTmemS + sb * kHalfKeys;
+            for (int c = 0; c < NC; ++c) {
+              if (j == U.j0 && !mbar_wait(&S.q_full[c], ucount & 1u, abort_flag)) { ok = false; break; }
+              const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
+              if (!mbar_wait(&S.k_full[st], ph, abort_flag)) { ok = false; break; }
               tc_fence_after();
-              const uint32_t d = tmem_base + kTmemS + sb * kHalfKeys;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = make_smem_desc(q_base + s_c * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
-                const uint64_t bd = make_smem_desc(k_base + st * kPlane64 + kk * 32, 16, 1024, LAYOUT_SW128);
-                mma_bf16_ss_pair(d, ad, bd, idesc_s, (s_c | kk) ? 1u : 0u);
-              }
+              // descriptor start addresses advance 32 B (encoded 2) per K step of 16
+              const uint64_t ad = q_desc + (uint64_t)(c * (kPlane64 >> 4));
+              const uint64_t bd = k_desc + (uint64_t)(st * (kPlane64 >> 4));
+              mma_bf16_ss_pair(d, ad + 0, bd + 0, idesc_s, c ? 1u : 0u);
+              mma_bf16_ss_pair(d, ad + 2, bd + 2, idesc_s, 1u);
+              mma_bf16_ss_pair(d, ad + 4, bd + 4, idesc_s, 1u);
+              mma_bf16_ss_pair(d, ad + 6, bd + 6, idesc_s, 1u);
               mma_commit_pair_mc(&S.k_empty[st], kBoth);
-              if (s_j == sU.j1 - 1) mma_commit_pair_mc(&S.q_empty[s_c], kBoth);   // Q plane free for the next unit
+              if (j == U.j1 - 1) mma_commit_pair_mc(&S.q_empty[c], kBoth);   // Q plane free for the next unit
               ++kc;
-              progress = true;
-              if (++s_c == NC) {
-                mma_commit_pair_mc(&S.s_full[sb], kBoth);
-                ++sc;
-                s_c = 0;
-                s_buf = false;
-                if (++s_j == sU.j1) {
-                  ++s_uc;
-                  s_u = next_unit(p, s_u + n_clusters, n_clusters, sU);
-                  s_j = sU.j0;
-                }
+            }
+            if (!ok) break;
+            mma_commit_pair_mc(&S.s_full[sb], kBoth);
+            ++sc;
+          }
+          ++ucount;
+        }
+        // Wait until every MMA this thread issued has completed before teardown.
+        mma_commit(&S.final_s);
+        mbar_wait(&S.final_s, 0, nullptr);
+      }
+    } else if (warp == kPvWarp) {
+      // ------------------------------------------------------------------ P.V issuer
+      // O += P V per tile: for each value stage (64 keys x kN value columns across
+      // the pair), 4 MMAs of K = 16 keys reading P buffer (tile ordinal % 2).
+      if (leader && elect_one()) {
+        constexpr uint32_t idesc_pv = make_idesc(1, 1, 128, VS::kN, 0, 1);         // P K-major, V MN-major
+        const uint64_t p_desc = make_smem_desc(smem_u32(p_sm), 16, 1024, LAYOUT_SW128);
+        const uint64_t v_desc = make_smem_desc(smem_u32(v_sm), kPlane64, 1024, LAYOUT_SW128);
+        uint32_t vc = 0, pc = 0, oc = 0;
+        bool ok = true;
+        Unit U;
+        for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
+             u = next_unit(p, u + n_clusters, n_clusters, U)) {
+          for (int j = U.j0; j < U.j1 && ok; ++j) {
+            const bool first = (j == U.j0);
+            ok = mbar_wait(&S.p_full[pc & 1u], (pc >> 1) & 1u, abort_flag, true);
+            if (ok && first) ok = mbar_wait(&S.o_empty, (oc & 1u) ^ 1u, abort_flag, true);
+            if (!ok) break;
+            tc_fence_after();
+            for (int kh = 0; kh < 2 && ok; ++kh) {
+              for (int h = 0; h < VS::kNpv; ++h) {
+                const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
+                if (!mbar_wait(&S.v_full[st], ph, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem_base + kTmemO + h * (VS::kN / 2);
+                // P advances 32 B (encoded 2) and V 16 keys = 2048 B (encoded 128) per K step
+                const uint64_t ad = p_desc + (uint64_t)(((pc & 1u) * 2 + kh) * (kPlane64 >> 4));
+                const uint64_t bd = v_desc + (uint64_t)(st * (VS::kStageBytes >> 4));
+                mma_bf16_ss_pair(d, ad + 0, bd + 0, idesc_pv, (first && kh == 0) ? 0u : 1u);
+                mma_bf16_ss_pair(d, ad + 2, bd + 128, idesc_pv, 1u);
+                mma_bf16_ss_pair(d, ad + 4, bd + 256, idesc_pv, 1u);
+                mma_bf16_ss_pair(d, ad + 6, bd + 384, idesc_pv, 1u);
+                mma_commit_pair_mc(&S.v_empty[st], kBoth);
+                ++vc;
               }
             }
+            if (!ok) break;
+            mma_commit_pair_mc(&S.p_empty[pc & 1u], kBoth);
+            if (j == U.j1 - 1) { mma_commit_pair_mc(&S.o_full, kBoth); ++oc; }
+            ++pc;
           }
         }
-        // ---- bounded idling
-        if (progress) {
-          idle = 0;
-        } else if ((++idle % kIdleCheck) == 0) {
-          if (*abort_flag) break;
-          const uint64_t now = global_timer_ns();
-          if (idle == kIdleCheck) {
-            idle_t0 = now;
-          } else if (now - idle_t0 > kWaitLimitNs) {
-            atomicExch(&g_device_error, DEV_ERR_TIMEOUT);
-            *abort_flag = 1u;
-            break;
-          }
-        }
+        mma_commit(&S.final_pv);
+        mbar_wait(&S.final_pv, 0, nullptr);
       }
-      // Wait until every MMA this thread issued has completed before teardown.
-      mma_commit(&S.final_bar);
-      mbar_wait(&S.final_bar, 0, nullptr);
     }
   } else {
+    regs_increase<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax / epilogue
     const uint32_t l = warp * 32 + lane;          // TMEM lane = (key half, head)
     const uint32_t h = l & 63u;                   // head within this CTA
@@ -681,6 +679,12 @@ cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorM
   auto kern = sparse_attn_kernel<NC, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // The register split must fit in what the CTA launches with, or the increase
+  // would wait forever: refuse to launch a build where it does not.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if ((uint32_t)fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
   kern<<<grid_clusters * 2, kThreads, smem, stream>>>(tq, tkv, p);
   return cudaGetLastError();
 }
@@ -715,5 +719,7 @@ cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t strea
   else return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
+
+cudaError_t read_attn_error(uint32_t* value, bool clear) { return read_unit_error(value, clear); }
 
 }  // namespace dsa

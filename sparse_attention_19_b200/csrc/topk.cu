@@ -213,4 +213,6 @@ cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+cudaError_t read_topk_error(uint32_t* value, bool clear) { return read_unit_error(value, clear); }
+
 }  // namespace dsa
