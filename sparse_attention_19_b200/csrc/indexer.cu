@@ -14,8 +14,9 @@
 // shared memory and streams key tiles through a TMA ring; two TMEM accumulators
 // let the epilogue of one sub-block overlap the MMA of the next.
 //
-// Warp roles (288 threads): warps 0..3 epilogue (warp w reads TMEM lanes 32w .. 32w+31),
-// warp 4 TMEM owner + MMA issuer, warps 5..8 TMA loaders.
+// Warp roles (416 threads): warps 0..7 epilogue (warp w reads TMEM lanes
+// 32(w%4) .. 32(w%4)+31 and every other 64-column group, starting at group w/4),
+// warp 8 TMEM owner + MMA issuer, warps 9..12 TMA loaders.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -31,10 +32,13 @@ namespace {
 
 constexpr int kKeysPerTile = 128;
 constexpr int kMaxStages = 8;
-constexpr int kThreads = 288;        // warps 0-3 epilogue, 4 MMA, 5-8 loaders
+constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, splitting the columns
+constexpr int kMmaWarp = kEpiWarps;
 constexpr int kLoaders = 4;          // TMA requests from one warp are served in order, so each
                                      // key tile is loaded as four 32-row boxes from four warps
-constexpr int kLoaderWarp0 = 5;
+constexpr int kLoaderWarp0 = kMmaWarp + 1;
+constexpr int kThreads = 32 * (kLoaderWarp0 + kLoaders);   // 416
+static_assert(kLoaders * 32 == kKeysPerTile, "one 32-row box per loader");
 constexpr int kTmemCols = 512;
 
 struct IndexerSmem {
@@ -43,7 +47,7 @@ struct IndexerSmem {
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];
   uint64_t acc_full[8], acc_empty[8];     // TMEM accumulators: 512 / N of them (at most 8)
   uint64_t final_bar;
-  uint64_t epi_bar;          // rendezvous of the 4 epilogue warps
+  uint64_t epi_bar;          // rendezvous of the epilogue warps
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -106,14 +110,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
     for (int s = 0; s < 8; ++s) {
       mbar_init(&S.acc_full[s], 1);
-      mbar_init(&S.acc_empty[s], 4);
+      mbar_init(&S.acc_empty[s], kEpiWarps);
     }
     mbar_init(&S.final_bar, 1);
-    mbar_init(&S.epi_bar, 4);
+    mbar_init(&S.epi_bar, kEpiWarps);
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -152,7 +156,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (!ok) break;
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       const uint32_t idesc = make_idesc(0, 0, 128, (uint32_t)N, 0, 0);  // e4m3 x e4m3 -> f32
@@ -195,21 +199,22 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t quarter = warp;                   // TMEM lane quarter this warp may read
+    const uint32_t quarter = warp & 3u;              // TMEM lane quarter this warp may read
+    const uint32_t half = warp >> 2;                 // which 64-column groups (even / odd)
     const uint32_t row = quarter * 32 + lane;        // key row within the tile
-    const int et = threadIdx.x;                      // 0..127
+    const int et = threadIdx.x;                      // 0 .. 32 * kEpiWarps - 1
     uint32_t seq = 0, epi_phase = 0;
     for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
       const UnitInfo U = decode_unit(p, u);
       if (!warps_rendezvous(&S.epi_bar, epi_phase, abort_flag)) break;   // previous unit done with w/sq
-      for (int x = et; x < QU * H_I; x += 128) {
+      for (int x = et; x < QU * H_I; x += 32 * kEpiWarps) {
         const int qq = x / H_I, j = x % H_I;
         const int i = U.i0 + qq;
         float wv = 0.f;
         if (i < p.Lq) wv = __bfloat162float(p.w[((size_t)U.b * p.Lq + i) * H_I + j]);
         w_smem[x] = wv;
       }
-      for (int x = et; x < QU; x += 128) {
+      for (int x = et; x < QU; x += 32 * kEpiWarps) {
         const int i = U.i0 + x;
         sq_smem[x] = (i < p.Lq) ? (p.q_scale ? p.q_scale[(size_t)U.b * p.Lq + i] : 1.f) : 0.f;
       }
@@ -232,9 +237,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t t_base = tmem_base + ((quarter * 32u) << 16) + slot * (uint32_t)N;
-          // 64 columns per TMEM round trip (two loads, one wait); each query owns H_I columns.
+          // 64 columns per TMEM round trip (two loads, one wait); each query owns H_I
+          // columns.  The head sum runs as two interleaved partial sums (packed FMA).
           constexpr int QPG = (H_I >= 64) ? 1 : 64 / H_I;      // queries per 64-column group
-          for (int g0 = 0; g0 < N; g0 += 64) {
+          constexpr int HE = (H_I >= 64) ? 64 : H_I;            // heads of one query in a group
+          for (int g0 = (int)half * 64; g0 < N; g0 += 128) {
             uint32_t v[64];
             tmem_ld32(t_base + (uint32_t)g0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             tmem_ld32(t_base + (uint32_t)g0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
@@ -242,11 +249,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 #pragma unroll
             for (int a = 0; a < QPG; ++a) {
               const int qi = g0 / H_I + a;                    // query within the sub-block
-              const float* wq = w_smem + (size_t)(sb * p.qb + qi) * H_I;
-              float acc = 0.f;
+              const float2* wq = reinterpret_cast<const float2*>(w_smem + (size_t)(sb * p.qb + qi) * H_I);
+              float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-              for (int e = 0; e < (H_I >= 64 ? 64 : H_I); ++e)
-                acc = fmaf(wq[e], fmaxf(__uint_as_float(v[a * (H_I >= 64 ? 64 : H_I) + e]), 0.f), acc);
+              for (int e = 0; e < HE; e += 2)
+                acc2 = ffma2(make_float2(fmaxf(__uint_as_float(v[a * HE + e]), 0.f),
+                                         fmaxf(__uint_as_float(v[a * HE + e + 1]), 0.f)),
+                             wq[e / 2], acc2);
+              const float acc = acc2.x + acc2.y;
               const int qq = sb * p.qb + qi;
               const int i = U.i0 + qq;
               if (i < p.Lq && s < p.Lk) {
@@ -272,7 +282,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         for (int kt = U.kt1; kt < nt_all; ++kt) {
           const int s = kt * kKeysPerTile + (int)row;
           if (s >= p.Lk) continue;
-          for (int qq = 0; qq < QU; ++qq) {
+          for (int qq = (int)half; qq < QU; qq += 2) {
             const int i = U.i0 + qq;
             if (i < p.Lq)
               __stcs(p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s, -INFINITY);
@@ -284,7 +294,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }

@@ -196,6 +196,17 @@ __device__ __forceinline__ bool warps_rendezvous(uint64_t* bar, uint32_t& phase,
   return ok;
 }
 
+// ---------------------------------------------------------------- packed fp32
+// Two independent round-to-nearest FMAs in one instruction: (a.x*b.x + c.x, a.y*b.y + c.y).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<const float2*>(&r);
+}
+
 // ---------------------------------------------------------------- register split
 // Per-warpgroup register budget (all 4 warps of a warpgroup execute the same one).
 // The increases of a CTA must fit within what its decreases release from the
