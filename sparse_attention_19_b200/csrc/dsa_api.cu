@@ -22,6 +22,7 @@ namespace {
 
 constexpr int kMaxK = 2048;
 constexpr int kAttnTile = 128;
+constexpr long long kTopkCacheMax = 8192;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -151,14 +152,14 @@ dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, in
                     cudaStream_t st) {
   TopkParams p{};
   p.scores = scores; p.B = B; p.Lq = Lq; p.Lk = Lk; p.q_offset = q_offset; p.k = k; p.indices = idx;
-  const long long nmax = (long long)q_offset + Lq < Lk ? (long long)q_offset + Lq : Lk;
-  if (nmax <= 32768) {
-    p.cache_cap = (int)round_up((size_t)nmax, 4);
-    p.cand_cap = 4096;
-  } else {
-    p.cache_cap = 0;
-    p.cand_cap = 16384;
-  }
+  const long long nmax = (long long)q_offset + Lq < Lk ? (long long)q_offset + Lq : Lk;   // longest row
+  // Rows up to kTopkCacheMax scores stay in shared memory between passes; longer
+  // ones are re-read from L2 (measured faster at 32K: the small CTA lets more rows
+  // share an SM, and their second pass still hits L2).
+  p.cache_cap = nmax <= kTopkCacheMax ? (int)round_up((size_t)nmax, 4) : 0;
+  p.bit_words = (int)round_up((size_t)(nmax + 31) / 32, 4);
+  p.cand_cap = 4096;
+  p.vec4 = (aligned16(scores) && Lk % 4 == 0) ? 1 : 0;
   return launch_topk(p, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

@@ -35,10 +35,12 @@ struct TopkParams {
   const float* scores;    // [B, Lq, Lk]
   int B, Lq, Lk, q_offset, k;
   int32_t* indices;       // [B, Lq, k]
-  int cache_cap;          // row elements cached in shared memory (0 = stream from global)
+  int cache_cap;          // row elements cached in shared memory (0 = re-read from global); multiple of 4
+  int bit_words;          // 32-bit words of each position bitmap (>= ceil(row length / 32)); multiple of 4
   int cand_cap;           // candidate (key, position) pairs held in shared memory
+  int vec4;               // rows start 16-byte aligned (scores aligned, Lk % 4 == 0): 16-byte loads
 };
-size_t topk_smem_bytes(int cache_cap, int cand_cap);
+size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap);
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sparse attention

@@ -1,19 +1,30 @@
-// topk.cu -- per-query top-k over the indexer scores (radix select).
+// topk.cu -- per-query top-k over the indexer scores.
 //
 // Row (b, i) sits at position t = q_offset + i and selects, among the n =
 // min(t+1, Lk) scores I[t, 0..n), the m = min(k, n) largest, ties to the smaller
 // position ("Отбор и основное внимание": the k KV entries with the largest
 // I_{t,s}).  The result is written in ascending position order, -1 padded.
 //
-// Method: fp32 scores become order-preserving 32-bit keys (-0.0 is first
-// canonicalised to +0.0).  The key of the m-th largest element is found digit by
-// digit (11 + 11 + 10 bits) from shared-memory histograms; after the first digit
-// only the elements of the boundary bin (copied to a candidate list) are
-// visited.  A final pass in position order takes every key above the threshold
-// and the first (m - #above) keys equal to it, placing each selected element at
-// (number of selected elements before it) via a block-wide prefix sum, so the
-// output is sorted and ties resolve to smaller positions.
-// One CTA per row; the row is cached in shared memory when it fits.
+// Method (one CTA per row).  fp32 scores become order-preserving 32-bit keys
+// (-0.0 is first canonicalised to +0.0).  The exact key of the m-th largest
+// element (the threshold) is found by histogram refinement:
+//   1. a strided sample of the row (1024 scores) gives a key range [lo, hi];
+//   2. one pass over the row builds a 2048-bin histogram over that range (bin =
+//      (key - lo) >> shift, so the bins follow the data rather than the float
+//      exponent; keys outside the range are clamped into the end bins) and
+//      yields the bin b that holds the m-th largest key and the count above it;
+//   3. a second pass records every element of a bin above b in a bitmap (warp
+//      ballots, no atomics) and collects the elements of bin b as candidates;
+//      the threshold is then refined on the candidates in shared memory, with
+//      2048-bin histograms over the candidates' own key range, down to an exact key.
+// The output takes every element above the threshold and the first
+// (m - #above) elements equal to it in position order: two bitmaps (above,
+// equal) are scanned word by word with warp prefix sums, so positions come out
+// sorted and ties resolve to smaller positions.  When bin b holds more elements
+// than the candidate buffer (many equal scores), the refinement runs over the
+// row instead and a final pass rebuilds both bitmaps.
+// Rows up to cache_cap elements are kept in shared memory after the first pass;
+// longer rows are re-read (from L2) by each pass.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -27,6 +38,11 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kBinBits = 11;
+constexpr int kBins = 1 << kBinBits;
+constexpr int kUnroll = 8;           // 4-byte loads in flight per thread in the row passes
+constexpr int kUnroll4 = 4;          // 16-byte loads in flight per thread in the histogram pass
+constexpr int kSample = 1024;        // strided sample that sets the first histogram's range
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -34,11 +50,11 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// 16-byte multiple, so the row cache and the 8-byte candidate pairs that follow
-// it in dynamic shared memory stay aligned.
+// 16-byte multiple, so the arrays that follow it in dynamic shared memory stay aligned.
 struct alignas(16) TopkShared {
-  uint32_t hist[2048];
+  uint32_t hist[kBins];
   uint32_t warp_tot[kWarps];
+  uint32_t warp_a[kWarps], warp_b[kWarps];
   uint32_t bin, above, ncand;
 };
 
@@ -71,14 +87,16 @@ __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* w
 
 // Find the bin b (searching from the top) where the running count from above first
 // reaches `need`; records b and the count strictly above it.
-__device__ void find_bin(TopkShared& sh, int nbins, uint32_t need) {
-  const int per = nbins / kThreads;                 // bins per thread (4 or 2)
+__device__ void find_bin(TopkShared& sh, uint32_t need) {
+  constexpr int per = kBins / kThreads;            // bins per thread
   const int lo = threadIdx.x * per;
   uint32_t mine = 0;
+#pragma unroll
   for (int x = 0; x < per; ++x) mine += sh.hist[lo + x];
   uint32_t total;
   const uint32_t incl = block_inclusive_scan(mine, sh.warp_tot, total);
   uint32_t acc = total - incl;                      // count in bins above this thread's range
+#pragma unroll
   for (int x = per - 1; x >= 0; --x) {
     const uint32_t c = sh.hist[lo + x];
     if (acc < need && acc + c >= need) {
@@ -90,12 +108,63 @@ __device__ void find_bin(TopkShared& sh, int nbins, uint32_t need) {
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
+// Right shift that maps a key range of width range+1 onto at most kBins bins.
+__device__ __forceinline__ int bin_shift(uint32_t range) {
+  return range == 0u ? 0 : max(0, 32 - __clz(range) - kBinBits);
+}
+
+// Block-wide min and max (every thread receives both).
+__device__ __forceinline__ void block_min_max(TopkShared& sh, uint32_t& mn, uint32_t& mx) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  __syncthreads();                                  // earlier readers of warp_a / warp_b are done
+  if (lane == 0) { sh.warp_a[warp] = mn; sh.warp_b[warp] = mx; }
+  __syncthreads();
+  mn = sh.warp_a[0];
+  mx = sh.warp_b[0];
+  for (int w = 1; w < kWarps; ++w) { mn = min(mn, sh.warp_a[w]); mx = max(mx, sh.warp_b[w]); }
+}
+
+__device__ __forceinline__ void clear_hist(TopkShared& sh) {
+  for (int x = threadIdx.x; x < kBins; x += kThreads) sh.hist[x] = 0u;
+  __syncthreads();
+}
+
+// Visits every position s < n of the row in warp-aligned groups of 32 (lane =
+// s % 32, so one warp's ballot covers one bitmap word), with kUnroll groups per
+// thread in flight: f(s, valid, key), key = 0 when !valid.  Every lane of a warp
+// calls f for the same groups.
+template <typename KeyAt, typename F>
+__device__ __forceinline__ void row_pass(int n, KeyAt key_at, F f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int base = warp * 32; base < n; base += kThreads * kUnroll) {
+    uint32_t key[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int s = base + u * kThreads + lane;
+      key[u] = (s < n) ? key_at(s) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int g = base + u * kThreads;           // warp-uniform
+      if (g < n) f(g + lane, g + lane < n, key[u]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
   uint32_t* cache = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
-  uint2* cand = reinterpret_cast<uint2*>(cache + (p.cache_cap + 3) / 4 * 4);
+  uint32_t* gt_bits = cache + p.cache_cap;          // cache_cap and bit_words are multiples of 4
+  uint32_t* eq_bits = gt_bits + p.bit_words;
+  uint2* cand = reinterpret_cast<uint2*>(eq_bits + p.bit_words);
 
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int row = blockIdx.x;                       // b * Lq + i
   const int i = row % p.Lq;
   const long long t = (long long)p.q_offset + i;
@@ -109,102 +178,198 @@ __global__ void __launch_bounds__(kThreads, 1) topk_kernel(const TopkParams p) {
     return;
   }
   const bool cached = n <= p.cache_cap;
+  auto key_at = [&](int s) -> uint32_t { return cached ? cache[s] : score_key(__ldg(src + s)); };
+  auto load_key = [&](int s) -> uint32_t { return score_key(__ldg(src + s)); };
 
-  // ---- digit 1: bits 31..21, over the whole row (also fills the cache)
-  for (int x = threadIdx.x; x < 2048; x += kThreads) sh.hist[x] = 0u;
-  if (threadIdx.x == 0) sh.ncand = 0u;
-  __syncthreads();
-  for (int s = threadIdx.x; s < n; s += kThreads) {
-    const uint32_t key = score_key(__ldcs(src + s));
-    if (cached) cache[s] = key;
-    atomicAdd(&sh.hist[key >> 21], 1u);
+  // ---- 1. key range of a strided sample
+  const int ns = n < kSample ? n : kSample;
+  uint32_t smin = 0xffffffffu, smax = 0u;
+  for (int j = threadIdx.x; j < ns; j += kThreads) {
+    const uint32_t key = load_key((int)(((long long)j * n) / ns));
+    smin = min(smin, key);
+    smax = max(smax, key);
+  }
+  block_min_max(sh, smin, smax);
+
+  // ---- 2. histogram over the sampled range (outliers clamped into the end bins)
+  const uint32_t lo = smin;
+  const int shift = bin_shift(smax - smin);
+  auto bin_of = [lo, shift](uint32_t key) -> uint32_t {
+    return key < lo ? 0u : min((uint32_t)(kBins - 1), (key - lo) >> shift);
+  };
+  clear_hist(sh);
+  if (p.vec4) {
+    // 16-byte loads (rows start 16-byte aligned): four scores per thread per step.
+    const float4* src4 = reinterpret_cast<const float4*>(src);
+    const int nq = n >> 2;
+    for (int q0 = threadIdx.x; q0 < nq; q0 += kThreads * kUnroll4) {
+      float4 f[kUnroll4];
+#pragma unroll
+      for (int u = 0; u < kUnroll4; ++u) {
+        const int q = q0 + u * kThreads;
+        f[u] = (q < nq) ? __ldg(src4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll4; ++u) {
+        const int q = q0 + u * kThreads;
+        if (q >= nq) break;
+        const uint4 key = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
+        if (cached) reinterpret_cast<uint4*>(cache)[q] = key;
+        atomicAdd(&sh.hist[bin_of(key.x)], 1u);
+        atomicAdd(&sh.hist[bin_of(key.y)], 1u);
+        atomicAdd(&sh.hist[bin_of(key.z)], 1u);
+        atomicAdd(&sh.hist[bin_of(key.w)], 1u);
+      }
+    }
+    for (int s = (nq << 2) + (int)threadIdx.x; s < n; s += kThreads) {
+      const uint32_t key = load_key(s);
+      if (cached) cache[s] = key;
+      atomicAdd(&sh.hist[bin_of(key)], 1u);
+    }
+  } else {
+    row_pass(n, load_key, [&](int s, bool valid, uint32_t key) {
+      if (!valid) return;
+      if (cached) cache[s] = key;
+      atomicAdd(&sh.hist[bin_of(key)], 1u);
+    });
   }
   __syncthreads();
-  find_bin(sh, 2048, (uint32_t)k);
-  const uint32_t b1 = sh.bin;
-  uint32_t need = (uint32_t)k - sh.above;           // still to take inside bin b1
-  auto key_at = [&](int s) -> uint32_t { return cached ? cache[s] : score_key(__ldcs(src + s)); };
+  uint32_t need = (uint32_t)k;                       // n > k, so m = k
+  find_bin(sh, need);
+  const uint32_t b = sh.bin;
+  need -= sh.above;
+  const uint32_t cnt_b = sh.hist[b];
 
-  // ---- compact the boundary bin
-  for (int s = threadIdx.x; s < n; s += kThreads) {
-    const uint32_t key = key_at(s);
-    if ((key >> 21) == b1) {
+  // ---- 3. bins above b are selected; bin b becomes the candidate list
+  if (threadIdx.x == 0) sh.ncand = 0u;
+  __syncthreads();
+  row_pass(n, key_at, [&](int s, bool valid, uint32_t key) {
+    const uint32_t d = bin_of(key);
+    const uint32_t gbal = __ballot_sync(0xffffffffu, valid && d > b);
+    if (lane == 0) { gt_bits[s >> 5] = gbal; eq_bits[s >> 5] = 0u; }
+    if (valid && d == b) {
       const uint32_t pos = atomicAdd(&sh.ncand, 1u);
       if (pos < (uint32_t)p.cand_cap) cand[pos] = make_uint2(key, (uint32_t)s);
     }
+  });
+  __syncthreads();
+  const bool fits = cnt_b <= (uint32_t)p.cand_cap;
+
+  // Exact threshold: the need-th largest key among the elements of bin b, found
+  // by 2048-bin histograms over a shrinking key window [wlo, whi] (inclusive).
+  uint32_t wlo, whi;
+  if (fits) {
+    uint32_t cmin = 0xffffffffu, cmax = 0u;
+    for (int x = threadIdx.x; x < (int)cnt_b; x += kThreads) {
+      cmin = min(cmin, cand[x].x);
+      cmax = max(cmax, cand[x].x);
+    }
+    block_min_max(sh, cmin, cmax);
+    wlo = cmin;
+    whi = cmax;
+  } else {
+    wlo = (b == 0) ? 0u : lo + (b << shift);
+    whi = (b == (uint32_t)(kBins - 1)) ? 0xffffffffu : lo + (((b + 1) << shift) - 1u);
+  }
+  uint32_t thr;
+  for (;;) {
+    const int wsh = bin_shift(whi - wlo);
+    const uint32_t l0 = wlo, h0 = whi;
+    clear_hist(sh);
+    if (fits) {
+      for (int x = threadIdx.x; x < (int)cnt_b; x += kThreads) {
+        const uint32_t key = cand[x].x;
+        if (key >= l0 && key <= h0) atomicAdd(&sh.hist[(key - l0) >> wsh], 1u);
+      }
+    } else {
+      row_pass(n, key_at, [&](int, bool valid, uint32_t key) {
+        if (valid && key >= l0 && key <= h0) atomicAdd(&sh.hist[(key - l0) >> wsh], 1u);
+      });
+    }
+    __syncthreads();
+    find_bin(sh, need);
+    const uint32_t bw = sh.bin;
+    need -= sh.above;
+    if (wsh == 0) { thr = wlo + bw; break; }
+    wlo = l0 + (bw << wsh);
+    const unsigned long long top = (unsigned long long)wlo + (1ull << wsh) - 1ull;
+    whi = top < (unsigned long long)h0 ? (uint32_t)top : h0;
+  }
+  if (fits) {
+    for (int x = threadIdx.x; x < (int)cnt_b; x += kThreads) {
+      const uint2 c = cand[x];
+      if (c.x > thr) atomicOr(&gt_bits[c.y >> 5], 1u << (c.y & 31u));
+      else if (c.x == thr) atomicOr(&eq_bits[c.y >> 5], 1u << (c.y & 31u));
+    }
+  } else {
+    // Bitmaps rebuilt from one pass over the row: above = key > thr, equal = key == thr.
+    row_pass(n, key_at, [&](int s, bool valid, uint32_t key) {
+      const uint32_t gbal = __ballot_sync(0xffffffffu, valid && key > thr);
+      const uint32_t ebal = __ballot_sync(0xffffffffu, valid && key == thr);
+      if (lane == 0) { gt_bits[s >> 5] = gbal; eq_bits[s >> 5] = ebal; }
+    });
   }
   __syncthreads();
-  const uint32_t ncand = sh.ncand;
-  const bool use_cand = ncand <= (uint32_t)p.cand_cap;
-  const int scan_n = use_cand ? (int)ncand : n;
 
-  // ---- digits 2 (bits 20..10) and 3 (bits 9..0) over the candidates
-  uint32_t prefix = b1;                              // known high bits of the threshold key
-  int known = 11;                                    // how many high bits are known
-  const int widths[2] = {11, 10};
-  for (int d = 0; d < 2; ++d) {
-    const int wbits = widths[d];
-    const int shift = 32 - known - wbits;
-    const int nbins = 1 << wbits;
-    for (int x = threadIdx.x; x < 2048; x += kThreads) sh.hist[x] = 0u;
-    __syncthreads();
-    for (int x = threadIdx.x; x < scan_n; x += kThreads) {
-      const uint32_t key = use_cand ? cand[x].x : key_at(x);
-      if ((key >> (32 - known)) == prefix) atomicAdd(&sh.hist[(key >> shift) & (nbins - 1)], 1u);
-    }
-    __syncthreads();
-    find_bin(sh, nbins < 2048 ? 2048 : nbins, need);   // unused upper bins are zero
-    prefix = (prefix << wbits) | sh.bin;
-    need -= sh.above;
-    known += wbits;
+  // ---- 4. ordered output: every "above" position and the first eq_take "equal" ones
+  const uint32_t eq_take = need;
+  const int W = (n + 31) >> 5;
+  const int wpw = (W + kWarps - 1) / kWarps;         // bitmap words per warp
+  const int w_begin = warp * wpw, w_end = min(W, w_begin + wpw);
+  uint32_t cg = 0, ce = 0;
+  for (int w = w_begin + lane; w < w_end; w += 32) { cg += __popc(gt_bits[w]); ce += __popc(eq_bits[w]); }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    cg += __shfl_xor_sync(0xffffffffu, cg, o);
+    ce += __shfl_xor_sync(0xffffffffu, ce, o);
   }
-  const uint32_t thr = prefix;                       // exact key of the m-th largest
-  const uint32_t eq_take = need;                     // how many keys == thr to take
-
-  // ---- ordered output pass
-  constexpr int E = 4;                               // consecutive elements per thread
-  uint32_t gt_off = 0, eq_off = 0;
-  for (int base = 0; base < n; base += kThreads * E) {
-    const int s0 = base + threadIdx.x * E;
-    uint32_t keys[E];
-    uint32_t gt = 0, eq = 0;
+  if (lane == 0) { sh.warp_a[warp] = cg; sh.warp_b[warp] = ce; }
+  __syncthreads();
+  uint32_t g = 0, e = 0;
+  for (int w = 0; w < warp; ++w) { g += sh.warp_a[w]; e += sh.warp_b[w]; }
+  for (int w0 = w_begin; w0 < w_end; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t gw = (w < w_end) ? gt_bits[w] : 0u;
+    const uint32_t ew = (w < w_end) ? eq_bits[w] : 0u;
+    // inclusive prefix of the per-word counts over the lanes (word order)
+    const uint32_t tg = __popc(gw), te = __popc(ew);
+    uint32_t pg = tg, pe = te;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int s = s0 + e;
-      keys[e] = (s < n) ? key_at(s) : 0u;
-      if (s < n) { gt += keys[e] > thr; eq += keys[e] == thr; }
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t yg = __shfl_up_sync(0xffffffffu, pg, o);
+      const uint32_t ye = __shfl_up_sync(0xffffffffu, pe, o);
+      if (lane >= o) { pg += yg; pe += ye; }
     }
-    uint32_t total;
-    const uint32_t incl = block_inclusive_scan(gt | (eq << 16), sh.warp_tot, total);
-    const uint32_t excl = incl - (gt | (eq << 16));
-    uint32_t g = gt_off + (excl & 0xFFFFu), q = eq_off + (excl >> 16);
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int s = s0 + e;
-      if (s >= n) break;
-      if (keys[e] > thr) {
-        const uint32_t pos = g + min(q, eq_take);
+    const uint32_t sum_g = __shfl_sync(0xffffffffu, pg, 31), sum_e = __shfl_sync(0xffffffffu, pe, 31);
+    uint32_t gg = g + pg - tg, ee = e + pe - te;
+    uint32_t sel = gw | ew;
+    while (sel) {
+      const int bit = __ffs(sel) - 1;
+      sel &= sel - 1u;
+      const int s = w * 32 + bit;
+      if ((gw >> bit) & 1u) {
+        const uint32_t pos = gg + min(ee, eq_take);
         if (pos < (uint32_t)k) out[pos] = s;
-        ++g;
-      } else if (keys[e] == thr) {
-        if (q < eq_take && g + q < (uint32_t)k) out[g + q] = s;
-        ++q;
+        ++gg;
+      } else {
+        if (ee < eq_take && gg + ee < (uint32_t)k) out[gg + ee] = s;
+        ++ee;
       }
     }
-    gt_off += total & 0xFFFFu;
-    eq_off += total >> 16;
+    g += sum_g;
+    e += sum_e;
   }
 }
 
 }  // namespace
 
-size_t topk_smem_bytes(int cache_cap, int cand_cap) {
-  static_assert(sizeof(TopkShared) % 16 == 0, "candidate pairs must stay 8-byte aligned");
-  return sizeof(TopkShared) + (size_t)((cache_cap + 3) / 4 * 4) * 4 + (size_t)cand_cap * 8;
+size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap) {
+  static_assert(sizeof(TopkShared) % 16 == 0, "arrays that follow must stay 16-byte aligned");
+  return sizeof(TopkShared) + ((size_t)cache_cap + 2 * (size_t)bit_words) * 4 + (size_t)cand_cap * 8;
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream) {
-  const size_t smem = topk_smem_bytes(p.cache_cap, p.cand_cap);
+  const size_t smem = topk_smem_bytes(p.cache_cap, p.bit_words, p.cand_cap);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int rows = p.B * p.Lq;
