@@ -41,7 +41,7 @@
 // Warp roles (768 threads per CTA): warps 0-3 softmax/epilogue (TMEM lane quarter
 // = warp), warp 4 TMEM owner + S issuer (leader), warp 5 P.V issuer (leader),
 // warps 6-14 key loaders, warps 15-23 value loaders + index staging.  The softmax
-// warpgroup holds 112 registers per thread, the others 72 (setmaxnreg).
+// warpgroup holds 120 registers per thread, the others 72 (setmaxnreg).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -75,10 +75,10 @@ constexpr int kVWarps = kVStages * kVWarpsPerSlot;
 constexpr int kThreads = 32 * (kVWarp0 + kVWarps);   // 768
 constexpr int kStageBatch = 8;       // index words in flight per warp while staging
 // Register split: the CTA launches with 80 registers per thread (6 warps per SM
-// sub-partition); the softmax warpgroup then takes 112 and the other warpgroups
+// sub-partition); the softmax warpgroup then takes 120 and the other warpgroups
 // (MMA issuers, loaders) keep 72.
 constexpr uint32_t kRegsLaunch = 80;
-constexpr uint32_t kRegsSoftmax = 112;
+constexpr uint32_t kRegsSoftmax = 120;
 constexpr uint32_t kRegsOther = 72;
 static_assert(128 * kRegsSoftmax + (kThreads - 128) * kRegsOther <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
@@ -99,7 +99,7 @@ struct AttnBarriers {
   uint64_t o_full, o_empty, final_s, final_pv;
   uint64_t idx_full[2], idx_empty[2];
   uint32_t valid_mask[2][kMaxIdx / 32];   // per 32 staged positions: bit set = valid entry
-  uint64_t xbar;             // rendezvous of the 4 softmax warps (max / sum exchange)
+  uint64_t xbar[2];          // rendezvous of softmax warps w and w ^ 2 (same heads, other key half)
   uint32_t tmem_base;
   uint32_t abort_flag;
   float red_max[2][128];
@@ -201,7 +201,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     mbar_init(&S.o_empty, 8);
     mbar_init(&S.final_s, 1);
     mbar_init(&S.final_pv, 1);
-    mbar_init(&S.xbar, 4);
+    mbar_init(&S.xbar[0], 2);
+    mbar_init(&S.xbar[1], 2);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -484,26 +485,27 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         ok = mbar_wait_warp(&S.s_full[sb], (sc >> 1) & 1u, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        // Two passes over this lane's 64 logits in TMEM (32 at a time, to stay within
-        // the register budget): the row maximum, then the probabilities, packed to
-        // bf16 pairs.
+        // This lane's 64 logits, read from TMEM once.  Invalid entries (padding,
+        // out-of-range) become -inf; whole groups are valid except in a row's last tile.
         const uint32_t s_addr = tmem_base + lane_addr + kTmemS + sb * kHalfKeys;
         const uint32_t* vm = &S.valid_mask[ib][((j - U.j0) * kTileKeys + (int)half * kHalfKeys) / 32];
-        const uint32_t vmask0 = vm[0], vmask1 = vm[1];
+        const uint32_t vmask0 = vm[0], vmask1 = vm[1];   // warp-uniform
+        uint32_t v[64];
+        tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
+        if ((vmask0 & vmask1) != 0xffffffffu) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (!((((c < 32) ? vmask0 : vmask1) >> (c & 31)) & 1u)) v[c] = __float_as_uint(-INFINITY);
+        }
         float smax = -INFINITY;                       // maximum of the raw logits (scale > 0)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t v[32];
-          tmem_ld32(s_addr + hh * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if ((((hh == 0) ? vmask0 : vmask1) >> c) & 1u) smax = fmaxf(smax, __uint_as_float(v[c]));
-        }
+        for (int c = 0; c < 64; ++c) smax = fmaxf(smax, __uint_as_float(v[c]));
         float tmax = smax * p.scale_log2;
         const uint32_t rb = sc & 1u;
         S.red_max[rb][l] = tmax;
-        ok = warps_rendezvous(&S.xbar, xph, abort_flag);
+        ok = warps_rendezvous(&S.xbar[warp & 1u], xph, abort_flag);
         if (!ok) break;
         tmax = fmaxf(tmax, S.red_max[rb][l ^ 64u]);
         const float m_new = fmaxf(m, tmax);
@@ -522,44 +524,39 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           if (!ok) break;
           tc_fence_after();
           const float alpha = need ? exp2f(m - m_new) : 1.f;
-          for (int c0 = 0; c0 < VS::kNpv * (VS::kN / 2); c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld32(tmem_base + lane_addr + kTmemO + c0, ov);
+          for (int c0 = 0; c0 < VS::kNpv * (VS::kN / 2); c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld16(tmem_base + lane_addr + kTmemO + c0, ov);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tmem_base + lane_addr + kTmemO + c0, ov);
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st16(tmem_base + lane_addr + kTmemO + c0, ov);
           }
           tmem_st_wait();
           if (need) lsum *= alpha;
         }
         if (need) m = m_new;
-        // probabilities in bf16, straight into P (the sum uses the rounded values, as P.V sees them)
+        // Probabilities 2^(z*scale*log2e - m), packed to bf16 straight into P (row h of
+        // this lane's key-half plane, 128-byte swizzle); the row sum is kept in fp32.
         uint8_t* prow = p_sm + (pbuf * 2 + half) * kPlane64 + (h >> 3) * 1024 + (h & 7) * 128;
-        float psum = 0.f;
-#pragma unroll 1   // one 32-column half at a time keeps the live registers low
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t v[32];
-          tmem_ld32(s_addr + hh * 32, v);
-          tmem_ld_wait();
+        const float2 scl = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm = make_float2(-m_use, -m_use);
+        float2 sum2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w4[4];
+        for (int q = 0; q < 8; ++q) {                   // 16-byte chunk q: keys 8q .. 8q+7
+          uint32_t w4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c0 = q4 * 8 + 2 * e, c1 = c0 + 1;
-              const uint32_t vmh = (hh == 0) ? vmask0 : vmask1;
-              const float x0 = ((vmh >> c0) & 1u) ? fmaf(__uint_as_float(v[c0]), p.scale_log2, -m_use) : -INFINITY;
-              const float x1 = ((vmh >> c1) & 1u) ? fmaf(__uint_as_float(v[c1]), p.scale_log2, -m_use) : -INFINITY;
-              const __nv_bfloat162 v2 = __floats2bfloat162_rn(exp2f(x0), exp2f(x1));
-              const float2 back = __bfloat1622float2(v2);
-              psum += back.x + back.y;
-              w4[e] = *reinterpret_cast<const uint32_t*>(&v2);
-            }
-            const int c = hh * 4 + q4;                      // 16-byte chunk within the 128-byte row
-            *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int e = 0; e < 4; ++e) {
+            const int c0 = q * 8 + 2 * e;
+            const float2 x = ffma2(make_float2(__uint_as_float(v[c0]), __uint_as_float(v[c0 + 1])), scl, nm);
+            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            sum2 = fadd2(sum2, pr);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(pr.x, pr.y);
+            w4[e] = *reinterpret_cast<const uint32_t*>(&b2);
           }
+          *reinterpret_cast<uint4*>(prow + ((q ^ (h & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
+        const float psum = sum2.x + sum2.y;
         lsum += psum;
         tc_fence_before();
         __syncwarp();
@@ -581,10 +578,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       if (!ok) break;
       tc_fence_after();
       S.red_sum[l] = lsum;
-      ok = warps_rendezvous(&S.xbar, xph, abort_flag);
+      ok = warps_rendezvous(&S.xbar[warp & 1u], xph, abort_flag);
       if (!ok) break;
       const float total = lsum + S.red_sum[l ^ 64u];
-      ok = warps_rendezvous(&S.xbar, xph, abort_flag);   // red_sum may be rewritten next unit
+      ok = warps_rendezvous(&S.xbar[warp & 1u], xph, abort_flag);   // red_sum may be rewritten next unit
       if (!ok) break;
       const float inv = total > 0.f ? 1.f / total : 0.f;
       const float lse_v = total > 0.f ? (m + log2f(total)) * kLn2 : -INFINITY;
