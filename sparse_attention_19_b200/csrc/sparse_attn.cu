@@ -63,13 +63,15 @@ constexpr int kPBufs = 2;            // P buffers (2 planes each: keys 0-63, 64-
 constexpr int kMaxIdx = 2048;        // selected positions per unit (staged in shared memory)
 constexpr int kMmaWarp = 4;           // TMEM owner + S issuer
 constexpr int kPvWarp = 5;            // P.V issuer
-// Loaders own ring slots: kKWarpsPerSlot warps fill every key chunk that lands
-// in their slot (so a warp waits only on its own slot, and the chunks of
-// different slots are issued in parallel); likewise for the value stages.
-constexpr int kKWarpsPerSlot = 2;
-constexpr int kVWarpsPerSlot = 2;
+// Loaders own ring slots, so a warp waits only on its own slots (in ring order)
+// and the stages of different slots are issued in parallel.  Key chunks: a team
+// of kKTeamWarps warps owns kKTeamSlots consecutive slots and splits each chunk's
+// 16 gathers; value stages: kVWarpsPerSlot warps per slot split its gathers.
+constexpr int kKTeamWarps = 3;
+constexpr int kKTeamSlots = 2;
+constexpr int kVWarpsPerSlot = 3;
 constexpr int kKWarp0 = 6;           // key-chunk loaders
-constexpr int kKWarps = kKStages * kKWarpsPerSlot;
+constexpr int kKWarps = kKStages / kKTeamSlots * kKTeamWarps;
 constexpr int kVWarp0 = kKWarp0 + kKWarps;   // value-stage loaders
 constexpr int kVWarps = kVStages * kVWarpsPerSlot;
 constexpr int kThreads = 32 * (kVWarp0 + kVWarps);   // 768
@@ -223,12 +225,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       // ------------------------------------------------------------------ key loaders
       // Per unit: the Q planes (plane c from warp c % kKWarps), then for each tile
       // its NC key chunks (this CTA's 64 keys x 64 columns).  Chunk kc goes to
-      // ring slot kc % kKStages; the warps that own that slot each issue their
-      // share of its 16 four-row gathers.
-      constexpr int kGroupsPerWarp = (kHalfKeys / 4) / kKWarpsPerSlot;
+      // ring slot kc % kKStages; the team that owns that slot issues its 16
+      // four-row gathers, groups g = part, part + kKTeamWarps, ...
       const int pw = (int)warp - kKWarp0;
-      const uint32_t my_slot = (uint32_t)(pw / kKWarpsPerSlot);
-      const int part = pw % kKWarpsPerSlot;
+      const uint32_t my_team = (uint32_t)(pw / kKTeamWarps);
+      const int part = pw % kKTeamWarps;
       uint32_t ucount = 0, kc = 0;
       bool ok = true;
       if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
@@ -253,7 +254,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         for (int j = U.j0; j < U.j1 && ok; ++j) {
           for (int c = 0; c < NC; ++c, ++kc) {
             const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
-            if (st != my_slot) continue;
+            if (st / kKTeamSlots != my_team) continue;
             bool w_ok = true;
             if (lane == 0) {
               w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
@@ -261,8 +262,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             }
             if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
             const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
-            if ((int)lane < kGroupsPerWarp) {
-              const int g = part * kGroupsPerWarp + (int)lane;      // 4-key group of this lane
+            const int g = part + kKTeamWarps * (int)lane;            // 4-key group of this lane
+            if (g < kHalfKeys / 4) {
               const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
               tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
                                gather_row(idx, base + 0), gather_row(idx, base + 1),
@@ -285,7 +286,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       // loaders and the softmax warps are done with the unit two back.
       // Value stages: per tile, 2 x kNpv stages of 64 keys (kh) x this CTA's kN/2
       // columns of value block h, i.e. all 128 keys of the tile across the two halves.
-      constexpr int kGroupsPerWarp = 16 * VS::kPlanes / kVWarpsPerSlot;
       const int pw = (int)warp - kVWarp0;
       const uint32_t my_slot = (uint32_t)(pw / kVWarpsPerSlot);
       const int part = pw % kVWarpsPerSlot;
@@ -344,8 +344,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
               }
               if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
               const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
-              if ((int)lane < kGroupsPerWarp) {
-                const int g = part * kGroupsPerWarp + (int)lane;
+              const int g = part + kVWarpsPerSlot * (int)lane;
+              if (g < 16 * VS::kPlanes) {
                 const int pl = g / 16, kg = g % 16;
                 const int base = (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4;
                 const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
