@@ -113,6 +113,33 @@ dsa_status dsa_sparse_attn(const dsa_attn_args *args, int B, int Lq, int Lk,
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * dsa_sparse_attn without a workspace argument.  The pages have no counterpart
+ * to this call: it is for callers that may not allocate device memory at the
+ * point of the call yet still reach the split-k path (few query rows, e.g.
+ * decode) -- a serving loop that committed all device memory to its own pool up
+ * front, or code that must not risk the implicit device synchronisation that
+ * freeing memory brings.
+ *
+ * Arguments, layouts, results and errors are those of dsa_sparse_attn.  The
+ * split-k partials (dsa_workspace_size(DSA_OP_SPARSE_ATTN, ...) bytes; 0 when
+ * B*Lq is large enough that no row is split) are kept in a fixed array of
+ * DSA_NOALLOC_SCRATCH_BYTES that is part of the library's device code, so the
+ * call allocates and frees nothing.  A call that needs more returns
+ * DSA_ERR_WORKSPACE before launching anything.  Nothing in the array has to
+ * start at zero: every partial is written before it is read.
+ * The first call on each device looks the array's address up (which may make the
+ * CUDA runtime load the library's device code); make that first call before any
+ * stream capture begins.
+ * The array is shared by all calls on a device: calls whose executions overlap
+ * (different streams, or host threads with no ordering between them) race on it
+ * and produce wrong results.  Order them, e.g. on one stream.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+dsa_status dsa_sparse_attn_noalloc(const dsa_attn_args *args, int B, int Lq, int Lk,
+                                   const int32_t *indices, int k, void *out, float *lse,
+                                   void *stream);
+
+/*
  * The whole forward pass: indexer -> top-k -> sparse attention.
  * `iargs` and `aargs` describe the same B, Lq, Lk, q_offset.
  *   indices: int32 [B, Lq, k] (as dsa_topk); out: bf16 [B, Lq, H, d_v];

@@ -19,7 +19,7 @@ import os
 import torch
 
 __all__ = [
-    "DSAError", "lib", "lib_path", "indexer_scores", "topk", "sparse_attn", "forward",
+    "DSAError", "lib", "lib_path", "indexer_scores", "topk", "sparse_attn", "sparse_attn_noalloc", "forward",
     "workspace_size", "status_string", "device_status", "selftest_wait_timeout", "version",
     "OP_TOPK", "OP_SPARSE_ATTN", "OP_FORWARD",
 ]
@@ -64,6 +64,7 @@ def lib():
         L.dsa_indexer_scores.argtypes = [ctypes.POINTER(IndexerArgs), P, P]
         L.dsa_topk.argtypes = [P, I, I, I, I, I, P, P, Z, P]
         L.dsa_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), I, I, I, P, I, P, P, P, Z, P]
+        L.dsa_sparse_attn_noalloc.argtypes = [ctypes.POINTER(AttnArgs), I, I, I, P, I, P, P, P]
         L.dsa_forward.argtypes = [ctypes.POINTER(IndexerArgs), ctypes.POINTER(AttnArgs), I, P, P, P, P, Z, P]
         L.dsa_forward_timed.argtypes = [ctypes.POINTER(IndexerArgs), ctypes.POINTER(AttnArgs), I, P, P, P, P, Z, P,
                                         ctypes.POINTER(ctypes.c_void_p)]
@@ -73,7 +74,8 @@ def lib():
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_device_status.argtypes = [I]
         L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
-        for f in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward", "dsa_forward_timed",
+        for f in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_sparse_attn_noalloc", "dsa_forward",
+                  "dsa_forward_timed",
                   "dsa_device_status",
                   "dsa_selftest_wait_timeout", "dsa_version"):
             getattr(L, f).restype = ctypes.c_int
@@ -194,6 +196,25 @@ def sparse_attn(q, kv, indices, d_v, scale, out=None, lse=None, want_lse=True, w
     workspace, nbytes = _workspace(OP_SPARSE_ATTN, B, Lq, Lk, k, H, d_v, q.device, workspace)
     _check(lib().dsa_sparse_attn(ctypes.byref(a), B, Lq, Lk, _ptr(indices), k, _ptr(out), _ptr(lse),
                                  _ptr(workspace), nbytes, _stream(stream)), "dsa_sparse_attn")
+    return out, lse
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20   # DSA_NOALLOC_SCRATCH_BYTES
+
+
+def sparse_attn_noalloc(q, kv, indices, d_v, scale, out, lse=None, stream=None):
+    """sparse_attn into caller-provided `out` (and `lse`), with no device allocation:
+    the split-k partials use the library's fixed scratch array (dsa_sparse_attn_noalloc)."""
+    a = _attn_args(q, kv, d_v, scale)
+    B, Lq, H, _ = q.shape
+    Lk = kv.shape[1]
+    k = indices.shape[-1]
+    _need(indices, torch.int32, (B, Lq, k), "indices")
+    _need(out, torch.bfloat16, (B, Lq, H, d_v), "out")
+    if lse is not None:
+        _need(lse, torch.float32, (B, Lq, H), "lse")
+    _check(lib().dsa_sparse_attn_noalloc(ctypes.byref(a), B, Lq, Lk, _ptr(indices), k, _ptr(out), _ptr(lse),
+                                         _stream(stream)), "dsa_sparse_attn_noalloc")
     return out, lse
 
 

@@ -285,6 +285,43 @@ size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_
   return 0;
 }
 
+// Split-k partials of dsa_sparse_attn_noalloc: a fixed array in this module's
+// device image, so that call allocates nothing.  Its address is looked up once
+// per device (with that device current) and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DSA_NOALLOC_SCRATCH_BYTES];
+static constexpr int kMaxDevices = 64;
+
+static dsa_status noalloc_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return DSA_OK;
+}
+
+dsa_status dsa_sparse_attn_noalloc(const dsa_attn_args* args, int B, int Lq, int Lk, const int32_t* indices,
+                                   int k, void* out, float* lse, void* stream) {
+  dsa_status s = check_attn(args, B, Lq, Lk);
+  if (s != DSA_OK) return s;
+  if (!indices || !out || !aligned16(indices) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+  if (lse && !aligned16(lse)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+  const size_t need = attn_ws_bytes(B, Lq, k, args->H, args->d_v);
+  if (need > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0 && (s = noalloc_scratch(&ws)) != DSA_OK) return s;
+  return run_attn(args, B, Lq, Lk, 0, false, indices, k, out, lse, ws, DSA_NOALLOC_SCRATCH_BYTES,
+                  static_cast<cudaStream_t>(stream));
+}
+
 dsa_status dsa_forward_timed(const dsa_indexer_args* iargs, const dsa_attn_args* aargs, int k, int32_t* indices,
                              void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream,
                              void* const* stage_events) {
