@@ -87,11 +87,24 @@ dsa_status check_attn(const dsa_attn_args* a, int B, int Lq, int Lk) {
 
 // Split-k factor for the attention: enough (row, split) units to cover the SM
 // pairs several times over; 1 for prefill-sized batches.
+// Split-k factor for the attention: each row's key tiles are spread over s units
+// (s a power of two).  Cost model in units of one tile's pipelined time on a CTA
+// pair (measured ~2.5 us): a unit costs its tiles plus about 1.8 tiles of fill,
+// drain and partial-result traffic; units run in waves over the pairs; merging
+// split partials adds about one tile.  Few rows (decode) get split, many do not.
 int attn_splits(int rows, int n_tiles) {
-  const int pairs = sm_count() / 2;
-  int s = 1;
-  while (s < n_tiles && (long long)rows * s < 4LL * pairs) s *= 2;
-  return s < n_tiles ? s : n_tiles;
+  constexpr double kUnitOverheadTiles = 1.8, kCombineTiles = 1.0;
+  const long long pairs = sm_count() / 2;
+  int best_s = 1;
+  double best = 1e300;
+  for (int s = 1; s <= n_tiles; s *= 2) {
+    const long long units = (long long)rows * s;
+    const long long waves = (units + pairs - 1) / pairs;
+    const int tiles = (n_tiles + s - 1) / s;
+    const double cost = (double)waves * (tiles + kUnitOverheadTiles) + (s > 1 ? kCombineTiles : 0.0);
+    if (cost < best) { best = cost; best_s = s; }
+  }
+  return best_s;
 }
 
 size_t attn_ws_bytes(int B, int Lq, int k, int H, int d_v) {

@@ -110,7 +110,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
     for (int s = 0; s < 8; ++s) {
       mbar_init(&S.acc_full[s], 1);
-      mbar_init(&S.acc_empty[s], kEpiWarps);
+      mbar_init(&S.acc_empty[s], N <= 64 ? kEpiWarps / 2 : kEpiWarps);
     }
     mbar_init(&S.final_bar, 1);
     mbar_init(&S.epi_bar, kEpiWarps);
@@ -201,6 +201,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // ------------------------------------------------------------ epilogue
     const uint32_t quarter = warp & 3u;              // TMEM lane quarter this warp may read
     const uint32_t half = warp >> 2;                 // which 64-column groups (even / odd)
+    // With a single 64-column group (decode: one query per sequence) the two warp
+    // halves take alternate accumulators instead of alternate groups.
+    const bool narrow = N <= 64;
     const uint32_t row = quarter * 32 + lane;        // key row within the tile
     const int et = threadIdx.x;                      // 0 .. 32 * kEpiWarps - 1
     uint32_t seq = 0, epi_phase = 0;
@@ -232,8 +235,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int s = kt * kKeysPerTile + (int)row;
         const float sk = sk_next;
         sk_next = key_scale(kt + 1);
-        for (int sb = 0; sb < p.nsub; ++sb) {
+        for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
           const uint32_t slot = seq % nslot, use = seq / nslot;
+          if (narrow && (seq & 1u) != half) continue;
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t t_base = tmem_base + ((quarter * 32u) << 16) + slot * (uint32_t)N;
@@ -241,7 +245,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           // columns.  The head sum runs as two interleaved partial sums (packed FMA).
           constexpr int QPG = (H_I >= 64) ? 1 : 64 / H_I;      // queries per 64-column group
           constexpr int HE = (H_I >= 64) ? 64 : H_I;            // heads of one query in a group
-          for (int g0 = (int)half * 64; g0 < N; g0 += 128) {
+          for (int g0 = narrow ? 0 : (int)half * 64; g0 < N; g0 += narrow ? 64 : 128) {
             uint32_t v[64];
             tmem_ld32(t_base + (uint32_t)g0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             tmem_ld32(t_base + (uint32_t)g0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
@@ -272,7 +276,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.acc_empty[slot]);
-          ++seq;
         }
       }
       if (!ok) break;

@@ -63,10 +63,12 @@ def test_noalloc_without_split_needs_no_scratch():
 
 
 def test_noalloc_rejects_calls_beyond_the_scratch_size():
-    # B = 64 single-query rows need 8-way split-k partials of ~134 MB > 64 MiB; the
-    # call must refuse on the host before touching CUDA (the pointers are never used).
+    # 160 single-query rows are split two ways (on 148 SMs): ~80 MiB of partials >
+    # 64 MiB.  The call must refuse on the host before touching CUDA (the pointers
+    # are never used).
     L = dsa.lib()
     a = dsa.AttnArgs(H=H, d_qk=D, d_v=DV, scale=SCALE, q=16, kv=16)
     fake = ctypes.c_void_p(256)
-    rc = L.dsa_sparse_attn_noalloc(ctypes.byref(a), 64, 1, 131072, fake, 2048, fake, None, None)
+    assert dsa.workspace_size(dsa.OP_SPARSE_ATTN, 160, 1, 131072, 2048, H, DV) > dsa.NOALLOC_SCRATCH_BYTES
+    rc = L.dsa_sparse_attn_noalloc(ctypes.byref(a), 160, 1, 131072, fake, 2048, fake, None, None)
     assert rc == 3 and dsa.status_string(rc).startswith("DSA_ERR_WORKSPACE")
