@@ -130,16 +130,24 @@ dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper
   }
   p.nsub = (a->Lq > p.qb) ? 2 : 1;
   p.queries_per_unit = p.qb * p.nsub;
+  if (p.queries_per_unit * a->H_I > 512) return DSA_ERR_UNSUPPORTED;   // epilogue staging limit
   p.n_qblocks = (a->Lq + p.queries_per_unit - 1) / p.queries_per_unit;
   const int sms = sm_count();
   const long long base_units = (long long)p.n_qblocks * a->B;
   const int max_tiles = (a->q_offset + a->Lq - 1) / 128 + 1;
+  // Few query blocks (decode): split each sequence's key tiles over kchunks units.
+  // Cost model in key tiles per CTA: waves of units over the SMs, each unit its
+  // tiles plus about two tiles of start-up; keep at least ~8 tiles per unit.
   int kch = 1;
   if (base_units < 4LL * sms) {
-    kch = (int)((4LL * sms + base_units - 1) / base_units);
-    const int cap = (max_tiles + 7) / 8;           // keep at least ~8 key tiles per unit
-    if (kch > cap) kch = cap;
-    if (kch < 1) kch = 1;
+    constexpr double kUnitOverheadTiles = 2.0;
+    const int cap = (max_tiles + 7) / 8;
+    double best = 1e300;
+    for (int c = 1; c <= cap; ++c) {
+      const long long waves = (base_units * c + sms - 1) / sms;
+      const double cost = (double)waves * ((double)(max_tiles + c - 1) / c + kUnitOverheadTiles);
+      if (cost < best) { best = cost; kch = c; }
+    }
   }
   p.kchunks = kch;
   p.n_units = (int)(base_units * kch);
@@ -148,6 +156,11 @@ dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper
   p.w = reinterpret_cast<const __nv_bfloat16*>(a->w);
   p.k_scale = a->k_scale;
   p.scores = scores;
+  // Decode-like calls (a small query block streaming many keys from HBM) take the
+  // key scales through a TMA-filled shared-memory ring, when the [B, Lk] fp32 array
+  // can be described to TMA (rows of a multiple of 16 bytes); prefill reads them
+  // directly (they stay in L2), one tile ahead.
+  p.scale_ring = (a->k_scale && a->Lk % 4 == 0 && p.nsub * p.qb * a->H_I <= 128) ? 1 : 0;
 
   const CUtensorMapSwizzle swz = (a->d_I == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap tq, tk;
@@ -157,8 +170,12 @@ dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper
   if (!make_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 32,
                  swz))                                     // key tiles arrive as four 32-row boxes
     return DSA_ERR_CUDA;
+  CUtensorMap ts = tk;                                     // unused unless scale_ring
+  if (p.scale_ring && !make_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a->k_scale, (uint64_t)a->B, a->Lk,
+                                 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return DSA_ERR_CUDA;
   const int grid = p.n_units < sms ? p.n_units : sms;
-  return launch_indexer(p, tq, tk, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return launch_indexer(p, tq, tk, ts, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, int k, int32_t* idx,

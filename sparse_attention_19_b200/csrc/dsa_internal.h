@@ -21,6 +21,7 @@ struct IndexerParams {
   int kchunks;            // key-tile ranges per query block (>1 splits long rows across CTAs)
   int n_units;            // n_qblocks * B * kchunks
   int fill_upper;         // write -inf for s > t (full-matrix output)
+  int scale_ring;         // key scales staged per tile by TMA (k_scale set, Lk % 4 == 0)
   const float* q_scale;   // [B, Lq] or null
   const __nv_bfloat16* w; // [B, Lq, H_I]
   const float* k_scale;   // [B, Lk] or null
@@ -28,7 +29,7 @@ struct IndexerParams {
 };
 size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages);
 cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                           int grid, cudaStream_t stream);
+                           const CUtensorMap& ts, int grid, cudaStream_t stream);
 
 // ---------------------------------------------------------------- top-k
 struct TopkParams {

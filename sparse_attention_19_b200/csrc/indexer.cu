@@ -11,8 +11,12 @@
 // axis, TMEM lane = key and the H_I columns of one query sit in that lane, so the
 // ReLU, the weighting and the head sum are a per-thread loop in the epilogue with
 // no cross-thread reduction.  Each CTA keeps NSUB query sub-blocks resident in
-// shared memory and streams key tiles through a TMA ring; two TMEM accumulators
-// let the epilogue of one sub-block overlap the MMA of the next.
+// shared memory and streams key tiles through a TMA ring; 512 / N TMEM
+// accumulators (up to 8) let the epilogue of one sub-block overlap the MMAs of the
+// next ones.  Prefill with H_I = 64 uses QB = 4 (N = 256, two accumulators, two
+// sub-blocks; fewer, larger steps measured faster than QB = 2 with four); decode
+// uses QB = 1 (N = 64) with a deeper key ring, the key scales staged through a TMA
+// ring, and the two epilogue warp halves taking alternate accumulators.
 //
 // Warp roles (416 threads): warps 0..7 epilogue (warp w reads TMEM lanes
 // 32(w%4) .. 32(w%4)+31 and every other 64-column group, starting at group w/4),
@@ -31,7 +35,7 @@ namespace dsa {
 namespace {
 
 constexpr int kKeysPerTile = 128;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, splitting the columns
 constexpr int kMmaWarp = kEpiWarps;
 constexpr int kLoaders = 4;          // TMA requests from one warp are served in order, so each
@@ -40,17 +44,23 @@ constexpr int kLoaderWarp0 = kMmaWarp + 1;
 constexpr int kThreads = 32 * (kLoaderWarp0 + kLoaders);   // 416
 static_assert(kLoaders * 32 == kKeysPerTile, "one 32-row box per loader");
 constexpr int kTmemCols = 512;
+constexpr int kScaleSlots = 16;      // key-scale ring: 128 fp32 per tile, released by the epilogue
 
 struct IndexerSmem {
   // Barriers and small per-unit data first; big tiles follow at a 1024-byte boundary.
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];         // query block buffers (two when the block is small)
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];
   uint64_t acc_full[8], acc_empty[8];     // TMEM accumulators: 512 / N of them (at most 8)
+  uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
   uint64_t final_bar;
   uint64_t epi_bar;          // rendezvous of the epilogue warps
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
+
+// Query-block buffers: two (the next unit's block loads while this one runs) when a
+// block is small, as in decode; one for the large prefill blocks.
+__host__ __device__ constexpr uint32_t query_buffers(uint32_t q_bytes) { return q_bytes <= 32768u ? 2u : 1u; }
 
 struct UnitInfo {
   int b, i0, kt0, kt1;  // batch, first query, key-tile range [kt0, kt1)
@@ -78,7 +88,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const IndexerParams& p, int u) {
 template <int H_I, int D_I, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-               const IndexerParams p) {
+               const __grid_constant__ CUtensorMap tmap_s, const IndexerParams p) {
   static_assert(D_I == 64 || D_I == 128, "d_I");
   constexpr uint32_t kRowBytes = D_I;                  // one e4m3 row
   constexpr uint32_t kLayout = (D_I == 128) ? LAYOUT_SW128 : LAYOUT_SW64;
@@ -92,18 +102,23 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   const int N = p.qb * H_I;                            // MMA N (queries x heads)
   const uint32_t nslot = min(8, kTmemCols / N);        // accumulators in flight (more when N is small)
   const int QU = p.queries_per_unit;                   // = qb * nsub
-  uint8_t* q_smem = tiles;                             // nsub * N rows
-  uint8_t* k_smem = tiles + (size_t)p.nsub * N * kRowBytes;
-  float* w_smem = reinterpret_cast<float*>(k_smem + (size_t)kStages * kKeysPerTile * kRowBytes);
-  float* sq_smem = w_smem + QU * H_I;
+  const uint32_t q_bytes = (uint32_t)(p.nsub * N) * kRowBytes;   // one query block
+  const uint32_t n_qbuf = query_buffers(q_bytes);
+  uint8_t* q_smem = tiles;                             // n_qbuf x (nsub * N rows)
+  uint8_t* k_smem = tiles + n_qbuf * (size_t)q_bytes;
+  float* sc_smem = reinterpret_cast<float*>(k_smem + (size_t)kStages * kKeysPerTile * kRowBytes);
+  float* w_smem = sc_smem + kScaleSlots * kKeysPerTile;   // 2 x QU * H_I (per unit, double-buffered)
+  float* sq_smem = w_smem + 2 * QU * H_I;                  // 2 x QU
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
   volatile uint32_t* abort_flag = &S.abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&S.q_full, 1);
-    mbar_init(&S.q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.q_full[i], 1);
+      mbar_init(&S.q_empty[i], 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.k_full[s], 1);
       mbar_init(&S.k_empty[s], 1);
@@ -111,6 +126,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     for (int s = 0; s < 8; ++s) {
       mbar_init(&S.acc_full[s], 1);
       mbar_init(&S.acc_empty[s], N <= 64 ? kEpiWarps / 2 : kEpiWarps);
+    }
+    for (int s = 0; s < kScaleSlots; ++s) {
+      mbar_init(&S.sc_full[s], 1);
+      mbar_init(&S.sc_empty[s], kEpiWarps);
     }
     mbar_init(&S.final_bar, 1);
     mbar_init(&S.epi_bar, kEpiWarps);
@@ -132,19 +151,21 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // of each key stage.
     const int pw = (int)warp - kLoaderWarp0;
     if (elect_one()) {
-      if (pw == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_k); }
-      uint32_t q_phase = 0, kstage = 0, kphase = 0;
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      if (pw == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_k); if (p.scale_ring) prefetch_tmap(&tmap_s); }
+      uint32_t ucount = 0, kstage = 0, kphase = 0, sc_use = 0;
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++ucount) {
         const UnitInfo U = decode_unit(p, u);
         if (pw == 0) {
-          if (!mbar_wait(&S.q_empty, q_phase ^ 1, abort_flag)) break;
-          mbar_arrive_expect_tx(&S.q_full, (uint32_t)(p.nsub * N) * kRowBytes);
+          // query block of this unit into buffer ucount % n_qbuf (free once the unit
+          // n_qbuf back is done)
+          const uint32_t qb_i = ucount % n_qbuf;
+          if (!mbar_wait(&S.q_empty[qb_i], ((ucount / n_qbuf) & 1u) ^ 1u, abort_flag)) break;
+          mbar_arrive_expect_tx(&S.q_full[qb_i], q_bytes);
           for (int sb = 0; sb < p.nsub; ++sb) {
             const int row = ((U.b * p.Lq) + U.i0 + sb * p.qb) * H_I;
-            tma_load_2d(q_smem + (size_t)sb * N * kRowBytes, &tmap_q, &S.q_full, 0, row);
+            tma_load_2d(q_smem + qb_i * q_bytes + (size_t)sb * N * kRowBytes, &tmap_q, &S.q_full[qb_i], 0, row);
           }
         }
-        q_phase ^= 1;
         bool ok = true;
         for (int kt = U.kt0; kt < U.kt1; ++kt) {
           if (!mbar_wait(&S.k_empty[kstage], kphase ^ 1, abort_flag)) { ok = false; break; }
@@ -152,6 +173,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           tma_load_2d(k_smem + (size_t)kstage * kKeysPerTile * kRowBytes + pw * 32 * kRowBytes, &tmap_k,
                       &S.k_full[kstage], 0, U.b * p.Lk + kt * kKeysPerTile + pw * 32);
           if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
+          if (pw == 0 && p.scale_ring) {
+            // the tile's 128 key scales (zero-filled past Lk) into the scale ring
+            const uint32_t ss = sc_use % kScaleSlots;
+            if (!mbar_wait(&S.sc_empty[ss], ((sc_use / kScaleSlots) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&S.sc_full[ss], kKeysPerTile * 4);
+            tma_load_2d(sc_smem + ss * kKeysPerTile, &tmap_s, &S.sc_full[ss], kt * kKeysPerTile, U.b);
+            ++sc_use;
+          }
         }
         if (!ok) break;
       }
@@ -160,12 +189,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       const uint32_t idesc = make_idesc(0, 0, 128, (uint32_t)N, 0, 0);  // e4m3 x e4m3 -> f32
-      uint32_t q_phase = 0, kstage = 0, kphase = 0, seq = 0;
-      const uint32_t q_base = smem_u32(q_smem), k_base = smem_u32(k_smem);
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      uint32_t ucount = 0, kstage = 0, kphase = 0, seq = 0;
+      const uint32_t k_base = smem_u32(k_smem);
+      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++ucount) {
         const UnitInfo U = decode_unit(p, u);
-        if (!mbar_wait(&S.q_full, q_phase, abort_flag)) break;
-        q_phase ^= 1;
+        const uint32_t qb_i = ucount % n_qbuf;
+        const uint32_t q_base = smem_u32(q_smem) + qb_i * q_bytes;
+        if (!mbar_wait(&S.q_full[qb_i], (ucount / n_qbuf) & 1u, abort_flag)) break;
         tc_fence_after();
         bool ok = true;
         for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
@@ -190,7 +220,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           mma_commit(&S.k_empty[kstage]);
           if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
         }
-        mma_commit(&S.q_empty);
+        mma_commit(&S.q_empty[qb_i]);
         if (!ok) break;
       }
       // Every MMA issued here completes before the TMEM is released.
@@ -206,35 +236,62 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     const bool narrow = N <= 64;
     const uint32_t row = quarter * 32 + lane;        // key row within the tile
     const int et = threadIdx.x;                      // 0 .. 32 * kEpiWarps - 1
-    uint32_t seq = 0, epi_phase = 0;
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    uint32_t seq = 0, epi_phase = 0, sc_use = 0, ucount = 0;
+    // A unit's weights and query scales sit in smem buffer (unit ordinal % 2).  The
+    // next unit's values are read into registers when a unit starts and stored when
+    // it ends, so their memory latency hides under the unit's work.
+    constexpr int kWPerThread = 512 / (32 * kEpiWarps);       // QU * H_I <= 512 (host-checked)
+    float wr[kWPerThread], sr = 0.f;
+    auto fetch = [&](const UnitInfo& V) {
+#pragma unroll
+      for (int e = 0; e < kWPerThread; ++e) {
+        const int x = et + e * 32 * kEpiWarps, qq = x / H_I, i = V.i0 + qq;
+        wr[e] = (x < QU * H_I && i < p.Lq)
+                    ? __bfloat162float(p.w[((size_t)V.b * p.Lq + i) * H_I + x % H_I]) : 0.f;
+      }
+      const int i = V.i0 + et;
+      sr = (et < QU && i < p.Lq) ? (p.q_scale ? p.q_scale[(size_t)V.b * p.Lq + i] : 1.f) : 0.f;
+    };
+    auto store = [&](uint32_t buf) {
+#pragma unroll
+      for (int e = 0; e < kWPerThread; ++e) {
+        const int x = et + e * 32 * kEpiWarps;
+        if (x < QU * H_I) w_smem[buf * QU * H_I + x] = wr[e];
+      }
+      if (et < QU) sq_smem[buf * QU + et] = sr;
+    };
+    if ((int)blockIdx.x < p.n_units) {
+      fetch(decode_unit(p, blockIdx.x));
+      store(0);
+    }
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++ucount) {
       const UnitInfo U = decode_unit(p, u);
-      if (!warps_rendezvous(&S.epi_bar, epi_phase, abort_flag)) break;   // previous unit done with w/sq
-      for (int x = et; x < QU * H_I; x += 32 * kEpiWarps) {
-        const int qq = x / H_I, j = x % H_I;
-        const int i = U.i0 + qq;
-        float wv = 0.f;
-        if (i < p.Lq) wv = __bfloat162float(p.w[((size_t)U.b * p.Lq + i) * H_I + j]);
-        w_smem[x] = wv;
-      }
-      for (int x = et; x < QU; x += 32 * kEpiWarps) {
-        const int i = U.i0 + x;
-        sq_smem[x] = (i < p.Lq) ? (p.q_scale ? p.q_scale[(size_t)U.b * p.Lq + i] : 1.f) : 0.f;
-      }
+      // this unit's buffer is complete and the other one is no longer read
       if (!warps_rendezvous(&S.epi_bar, epi_phase, abort_flag)) break;
+      const bool has_next = u + (int)gridDim.x < p.n_units;
+      if (has_next) fetch(decode_unit(p, u + gridDim.x));
+      const float* wbuf = w_smem + (ucount & 1u) * QU * H_I;
+      const float* sqbuf = sq_smem + (ucount & 1u) * QU;
       bool ok = true;
-      // The key scale of the next tile is loaded one iteration ahead, so its
-      // memory latency overlaps the current tile's epilogue.
+      // Key scales: from the TMA-filled ring when staged (scale_ring), else loaded
+      // one tile ahead, so their memory latency overlaps the current tile's epilogue.
       auto key_scale = [&](int kt) -> float {
         const int s = kt * kKeysPerTile + (int)row;
         if (kt >= U.kt1 || s >= p.Lk) return 0.f;
         return p.k_scale ? __ldg(p.k_scale + (size_t)U.b * p.Lk + s) : 1.f;
       };
-      float sk_next = key_scale(U.kt0);
+      float sk_next = p.scale_ring ? 0.f : key_scale(U.kt0);
       for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
         const int s = kt * kKeysPerTile + (int)row;
-        const float sk = sk_next;
-        sk_next = key_scale(kt + 1);
+        float sk;
+        const uint32_t ss = sc_use % kScaleSlots;
+        if (p.scale_ring) {
+          if (!mbar_wait_warp(&S.sc_full[ss], (sc_use / kScaleSlots) & 1u, abort_flag)) { ok = false; break; }
+          sk = sc_smem[ss * kKeysPerTile + row];
+        } else {
+          sk = sk_next;
+          sk_next = key_scale(kt + 1);
+        }
         for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
           const uint32_t slot = seq % nslot, use = seq / nslot;
           if (narrow && (seq & 1u) != half) continue;
@@ -253,7 +310,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 #pragma unroll
             for (int a = 0; a < QPG; ++a) {
               const int qi = g0 / H_I + a;                    // query within the sub-block
-              const float2* wq = reinterpret_cast<const float2*>(w_smem + (size_t)(sb * p.qb + qi) * H_I);
+              const float2* wq = reinterpret_cast<const float2*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
               float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
               for (int e = 0; e < HE; e += 2)
@@ -267,7 +324,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                 const int t = p.q_offset + i;
                 float* dst = p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s;
                 if (s <= t)
-                  __stcs(dst, acc * sq_smem[qq] * sk);
+                  __stcs(dst, acc * sqbuf[qq] * sk);
                 else if (p.fill_upper)
                   __stcs(dst, -INFINITY);
               }
@@ -276,6 +333,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.acc_empty[slot]);
+        }
+        if (p.scale_ring) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.sc_empty[ss]);
+          ++sc_use;
         }
       }
       if (!ok) break;
@@ -292,6 +354,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           }
         }
       }
+      if (has_next) store((ucount + 1) & 1u);
     }
   }
 
@@ -305,13 +368,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 
 template <int H_I, int D_I, int kStages>
 cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& ts,
                              int grid, cudaStream_t stream) {
   const size_t smem = indexer_smem_bytes(p.nsub * p.qb * H_I, D_I, p.queries_per_unit * H_I,
                                          p.queries_per_unit, kStages);
   auto kern = indexer_kernel<H_I, D_I, kStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(tq, tk, p);
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, ts, p);
   return cudaGetLastError();
 }
 
@@ -319,21 +383,23 @@ cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, cons
 
 size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages) {
   size_t b = sizeof(IndexerSmem) + 1024;                       // barriers + alignment slack
-  b += (size_t)q_rows * d_I;                                   // resident query block
+  b += query_buffers((uint32_t)(q_rows * d_I)) * (size_t)q_rows * d_I;   // query block buffers
   b += (size_t)stages * kKeysPerTile * d_I;                    // key ring
-  b += (size_t)(w_floats + sq_floats) * sizeof(float);
+  b += (size_t)kScaleSlots * kKeysPerTile * sizeof(float);      // key-scale ring
+  b += 2 * (size_t)(w_floats + sq_floats) * sizeof(float);     // weights / query scales, double-buffered
   // At least ~116 KB so that one CTA (and its 512 TMEM columns) owns each SM.
   return b < 118784 ? 118784 : b;
 }
 
 cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                           const CUtensorMap& ts,
                            int grid, cudaStream_t stream) {
   // A small resident query block (decode) leaves room for a deeper key ring.
   const bool deep = p.nsub * p.qb * p.H_I <= 128;
   if (p.H_I == 64 && p.d_I == 128)
-    return deep ? launch_indexer_t<64, 128, 8>(p, tq, tk, grid, stream)
-                : launch_indexer_t<64, 128, 4>(p, tq, tk, grid, stream);
-  if (p.H_I == 4 && p.d_I == 64) return launch_indexer_t<4, 64, 4>(p, tq, tk, grid, stream);
+    return deep ? launch_indexer_t<64, 128, 12>(p, tq, tk, ts, grid, stream)
+                : launch_indexer_t<64, 128, 4>(p, tq, tk, ts, grid, stream);
+  if (p.H_I == 4 && p.d_I == 64) return launch_indexer_t<4, 64, 4>(p, tq, tk, ts, grid, stream);
   return cudaErrorInvalidValue;
 }
 
