@@ -189,6 +189,15 @@ dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, in
   p.cache_cap = nmax <= kTopkCacheMax ? (int)round_up((size_t)nmax, 4) : 0;
   p.bit_words = (int)round_up((size_t)(nmax + 31) / 32, 4);
   p.cand_cap = 4096;
+  // Too few rows to fill the GPU (decode) and long ones: a cluster of CTAs per row,
+  // each CTA owning a 32-aligned segment of it.
+  const long long rows = (long long)B * Lq;
+  if (rows * kTopkClusterCtas <= 2LL * sm_count() && nmax > 16384) {
+    const long long seg = ((nmax + kTopkClusterCtas - 1) / kTopkClusterCtas + 31) / 32 * 32;
+    p.cluster = 1;
+    p.cache_cap = 0;
+    p.bit_words = (int)round_up((size_t)(seg / 32), 4);
+  }
   p.vec4 = (aligned16(scores) && Lk % 4 == 0) ? 1 : 0;
   return launch_topk(p, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

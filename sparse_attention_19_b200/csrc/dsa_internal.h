@@ -40,8 +40,11 @@ struct TopkParams {
   int bit_words;          // 32-bit words of each position bitmap (>= ceil(row length / 32)); multiple of 4
   int cand_cap;           // candidate (key, position) pairs held in shared memory
   int vec4;               // rows start 16-byte aligned (scores aligned, Lk % 4 == 0): 16-byte loads
+  int cluster;            // each row spread over a cluster of kTopkClusterCtas CTAs (few long rows);
+                          // bit_words then covers one CTA's segment
 };
-size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap);
+constexpr int kTopkClusterCtas = 4;
+size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap, bool cluster);
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- sparse attention

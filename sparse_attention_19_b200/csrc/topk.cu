@@ -50,12 +50,17 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// 16-byte multiple, so the arrays that follow it in dynamic shared memory stay aligned.
-struct alignas(16) TopkShared {
-  uint32_t hist[kBins];
+// Block-wide scratch for scans and reductions.
+struct ScanScratch {
   uint32_t warp_tot[kWarps];
   uint32_t warp_a[kWarps], warp_b[kWarps];
   uint32_t bin, above, ncand;
+};
+
+// 16-byte multiple, so the arrays that follow it in dynamic shared memory stay aligned.
+struct alignas(16) TopkShared {
+  uint32_t hist[kBins];
+  ScanScratch x;
 };
 
 // Block-wide inclusive scan of one value per thread (thread order).
@@ -86,22 +91,22 @@ __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* w
 }
 
 // Find the bin b (searching from the top) where the running count from above first
-// reaches `need`; records b and the count strictly above it.
-__device__ void find_bin(TopkShared& sh, uint32_t need) {
+// reaches `need`; records b and the count strictly above it in x.bin / x.above.
+__device__ void find_bin(const uint32_t* hist, ScanScratch& x, uint32_t need) {
   constexpr int per = kBins / kThreads;            // bins per thread
   const int lo = threadIdx.x * per;
   uint32_t mine = 0;
 #pragma unroll
-  for (int x = 0; x < per; ++x) mine += sh.hist[lo + x];
+  for (int i = 0; i < per; ++i) mine += hist[lo + i];
   uint32_t total;
-  const uint32_t incl = block_inclusive_scan(mine, sh.warp_tot, total);
+  const uint32_t incl = block_inclusive_scan(mine, x.warp_tot, total);
   uint32_t acc = total - incl;                      // count in bins above this thread's range
 #pragma unroll
-  for (int x = per - 1; x >= 0; --x) {
-    const uint32_t c = sh.hist[lo + x];
+  for (int i = per - 1; i >= 0; --i) {
+    const uint32_t c = hist[lo + i];
     if (acc < need && acc + c >= need) {
-      sh.bin = (uint32_t)(lo + x);
-      sh.above = acc;
+      x.bin = (uint32_t)(lo + i);
+      x.above = acc;
     }
     acc += c;
   }
@@ -114,7 +119,7 @@ __device__ __forceinline__ int bin_shift(uint32_t range) {
 }
 
 // Block-wide min and max (every thread receives both).
-__device__ __forceinline__ void block_min_max(TopkShared& sh, uint32_t& mn, uint32_t& mx) {
+__device__ __forceinline__ void block_min_max(ScanScratch& x, uint32_t& mn, uint32_t& mx) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -122,15 +127,15 @@ __device__ __forceinline__ void block_min_max(TopkShared& sh, uint32_t& mn, uint
     mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
   __syncthreads();                                  // earlier readers of warp_a / warp_b are done
-  if (lane == 0) { sh.warp_a[warp] = mn; sh.warp_b[warp] = mx; }
+  if (lane == 0) { x.warp_a[warp] = mn; x.warp_b[warp] = mx; }
   __syncthreads();
-  mn = sh.warp_a[0];
-  mx = sh.warp_b[0];
-  for (int w = 1; w < kWarps; ++w) { mn = min(mn, sh.warp_a[w]); mx = max(mx, sh.warp_b[w]); }
+  mn = x.warp_a[0];
+  mx = x.warp_b[0];
+  for (int w = 1; w < kWarps; ++w) { mn = min(mn, x.warp_a[w]); mx = max(mx, x.warp_b[w]); }
 }
 
-__device__ __forceinline__ void clear_hist(TopkShared& sh) {
-  for (int x = threadIdx.x; x < kBins; x += kThreads) sh.hist[x] = 0u;
+__device__ __forceinline__ void clear_hist(uint32_t* hist) {
+  for (int i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0u;
   __syncthreads();
 }
 
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
     smin = min(smin, key);
     smax = max(smax, key);
   }
-  block_min_max(sh, smin, smax);
+  block_min_max(sh.x, smin, smax);
 
   // ---- 2. histogram over the sampled range (outliers clamped into the end bins)
   const uint32_t lo = smin;
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
   auto bin_of = [lo, shift](uint32_t key) -> uint32_t {
     return key < lo ? 0u : min((uint32_t)(kBins - 1), (key - lo) >> shift);
   };
-  clear_hist(sh);
+  clear_hist(sh.hist);
   if (p.vec4) {
     // 16-byte loads (rows start 16-byte aligned): four scores per thread per step.
     const float4* src4 = reinterpret_cast<const float4*>(src);
@@ -235,20 +240,20 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
   }
   __syncthreads();
   uint32_t need = (uint32_t)k;                       // n > k, so m = k
-  find_bin(sh, need);
-  const uint32_t b = sh.bin;
-  need -= sh.above;
+  find_bin(sh.hist, sh.x, need);
+  const uint32_t b = sh.x.bin;
+  need -= sh.x.above;
   const uint32_t cnt_b = sh.hist[b];
 
   // ---- 3. bins above b are selected; bin b becomes the candidate list
-  if (threadIdx.x == 0) sh.ncand = 0u;
+  if (threadIdx.x == 0) sh.x.ncand = 0u;
   __syncthreads();
   row_pass(n, key_at, [&](int s, bool valid, uint32_t key) {
     const uint32_t d = bin_of(key);
     const uint32_t gbal = __ballot_sync(0xffffffffu, valid && d > b);
     if (lane == 0) { gt_bits[s >> 5] = gbal; eq_bits[s >> 5] = 0u; }
     if (valid && d == b) {
-      const uint32_t pos = atomicAdd(&sh.ncand, 1u);
+      const uint32_t pos = atomicAdd(&sh.x.ncand, 1u);
       if (pos < (uint32_t)p.cand_cap) cand[pos] = make_uint2(key, (uint32_t)s);
     }
   });
@@ -264,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
       cmin = min(cmin, cand[x].x);
       cmax = max(cmax, cand[x].x);
     }
-    block_min_max(sh, cmin, cmax);
+    block_min_max(sh.x, cmin, cmax);
     wlo = cmin;
     whi = cmax;
   } else {
@@ -275,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
   for (;;) {
     const int wsh = bin_shift(whi - wlo);
     const uint32_t l0 = wlo, h0 = whi;
-    clear_hist(sh);
+    clear_hist(sh.hist);
     if (fits) {
       for (int x = threadIdx.x; x < (int)cnt_b; x += kThreads) {
         const uint32_t key = cand[x].x;
@@ -287,9 +292,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
       });
     }
     __syncthreads();
-    find_bin(sh, need);
-    const uint32_t bw = sh.bin;
-    need -= sh.above;
+    find_bin(sh.hist, sh.x, need);
+    const uint32_t bw = sh.x.bin;
+    need -= sh.x.above;
     if (wsh == 0) { thr = wlo + bw; break; }
     wlo = l0 + (bw << wsh);
     const unsigned long long top = (unsigned long long)wlo + (1ull << wsh) - 1ull;
@@ -323,10 +328,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
     cg += __shfl_xor_sync(0xffffffffu, cg, o);
     ce += __shfl_xor_sync(0xffffffffu, ce, o);
   }
-  if (lane == 0) { sh.warp_a[warp] = cg; sh.warp_b[warp] = ce; }
+  if (lane == 0) { sh.x.warp_a[warp] = cg; sh.x.warp_b[warp] = ce; }
   __syncthreads();
   uint32_t g = 0, e = 0;
-  for (int w = 0; w < warp; ++w) { g += sh.warp_a[w]; e += sh.warp_b[w]; }
+  for (int w = 0; w < warp; ++w) { g += sh.x.warp_a[w]; e += sh.x.warp_b[w]; }
   for (int w0 = w_begin; w0 < w_end; w0 += 32) {
     const int w = w0 + lane;
     const uint32_t gw = (w < w_end) ? gt_bits[w] : 0u;
@@ -361,18 +366,255 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
   }
 }
 
+// ------------------------------------------------------------------ few long rows
+// The same selection with each row spread over a cluster of kClusterCtas CTAs
+// (used when there are too few rows to fill the GPU, as in decode).  CTA r owns the
+// 32-aligned segment [s0, s1) of the row.  Every CTA draws the same sample, so all
+// agree on the first histogram's range; histograms are summed over the cluster
+// through distributed shared memory, so every CTA finds the same bins and the same
+// threshold; each CTA marks its own segment's bitmaps and candidates, and writes
+// its selected positions after those of the lower-ranked CTAs.
+constexpr int kClusterCtas = kTopkClusterCtas;
+
+struct alignas(16) TopkClusterShared {
+  uint32_t hist[kBins];        // this CTA's histogram
+  uint32_t tot[kBins];         // the cluster's
+  ScanScratch x;
+  uint32_t pub_a, pub_b;       // values this CTA publishes to the cluster
+  uint32_t pad[2];
+};
+
+// tot = sum over the cluster's CTAs of hist.
+__device__ void cluster_sum_hist(TopkClusterShared& sh) {
+  cluster_sync();                                   // every CTA's hist is complete
+  const uint32_t base = smem_u32(sh.hist);
+  for (int i = threadIdx.x; i < kBins; i += kThreads) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int c = 0; c < kClusterCtas; ++c) t += ld_shared_cluster_u32(mapa_shared(base + 4u * i, c));
+    sh.tot[i] = t;
+  }
+  cluster_sync();                                   // no CTA rewrites hist while others read it
+}
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads, 2)
+topk_cluster_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TopkClusterShared& sh = *reinterpret_cast<TopkClusterShared*>(smem_raw);
+  uint32_t* gt_bits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkClusterShared));   // segment words
+  uint32_t* eq_bits = gt_bits + p.bit_words;
+  uint2* cand = reinterpret_cast<uint2*>(eq_bits + p.bit_words);
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t r = cluster_ctarank();
+  const int row = blockIdx.x / kClusterCtas;        // b * Lq + i
+  const int i = row % p.Lq;
+  const long long t = (long long)p.q_offset + i;
+  const int n = (int)((t + 1 < p.Lk) ? t + 1 : p.Lk);
+  const int k = p.k;
+  int32_t* out = p.indices + (size_t)row * k;
+  const float* src = p.scores + (size_t)row * p.Lk;
+
+  if (n <= k) {                                     // the whole cluster leaves together
+    if (r == 0)
+      for (int x = threadIdx.x; x < k; x += kThreads) out[x] = (x < n) ? x : -1;
+    return;
+  }
+  const int seg = ((n + kClusterCtas - 1) / kClusterCtas + 31) / 32 * 32;
+  const int s0 = min(n, (int)r * seg), s1 = min(n, s0 + seg);
+  auto load_key = [&](int s) -> uint32_t { return score_key(__ldg(src + s)); };
+  // row passes over this CTA's segment: positions s0 + (0 .. s1 - s0)
+  auto seg_key = [&](int s) -> uint32_t { return load_key(s0 + s); };
+
+  // ---- 1. sampled key range (the same in every CTA)
+  const int ns = n < kSample ? n : kSample;
+  uint32_t smin = 0xffffffffu, smax = 0u;
+  for (int j = threadIdx.x; j < ns; j += kThreads) {
+    const uint32_t key = load_key((int)(((long long)j * n) / ns));
+    smin = min(smin, key);
+    smax = max(smax, key);
+  }
+  block_min_max(sh.x, smin, smax);
+  const uint32_t lo = smin;
+  const int shift = bin_shift(smax - smin);
+  auto bin_of = [lo, shift](uint32_t key) -> uint32_t {
+    return key < lo ? 0u : min((uint32_t)(kBins - 1), (key - lo) >> shift);
+  };
+
+  // ---- 2. segment histogram, summed over the cluster
+  clear_hist(sh.hist);
+  row_pass(s1 - s0, seg_key, [&](int, bool valid, uint32_t key) {
+    if (valid) atomicAdd(&sh.hist[bin_of(key)], 1u);
+  });
+  __syncthreads();
+  cluster_sum_hist(sh);
+  uint32_t need = (uint32_t)k;
+  find_bin(sh.tot, sh.x, need);
+  const uint32_t b = sh.x.bin;
+  need -= sh.x.above;
+  const uint32_t cnt_b = sh.tot[b];
+
+  // ---- 3. this segment's bins above b into the bitmap; its bin-b elements as candidates
+  if (threadIdx.x == 0) sh.x.ncand = 0u;
+  __syncthreads();
+  row_pass(s1 - s0, seg_key, [&](int s, bool valid, uint32_t key) {
+    const uint32_t d = bin_of(key);
+    const uint32_t gbal = __ballot_sync(0xffffffffu, valid && d > b);
+    if (lane == 0) { gt_bits[s >> 5] = gbal; eq_bits[s >> 5] = 0u; }
+    if (valid && d == b) {
+      const uint32_t pos = atomicAdd(&sh.x.ncand, 1u);
+      if (pos < (uint32_t)p.cand_cap) cand[pos] = make_uint2(key, (uint32_t)s);
+    }
+  });
+  __syncthreads();
+  const bool fits = cnt_b <= (uint32_t)p.cand_cap;  // then every CTA's share fits as well
+  const int own = (int)sh.x.ncand;
+
+  // Exact threshold, refined over the window [wlo, whi] with cluster-summed histograms
+  // of the candidates (or of the segments when the candidates do not fit).
+  uint32_t wlo, whi;
+  if (fits) {
+    uint32_t cmin = 0xffffffffu, cmax = 0u;
+    for (int x = threadIdx.x; x < own; x += kThreads) {
+      cmin = min(cmin, cand[x].x);
+      cmax = max(cmax, cand[x].x);
+    }
+    block_min_max(sh.x, cmin, cmax);
+    if (threadIdx.x == 0) { sh.pub_a = cmin; sh.pub_b = cmax; }
+    cluster_sync();
+    wlo = 0xffffffffu;
+    whi = 0u;
+#pragma unroll
+    for (int c = 0; c < kClusterCtas; ++c) {
+      wlo = min(wlo, ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c)));
+      whi = max(whi, ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_b), c)));
+    }
+    cluster_sync();
+  } else {
+    wlo = (b == 0) ? 0u : lo + (b << shift);
+    whi = (b == (uint32_t)(kBins - 1)) ? 0xffffffffu : lo + (((b + 1) << shift) - 1u);
+  }
+  uint32_t thr;
+  for (;;) {
+    const int wsh = bin_shift(whi - wlo);
+    const uint32_t l0 = wlo, h0 = whi;
+    clear_hist(sh.hist);
+    if (fits) {
+      for (int x = threadIdx.x; x < own; x += kThreads) {
+        const uint32_t key = cand[x].x;
+        if (key >= l0 && key <= h0) atomicAdd(&sh.hist[(key - l0) >> wsh], 1u);
+      }
+    } else {
+      row_pass(s1 - s0, seg_key, [&](int, bool valid, uint32_t key) {
+        if (valid && key >= l0 && key <= h0) atomicAdd(&sh.hist[(key - l0) >> wsh], 1u);
+      });
+    }
+    __syncthreads();
+    cluster_sum_hist(sh);
+    find_bin(sh.tot, sh.x, need);
+    const uint32_t bw = sh.x.bin;
+    need -= sh.x.above;
+    if (wsh == 0) { thr = wlo + bw; break; }
+    wlo = l0 + (bw << wsh);
+    const unsigned long long top = (unsigned long long)wlo + (1ull << wsh) - 1ull;
+    whi = top < (unsigned long long)h0 ? (uint32_t)top : h0;
+  }
+  if (fits) {
+    for (int x = threadIdx.x; x < own; x += kThreads) {
+      const uint2 c = cand[x];
+      if (c.x > thr) atomicOr(&gt_bits[c.y >> 5], 1u << (c.y & 31u));
+      else if (c.x == thr) atomicOr(&eq_bits[c.y >> 5], 1u << (c.y & 31u));
+    }
+  } else {
+    row_pass(s1 - s0, seg_key, [&](int s, bool valid, uint32_t key) {
+      const uint32_t gbal = __ballot_sync(0xffffffffu, valid && key > thr);
+      const uint32_t ebal = __ballot_sync(0xffffffffu, valid && key == thr);
+      if (lane == 0) { gt_bits[s >> 5] = gbal; eq_bits[s >> 5] = ebal; }
+    });
+  }
+  __syncthreads();
+
+  // ---- 4. ordered output: offsets from the lower-ranked CTAs, then this segment
+  const uint32_t eq_take = need;
+  const int W = (s1 - s0 + 31) >> 5;
+  const int wpw = (W + kWarps - 1) / kWarps;         // bitmap words per warp
+  const int w_begin = warp * wpw, w_end = min(W, w_begin + wpw);
+  uint32_t cg = 0, ce = 0;
+  for (int w = w_begin + lane; w < w_end; w += 32) { cg += __popc(gt_bits[w]); ce += __popc(eq_bits[w]); }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    cg += __shfl_xor_sync(0xffffffffu, cg, o);
+    ce += __shfl_xor_sync(0xffffffffu, ce, o);
+  }
+  if (lane == 0) { sh.x.warp_a[warp] = cg; sh.x.warp_b[warp] = ce; }
+  __syncthreads();
+  uint32_t g = 0, e = 0, seg_g = 0, seg_e = 0;
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) { g += sh.x.warp_a[w]; e += sh.x.warp_b[w]; }
+    seg_g += sh.x.warp_a[w];
+    seg_e += sh.x.warp_b[w];
+  }
+  if (threadIdx.x == 0) { sh.pub_a = seg_g; sh.pub_b = seg_e; }
+  cluster_sync();
+  for (uint32_t c = 0; c < r; ++c) {
+    g += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c));
+    e += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_b), c));
+  }
+  cluster_sync();                                   // peers' shared memory is no longer read
+  for (int w0 = w_begin; w0 < w_end; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t gw = (w < w_end) ? gt_bits[w] : 0u;
+    const uint32_t ew = (w < w_end) ? eq_bits[w] : 0u;
+    const uint32_t tg = __popc(gw), te = __popc(ew);
+    uint32_t pg = tg, pe = te;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t yg = __shfl_up_sync(0xffffffffu, pg, o);
+      const uint32_t ye = __shfl_up_sync(0xffffffffu, pe, o);
+      if (lane >= o) { pg += yg; pe += ye; }
+    }
+    const uint32_t sum_g = __shfl_sync(0xffffffffu, pg, 31), sum_e = __shfl_sync(0xffffffffu, pe, 31);
+    uint32_t gg = g + pg - tg, ee = e + pe - te;
+    uint32_t sel = gw | ew;
+    while (sel) {
+      const int bit = __ffs(sel) - 1;
+      sel &= sel - 1u;
+      const int s = s0 + w * 32 + bit;
+      if ((gw >> bit) & 1u) {
+        const uint32_t pos = gg + min(ee, eq_take);
+        if (pos < (uint32_t)k) out[pos] = s;
+        ++gg;
+      } else {
+        if (ee < eq_take && gg + ee < (uint32_t)k) out[gg + ee] = s;
+        ++ee;
+      }
+    }
+    g += sum_g;
+    e += sum_e;
+  }
+}
+
 }  // namespace
 
-size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap) {
+size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap, bool cluster) {
   static_assert(sizeof(TopkShared) % 16 == 0, "arrays that follow must stay 16-byte aligned");
+  static_assert(sizeof(TopkClusterShared) % 16 == 0, "arrays that follow must stay 16-byte aligned");
+  if (cluster) return sizeof(TopkClusterShared) + 2 * (size_t)bit_words * 4 + (size_t)cand_cap * 8;
   return sizeof(TopkShared) + ((size_t)cache_cap + 2 * (size_t)bit_words) * 4 + (size_t)cand_cap * 8;
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream) {
-  const size_t smem = topk_smem_bytes(p.cache_cap, p.bit_words, p.cand_cap);
+  const size_t smem = topk_smem_bytes(p.cache_cap, p.bit_words, p.cand_cap, p.cluster != 0);
+  const int rows = p.B * p.Lq;
+  if (p.cluster) {
+    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (rows == 0) return cudaSuccess;
+    topk_cluster_kernel<<<rows * kClusterCtas, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int rows = p.B * p.Lq;
   if (rows == 0) return cudaSuccess;
   topk_kernel<<<rows, kThreads, smem, stream>>>(p);
   return cudaGetLastError();

@@ -139,6 +139,20 @@ def test_topk_boundary_bin_larger_than_candidate_buffer():
     _topk_case(s.to(DEV), 32998, 2048)
 
 
+def test_topk_few_long_rows_spread_over_a_cluster():
+    # Three rows of 131072 scores (fewer rows than SMs): each row is spread over a
+    # cluster of CTAs.  Row 0 random; row 1 has 100000 equal scores at the threshold
+    # spanning every CTA's segment (candidate overflow, ties to smaller positions);
+    # row 2 rounded scores with +-0.
+    g = torch.Generator().manual_seed(13)
+    Lk = 131072
+    s = torch.randn(1, 3, Lk, generator=g)
+    s[0, 1, 20000:120000] = 3.0
+    s[0, 2] = torch.round(s[0, 2] * 4) / 4
+    s[0, 2, 60000:70000:2] = -0.0
+    _topk_case(s.to(DEV), Lk - 3, 2048)
+
+
 # ------------------------------------------------------------------ sparse attention
 
 def _attn_case(B, Lq, Lk, k, H, D, Dv, idx_np, seed, q_offset_for_oracle=0):
