@@ -298,35 +298,68 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t t_base = tmem_base + ((quarter * 32u) << 16) + slot * (uint32_t)N;
-          // 64 columns per TMEM round trip (two loads, one wait); each query owns H_I
-          // columns.  The head sum runs as two interleaved partial sums (packed FMA).
-          constexpr int QPG = (H_I >= 64) ? 1 : 64 / H_I;      // queries per 64-column group
-          constexpr int HE = (H_I >= 64) ? 64 : H_I;            // heads of one query in a group
-          for (int g0 = narrow ? 0 : (int)half * 64; g0 < N; g0 += narrow ? 64 : 128) {
-            uint32_t v[64];
-            tmem_ld32(t_base + (uint32_t)g0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-            tmem_ld32(t_base + (uint32_t)g0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          // One query's score for this lane's key: ReLU, weighting and head sum over its
+          // H_I columns (two interleaved partial sums, packed FMA), then the scales and
+          // the causal mask.
+          auto finish = [&](int qi, float acc) {
+            const int qq = sb * p.qb + qi;
+            const int i = U.i0 + qq;
+            if (i < p.Lq && s < p.Lk) {
+              const int t = p.q_offset + i;
+              float* dst = p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s;
+              if (s <= t)
+                __stcs(dst, acc * sqbuf[qq] * sk);
+              else if (p.fill_upper)
+                __stcs(dst, -INFINITY);
+            }
+          };
+          auto relu_dot = [&](const uint32_t* v, const float4* wq, int n, float2 acc2) -> float2 {
+            float2 acc_b = make_float2(0.f, 0.f);   // second chain: independent FMAs in flight
+#pragma unroll
+            for (int e = 0; e < n; e += 4) {
+              const float4 w4 = wq[e / 4];       // weights as 16-byte loads
+              acc2 = ffma2(make_float2(fmaxf(__uint_as_float(v[e]), 0.f), fmaxf(__uint_as_float(v[e + 1]), 0.f)),
+                           make_float2(w4.x, w4.y), acc2);
+              acc_b = ffma2(make_float2(fmaxf(__uint_as_float(v[e + 2]), 0.f), fmaxf(__uint_as_float(v[e + 3]), 0.f)),
+                            make_float2(w4.z, w4.w), acc_b);
+            }
+            return fadd2(acc2, acc_b);
+          };
+          const int g_first = narrow ? 0 : (int)half * 64, g_step = narrow ? 64 : 128;
+          if constexpr (H_I == 64) {
+            // This warp's 64-column groups (one query each) are read in 32-column parts
+            // through two register buffers: the next part's TMEM load is in flight
+            // while the current part is reduced.
+            const int n_parts = 2 * ((N - g_first + g_step - 1) / g_step);
+            auto col = [&](int pp) { return (uint32_t)(g_first + (pp >> 1) * g_step + (pp & 1) * 32); };
+            uint32_t va[32], vb[32];
+            tmem_ld32(t_base + col(0), va);
             tmem_ld_wait();
+            for (int pp = 0; pp < n_parts; pp += 2) {
+              tmem_ld32(t_base + col(pp + 1), vb);
+              const int qi = (int)col(pp) / 64;                  // query within the sub-block
+              const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
+              float2 acc2 = relu_dot(va, wq, 32, make_float2(0.f, 0.f));
+              tmem_ld_wait();
+              if (pp + 2 < n_parts) tmem_ld32(t_base + col(pp + 2), va);
+              acc2 = relu_dot(vb, wq + 8, 32, acc2);
+              finish(qi, acc2.x + acc2.y);
+              if (pp + 2 < n_parts) tmem_ld_wait();
+            }
+          } else {
+            // Small H_I: each 64-column group holds 64 / H_I queries.
+            constexpr int QPG = 64 / H_I;
+            for (int g0 = g_first; g0 < N; g0 += g_step) {
+              uint32_t v[64];
+              tmem_ld32(t_base + (uint32_t)g0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+              tmem_ld32(t_base + (uint32_t)g0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+              tmem_ld_wait();
 #pragma unroll
-            for (int a = 0; a < QPG; ++a) {
-              const int qi = g0 / H_I + a;                    // query within the sub-block
-              const float2* wq = reinterpret_cast<const float2*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
-              float2 acc2 = make_float2(0.f, 0.f);
-#pragma unroll
-              for (int e = 0; e < HE; e += 2)
-                acc2 = ffma2(make_float2(fmaxf(__uint_as_float(v[a * HE + e]), 0.f),
-                                         fmaxf(__uint_as_float(v[a * HE + e + 1]), 0.f)),
-                             wq[e / 2], acc2);
-              const float acc = acc2.x + acc2.y;
-              const int qq = sb * p.qb + qi;
-              const int i = U.i0 + qq;
-              if (i < p.Lq && s < p.Lk) {
-                const int t = p.q_offset + i;
-                float* dst = p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s;
-                if (s <= t)
-                  __stcs(dst, acc * sqbuf[qq] * sk);
-                else if (p.fill_upper)
-                  __stcs(dst, -INFINITY);
+              for (int a = 0; a < QPG; ++a) {
+                const int qi = g0 / H_I + a;
+                const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
+                const float2 acc2 = relu_dot(v + a * H_I, wq, H_I, make_float2(0.f, 0.f));
+                finish(qi, acc2.x + acc2.y);
               }
             }
           }
