@@ -18,9 +18,10 @@
 // uses QB = 1 (N = 64) with a deeper key ring, the key scales staged through a TMA
 // ring, and the two epilogue warp halves taking alternate accumulators.
 //
-// Warp roles (416 threads): warps 0..7 epilogue (warp w reads TMEM lanes
-// 32(w%4) .. 32(w%4)+31 and every other 64-column group, starting at group w/4),
-// warp 8 TMEM owner + MMA issuer, warps 9..12 TMA loaders.
+// Warp roles (768 threads): warps 0..15 epilogue (warp w reads TMEM lanes
+// 32(w%4) .. 32(w%4)+31 of the 64-column groups w/4, w/4 + 4, ...), warp 16 TMEM
+// owner + MMA issuer, warps 20..23 TMA loaders.  Four epilogue warps per SM
+// sub-partition hide the latency of the per-element ReLU / weighting / head sum.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -36,12 +37,18 @@ namespace {
 
 constexpr int kKeysPerTile = 128;
 constexpr int kMaxStages = 12;
-constexpr int kEpiWarps = 8;         // two per TMEM lane quarter, splitting the columns
-constexpr int kMmaWarp = kEpiWarps;
+constexpr int kEpiWarps = 16;        // four per TMEM lane quarter ("quads" of four warps)
+constexpr int kQuads = kEpiWarps / 4;
+constexpr int kMmaWarp = kEpiWarps;  // warps 16-19: MMA issuer (+ three idle warps of its warpgroup)
 constexpr int kLoaders = 4;          // TMA requests from one warp are served in order, so each
                                      // key tile is loaded as four 32-row boxes from four warps
-constexpr int kLoaderWarp0 = kMmaWarp + 1;
-constexpr int kThreads = 32 * (kLoaderWarp0 + kLoaders);   // 416
+constexpr int kLoaderWarp0 = kMmaWarp + 4;
+constexpr int kThreads = 32 * (kLoaderWarp0 + kLoaders);   // 768
+// Register split: 80 per thread at launch (6 warps per SM sub-partition); the four
+// epilogue warpgroups take 88, the MMA / loader warpgroups keep 64.
+constexpr uint32_t kRegsLaunch = 80, kRegsEpi = 88, kRegsOther = 64;
+static_assert(32 * kEpiWarps * kRegsEpi + (kThreads - 32 * kEpiWarps) * kRegsOther <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 static_assert(kLoaders * 32 == kKeysPerTile, "one 32-row box per loader");
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 16;      // key-scale ring: 128 fp32 per tile, released by the epilogue
@@ -125,7 +132,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
     for (int s = 0; s < 8; ++s) {
       mbar_init(&S.acc_full[s], 1);
-      mbar_init(&S.acc_empty[s], N <= 64 ? kEpiWarps / 2 : kEpiWarps);
+      mbar_init(&S.acc_empty[s], N <= 64 ? 4 : kEpiWarps);
     }
     for (int s = 0; s < kScaleSlots; ++s) {
       mbar_init(&S.sc_full[s], 1);
@@ -145,6 +152,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
 
+  if (warp >= (uint32_t)kEpiWarps) {
+    regs_decrease<kRegsOther>();
   if (warp >= kLoaderWarp0) {
     // ------------------------------------------------------------ TMA loaders
     // Loader 0 also loads the query block; every loader fills rows [32*pw, 32*pw+32)
@@ -227,12 +236,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       mma_commit(&S.final_bar);
       mbar_wait(&S.final_bar, 0, nullptr);
     }
+  }
   } else {
+    regs_increase<kRegsEpi>();
     // ------------------------------------------------------------ epilogue
     const uint32_t quarter = warp & 3u;              // TMEM lane quarter this warp may read
-    const uint32_t half = warp >> 2;                 // which 64-column groups (even / odd)
-    // With a single 64-column group (decode: one query per sequence) the two warp
-    // halves take alternate accumulators instead of alternate groups.
+    const uint32_t quad = warp >> 2;                 // which 64-column groups: quad, quad + 4, ...
+    // With a single 64-column group (decode: one query per sequence) the quads take
+    // accumulators in turn instead of column groups.
     const bool narrow = N <= 64;
     const uint32_t row = quarter * 32 + lane;        // key row within the tile
     const int et = threadIdx.x;                      // 0 .. 32 * kEpiWarps - 1
@@ -294,7 +305,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
         for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
           const uint32_t slot = seq % nslot, use = seq / nslot;
-          if (narrow && (seq & 1u) != half) continue;
+          if (narrow && seq % kQuads != quad) continue;
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t t_base = tmem_base + ((quarter * 32u) << 16) + slot * (uint32_t)N;
@@ -313,8 +324,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                 __stcs(dst, -INFINITY);
             }
           };
+          // sum_j w_j ReLU(x_j): packed FMAs, two independent chains.
           auto relu_dot = [&](const uint32_t* v, const float4* wq, int n, float2 acc2) -> float2 {
-            float2 acc_b = make_float2(0.f, 0.f);   // second chain: independent FMAs in flight
+            float2 acc_b = make_float2(0.f, 0.f);
 #pragma unroll
             for (int e = 0; e < n; e += 4) {
               const float4 w4 = wq[e / 4];       // weights as 16-byte loads
@@ -325,41 +337,37 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             }
             return fadd2(acc2, acc_b);
           };
-          const int g_first = narrow ? 0 : (int)half * 64, g_step = narrow ? 64 : 128;
+          const int g_first = narrow ? 0 : (int)quad * 64, g_step = narrow ? 64 : 64 * kQuads;
           if constexpr (H_I == 64) {
-            // This warp's 64-column groups (one query each) are read in 32-column parts
-            // through two register buffers: the next part's TMEM load is in flight
-            // while the current part is reduced.
-            const int n_parts = 2 * ((N - g_first + g_step - 1) / g_step);
-            auto col = [&](int pp) { return (uint32_t)(g_first + (pp >> 1) * g_step + (pp & 1) * 32); };
-            uint32_t va[32], vb[32];
-            tmem_ld32(t_base + col(0), va);
-            tmem_ld_wait();
-            for (int pp = 0; pp < n_parts; pp += 2) {
-              tmem_ld32(t_base + col(pp + 1), vb);
-              const int qi = (int)col(pp) / 64;                  // query within the sub-block
+            // This warp's 64-column groups (one query each), 32 columns per TMEM load.
+            for (int g0 = g_first; g0 < N; g0 += g_step) {
+              const int qi = g0 / 64;                            // query within the sub-block
               const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
-              float2 acc2 = relu_dot(va, wq, 32, make_float2(0.f, 0.f));
+              uint32_t v[32];
+              tmem_ld32(t_base + (uint32_t)g0, v);
               tmem_ld_wait();
-              if (pp + 2 < n_parts) tmem_ld32(t_base + col(pp + 2), va);
-              acc2 = relu_dot(vb, wq + 8, 32, acc2);
+              float2 acc2 = relu_dot(v, wq, 32, make_float2(0.f, 0.f));
+              tmem_ld32(t_base + (uint32_t)g0 + 32, v);
+              tmem_ld_wait();
+              acc2 = relu_dot(v, wq + 8, 32, acc2);
               finish(qi, acc2.x + acc2.y);
-              if (pp + 2 < n_parts) tmem_ld_wait();
             }
           } else {
-            // Small H_I: each 64-column group holds 64 / H_I queries.
-            constexpr int QPG = 64 / H_I;
+            // Small H_I: each 64-column group holds 64 / H_I queries, 32 / H_I per load.
+            constexpr int QPL = 32 / H_I;
             for (int g0 = g_first; g0 < N; g0 += g_step) {
-              uint32_t v[64];
-              tmem_ld32(t_base + (uint32_t)g0, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-              tmem_ld32(t_base + (uint32_t)g0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-              tmem_ld_wait();
 #pragma unroll
-              for (int a = 0; a < QPG; ++a) {
-                const int qi = g0 / H_I + a;
-                const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
-                const float2 acc2 = relu_dot(v + a * H_I, wq, H_I, make_float2(0.f, 0.f));
-                finish(qi, acc2.x + acc2.y);
+              for (int part = 0; part < 2; ++part) {
+                uint32_t v[32];
+                tmem_ld32(t_base + (uint32_t)(g0 + part * 32), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int a = 0; a < QPL; ++a) {
+                  const int qi = (g0 + part * 32) / H_I + a;
+                  const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
+                  const float2 acc2 = relu_dot(v + a * H_I, wq, H_I, make_float2(0.f, 0.f));
+                  finish(qi, acc2.x + acc2.y);
+                }
               }
             }
           }
@@ -380,7 +388,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         for (int kt = U.kt1; kt < nt_all; ++kt) {
           const int s = kt * kKeysPerTile + (int)row;
           if (s >= p.Lk) continue;
-          for (int qq = (int)half; qq < QU; qq += 2) {
+          for (int qq = (int)quad; qq < QU; qq += kQuads) {
             const int i = U.i0 + qq;
             if (i < p.Lq)
               __stcs(p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s, -INFINITY);
@@ -408,6 +416,12 @@ cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, cons
   auto kern = indexer_kernel<H_I, D_I, kStages>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  // The register split must fit in what the CTA launches with, or the increase
+  // would wait forever: refuse to launch a build where it does not.
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if ((uint32_t)fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, ts, p);
   return cudaGetLastError();
 }
