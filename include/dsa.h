@@ -142,6 +142,10 @@ dsa_status dsa_sparse_attn_noalloc(const dsa_attn_args *args, int B, int Lq, int
 /*
  * The whole forward pass: indexer -> top-k -> sparse attention.
  * `iargs` and `aargs` describe the same B, Lq, Lk, q_offset.
+ * Short sequences (q_offset + Lq <= k): every row selects all of its positions
+ * 0..t whatever the indexer says, so the pass is dense causal MLA attention; the
+ * indexer is not run (the short-sequence mode of the DSA report's "Стоимость"
+ * section, where attention falls back to the masked dense form).
  *   indices: int32 [B, Lq, k] (as dsa_topk); out: bf16 [B, Lq, H, d_v];
  *   lse: fp32 [B, Lq, H] or NULL.
  * The workspace holds the indexer scores of the call ([B, Lq, Lk] fp32) and

@@ -382,8 +382,15 @@ dsa_status dsa_forward_timed(const dsa_indexer_args* iargs, const dsa_attn_args*
   char* attn_ws = static_cast<char*>(workspace) + score_bytes;
   const size_t attn_ws_size = workspace_bytes - score_bytes;
   if (!mark(0)) return DSA_ERR_CUDA;
-  s = run_indexer(iargs, scores, false, st);
-  if (s != DSA_OK) return s;
+  // Short sequences: when every row's causal range fits in k (q_offset + Lq <= k),
+  // every position is selected whatever the scores, and the pass is dense causal
+  // attention.  The indexer is skipped; the top-k step writes the index lists
+  // 0..t without reading scores.
+  const bool dense = (long long)iargs->q_offset + iargs->Lq <= k;
+  if (!dense) {
+    s = run_indexer(iargs, scores, false, st);
+    if (s != DSA_OK) return s;
+  }
   if (!mark(1)) return DSA_ERR_CUDA;
   s = run_topk(scores, iargs->B, iargs->Lq, iargs->Lk, iargs->q_offset, k, indices, st);
   if (s != DSA_OK) return s;

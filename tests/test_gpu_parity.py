@@ -243,6 +243,28 @@ def test_forward_tiny_all_rows_exact_indices():
     _check_forward_rows(inp, wl, idx, out, lse, np.arange(wl.Lq), wl.Lq, 0, exact_idx=True)
 
 
+def test_forward_short_sequence_is_dense_causal_attention():
+    # q_offset + Lq <= k: every row selects all of 0..t, the pass is dense causal
+    # attention and the indexer is not consulted -- garbage indexer inputs give the
+    # same result.
+    wl = WORKLOADS["prefill_8k"].with_(Lq=1024, Lk=1024)
+    inp = make_inputs(wl, DEV, 3)
+    idx, out, lse = _forward(inp, wl)
+    n = np.arange(wl.Lq) + 1
+    want = np.where(np.arange(wl.k)[None, :] < n[:, None], np.arange(wl.k)[None, :], -1)
+    assert np.array_equal(idx.reshape(-1, wl.k).cpu().numpy(), want)
+    rows = np.r_[0, 1, 63, 500, 1022, 1023]
+    keys = oracle.keys_from_inputs(inp)
+    r = oracle.rows_from_inputs(inp, rows, wl.Lq, 0)
+    oo, ol = oracle.sparse_attn(r["row_b"], r["q"], keys["kv"], want[rows].astype(np.int32), wl.scale, wl.Dv)
+    P.check_attention(out.reshape(-1, wl.H, wl.Dv)[torch.as_tensor(rows, device=DEV)],
+                      lse.reshape(-1, wl.H)[torch.as_tensor(rows, device=DEV)], oo, ol)
+    garbage = dict(inp)
+    garbage["q_I"] = torch.randint(0, 255, inp["q_I"].shape, dtype=inp["q_I"].dtype, device=DEV)
+    idx2, out2, lse2 = _forward(garbage, wl)
+    assert torch.equal(idx2, idx) and torch.equal(out2, out)
+
+
 def test_forward_prefill_8k_sampled_rows():
     wl = WORKLOADS["prefill_8k"]
     inp = make_inputs(wl, DEV, 0)
