@@ -55,6 +55,8 @@ def _load():
             lib.oracle_topk.argtypes = [P, i64, i32, P, i32, P]
             lib.oracle_sparse_attn.restype = i32
             lib.oracle_sparse_attn.argtypes = [i64, P, i32, i32, i32, f64, P, i32, P, P, i32, P, P]
+            lib.oracle_indexer_kl.restype = i32
+            lib.oracle_indexer_kl.argtypes = [i64, P, i32, i32, f64, P, i32, P, P, i32, P, P, P]
             lib.oracle_dsa_forward.restype = i32
             lib.oracle_dsa_forward.argtypes = [i64, P, P, i32, i32, P, P, P, i32, P, P,
                                                i32, i32, i32, f64, P, P, i32, P, P, P, P]
@@ -142,6 +144,37 @@ def sparse_attn(row_b, q, kv, indices, scale, Dv):
     if rc != 0:
         raise ValueError(f"oracle_sparse_attn failed ({rc})")
     return out, lse
+
+
+def indexer_kl(row_b, q, kv, indices, scores, scale):
+    """The indexer's training loss over the selected positions, per query row.
+
+    DeepSeek-V3.2 technical-report summary, section "Как учили индексатор": the
+    target p is the main attention's probabilities summed over the heads and
+    L1-normalised; the loss is D_KL(p || softmax(I)) over the selected positions
+    (the sparse stage).  q: uint16 bf16 bits [n, H, D]; kv: uint16 [B, Lk, D];
+    indices: int32 [n, k] (negative = padding); scores: float [n, Lk], row r's
+    indexer scores.  Returns (target f64 [n, k] aligned with the index slots,
+    kl f64 [n]).
+    """
+    qa, pq = _c(q, np.uint16)
+    n, H, D = qa.shape
+    kva, pkv = _c(kv, np.uint16)
+    Lk = kva.shape[1]
+    ia, pi = _c(indices, np.int32)
+    k = ia.shape[1]
+    sa, ps = _c(scores, np.float64)
+    if sa.shape != (n, Lk):
+        raise ValueError("scores must be [n, Lk]")
+    rb, prb = _c(row_b, np.int64)
+    target = np.empty((n, k), dtype=np.float64)
+    kl = np.empty(n, dtype=np.float64)
+    rc = _load().oracle_indexer_kl(n, prb, H, D, float(scale), pq, Lk, pkv, pi, k, ps,
+                                   target.ctypes.data_as(ctypes.c_void_p),
+                                   kl.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise ValueError(f"oracle_indexer_kl failed ({rc})")
+    return target, kl
 
 
 def dsa_forward(row_b, row_t, q_I, q_scale, w, k_I, k_scale, q, kv, k, scale, Dv,

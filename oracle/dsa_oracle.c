@@ -14,7 +14,12 @@
  *     computed in FP8 (third bullet under that equation);
  *   - subsection "Отбор и основное внимание", equation for u_t:
  *       u_t = Attn(h_t, { c_s : I[t,s] in Top-k(I[t,:]) }),  k = 2048,
- *     with MLA in MQA mode: one latent KV row c_s serves every query head.
+ *     with MLA in MQA mode: one latent KV row c_s serves every query head;
+ *   - section "Как учили индексатор" (the indexer's training loss): the target
+ *     p[t,:] is the main attention's probabilities summed over all heads and
+ *     L1-normalised along the keys; the loss is the KL divergence between p[t,:]
+ *     and the softmax of the indexer's scores, over the selected positions only
+ *     in the sparse stage (item 2 of that section).
  *
  * Readings where the page is silent (each one is listed with its reason in the
  * repository's design notes):
@@ -22,7 +27,10 @@
  *   - FP8 values are dequantised with one positive fp32 scale per token;
  *   - top-k ties go to the smaller position; -0.0 equals +0.0;
  *   - a row with t+1 <= k selects every position 0..t;
- *   - V is the leading Dv columns of the latent KV row; K is the whole row.
+ *   - V is the leading Dv columns of the latent KV row; K is the whole row;
+ *   - the loss is D_KL(p || softmax(I)) (target first), both distributions over
+ *     the row's valid selected positions; 0 log 0 = 0; a row with no valid
+ *     selected position has loss 0 and target 0.
  *
  * Every sum is a plain loop in fp64, in index order.  OpenMP only splits the
  * independent query rows across host threads.
@@ -252,6 +260,104 @@ int oracle_sparse_attn(int64_t n_rows, const int64_t *row_b, int H, int D, int D
                 o[v] /= l;
             if (lse) lse[r * H + h] = zmax + log(l);
         }
+        free(z);
+    }
+    return bad ? 2 : 0;
+}
+
+/* ---- the indexer's training loss (forward) ---------------------------------- */
+
+/*
+ * For each of n_rows query rows (row r of batch row_b[r], query q[r], selection
+ * indices[r], the row's indexer scores scores[r][0..Lk)):
+ *   per head h, the attention probabilities a_h[x] over the valid selected
+ *   positions (the same softmax as oracle_sparse_attn);
+ *   P[x] = sum_h a_h[x];  target[r][x] = P[x] / sum_x P[x]    (0 on invalid slots);
+ *   lq[x] = log softmax over the valid selected x of scores[r][indices[r][x]];
+ *   kl[r] = sum over valid x with target > 0 of target[x] * (log target[x] - lq[x]).
+ * Slot x of target corresponds to slot x of indices.  Negative indices are
+ * padding; an index >= Lk is an error (returns 2).
+ */
+int oracle_indexer_kl(int64_t n_rows, const int64_t *row_b, int H, int D, double scale,
+                      const uint16_t *q, int Lk, const uint16_t *kv,
+                      const int32_t *indices, int k, const double *scores,
+                      double *target, double *kl)
+{
+    if (n_rows < 0 || H <= 0 || D <= 0 || k <= 0 || Lk <= 0)
+        return 1;
+    int bad = 0;
+    int64_t r;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (r = 0; r < n_rows; ++r) {
+        int64_t b = row_b[r];
+        const int32_t *idx = indices + r * (int64_t)k;
+        const double *I = scores + r * (int64_t)Lk;
+        double *tg = target + r * (int64_t)k;
+        double *z = (double *)malloc(sizeof(double) * (size_t)k);
+        int nvalid = 0;
+        for (int x = 0; x < k; ++x) {
+            tg[x] = 0.0;
+            if (idx[x] >= Lk) bad = 1;
+            else if (idx[x] >= 0) ++nvalid;
+        }
+        kl[r] = 0.0;
+        if (nvalid == 0) {
+            free(z);
+            continue;
+        }
+        /* Main attention, head by head, accumulated into tg[] (= P before normalising). */
+        for (int h = 0; h < H; ++h) {
+            const uint16_t *qh = q + (r * H + h) * (int64_t)D;
+            double zmax = -INFINITY;
+            for (int x = 0; x < k; ++x) {
+                int32_t s = idx[x];
+                if (s < 0 || s >= Lk) continue;
+                const uint16_t *kr = kv + (b * Lk + s) * (int64_t)D;
+                double dot = 0.0;
+                for (int d = 0; d < D; ++d)
+                    dot += oracle_bf16_value(qh[d]) * oracle_bf16_value(kr[d]);
+                z[x] = scale * dot;
+                if (z[x] > zmax) zmax = z[x];
+            }
+            double l = 0.0;
+            for (int x = 0; x < k; ++x) {
+                int32_t s = idx[x];
+                if (s < 0 || s >= Lk) continue;
+                l += exp(z[x] - zmax);
+            }
+            for (int x = 0; x < k; ++x) {
+                int32_t s = idx[x];
+                if (s < 0 || s >= Lk) continue;
+                tg[x] += exp(z[x] - zmax) / l;
+            }
+        }
+        /* L1 normalisation of the head sum. */
+        double total = 0.0;
+        for (int x = 0; x < k; ++x)
+            total += tg[x];
+        for (int x = 0; x < k; ++x)
+            tg[x] /= total;
+        /* log softmax of the indexer scores over the same positions. */
+        double imax = -INFINITY;
+        for (int x = 0; x < k; ++x) {
+            int32_t s = idx[x];
+            if (s < 0 || s >= Lk) continue;
+            if (I[s] > imax) imax = I[s];
+        }
+        double li = 0.0;
+        for (int x = 0; x < k; ++x) {
+            int32_t s = idx[x];
+            if (s < 0 || s >= Lk) continue;
+            li += exp(I[s] - imax);
+        }
+        double log_norm = imax + log(li);
+        double acc = 0.0;
+        for (int x = 0; x < k; ++x) {
+            int32_t s = idx[x];
+            if (s < 0 || s >= Lk || tg[x] <= 0.0) continue;
+            acc += tg[x] * (log(tg[x]) - (I[s] - log_norm));
+        }
+        kl[r] = acc;
         free(z);
     }
     return bad ? 2 : 0;

@@ -385,3 +385,117 @@ def test_work_ratio_matches_the_page_exercise():
     assert wl.selected_pairs == 128000 * 2048 - 2048 * 2047 // 2
     assert wl.selected_pairs / 128000 ** 2 == pytest.approx(0.016, rel=0.01)
     assert wl.causal_pairs == 128000 * 128001 // 2
+
+
+# ---------------------------------------------------------------- indexer training loss
+# Section "Как учили индексатор": target p = main-attention probabilities summed over
+# the heads, L1-normalised; loss = D_KL(p || softmax(I)) over the selected positions.
+
+def _num(x):
+    return math.log(2.0) if x == "ln2" else float(x)
+
+
+def test_kl_hand_worked_case():
+    g = json.load(open(os.path.join(GOLD, "indexer_kl_hand.json")))
+    q = bf16_bits(g["q"])
+    kv = bf16_bits(g["kv"])
+    scores = np.array([[_num(v) for v in row] for row in g["scores"]])
+    target, kl = oracle.indexer_kl(np.array(g["row_b"]), q, kv, np.array(g["indices"], np.int32), scores,
+                                   _num(g["scale"]))
+    want_t = np.array([[a / b for a, b in row] for row in g["target_fractions"]])
+    np.testing.assert_allclose(target, want_t, rtol=1e-14, atol=1e-16)
+    want_kl = [sum((pn / pd) * math.log((pn / pd) / (qn / qd)) for pn, pd, qn, qd in row)
+               for row in g["kl_terms_p_q"]]
+    np.testing.assert_allclose(kl, want_kl, rtol=1e-13)
+    # the reversed divergence D_KL(softmax(I) || p) differs, so the direction is pinned
+    rev = sum((qn / qd) * math.log((qn / qd) / (pn / pd)) for pn, pd, qn, qd in g["kl_terms_p_q"][0])
+    assert abs(kl[0] - rev) > 1e-3
+
+
+def _kl_case(rng, n=3, H=4, D=64, Lk=40, k=16, B=2):
+    q_t, q_b = _bf16_rand((n, H, D), rng)
+    kv_t, kv_b = _bf16_rand((B, Lk, D), rng)
+    row_b = rng.integers(0, B, size=n)
+    idx = np.full((n, k), -1, np.int32)
+    for r in range(n):
+        m = int(rng.integers(1, k + 1))
+        slots = rng.choice(k, size=m, replace=False)
+        idx[r, slots] = rng.choice(Lk, size=m, replace=False)
+    scores = rng.normal(size=(n, Lk)) * 3.0
+    return q_t, q_b, kv_t, kv_b, row_b, idx, scores
+
+
+def test_kl_matches_library_softmax_and_entropy():
+    # target through torch.softmax per head; KL through scipy.stats.entropy(p, q),
+    # which computes sum p log(p/q) for two distributions.
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    rng = np.random.default_rng(40)
+    q_t, q_b, kv_t, kv_b, row_b, idx, scores = _kl_case(rng)
+    scale = 1.0 / math.sqrt(192.0)
+    target, kl = oracle.indexer_kl(row_b, q_b, kv_b, idx, scores, scale)
+    for r in range(len(row_b)):
+        valid = idx[r] >= 0
+        pos = idx[r][valid]
+        keys = kv_t[row_b[r]].double()[torch.as_tensor(pos)]                 # [m, D]
+        logits = torch.einsum("hd,md->hm", q_t[r].double(), keys) * scale
+        p = torch.softmax(logits, dim=-1).sum(0)
+        p = (p / p.sum()).numpy()
+        np.testing.assert_allclose(target[r][valid], p, rtol=1e-12, atol=1e-15)
+        assert np.all(target[r][~valid] == 0.0)
+        qdist = softmax(scores[r][pos])
+        assert kl[r] == pytest.approx(entropy(p, qdist), rel=1e-11, abs=1e-14)
+
+
+def test_kl_is_zero_exactly_when_the_indexer_reproduces_the_target():
+    rng = np.random.default_rng(41)
+    q_t, q_b, kv_t, kv_b, row_b, idx, scores = _kl_case(rng)
+    target, kl = oracle.indexer_kl(row_b, q_b, kv_b, idx, scores, 0.2)
+    nv = (idx >= 0).sum(1)
+    assert np.all(kl[nv > 1] > 0.0) and np.all(kl[nv == 1] == 0.0)      # Gibbs: > 0 unless equal
+    matched = scores.copy()
+    for r in range(len(row_b)):
+        valid = idx[r] >= 0
+        matched[r, idx[r][valid]] = np.log(target[r][valid]) + 3.7        # softmax(log p + c) = p
+    _, kl0 = oracle.indexer_kl(row_b, q_b, kv_b, idx, matched, 0.2)
+    np.testing.assert_allclose(kl0, 0.0, atol=1e-13)
+
+
+def test_kl_ignores_score_shifts_and_everything_unselected():
+    rng = np.random.default_rng(42)
+    q_t, q_b, kv_t, kv_b, row_b, idx, scores = _kl_case(rng)
+    t0, kl0 = oracle.indexer_kl(row_b, q_b, kv_b, idx, scores, 0.3)
+    _, kl1 = oracle.indexer_kl(row_b, q_b, kv_b, idx, scores - 11.5, 0.3)
+    np.testing.assert_allclose(kl1, kl0, rtol=1e-12)
+    sc2, kv2 = scores.copy(), kv_b.copy()
+    for r in range(len(row_b)):
+        unsel = np.setdiff1d(np.arange(scores.shape[1]), idx[r][idx[r] >= 0])
+        sc2[r, unsel] = rng.normal(size=len(unsel)) * 50.0
+    used = {(int(row_b[r]), int(s)) for r in range(len(row_b)) for s in idx[r] if s >= 0}
+    for b in range(kv_b.shape[0]):
+        for s in range(kv_b.shape[1]):
+            if (b, s) not in used:
+                kv2[b, s] = bf16_bits(rng.normal(size=kv_b.shape[2]) * 4.0)
+    t2, kl2 = oracle.indexer_kl(row_b, q_b, kv2, idx, sc2, 0.3)
+    np.testing.assert_array_equal(t2, t0)
+    np.testing.assert_array_equal(kl2, kl0)
+
+
+def test_kl_follows_slot_order_and_padding():
+    rng = np.random.default_rng(43)
+    q_t, q_b, kv_t, kv_b, row_b, idx, scores = _kl_case(rng, n=1)
+    t0, kl0 = oracle.indexer_kl(row_b, q_b, kv_b, idx, scores, 0.25)
+    perm = rng.permutation(idx.shape[1])
+    t1, kl1 = oracle.indexer_kl(row_b, q_b, kv_b, idx[:, perm], scores, 0.25)
+    np.testing.assert_allclose(t1, t0[:, perm], rtol=1e-13, atol=1e-16)
+    assert kl1[0] == pytest.approx(kl0[0], rel=1e-12)
+
+
+def test_kl_degenerate_selections():
+    rng = np.random.default_rng(44)
+    q_t, q_b, kv_t, kv_b, row_b, idx, scores = _kl_case(rng, n=2)
+    one = np.full_like(idx, -1)
+    one[0, 5] = 7                                                        # a single selected position
+    target, kl = oracle.indexer_kl(row_b, q_b, kv_b, one, scores, 0.25)
+    assert target[0, 5] == 1.0 and np.count_nonzero(target[0]) == 1 and kl[0] == 0.0
+    assert np.all(target[1] == 0.0) and kl[1] == 0.0                      # nothing selected
