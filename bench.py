@@ -13,7 +13,8 @@ workload, with inputs resident in HBM.  Prints ONE JSON line (rank 0).
              CUDA-event duration, against the measured peak in MEASURED_PEAKS.json
   stages     the same for every kernel of the step
   workloads  the other workloads the metric names (decode at 128K context; 128K prefill
-             in 4096-query chunks), measured the same way with fewer steps
+             in 4096-query chunks), measured the same way with fewer steps; and the
+             indexer's training loss (forward) on the headline step's own outputs
   cpu_baseline  the fp64 oracle on a bounded sample of the headline workload, host cores
 
 Multi-GPU (torchrun): every rank runs its own independent problem (weak scaling, no
@@ -57,6 +58,7 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the supplementary workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--loss", action="store_true", help="time the indexer loss even with --no-extra")
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
 
@@ -360,6 +362,50 @@ def measure_e2e(wl, runner, steps, warmup, world):
     return ms, bi, bo
 
 
+def time_indexer_kl(wl, runner, steps, warmup, world, peaks, peak_src):
+    """The indexer's training loss (forward) on the step's own outputs: the scores the
+    forward left in its workspace, its selection and its lse.  One launch per call."""
+    dsa = runner.dsa
+    if wl.chunk or len(runner.chunks) != 1 or wl.q_offset + wl.Lq <= wl.k:
+        return None                       # needs the scores of a single indexer call
+    _, qs = runner.chunks[0]
+    B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
+    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B, Lq, Lk)
+    target = torch.empty(B, Lq, k, dtype=torch.float32, device=runner.device)
+    kl = torch.empty(B, Lq, dtype=torch.float32, device=runner.device)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        dsa.indexer_kl_loss(qs["q"], runner.keys["kv"], runner.indices, runner.lse, scores, wl.Dv, wl.scale,
+                            target=target, kl=kl, stream=stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        call()
+    e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world)
+    tot = runner.totals()
+    # S = q . c over every (selected pair, head); gathered latent rows as the bytes
+    flops = 2.0 * tot["selected_pairs"] * wl.H * wl.D
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"workload": wl.name, "value": tot["rows"] * world / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": steps, "warmup": warmup, "gpu_launches": steps,
+            "roofline": {"kernel": "indexer_kl_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "per_launch_algorithmic": flops,
+                         "peak_source": f"{peak_src} burst bf16 (MEASURED_PEAKS.json)",
+                         "gathered_gb": tot["selected_pairs"] * wl.D * 2 / 1e9,
+                         "traffic": traffic_from_profiles("indexer_kl_kernel", wl.name)},
+            "kl_mean": float(kl.mean())}
+
+
 # ------------------------------------------------------------------------------------ CPU oracle
 
 def oracle_sample(wl, inp_dev_or_host, n_rows, seed=0):
@@ -495,6 +541,11 @@ def main():
         line["e2e"] = {"value": tokens / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
                        "d2h_bytes_per_step": bo, "ms_per_step": e_ms}
     extra = {}
+    if not args.no_extra or args.loss:
+        kl_line = time_indexer_kl(wl, runner, max(3, args.steps // 2), args.warmup, world, peaks, peak_src)
+        if kl_line is not None:
+            extra["indexer_kl_loss"] = kl_line
+        line["workloads"] = extra
     if not args.no_extra:
         for name in ("decode_128k", "prefill_128k"):
             if name == wl.name:

@@ -166,6 +166,29 @@ dsa_status dsa_forward_timed(const dsa_indexer_args *iargs, const dsa_attn_args 
                              void *workspace, size_t workspace_bytes, void *stream,
                              void *const *stage_events);
 
+/*
+ * Forward of the lightning indexer's training loss (section "Как учили
+ * индексатор": the indexer learns the main attention's distribution through a
+ * KL divergence; in the sparse stage only over the selected positions).
+ * For query row (b,i) with the valid selected positions S (indices entries in
+ * [0, Lk); others are padding):
+ *   a_h[s]  = exp(scale * q[b,i,h,:] . kv[b,s,:] - lse[b,i,h])   (the attention
+ *             probabilities of head h, as dsa_sparse_attn computes them);
+ *   p[s]    = sum_h a_h[s] / sum_{s' in S} sum_h a_h[s']          (target, L1-normalised);
+ *   kl[b,i] = sum_{s in S} p[s] * (log p[s] - log softmax_S(scores[b,i,:])[s]).
+ *   args, B, Lq, Lk, indices, k: as dsa_sparse_attn (same shapes and limits);
+ *   lse:    fp32 [B, Lq, H], the natural-log log-sum-exp that dsa_sparse_attn
+ *           returned for the same q, kv and indices;
+ *   scores: fp32 [B, Lq, Lk], the indexer scores (dsa_indexer_scores layout);
+ *           only the selected entries are read, and they must be finite;
+ *   target: fp32 [B, Lq, k] or NULL: p at each index slot, 0 on padding slots;
+ *   kl:     fp32 [B, Lq]: the per-row loss, 0 for a row with no valid entry.
+ * The reduction over rows (sum or mean) is left to the caller.  No workspace.
+ */
+dsa_status dsa_indexer_kl_loss(const dsa_attn_args *args, int B, int Lq, int Lk,
+                               const int32_t *indices, int k, const float *lse,
+                               const float *scores, float *target, float *kl, void *stream);
+
 /* Bytes of device workspace the entry point `op` needs for these sizes (0 = none). */
 size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_v);
 

@@ -20,6 +20,7 @@ import torch
 
 __all__ = [
     "DSAError", "lib", "lib_path", "indexer_scores", "topk", "sparse_attn", "sparse_attn_noalloc", "forward",
+    "indexer_kl_loss",
     "workspace_size", "status_string", "device_status", "selftest_wait_timeout", "version",
     "OP_TOPK", "OP_SPARSE_ATTN", "OP_FORWARD",
 ]
@@ -68,6 +69,7 @@ def lib():
         L.dsa_forward.argtypes = [ctypes.POINTER(IndexerArgs), ctypes.POINTER(AttnArgs), I, P, P, P, P, Z, P]
         L.dsa_forward_timed.argtypes = [ctypes.POINTER(IndexerArgs), ctypes.POINTER(AttnArgs), I, P, P, P, P, Z, P,
                                         ctypes.POINTER(ctypes.c_void_p)]
+        L.dsa_indexer_kl_loss.argtypes = [ctypes.POINTER(AttnArgs), I, I, I, P, I, P, P, P, P, P]
         L.dsa_workspace_size.argtypes = [I, I, I, I, I, I, I]
         L.dsa_workspace_size.restype = ctypes.c_size_t
         L.dsa_status_string.argtypes = [I]
@@ -75,7 +77,7 @@ def lib():
         L.dsa_device_status.argtypes = [I]
         L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
         for f in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_sparse_attn_noalloc", "dsa_forward",
-                  "dsa_forward_timed",
+                  "dsa_forward_timed", "dsa_indexer_kl_loss",
                   "dsa_device_status",
                   "dsa_selftest_wait_timeout", "dsa_version"):
             getattr(L, f).restype = ctypes.c_int
@@ -248,6 +250,34 @@ def forward(q_I, q_scale, w, k_I, k_scale, q, kv, k, d_v, scale, q_offset=0, ind
     _check(lib().dsa_forward_timed(ctypes.byref(ia), ctypes.byref(aa), int(k), _ptr(indices), _ptr(out), _ptr(lse),
                                    _ptr(workspace), nbytes, _stream(stream), ev), "dsa_forward")
     return indices, out, lse
+
+
+def indexer_kl_loss(q, kv, indices, lse, scores, d_v, scale, target=None, want_target=True, kl=None,
+                    stream=None):
+    """Forward of the indexer's training loss over the selected positions.
+
+    Target p = the attention probabilities (from ``lse`` of sparse_attn on the same
+    selection) summed over the heads and L1-normalised; loss per row =
+    D_KL(p || softmax over the selected positions of ``scores``).  Returns
+    (target fp32 [B, Lq, k] or None, kl fp32 [B, Lq]).
+    """
+    a = _attn_args(q, kv, d_v, scale)
+    B, Lq, H, _ = q.shape
+    Lk = kv.shape[1]
+    k = indices.shape[-1]
+    _need(indices, torch.int32, (B, Lq, k), "indices")
+    _need(lse, torch.float32, (B, Lq, H), "lse")
+    _need(scores, torch.float32, (B, Lq, Lk), "scores")
+    if target is None and want_target:
+        target = torch.empty(B, Lq, k, dtype=torch.float32, device=q.device)
+    if target is not None:
+        _need(target, torch.float32, (B, Lq, k), "target")
+    if kl is None:
+        kl = torch.empty(B, Lq, dtype=torch.float32, device=q.device)
+    _need(kl, torch.float32, (B, Lq), "kl")
+    _check(lib().dsa_indexer_kl_loss(ctypes.byref(a), B, Lq, Lk, _ptr(indices), k, _ptr(lse), _ptr(scores),
+                                     _ptr(target), _ptr(kl), _stream(stream)), "dsa_indexer_kl_loss")
+    return target, kl
 
 
 def device_status(clear: bool = True) -> int:

@@ -1,8 +1,8 @@
 // dsa_api.cu -- the C ABI of libdsa.so (declared in include/dsa.h): argument
 // checks, TMA descriptor set-up, workspace layout and kernel dispatch for the
 // DeepSeek Sparse Attention forward pass.  Every step of the computation runs in
-// the kernels of indexer.cu, topk.cu and sparse_attn.cu; this file only checks,
-// describes and launches.
+// the kernels of indexer.cu, topk.cu, sparse_attn.cu and indexer_loss.cu; this
+// file only checks, describes and launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -239,6 +239,31 @@ dsa_status run_attn(const dsa_attn_args* a, int B, int Lq, int Lk, int q_offset,
   return DSA_OK;
 }
 
+dsa_status run_indexer_kl(const dsa_attn_args* a, int B, int Lq, int Lk, const int32_t* indices, int k,
+                          const float* lse, const float* scores, float* target, float* kl, cudaStream_t st) {
+  KlParams p{};
+  p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = a->H; p.k = k;
+  p.n_rows = B * Lq;
+  p.n_tiles = (k + 63) / 64;
+  p.scale_log2 = a->scale * 1.4426950408889634f;
+  p.indices = indices;
+  p.lse = lse;
+  p.scores = scores;
+  p.target = target;
+  p.kl = kl;
+  CUtensorMap tq, tkv;
+  if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->q, (uint64_t)p.n_rows * a->H, a->d_qk, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  if (!make_tmap(&tkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->kv, (uint64_t)B * Lk, a->d_qk, 64, 1,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  const int sms = sm_count();
+  const int grid = p.n_rows < sms ? p.n_rows : sms;
+  if (launch_indexer_kl(p, a->d_qk, tq, tkv, grid, st) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 __global__ void wait_selftest_kernel(uint32_t limit) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -261,12 +286,13 @@ cudaError_t read_device_error(uint32_t* value, bool clear) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return e;
   // Every unit's word holds DEV_ERR_NONE or the one code a failed wait records.
-  uint32_t words[4] = {0, 0, 0, 0};
+  uint32_t words[5] = {0, 0, 0, 0, 0};
   if ((e = read_unit_error(&words[0], clear)) != cudaSuccess) return e;
   if ((e = read_indexer_error(&words[1], clear)) != cudaSuccess) return e;
   if ((e = read_topk_error(&words[2], clear)) != cudaSuccess) return e;
   if ((e = read_attn_error(&words[3], clear)) != cudaSuccess) return e;
-  *value = words[0] | words[1] | words[2] | words[3];
+  if ((e = read_kl_error(&words[4], clear)) != cudaSuccess) return e;
+  *value = words[0] | words[1] | words[2] | words[3] | words[4];
   return cudaSuccess;
 }
 
@@ -309,6 +335,17 @@ dsa_status dsa_sparse_attn(const dsa_attn_args* args, int B, int Lq, int Lk, con
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
   return run_attn(args, B, Lq, Lk, 0, false, indices, k, out, lse, workspace, workspace_bytes,
                   static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_indexer_kl_loss(const dsa_attn_args* args, int B, int Lq, int Lk, const int32_t* indices, int k,
+                               const float* lse, const float* scores, float* target, float* kl, void* stream) {
+  dsa_status s = check_attn(args, B, Lq, Lk);
+  if (s != DSA_OK) return s;
+  if (!indices || !lse || !scores || !kl) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(indices) || !aligned16(lse) || !aligned16(scores) || !aligned16(kl)) return DSA_ERR_INVALID_ARG;
+  if (target && !aligned16(target)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+  return run_indexer_kl(args, B, Lq, Lk, indices, k, lse, scores, target, kl, static_cast<cudaStream_t>(stream));
 }
 
 size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_v) {

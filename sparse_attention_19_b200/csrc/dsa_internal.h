@@ -68,11 +68,28 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int d_qk, int d_v, const CUt
                                const CUtensorMap& tkv, int grid_clusters, cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t stream);
 
+// ---------------------------------------------------------------- indexer training loss
+struct KlParams {
+  int B, Lq, Lk, H, k;
+  int n_rows;             // B * Lq
+  int n_tiles;            // ceil(k / 64)
+  float scale_log2;       // softmax scale * log2(e)
+  const int32_t* indices; // [B, Lq, k]
+  const float* lse;       // [B, Lq, H], natural log
+  const float* scores;    // [B, Lq, Lk]
+  float* target;          // [B, Lq, k] or null
+  float* kl;              // [B, Lq]
+};
+size_t indexer_kl_smem_bytes(int d_qk);
+cudaError_t launch_indexer_kl(const KlParams& p, int d_qk, const CUtensorMap& tq, const CUtensorMap& tkv, int grid,
+                              cudaStream_t stream);
+
 // ---------------------------------------------------------------- misc
 // Error words of the kernel units (one per translation unit), and their union.
 cudaError_t read_indexer_error(uint32_t* value, bool clear);
 cudaError_t read_topk_error(uint32_t* value, bool clear);
 cudaError_t read_attn_error(uint32_t* value, bool clear);
+cudaError_t read_kl_error(uint32_t* value, bool clear);
 cudaError_t read_device_error(uint32_t* value, bool clear);
 cudaError_t launch_wait_selftest(uint32_t spin_limit, cudaStream_t stream);
 

@@ -109,3 +109,16 @@ def test_workspace_sizes():
     fwd = dsa.workspace_size(dsa.OP_FORWARD, 1, 4096, 131072, 2048, 128, 512)
     assert fwd >= 4096 * 131072 * 4
     assert dsa.workspace_size(dsa.OP_FORWARD, 0, 1, 1, 1, 1, 1) == 0
+
+
+def test_indexer_kl_loss_rejects_bad_arguments(L):
+    good = dsa.AttnArgs(128, 576, 512, 0.07, 16, 16)
+    p = ctypes.c_void_p(16)
+    f = L.dsa_indexer_kl_loss
+    assert f(ctypes.byref(good), 1, 1, 8, p, 8, None, p, None, p, None) == 1           # no lse
+    assert f(ctypes.byref(good), 1, 1, 8, p, 8, p, None, None, p, None) == 1           # no scores
+    assert f(ctypes.byref(good), 1, 1, 8, p, 8, p, p, None, None, None) == 1           # no kl
+    assert f(ctypes.byref(good), 1, 1, 8, p, 8, p, p, ctypes.c_void_p(8), p, None) == 1   # misaligned target
+    assert f(ctypes.byref(good), 1, 1, 8, p, 0, p, p, None, p, None) == 2              # k < 1
+    assert f(ctypes.byref(good), 1, 1, 8, p, 4096, p, p, None, p, None) == 2           # k > 2048
+    assert f(ctypes.byref(dsa.AttnArgs(64, 576, 512, 0.07, 16, 16)), 1, 1, 8, p, 8, p, p, None, p, None) == 2
