@@ -244,7 +244,7 @@ dsa_status run_indexer_kl(const dsa_attn_args* a, int B, int Lq, int Lk, const i
   KlParams p{};
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = a->H; p.k = k;
   p.n_rows = B * Lq;
-  p.n_tiles = (k + 63) / 64;
+  p.n_tiles = (k + 127) / 128;
   p.scale_log2 = a->scale * 1.4426950408889634f;
   p.indices = indices;
   p.lse = lse;
@@ -252,14 +252,14 @@ dsa_status run_indexer_kl(const dsa_attn_args* a, int B, int Lq, int Lk, const i
   p.target = target;
   p.kl = kl;
   CUtensorMap tq, tkv;
-  if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->q, (uint64_t)p.n_rows * a->H, a->d_qk, 64, 128,
+  if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->q, (uint64_t)p.n_rows * a->H, a->d_qk, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   if (!make_tmap(&tkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->kv, (uint64_t)B * Lk, a->d_qk, 64, 1,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  const int sms = sm_count();
-  const int grid = p.n_rows < sms ? p.n_rows : sms;
+  const int pairs = sm_count() / 2;
+  const int grid = p.n_rows < pairs ? p.n_rows : pairs;
   if (launch_indexer_kl(p, a->d_qk, tq, tkv, grid, st) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }

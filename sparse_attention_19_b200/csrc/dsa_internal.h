@@ -72,7 +72,7 @@ cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t strea
 struct KlParams {
   int B, Lq, Lk, H, k;
   int n_rows;             // B * Lq
-  int n_tiles;            // ceil(k / 64)
+  int n_tiles;            // ceil(k / 128)
   float scale_log2;       // softmax scale * log2(e)
   const int32_t* indices; // [B, Lq, k]
   const float* lse;       // [B, Lq, H], natural log
@@ -81,8 +81,8 @@ struct KlParams {
   float* kl;              // [B, Lq]
 };
 size_t indexer_kl_smem_bytes(int d_qk);
-cudaError_t launch_indexer_kl(const KlParams& p, int d_qk, const CUtensorMap& tq, const CUtensorMap& tkv, int grid,
-                              cudaStream_t stream);
+cudaError_t launch_indexer_kl(const KlParams& p, int d_qk, const CUtensorMap& tq, const CUtensorMap& tkv,
+                              int grid_clusters, cudaStream_t stream);
 
 // ---------------------------------------------------------------- misc
 // Error words of the kernel units (one per translation unit), and their union.

@@ -12,24 +12,32 @@
 // of that section).  lse is the log-sum-exp the attention kernel returns for the
 // same selection, so the logits are recomputed but never renormalised here.
 //
-// One CTA per query row at a time (persistent over rows), no cluster:
-//   * Q (128 head rows x d_qk bf16, 9 planes of 128 x 64 columns) stays in shared
-//     memory for the row; keys come in tiles of 64 selected positions, gathered
-//     in 64-column chunks (TMA tile::gather4, 128-byte swizzle) through a ring.
-//   * S = Q K^T per tile is a chain of tcgen05.mma (M = 128 heads, N = 64 keys,
-//     K = 16), issued by one thread, double-buffered in TMEM (2 x 64 columns).
-//   * Eight epilogue warps read S: warp w holds heads 32(w%4)..+31 (its TMEM lane
-//     quarter) for keys 32(w/4)..+31.  Each lane turns its 32 logits into
-//     probabilities with the row's lse, then the warp sums them over its 32 heads
-//     by a butterfly transpose-reduction (31 shuffles leave lane i holding key
-//     i's sum); the four head quarters meet in shared memory.
-//   * Warps 0-1 then own one key each: they fold P into the row's running sums
-//     (sum P, sum P log P, sum P (I - m), and the indexer log-sum-exp with a
-//     running maximum m), write P to the target, and at the row's end combine
-//     the sums into KL and rescale the target row by 1 / sum P.
-// Warp roles (800 threads): 0-7 epilogue, 8 TMEM owner + MMA issuer, 9-22 key
-// loaders (two warps per ring slot, each issuing half of a chunk's 16 gathers),
-// 23-24 stage each row's selected positions one row ahead.
+// Mapping onto a pair of SMs (a 2-CTA cluster, tcgen05 .cta_group::2), one query
+// row at a time per pair:
+//   * Each CTA holds 64 of the 128 heads' Q rows (64 x d_qk bf16) in shared
+//     memory, so most of the shared memory is left for keys in flight: a ring of
+//     16 chunks of 64 gathered latent rows x 64 columns per CTA (TMA
+//     tile::gather4, 128-byte swizzle).
+//   * Keys come in tiles of 128 selected positions; S = Q K^T is one pair-MMA
+//     chain (M = 128 heads, N = 128 keys, K = 16 per instruction) issued by one
+//     thread of the leader CTA, double-buffered in TMEM.  Each CTA's TMEM holds
+//     its 64 heads: lanes 0-63 keys 0-63 of the tile, lanes 64-127 keys 64-127.
+//   * Eight reduction warps per CTA read S: warp w holds TMEM lane quarter w % 4
+//     (32 heads, one key half) for 32 of the half's 64 keys.  Each lane turns its
+//     logits into probabilities with its head's lse, then the warp sums them over
+//     its 32 heads by a butterfly transpose-reduction (31 shuffles leave lane i
+//     holding key i's sum) and posts the sums to a 4-tile ring in the leader's
+//     shared memory: the leader's warps with plain stores and an arrive, the
+//     other CTA's with st.async, whose bytes complete the same barrier.
+//   * Four loss warps of the leader own one key each: per tile they add the four
+//     head-quarter sums into P, fold it into the row's running sums (sum P,
+//     sum P log P, sum P (I - m), and the indexer log-sum-exp with a running
+//     maximum m) and write P to the target; at the row's end they combine the
+//     sums into KL and rescale the target row by 1 / sum P.  The ring keeps this
+//     chain off the path of the TMEM reads.
+// Warp roles (1024 threads per CTA): 0-7 reduction, 8-11 loss (leader), 12 TMEM
+// owner + MMA issuer (leader), 13-14 stage each row's selected positions one row
+// ahead, 16-31 key loaders (one per ring slot).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -43,22 +51,25 @@ namespace dsa {
 
 namespace {
 
-constexpr int kTileKeys = 64;          // selected positions per S tile
-constexpr int kStages = 7;             // key-chunk ring depth (8 KB stages)
-constexpr int kWarpsPerSlot = 2;
-constexpr int kEpiWarps = 8;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp0 = 9;
-constexpr int kLoadWarps = kStages * kWarpsPerSlot;   // 14
-constexpr int kStageWarp0 = kLoadWarp0 + kLoadWarps;  // 23
+constexpr int kTileKeys = 128;         // selected positions per S tile (pair)
+constexpr int kHalfKeys = 64;          // keys per CTA in B, and per TMEM lane half
+constexpr int kStages = 16;            // key-chunk ring depth (8 KB stages)
+constexpr int kRedWarps = 8;           // reduction warps (warpgroups 0-1)
+constexpr int kLossWarp0 = 8;          // loss warps (warpgroup 2, leader)
+constexpr int kLossWarps = kTileKeys / 32;
+constexpr int kMmaWarp = 12;
+constexpr int kStageWarp0 = 13;
 constexpr int kStageWarps = 2;
-constexpr int kThreads = 32 * (kStageWarp0 + kStageWarps);   // 800
+constexpr int kLoadWarp0 = 16;
+constexpr int kLoadWarps = kStages;    // one loader warp per ring slot
+constexpr int kThreads = 32 * (kLoadWarp0 + kLoadWarps);   // 1024
+constexpr int kRedSlots = 4;           // tiles of head sums in flight to the loss warps
+constexpr uint32_t kPeerBytes = kRedWarps * 32 * 4;       // the other CTA's sums per tile
 constexpr int kStageBatch = 8;         // index words in flight per staging warp
 constexpr int kMaxIdx = 2048;
 constexpr int kMaxChunks = 9;
-constexpr uint32_t kQPlane = 128 * 128;   // 128 head rows x 128 B
-constexpr uint32_t kChunk = 64 * 128;     // 64 key rows x 128 B
-constexpr uint32_t kTmemCols = 128;       // two S buffers of 64 columns
+constexpr uint32_t kPlane = 64 * 128;  // 64 rows x 128 B (Q plane, key chunk)
+constexpr uint32_t kTmemCols = 128;    // two S buffers of 64 columns
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct KlShared {
@@ -66,13 +77,15 @@ struct KlShared {
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t s_full[2], s_empty[2];
   uint64_t idx_full[2], idx_empty[2];
-  uint64_t xbar;                        // rendezvous of the eight epilogue warps
+  uint64_t red_full[kRedSlots];          // leader: its reduction warps + the other CTA's bytes
+  uint64_t red_empty[kRedSlots];         // both CTAs: the leader's loss warps
+  uint64_t lbar;                         // rendezvous of the loss warps
   uint64_t final_mma;
   uint32_t tmem_base;
   uint32_t abort_flag;
-  uint32_t valid_mask[2][kMaxIdx / 32]; // per 32 staged slots: bit set = valid position
-  float red[2][4][kTileKeys];           // per S buffer: head-quarter partial sums per key
-  float fin[2][5];                      // per key warp: (Z, A, Bs, m, s) of the row
+  uint32_t valid_mask[2][kMaxIdx / 32];  // per 32 staged slots: bit set = valid position
+  float red[kRedSlots][4][kTileKeys];    // leader: per tile, 32-head sums (rank * 2 + quarter), per key
+  float fin[kLossWarps][5];              // leader: per loss warp (Z, A, Bs, m, s) of the row
 };
 
 // Row of kv (in the [B*Lk, d_qk] view) staged for a slot; bit 31 marks padding,
@@ -101,7 +114,7 @@ __device__ __forceinline__ RowSums merge(const RowSums& x, const RowSums& y) {
 }
 
 template <int NC>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
                   const KlParams p) {
   static_assert(NC <= kMaxChunks, "d_qk");
@@ -110,11 +123,15 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t area_off = ((raw_addr + sizeof(KlShared) + 1023u) & ~1023u) - raw_addr;
   uint8_t* q_sm = smem_raw + area_off;                              // NC planes
-  uint8_t* k_sm = q_sm + NC * kQPlane;                              // kStages chunks
-  int32_t* idx_sm = reinterpret_cast<int32_t*>(k_sm + kStages * kChunk);   // 2 x kMaxIdx
+  uint8_t* k_sm = q_sm + NC * kPlane;                               // kStages chunks
+  int32_t* idx_sm = reinterpret_cast<int32_t*>(k_sm + kStages * kPlane);   // 2 x kMaxIdx
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int cluster_id = blockIdx.x >> 1;
+  const int n_clusters = gridDim.x >> 1;
   volatile uint32_t* abort_flag = &S.abort_flag;
 
   if (threadIdx.x == 0) {
@@ -122,34 +139,88 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
     for (int i = 0; i < kStages; ++i) { mbar_init(&S.k_full[i], 1); mbar_init(&S.k_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_empty[i], kEpiWarps);
+      mbar_init(&S.s_empty[i], 2 * kRedWarps);           // both CTAs' reduction warps
       mbar_init(&S.idx_full[i], kStageWarps);
-      mbar_init(&S.idx_empty[i], kLoadWarps + kEpiWarps);
+      // readers of the staged positions: loaders, reduction warps, and the leader's loss warps
+      mbar_init(&S.idx_empty[i], kLoadWarps + kRedWarps + (leader ? kLossWarps : 0));
     }
-    mbar_init(&S.xbar, kEpiWarps);
+    for (int i = 0; i < kRedSlots; ++i) {
+      mbar_init(&S.red_full[i], kRedWarps);              // + kPeerBytes of transaction count
+      mbar_init(&S.red_empty[i], kLossWarps);
+    }
+    mbar_init(&S.lbar, kLossWarps);
     mbar_init(&S.final_mma, 1);
     S.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&S.tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&S.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
+  const uint16_t kBoth = 0x3;
   bool ok = true;
 
-  if (warp >= kStageWarp0) {
+  if (warp >= kLoadWarp0) {
+    // ------------------------------------------------------------------ key loaders
+    // Per row: this CTA's Q planes (plane c from loader c % kLoadWarps), then for
+    // each tile its NC key chunks (this CTA's 64 keys x 64 columns).  Chunk kc goes
+    // to ring slot kc % kStages, which loader warp kc % kStages owns; lanes 0-15
+    // issue its 16 four-row gathers.  Both CTAs' loads complete on the leader's
+    // barriers.
+    const int pw = (int)warp - kLoadWarp0;
+    uint32_t ucount = 0, kc = 0;
+    if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
+    for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
+      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+      if (lane == 0) {
+        const int qrow = row * p.H + (int)rank * 64;
+        for (int c = pw; c < NC && ok; c += kLoadWarps) {
+          ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
+          if (!ok) break;
+          if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane);
+          tma_load_2d_pair(q_sm + c * kPlane, &tmap_q, mapa_shared(smem_u32(&S.q_full[c]), 0), c * 64, qrow);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
+      if (!ok) break;
+      const int32_t* idx = idx_sm + ib * kMaxIdx;
+      for (int j = 0; j < p.n_tiles && ok; ++j) {
+        for (int c = 0; c < NC; ++c, ++kc) {
+          const uint32_t st = kc % kStages, ph = (kc / kStages) & 1u;
+          if ((int)st != pw) continue;
+          bool w_ok = true;
+          if (lane == 0) {
+            w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
+            if (w_ok && leader) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane);
+          }
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+          if (lane < kHalfKeys / 4) {
+            const int base = j * kTileKeys + (int)rank * kHalfKeys + (int)lane * 4;
+            tma_gather4_pair(k_sm + st * kPlane + lane * 512, &tmap_kv, mapa_shared(smem_u32(&S.k_full[st]), 0),
+                             c * 64, gather_row(idx, base + 0), gather_row(idx, base + 1),
+                             gather_row(idx, base + 2), gather_row(idx, base + 3));
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+    }
+  } else if (warp >= kStageWarp0 && warp < kStageWarp0 + kStageWarps) {
     // ------------------------------------------------------------------ index staging
     // Row ordinal n goes to buffer n % 2 as kv rows to gather (batch offset applied,
     // bit 31 on padding and out-of-range entries) plus one validity ballot per 32
-    // slots.  Slots past k are padding.
+    // slots.  Slots past k are padding.  Both CTAs stage the whole row.
     const int sw = (int)warp - kStageWarp0;
     const int nwords = p.n_tiles * (kTileKeys / 32);
     uint32_t ucount = 0;
-    for (int row = blockIdx.x; row < p.n_rows && ok; row += gridDim.x, ++ucount) {
+    for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
       const uint32_t buf = ucount & 1u, ph = (ucount >> 1) & 1u;
       ok = mbar_wait_warp(&S.idx_empty[buf], ph ^ 1u, abort_flag);
       if (!ok) break;
@@ -177,135 +248,78 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.idx_full[buf]);
     }
-  } else if (warp >= kLoadWarp0) {
-    // ------------------------------------------------------------------ key loaders
-    // Per row: the Q planes (plane c from loader c % kLoadWarps), then for each
-    // tile its NC key chunks (64 keys x 64 columns).  Chunk kc goes to ring slot
-    // kc % kStages; the slot's two warps issue its 16 four-row gathers, groups
-    // g = part, part + 2, ...
-    const int pw = (int)warp - kLoadWarp0;
-    const uint32_t my_slot = (uint32_t)(pw / kWarpsPerSlot);
-    const int part = pw % kWarpsPerSlot;
-    uint32_t ucount = 0, kc = 0;
-    if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
-    for (int row = blockIdx.x; row < p.n_rows && ok; row += gridDim.x, ++ucount) {
-      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
-      if (lane == 0) {
-        for (int c = pw; c < NC && ok; c += kLoadWarps) {
-          ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&S.q_full[c], kQPlane);
-          tma_load_2d(q_sm + c * kQPlane, &tmap_q, &S.q_full[c], c * 64, row * p.H);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
-      if (!ok) break;
-      const int32_t* idx = idx_sm + ib * kMaxIdx;
-      for (int j = 0; j < p.n_tiles && ok; ++j) {
-        for (int c = 0; c < NC; ++c, ++kc) {
-          const uint32_t st = kc % kStages, ph = (kc / kStages) & 1u;
-          if (st != my_slot) continue;
-          bool w_ok = true;
-          if (lane == 0) {
-            w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
-            if (w_ok && part == 0) mbar_arrive_expect_tx(&S.k_full[st], kChunk);
-          }
-          if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-          const int g = part + kWarpsPerSlot * (int)lane;         // 4-key group of this lane
-          if (g < kTileKeys / 4) {
-            const int base = j * kTileKeys + g * 4;
-            tma_gather4(k_sm + st * kChunk + g * 512, &tmap_kv, &S.k_full[st], c * 64, gather_row(idx, base + 0),
-                        gather_row(idx, base + 1), gather_row(idx, base + 2), gather_row(idx, base + 3));
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
-    }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     // S = Q K^T for each tile into TMEM buffer (tile ordinal % 2): per key chunk,
-    // 4 MMAs of K = 16 (descriptor start addresses advance 32 B, encoded 2).
-    if (elect_one()) {
+    // 4 pair-MMAs of K = 16 (descriptor start addresses advance 32 B, encoded 2).
+    if (leader && elect_one()) {
       constexpr uint32_t idesc = make_idesc(1, 1, 128, kTileKeys, 0, 0);   // bf16, K-major x K-major
       const uint64_t q_desc = make_smem_desc(smem_u32(q_sm), 16, 1024, LAYOUT_SW128);
       const uint64_t k_desc = make_smem_desc(smem_u32(k_sm), 16, 1024, LAYOUT_SW128);
       uint32_t ucount = 0, kc = 0, sc = 0;
-      for (int row = blockIdx.x; row < p.n_rows && ok; row += gridDim.x, ++ucount) {
+      for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
         for (int j = 0; j < p.n_tiles && ok; ++j, ++sc) {
           const uint32_t sb = sc & 1u;
-          ok = mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag);
+          ok = mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag, true);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t d = tmem_base + sb * kTileKeys;
+          const uint32_t d = tmem_base + sb * kHalfKeys;
           for (int c = 0; c < NC; ++c, ++kc) {
             if (j == 0 && !mbar_wait(&S.q_full[c], ucount & 1u, abort_flag)) { ok = false; break; }
             const uint32_t st = kc % kStages, ph = (kc / kStages) & 1u;
             if (!mbar_wait(&S.k_full[st], ph, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t ad = q_desc + (uint64_t)(c * (kQPlane >> 4));
-            const uint64_t bd = k_desc + (uint64_t)(st * (kChunk >> 4));
-            mma_bf16_ss(d, ad + 0, bd + 0, idesc, c ? 1u : 0u);
-            mma_bf16_ss(d, ad + 2, bd + 2, idesc, 1u);
-            mma_bf16_ss(d, ad + 4, bd + 4, idesc, 1u);
-            mma_bf16_ss(d, ad + 6, bd + 6, idesc, 1u);
-            mma_commit(&S.k_empty[st]);
-            if (j == p.n_tiles - 1) mma_commit(&S.q_empty[c]);   // plane free for the next row
+            const uint64_t ad = q_desc + (uint64_t)(c * (kPlane >> 4));
+            const uint64_t bd = k_desc + (uint64_t)(st * (kPlane >> 4));
+            mma_bf16_ss_pair(d, ad + 0, bd + 0, idesc, c ? 1u : 0u);
+            mma_bf16_ss_pair(d, ad + 2, bd + 2, idesc, 1u);
+            mma_bf16_ss_pair(d, ad + 4, bd + 4, idesc, 1u);
+            mma_bf16_ss_pair(d, ad + 6, bd + 6, idesc, 1u);
+            mma_commit_pair_mc(&S.k_empty[st], kBoth);
+            if (j == p.n_tiles - 1) mma_commit_pair_mc(&S.q_empty[c], kBoth);   // plane free for the next row
           }
           if (!ok) break;
-          mma_commit(&S.s_full[sb]);
+          mma_commit_pair_mc(&S.s_full[sb], kBoth);
         }
       }
       // Every MMA this thread issued completes before the TMEM is released.
       mma_commit(&S.final_mma);
       mbar_wait(&S.final_mma, 0, nullptr);
     }
-  } else {
-    // ------------------------------------------------------------------ epilogue
-    const uint32_t quarter = warp & 3u;            // TMEM lane quarter = head group
-    const int c0 = (int)(warp >> 2) * 32;          // this warp's 32 keys of the tile
-    const int head = (int)quarter * 32 + (int)lane;
+  } else if (warp < (uint32_t)kRedWarps) {
+    // ------------------------------------------------------------------ reduction warps
+    const uint32_t quarter = warp & 3u;            // TMEM lane quarter
+    const int hq = (int)(quarter & 1u);            // head quarter within this CTA's 64 heads
+    const int kh = (int)(quarter >> 1);            // key half of the tile held by these lanes
+    const int c0 = (int)(warp >> 2) * 32;          // this warp's 32 of the half's 64 keys
+    const int kk0 = kh * kHalfKeys + c0;           // first key of the tile this warp reduces
+    const int head = (int)rank * 64 + hq * 32 + (int)lane;
     const bool head_ok = head < p.H;
     const uint32_t lane_addr = (quarter * 32u) << 16;
-    const bool keyer = warp < 2;                   // owns key `key` of every tile
-    const int key = (int)warp * 32 + (int)lane;
     const float2 scl = make_float2(p.scale_log2, p.scale_log2);
-    uint32_t ucount = 0, sc = 0, xph = 0;
-    for (int row = blockIdx.x; row < p.n_rows && ok; row += gridDim.x, ++ucount) {
+    // where this warp's 32 sums go in the leader's ring, and the barrier that counts them
+    const uint32_t red_dst = mapa_shared(smem_u32(&S.red[0][(int)rank * 2 + hq][kk0 + (int)lane]), 0);
+    const uint32_t red_full0 = mapa_shared(smem_u32(&S.red_full[0]), 0);
+    uint32_t ucount = 0, sc = 0;
+    for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
       const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
-      const int32_t* idx = idx_sm + ib * kMaxIdx;
-      const int bLk = (row / p.Lq) * p.Lk;
-      const float* srow = p.scores + (size_t)row * p.Lk;
-      float* trow = p.target ? p.target + (size_t)row * p.k : nullptr;
       // exponent offset: a_h[s] = 2^(z * scale * log2 e - lse * log2 e)
       const float nl = head_ok ? -p.lse[(size_t)row * p.H + head] * kLog2e : 0.f;
       const float2 nl2 = make_float2(nl, nl);
-      RowSums acc{0.f, 0.f, 0.f, -INFINITY, 0.f};
       for (int j = 0; j < p.n_tiles && ok; ++j, ++sc) {
-        // The key warps fetch this tile's indexer scores before waiting for S.
-        const int slot = j * kTileKeys + key;
-        bool kvalid = false;
-        float iv = 0.f;
-        if (keyer) {
-          const int32_t gr = idx[slot];
-          kvalid = gr >= 0;
-          if (kvalid) iv = __ldg(srow + (gr - bLk));
-        }
         const uint32_t sb = sc & 1u;
         ok = mbar_wait_warp(&S.s_full[sb], (sc >> 1) & 1u, abort_flag);
         if (!ok) break;
         tc_fence_after();
         uint32_t v[32];
-        tmem_ld32(tmem_base + lane_addr + sb * kTileKeys + c0, v);
+        tmem_ld32(tmem_base + lane_addr + sb * kHalfKeys + c0, v);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.s_empty[sb]);
-        const uint32_t vm = head_ok ? S.valid_mask[ib][(j * kTileKeys + c0) >> 5] : 0u;
+        if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
+        const uint32_t vm = head_ok ? S.valid_mask[ib][(j * kTileKeys + kk0) >> 5] : 0u;
         float pr[32];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -315,7 +329,7 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
         }
         // Butterfly transpose-reduction over the warp's 32 heads: at each step a lane
         // keeps the half of its columns selected by one bit of its lane number and
-        // adds the partner's copy of that half.  Lane i ends with key c0 + i.
+        // adds the partner's copy of that half.  Lane i ends with key kk0 + i.
 #pragma unroll
         for (int half = 16; half >= 1; half >>= 1) {
           const bool up = (lane & (uint32_t)half) != 0u;
@@ -327,60 +341,128 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
             pr[e] = keep + __shfl_xor_sync(0xffffffffu, send, half);
           }
         }
-        S.red[sb][quarter][c0 + (int)lane] = pr[0];
-        ok = warps_rendezvous(&S.xbar, xph, abort_flag);
+        // Post to ring slot sc % kRedSlots once the loss warps are done with it.
+        const uint32_t slot = sc % kRedSlots, rph = (sc / kRedSlots) & 1u;
+        ok = mbar_wait_warp(&S.red_empty[slot], rph ^ 1u, abort_flag, true);
         if (!ok) break;
-        if (keyer) {
-          const float P = (S.red[sb][0][key] + S.red[sb][1][key]) + (S.red[sb][2][key] + S.red[sb][3][key]);
-          if (kvalid) {
-            if (iv > acc.m) {                          // move the references to the new maximum
-              if (acc.Z > 0.f) acc.Bs = fmaf(-acc.Z, iv - acc.m, acc.Bs);
-              acc.s = acc.m == -INFINITY ? 0.f : acc.s * ex2_approx((acc.m - iv) * kLog2e);
-              acc.m = iv;
-            }
-            if (iv != -INFINITY) acc.s += ex2_approx((iv - acc.m) * kLog2e);
-            acc.Z += P;
-            if (P > 0.f) {
-              acc.Bs = fmaf(P, iv - acc.m, acc.Bs);
-              acc.A = fmaf(P, __logf(P), acc.A);
-            }
+        const uint32_t off = slot * (uint32_t)sizeof(S.red[0]);
+        if (leader) {
+          S.red[slot][hq][kk0 + (int)lane] = pr[0];
+          __syncwarp();
+          if (lane == 0) {
+            if (warp == 0) mbar_arrive_expect_tx(&S.red_full[slot], kPeerBytes);
+            else mbar_arrive(&S.red_full[slot]);
           }
-          if (trow && slot < p.k) trow[slot] = P;      // rescaled once the row's sum is known
+        } else {
+          st_async_f32(red_dst + off, pr[0], red_full0 + slot * 8u);
         }
       }
       if (!ok) break;
-      // ---- end of the row: combine the key warps' sums into KL and normalise the target
-      if (keyer) {
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          RowSums o;
-          o.Z = __shfl_xor_sync(0xffffffffu, acc.Z, off);
-          o.A = __shfl_xor_sync(0xffffffffu, acc.A, off);
-          o.Bs = __shfl_xor_sync(0xffffffffu, acc.Bs, off);
-          o.m = __shfl_xor_sync(0xffffffffu, acc.m, off);
-          o.s = __shfl_xor_sync(0xffffffffu, acc.s, off);
-          acc = merge(acc, o);
-        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
+    }
+  } else if (warp >= (uint32_t)kLossWarp0 && warp < (uint32_t)(kLossWarp0 + kLossWarps) && leader) {
+    // ------------------------------------------------------------------ loss warps (leader)
+    const int key = ((int)warp - kLossWarp0) * 32 + (int)lane;   // key of every tile this thread owns
+    uint32_t ucount = 0, sc = 0, lph = 0;
+    const uint32_t peer_empty0 = mapa_shared(smem_u32(&S.red_empty[0]), 1);
+    for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
+      const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
+      ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
+      if (!ok) break;
+      const int32_t* idx = idx_sm + ib * kMaxIdx;
+      const int bLk = (row / p.Lq) * p.Lk;
+      const float* srow = p.scores + (size_t)row * p.Lk;
+      float* trow = p.target ? p.target + (size_t)row * p.k : nullptr;
+      RowSums acc{0.f, 0.f, 0.f, -INFINITY, 0.f};
+      // The indexer score of this thread's key in tile j (0 for padding or past the
+      // row's tiles); fetched four tiles before it is used, so that its DRAM latency
+      // stays off the chain.
+      auto fetch = [&](int j) -> float {
+        if (j >= p.n_tiles) return 0.f;
+        const int32_t gr = idx[j * kTileKeys + key];
+        return gr >= 0 ? __ldg(srow + (gr - bLk)) : 0.f;
+      };
+      auto consume = [&](int j, float iv) -> bool {
+        const int slot_x = j * kTileKeys + key;
+        const bool kvalid = idx[slot_x] >= 0;
+        const uint32_t slot = sc % kRedSlots, rph = (sc / kRedSlots) & 1u;
+        ++sc;
+        if (!mbar_wait_warp(&S.red_full[slot], rph, abort_flag, true)) return false;
+        const float P = (S.red[slot][0][key] + S.red[slot][1][key]) + (S.red[slot][2][key] + S.red[slot][3][key]);
+        __syncwarp();
         if (lane == 0) {
-          S.fin[warp][0] = acc.Z; S.fin[warp][1] = acc.A; S.fin[warp][2] = acc.Bs;
-          S.fin[warp][3] = acc.m; S.fin[warp][4] = acc.s;
+          mbar_arrive(&S.red_empty[slot]);
+          mbar_arrive_cluster(peer_empty0 + slot * 8u);
         }
+        if (kvalid) {
+          if (iv > acc.m) {                            // move the references to the new maximum
+            if (acc.Z > 0.f) acc.Bs = fmaf(-acc.Z, iv - acc.m, acc.Bs);
+            acc.s = acc.m == -INFINITY ? 0.f : acc.s * ex2_approx((acc.m - iv) * kLog2e);
+            acc.m = iv;
+          }
+          if (iv != -INFINITY) acc.s += ex2_approx((iv - acc.m) * kLog2e);
+          acc.Z += P;
+          if (P > 0.f) {
+            acc.Bs = fmaf(P, iv - acc.m, acc.Bs);
+            acc.A = fmaf(P, __logf(P), acc.A);
+          }
+        }
+        if (trow && slot_x < p.k) trow[slot_x] = P;    // rescaled once the row's sum is known
+        return true;
+      };
+      float iv0 = fetch(0), iv1 = fetch(1), iv2 = fetch(2), iv3 = fetch(3);
+      for (int j = 0; j < p.n_tiles && ok; j += 4) {
+        ok = consume(j, iv0);
+        iv0 = fetch(j + 4);
+        if (ok && j + 1 < p.n_tiles) { ok = consume(j + 1, iv1); iv1 = fetch(j + 5); }
+        if (ok && j + 2 < p.n_tiles) { ok = consume(j + 2, iv2); iv2 = fetch(j + 6); }
+        if (ok && j + 3 < p.n_tiles) { ok = consume(j + 3, iv3); iv3 = fetch(j + 7); }
       }
-      ok = warps_rendezvous(&S.xbar, xph, abort_flag);
+      if (!ok) break;
+      // ---- end of the row: combine the loss warps' sums into KL and normalise the target
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        RowSums y;
+        y.Z = __shfl_xor_sync(0xffffffffu, acc.Z, o);
+        y.A = __shfl_xor_sync(0xffffffffu, acc.A, o);
+        y.Bs = __shfl_xor_sync(0xffffffffu, acc.Bs, o);
+        y.m = __shfl_xor_sync(0xffffffffu, acc.m, o);
+        y.s = __shfl_xor_sync(0xffffffffu, acc.s, o);
+        acc = merge(acc, y);
+      }
+      const int lw = (int)warp - kLossWarp0;
+      if (lane == 0) {
+        S.fin[lw][0] = acc.Z; S.fin[lw][1] = acc.A; S.fin[lw][2] = acc.Bs;
+        S.fin[lw][3] = acc.m; S.fin[lw][4] = acc.s;
+      }
+      ok = warps_rendezvous(&S.lbar, lph, abort_flag);
+      if (!ok) break;
+      RowSums r{S.fin[0][0], S.fin[0][1], S.fin[0][2], S.fin[0][3], S.fin[0][4]};
+#pragma unroll
+      for (int w = 1; w < kLossWarps; ++w)
+        r = merge(r, RowSums{S.fin[w][0], S.fin[w][1], S.fin[w][2], S.fin[w][3], S.fin[w][4]});
+      ok = warps_rendezvous(&S.lbar, lph, abort_flag);   // fin is rewritten at the next row's end
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
       if (!ok) break;
-      if (keyer) {
-        const RowSums r0{S.fin[0][0], S.fin[0][1], S.fin[0][2], S.fin[0][3], S.fin[0][4]};
-        const RowSums r1{S.fin[1][0], S.fin[1][1], S.fin[1][2], S.fin[1][3], S.fin[1][4]};
-        const RowSums r = merge(r0, r1);
-        // KL = sum p log p - sum p (I - lse_I) with p = P / Z:
-        //    = (A - Bs) / Z - log Z + log s    (lse_I = m + log s; Bs is relative to m)
-        if (warp == 0 && lane == 0)
-          p.kl[row] = r.Z > 0.f ? (r.A - r.Bs) / r.Z - logf(r.Z) + logf(r.s) : 0.f;
-        if (trow && r.Z > 0.f) {
-          const float inv = 1.f / r.Z;
-          for (int x = key; x < p.k; x += kTileKeys) trow[x] *= inv;
+      // KL = sum p log p - sum p (I - lse_I) with p = P / Z:
+      //    = (A - Bs) / Z - log Z + log s    (lse_I = m + log s; Bs is relative to m)
+      if (lw == 0 && lane == 0) p.kl[row] = r.Z > 0.f ? (r.A - r.Bs) / r.Z - logf(r.Z) + logf(r.s) : 0.f;
+      if (trow && r.Z > 0.f) {
+        // all of this thread's loads first, then the stores: one round trip per row
+        const float inv = 1.f / r.Z;
+        constexpr int kPer = kMaxIdx / kTileKeys;
+        float t[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          const int x = key + i * kTileKeys;
+          t[i] = x < p.k ? trow[x] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          const int x = key + i * kTileKeys;
+          if (x < p.k) trow[x] = t[i] * inv;
         }
       }
     }
@@ -388,20 +470,21 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
 template <int NC>
-cudaError_t launch_t(const KlParams& p, const CUtensorMap& tq, const CUtensorMap& tkv, int grid,
+cudaError_t launch_t(const KlParams& p, const CUtensorMap& tq, const CUtensorMap& tkv, int grid_clusters,
                      cudaStream_t stream) {
   const size_t smem = indexer_kl_smem_bytes(NC * 64);
   auto kern = indexer_kl_kernel<NC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(tq, tkv, p);
+  kern<<<grid_clusters * 2, kThreads, smem, stream>>>(tq, tkv, p);
   return cudaGetLastError();
 }
 
@@ -410,16 +493,16 @@ cudaError_t launch_t(const KlParams& p, const CUtensorMap& tq, const CUtensorMap
 size_t indexer_kl_smem_bytes(int d_qk) {
   const int nc = d_qk / 64;
   size_t b = sizeof(KlShared) + 1024;              // shared state + alignment slack
-  b += (size_t)nc * kQPlane;                       // Q
-  b += (size_t)kStages * kChunk;                   // key ring
+  b += (size_t)nc * kPlane;                        // this CTA's Q rows
+  b += (size_t)kStages * kPlane;                   // key ring
   b += 2 * (size_t)kMaxIdx * sizeof(int32_t);      // staged positions, two rows
   return b;
 }
 
-cudaError_t launch_indexer_kl(const KlParams& p, int d_qk, const CUtensorMap& tq, const CUtensorMap& tkv, int grid,
-                              cudaStream_t stream) {
-  if (d_qk == 576) return launch_t<9>(p, tq, tkv, grid, stream);
-  if (d_qk == 192) return launch_t<3>(p, tq, tkv, grid, stream);
+cudaError_t launch_indexer_kl(const KlParams& p, int d_qk, const CUtensorMap& tq, const CUtensorMap& tkv,
+                              int grid_clusters, cudaStream_t stream) {
+  if (d_qk == 576) return launch_t<9>(p, tq, tkv, grid_clusters, stream);
+  if (d_qk == 192) return launch_t<3>(p, tq, tkv, grid_clusters, stream);
   return cudaErrorInvalidValue;
 }
 

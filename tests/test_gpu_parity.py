@@ -306,3 +306,27 @@ def test_wait_timeout_is_reported_not_trapped():
     assert dsa.device_status() == 0
     x = torch.ones(4, device=DEV)
     assert float(x.sum()) == 4.0          # the context is still usable
+
+
+# ------------------------------------------------------------------ context-parallel prefill
+
+def test_context_parallel_single_rank_matches_the_whole_sequence():
+    # One rank owning both zig-zag chunks: per-chunk forwards over the gathered
+    # key prefix reproduce the one-call forward of the whole sequence.
+    from sparse_attention_19_b200 import context_parallel as cp
+    wl = WORKLOADS["prefill_8k"].with_(Lq=4096, Lk=4096)
+    inp = to_dev(make_inputs(wl, "cpu", 3))
+    idx, out, lse = _forward(inp, wl)
+    chunk = 2048
+    mine = cp.zigzag_chunks(2, 1, 0)
+    local = cp.local_key_side(inp, mine, chunk)
+    queries = {c: {f: inp[f][:, c * chunk:(c + 1) * chunk].contiguous() for f in ("q_I", "q_scale", "w", "q")}
+               for c in mine}
+    res = cp.cp_forward(queries, local, 2, chunk, wl.k, wl.Dv, wl.scale, world=1, rank=0)
+    torch.cuda.synchronize()
+    for c in mine:
+        ci, co, cl = res[c]
+        sl = slice(c * chunk, (c + 1) * chunk)
+        assert torch.equal(ci, idx[:, sl])
+        assert float((co.float() - out[:, sl].float()).abs().max()) <= 1e-2
+        assert float((cl - lse[:, sl]).abs().max()) <= 1e-4
