@@ -17,7 +17,8 @@
 //   * Each CTA holds 64 of the 128 heads' Q rows (64 x d_qk bf16) in shared
 //     memory, so most of the shared memory is left for keys in flight: a ring of
 //     16 chunks of 64 gathered latent rows x 64 columns per CTA (TMA
-//     tile::gather4, 128-byte swizzle).
+//     tile::gather4, 128-byte swizzle).  One warp issues its TMA requests in
+//     order, so each chunk's 16 gathers are split over a team of four warps.
 //   * Keys come in tiles of 128 selected positions; S = Q K^T is one pair-MMA
 //     chain (M = 128 heads, N = 128 keys, K = 16 per instruction) issued by one
 //     thread of the leader CTA, double-buffered in TMEM.  Each CTA's TMEM holds
@@ -35,9 +36,12 @@
 //     maximum m) and write P to the target; at the row's end they combine the
 //     sums into KL and rescale the target row by 1 / sum P.  The ring keeps this
 //     chain off the path of the TMEM reads.
+// A row's tiles end at the last one holding a valid position (for top-k output,
+// which is valid-first, the all-padding tail of short rows is skipped).
 // Warp roles (1024 threads per CTA): 0-7 reduction, 8-11 loss (leader), 12 TMEM
 // owner + MMA issuer (leader), 13-14 stage each row's selected positions one row
-// ahead, 16-31 key loaders (one per ring slot).
+// ahead, 16-31 key loaders (four teams of four warps, each team owning four ring
+// slots and splitting each chunk's gathers).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -61,7 +65,9 @@ constexpr int kMmaWarp = 12;
 constexpr int kStageWarp0 = 13;
 constexpr int kStageWarps = 2;
 constexpr int kLoadWarp0 = 16;
-constexpr int kLoadWarps = kStages;    // one loader warp per ring slot
+constexpr int kTeamWarps = 4;          // loader warps sharing each chunk's 16 gathers
+constexpr int kTeamSlots = 4;          // consecutive ring slots a team owns
+constexpr int kLoadWarps = kStages / kTeamSlots * kTeamWarps;   // 16
 constexpr int kThreads = 32 * (kLoadWarp0 + kLoadWarps);   // 1024
 constexpr int kRedSlots = 4;           // tiles of head sums in flight to the loss warps
 constexpr uint32_t kPeerBytes = kRedWarps * 32 * 4;       // the other CTA's sums per tile
@@ -84,6 +90,7 @@ struct KlShared {
   uint32_t tmem_base;
   uint32_t abort_flag;
   uint32_t valid_mask[2][kMaxIdx / 32];  // per 32 staged slots: bit set = valid position
+  int32_t last_word[2][kStageWarps];     // per staging warp: last 32-slot word with a valid position
   float red[kRedSlots][4][kTileKeys];    // leader: per tile, 32-head sums (rank * 2 + quarter), per key
   float fin[kLossWarps][5];              // leader: per loss warp (Z, A, Bs, m, s) of the row
 };
@@ -91,6 +98,15 @@ struct KlShared {
 // Row of kv (in the [B*Lk, d_qk] view) staged for a slot; bit 31 marks padding,
 // which gathers row b*Lk (a valid row) and is masked.
 __device__ __forceinline__ int gather_row(const int32_t* rows, int pos) { return rows[pos] & 0x7fffffff; }
+
+// Tiles of the staged row in buffer `buf`: up to the last one that holds a valid
+// position (top-k output is valid-first, so this skips its all-padding tail).
+__device__ __forceinline__ int row_tiles(const volatile int32_t (*last_word)[kStageWarps], uint32_t buf) {
+  int last = -1;
+#pragma unroll
+  for (int w = 0; w < kStageWarps; ++w) last = max(last, (int)last_word[buf][w]);
+  return (last + 1 + (kTileKeys / 32) - 1) / (kTileKeys / 32);
+}
 
 // Running sums of one row: Z = sum P, A = sum P log P, Bs = sum P (I - m),
 // m = max I, s = sum exp(I - m), over the valid selected positions seen so far.
@@ -141,8 +157,9 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_empty[i], 2 * kRedWarps);           // both CTAs' reduction warps
       mbar_init(&S.idx_full[i], kStageWarps);
-      // readers of the staged positions: loaders, reduction warps, and the leader's loss warps
-      mbar_init(&S.idx_empty[i], kLoadWarps + kRedWarps + (leader ? kLossWarps : 0));
+      // readers of the staged positions: loaders, reduction warps, and the leader's loss
+      // warps and MMA issuer
+      mbar_init(&S.idx_empty[i], kLoadWarps + kRedWarps + (leader ? kLossWarps + 1 : 0));
     }
     for (int i = 0; i < kRedSlots; ++i) {
       mbar_init(&S.red_full[i], kRedWarps);              // + kPeerBytes of transaction count
@@ -167,43 +184,49 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
 
   if (warp >= kLoadWarp0) {
     // ------------------------------------------------------------------ key loaders
-    // Per row: this CTA's Q planes (plane c from loader c % kLoadWarps), then for
-    // each tile its NC key chunks (this CTA's 64 keys x 64 columns).  Chunk kc goes
-    // to ring slot kc % kStages, which loader warp kc % kStages owns; lanes 0-15
-    // issue its 16 four-row gathers.  Both CTAs' loads complete on the leader's
-    // barriers.
+    // Per row with tiles: this CTA's Q planes (plane c from loader c % kLoadWarps),
+    // then for each tile its NC key chunks (this CTA's 64 keys x 64 columns).  Chunk
+    // kc goes to ring slot kc % kStages; the team of kTeamWarps warps that owns that
+    // slot splits its 16 four-row gathers (groups g = part, part + kTeamWarps, ...).
+    // Both CTAs' loads complete on the leader's barriers.
     const int pw = (int)warp - kLoadWarp0;
-    uint32_t ucount = 0, kc = 0;
+    const uint32_t my_team = (uint32_t)(pw / kTeamWarps);
+    const int part = pw % kTeamWarps;
+    uint32_t ucount = 0, qcount = 0, kc = 0;
     if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
     for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
       const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
-      if (lane == 0) {
-        const int qrow = row * p.H + (int)rank * 64;
-        for (int c = pw; c < NC && ok; c += kLoadWarps) {
-          ok = mbar_wait(&S.q_empty[c], (ucount & 1u) ^ 1u, abort_flag);
-          if (!ok) break;
-          if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane);
-          tma_load_2d_pair(q_sm + c * kPlane, &tmap_q, mapa_shared(smem_u32(&S.q_full[c]), 0), c * 64, qrow);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
+      const int nt = row_tiles(S.last_word, ib);
+      if (nt > 0) {
+        if (lane == 0) {
+          const int qrow = row * p.H + (int)rank * 64;
+          for (int c = pw; c < NC && ok; c += kLoadWarps) {
+            ok = mbar_wait(&S.q_empty[c], (qcount & 1u) ^ 1u, abort_flag);
+            if (!ok) break;
+            if (leader) mbar_arrive_expect_tx(&S.q_full[c], 2u * kPlane);
+            tma_load_2d_pair(q_sm + c * kPlane, &tmap_q, mapa_shared(smem_u32(&S.q_full[c]), 0), c * 64, qrow);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ++qcount;
+      }
       const int32_t* idx = idx_sm + ib * kMaxIdx;
-      for (int j = 0; j < p.n_tiles && ok; ++j) {
+      for (int j = 0; j < nt && ok; ++j) {
         for (int c = 0; c < NC; ++c, ++kc) {
           const uint32_t st = kc % kStages, ph = (kc / kStages) & 1u;
-          if ((int)st != pw) continue;
+          if (st / kTeamSlots != my_team) continue;
           bool w_ok = true;
           if (lane == 0) {
             w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
-            if (w_ok && leader) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane);
+            if (w_ok && leader && part == 0) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane);
           }
           if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-          if (lane < kHalfKeys / 4) {
-            const int base = j * kTileKeys + (int)rank * kHalfKeys + (int)lane * 4;
-            tma_gather4_pair(k_sm + st * kPlane + lane * 512, &tmap_kv, mapa_shared(smem_u32(&S.k_full[st]), 0),
+          const int g = part + kTeamWarps * (int)lane;             // 4-key group of this lane
+          if (g < kHalfKeys / 4) {
+            const int base = j * kTileKeys + (int)rank * kHalfKeys + g * 4;
+            tma_gather4_pair(k_sm + st * kPlane + g * 512, &tmap_kv, mapa_shared(smem_u32(&S.k_full[st]), 0),
                              c * 64, gather_row(idx, base + 0), gather_row(idx, base + 1),
                              gather_row(idx, base + 2), gather_row(idx, base + 3));
           }
@@ -225,6 +248,7 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       ok = mbar_wait_warp(&S.idx_empty[buf], ph ^ 1u, abort_flag);
       if (!ok) break;
       const int b = row / p.Lq;
+      int last = -1;
       int32_t* dst = idx_sm + buf * kMaxIdx;
       const int32_t* src = p.indices + (size_t)row * p.k;
       for (int w0 = sw; w0 < nwords; w0 += kStageWarps * kStageBatch) {
@@ -243,8 +267,10 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
           dst[w * 32 + (int)lane] = valid ? grow : (int)((uint32_t)grow | 0x80000000u);
           const uint32_t bal = __ballot_sync(0xffffffffu, valid);
           if (lane == 0) S.valid_mask[buf][w] = bal;
+          if (bal) last = w;                          // words are visited in increasing order
         }
       }
+      if (lane == 0) S.last_word[buf][sw] = last;
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.idx_full[buf]);
     }
@@ -256,16 +282,20 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       constexpr uint32_t idesc = make_idesc(1, 1, 128, kTileKeys, 0, 0);   // bf16, K-major x K-major
       const uint64_t q_desc = make_smem_desc(smem_u32(q_sm), 16, 1024, LAYOUT_SW128);
       const uint64_t k_desc = make_smem_desc(smem_u32(k_sm), 16, 1024, LAYOUT_SW128);
-      uint32_t ucount = 0, kc = 0, sc = 0;
+      uint32_t ucount = 0, qcount = 0, kc = 0, sc = 0;
       for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
-        for (int j = 0; j < p.n_tiles && ok; ++j, ++sc) {
+        const uint32_t ib = ucount & 1u;
+        ok = mbar_wait(&S.idx_full[ib], (ucount >> 1) & 1u, abort_flag);
+        if (!ok) break;
+        const int nt = row_tiles(S.last_word, ib);
+        for (int j = 0; j < nt && ok; ++j, ++sc) {
           const uint32_t sb = sc & 1u;
           ok = mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag, true);
           if (!ok) break;
           tc_fence_after();
           const uint32_t d = tmem_base + sb * kHalfKeys;
           for (int c = 0; c < NC; ++c, ++kc) {
-            if (j == 0 && !mbar_wait(&S.q_full[c], ucount & 1u, abort_flag)) { ok = false; break; }
+            if (j == 0 && !mbar_wait(&S.q_full[c], qcount & 1u, abort_flag)) { ok = false; break; }
             const uint32_t st = kc % kStages, ph = (kc / kStages) & 1u;
             if (!mbar_wait(&S.k_full[st], ph, abort_flag)) { ok = false; break; }
             tc_fence_after();
@@ -276,11 +306,13 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
             mma_bf16_ss_pair(d, ad + 4, bd + 4, idesc, 1u);
             mma_bf16_ss_pair(d, ad + 6, bd + 6, idesc, 1u);
             mma_commit_pair_mc(&S.k_empty[st], kBoth);
-            if (j == p.n_tiles - 1) mma_commit_pair_mc(&S.q_empty[c], kBoth);   // plane free for the next row
+            if (j == nt - 1) mma_commit_pair_mc(&S.q_empty[c], kBoth);   // plane free for the next row
           }
           if (!ok) break;
           mma_commit_pair_mc(&S.s_full[sb], kBoth);
         }
+        if (nt > 0) ++qcount;
+        mbar_arrive(&S.idx_empty[ib]);
       }
       // Every MMA this thread issued completes before the TMEM is released.
       mma_commit(&S.final_mma);
@@ -305,10 +337,11 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
+      const int nt = row_tiles(S.last_word, ib);
       // exponent offset: a_h[s] = 2^(z * scale * log2 e - lse * log2 e)
-      const float nl = head_ok ? -p.lse[(size_t)row * p.H + head] * kLog2e : 0.f;
+      const float nl = (head_ok && nt > 0) ? -p.lse[(size_t)row * p.H + head] * kLog2e : 0.f;
       const float2 nl2 = make_float2(nl, nl);
-      for (int j = 0; j < p.n_tiles && ok; ++j, ++sc) {
+      for (int j = 0; j < nt && ok; ++j, ++sc) {
         const uint32_t sb = sc & 1u;
         ok = mbar_wait_warp(&S.s_full[sb], (sc >> 1) & 1u, abort_flag);
         if (!ok) break;
@@ -371,6 +404,7 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
       const int32_t* idx = idx_sm + ib * kMaxIdx;
+      const int nt = row_tiles(S.last_word, ib);
       const int bLk = (row / p.Lq) * p.Lk;
       const float* srow = p.scores + (size_t)row * p.Lk;
       float* trow = p.target ? p.target + (size_t)row * p.k : nullptr;
@@ -379,7 +413,7 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       // row's tiles); fetched four tiles before it is used, so that its DRAM latency
       // stays off the chain.
       auto fetch = [&](int j) -> float {
-        if (j >= p.n_tiles) return 0.f;
+        if (j >= nt) return 0.f;
         const int32_t gr = idx[j * kTileKeys + key];
         return gr >= 0 ? __ldg(srow + (gr - bLk)) : 0.f;
       };
@@ -412,12 +446,12 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
         return true;
       };
       float iv0 = fetch(0), iv1 = fetch(1), iv2 = fetch(2), iv3 = fetch(3);
-      for (int j = 0; j < p.n_tiles && ok; j += 4) {
+      for (int j = 0; j < nt && ok; j += 4) {
         ok = consume(j, iv0);
         iv0 = fetch(j + 4);
-        if (ok && j + 1 < p.n_tiles) { ok = consume(j + 1, iv1); iv1 = fetch(j + 5); }
-        if (ok && j + 2 < p.n_tiles) { ok = consume(j + 2, iv2); iv2 = fetch(j + 6); }
-        if (ok && j + 3 < p.n_tiles) { ok = consume(j + 3, iv3); iv3 = fetch(j + 7); }
+        if (ok && j + 1 < nt) { ok = consume(j + 1, iv1); iv1 = fetch(j + 5); }
+        if (ok && j + 2 < nt) { ok = consume(j + 2, iv2); iv2 = fetch(j + 6); }
+        if (ok && j + 3 < nt) { ok = consume(j + 3, iv3); iv3 = fetch(j + 7); }
       }
       if (!ok) break;
       // ---- end of the row: combine the loss warps' sums into KL and normalise the target
@@ -449,20 +483,24 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       // KL = sum p log p - sum p (I - lse_I) with p = P / Z:
       //    = (A - Bs) / Z - log Z + log s    (lse_I = m + log s; Bs is relative to m)
       if (lw == 0 && lane == 0) p.kl[row] = r.Z > 0.f ? (r.A - r.Bs) / r.Z - logf(r.Z) + logf(r.s) : 0.f;
-      if (trow && r.Z > 0.f) {
-        // all of this thread's loads first, then the stores: one round trip per row
-        const float inv = 1.f / r.Z;
-        constexpr int kPer = kMaxIdx / kTileKeys;
-        float t[kPer];
+      if (trow) {
+        // loads in batches of eight, then their stores: two round trips per row;
+        // slots past the processed tiles are padding and get 0
+        const float inv = r.Z > 0.f ? 1.f / r.Z : 0.f;
+        const int done = nt * kTileKeys;
+        constexpr int kBatch = 8;
+        for (int i0 = 0; i0 < kMaxIdx / kTileKeys; i0 += kBatch) {
+          float t[kBatch];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-          const int x = key + i * kTileKeys;
-          t[i] = x < p.k ? trow[x] : 0.f;
-        }
+          for (int i = 0; i < kBatch; ++i) {
+            const int x = key + (i0 + i) * kTileKeys;
+            t[i] = (x < p.k && x < done) ? trow[x] : 0.f;
+          }
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-          const int x = key + i * kTileKeys;
-          if (x < p.k) trow[x] = t[i] * inv;
+          for (int i = 0; i < kBatch; ++i) {
+            const int x = key + (i0 + i) * kTileKeys;
+            if (x < p.k) trow[x] = t[i] * inv;
+          }
         }
       }
     }
