@@ -213,10 +213,14 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
         ++qcount;
       }
       const int32_t* idx = idx_sm + ib * kMaxIdx;
-      for (int j = 0; j < nt && ok; ++j) {
-        for (int c = 0; c < NC; ++c, ++kc) {
+      // This row's chunks are kc0 .. kc0 + nt*NC - 1; visit only the team's slots.
+      const uint32_t kc0 = kc, kc_end = kc0 + (uint32_t)(nt * NC);
+      while (kc < kc_end && (kc % kStages) / kTeamSlots != my_team) ++kc;
+      for (; kc < kc_end && ok;
+           kc += ((kc % kTeamSlots) == kTeamSlots - 1) ? (uint32_t)(kStages - kTeamSlots + 1) : 1u) {
+        {
           const uint32_t st = kc % kStages, ph = (kc / kStages) & 1u;
-          if (st / kTeamSlots != my_team) continue;
+          const int j = (int)((kc - kc0) / NC), c = (int)((kc - kc0) % NC);
           bool w_ok = true;
           if (lane == 0) {
             w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
@@ -232,6 +236,7 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
           }
         }
       }
+      kc = kc_end;                                     // every warp's count moves past the row
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
     }
@@ -354,11 +359,20 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
         if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
         const uint32_t vm = head_ok ? S.valid_mask[ib][(j * kTileKeys + kk0) >> 5] : 0u;
         float pr[32];
+        if (vm == 0xffffffffu) {                       // warp-uniform: every key valid
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scl, nl2);
-          pr[e] = ((vm >> e) & 1u) ? ex2_approx(x.x) : 0.f;
-          pr[e + 1] = ((vm >> (e + 1)) & 1u) ? ex2_approx(x.y) : 0.f;
+          for (int e = 0; e < 32; e += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scl, nl2);
+            pr[e] = ex2_approx(x.x);
+            pr[e + 1] = ex2_approx(x.y);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scl, nl2);
+            pr[e] = ((vm >> e) & 1u) ? ex2_approx(x.x) : 0.f;
+            pr[e + 1] = ((vm >> (e + 1)) & 1u) ? ex2_approx(x.y) : 0.f;
+          }
         }
         // Butterfly transpose-reduction over the warp's 32 heads: at each step a lane
         // keeps the half of its columns selected by one bit of its lane number and
