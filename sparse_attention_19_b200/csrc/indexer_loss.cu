@@ -21,7 +21,7 @@
 //     order, so each chunk's 16 gathers are split over a team of four warps.
 //   * Keys come in tiles of 128 selected positions; S = Q K^T is one pair-MMA
 //     chain (M = 128 heads, N = 128 keys, K = 16 per instruction) issued by one
-//     thread of the leader CTA, double-buffered in TMEM.  Each CTA's TMEM holds
+//     thread of the leader CTA, into four S buffers in TMEM.  Each CTA's TMEM holds
 //     its 64 heads: lanes 0-63 keys 0-63 of the tile, lanes 64-127 keys 64-127.
 //   * Eight reduction warps per CTA read S: warp w holds TMEM lane quarter w % 4
 //     (32 heads, one key half) for 32 of the half's 64 keys.  Each lane turns its
@@ -75,13 +75,14 @@ constexpr int kStageBatch = 8;         // index words in flight per staging warp
 constexpr int kMaxIdx = 2048;
 constexpr int kMaxChunks = 9;
 constexpr uint32_t kPlane = 64 * 128;  // 64 rows x 128 B (Q plane, key chunk)
-constexpr uint32_t kTmemCols = 128;    // two S buffers of 64 columns
+constexpr int kSBufs = 4;              // S buffers in TMEM (64 columns each per CTA)
+constexpr uint32_t kTmemCols = kSBufs * 64;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct KlShared {
   uint64_t q_full[kMaxChunks], q_empty[kMaxChunks];
   uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[kSBufs], s_empty[kSBufs];
   uint64_t idx_full[2], idx_empty[2];
   uint64_t red_full[kRedSlots];          // leader: its reduction warps + the other CTA's bytes
   uint64_t red_empty[kRedSlots];         // both CTAs: the leader's loss warps
@@ -153,9 +154,11 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMaxChunks; ++i) { mbar_init(&S.q_full[i], 1); mbar_init(&S.q_empty[i], 1); }
     for (int i = 0; i < kStages; ++i) { mbar_init(&S.k_full[i], 1); mbar_init(&S.k_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_empty[i], 2 * kRedWarps);           // both CTAs' reduction warps
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&S.idx_full[i], kStageWarps);
       // readers of the staged positions: loaders, reduction warps, and the leader's loss
       // warps and MMA issuer
@@ -294,8 +297,8 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
         if (!ok) break;
         const int nt = row_tiles(S.last_word, ib);
         for (int j = 0; j < nt && ok; ++j, ++sc) {
-          const uint32_t sb = sc & 1u;
-          ok = mbar_wait(&S.s_empty[sb], ((sc >> 1) & 1u) ^ 1u, abort_flag, true);
+          const uint32_t sb = sc % kSBufs;
+          ok = mbar_wait(&S.s_empty[sb], ((sc / kSBufs) & 1u) ^ 1u, abort_flag, true);
           if (!ok) break;
           tc_fence_after();
           const uint32_t d = tmem_base + sb * kHalfKeys;
@@ -347,8 +350,8 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       const float nl = (head_ok && nt > 0) ? -p.lse[(size_t)row * p.H + head] * kLog2e : 0.f;
       const float2 nl2 = make_float2(nl, nl);
       for (int j = 0; j < nt && ok; ++j, ++sc) {
-        const uint32_t sb = sc & 1u;
-        ok = mbar_wait_warp(&S.s_full[sb], (sc >> 1) & 1u, abort_flag);
+        const uint32_t sb = sc % kSBufs;
+        ok = mbar_wait_warp(&S.s_full[sb], (sc / kSBufs) & 1u, abort_flag);
         if (!ok) break;
         tc_fence_after();
         uint32_t v[32];
