@@ -111,3 +111,33 @@ def test_two_gloo_ranks_gather_the_key_side_and_split_the_work():
         sl = slice(c * chunk, (c + 1) * chunk)
         assert np.array_equal(per_chunk[c][0], whole["indices"][sl])
         assert np.array_equal(per_chunk[c][1], whole["out"][sl])
+
+
+def _gather_only(rank, world, port, n_chunks, chunk, q):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        full, _ = _key_side(n_chunks * chunk, seed=7)
+        local = cp.local_key_side(full, cp.zigzag_chunks(n_chunks, world, rank), chunk)
+        keys = cp.gather_key_side(local, n_chunks, chunk, world, rank)
+        q.put((rank, all(torch.equal(keys[f], full[f]) for f in cp.KEY_FIELDS)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_four_gloo_ranks_two_rounds_gather_the_whole_sequence():
+    world, n_chunks, chunk = 4, 16, 16
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_only, args=(r, world, port, n_chunks, chunk, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=300) for _ in range(world))
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert res == {r: True for r in range(world)}
