@@ -406,6 +406,35 @@ def time_indexer_kl(wl, runner, steps, warmup, world, peaks, peak_src):
             "kl_mean": float(kl.mean())}
 
 
+def cpu_baseline_kl(wl, runner, budget_s=8.0):
+    """The oracle's indexer loss on rows spread evenly over the workload (host cores),
+    on the step's own scores, selection and lse inputs."""
+    import oracle
+    cores = oracle.num_threads()
+    _, qs = runner.chunks[0]
+    B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
+    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B * Lq, Lk)
+    kv = runner.keys["kv"].cpu().view(torch.int16).numpy().view(np.uint16)
+
+    def sample(n):
+        rows = np.unique(np.linspace(0, B * Lq - 1, n).astype(np.int64))
+        sel = torch.as_tensor(rows, device=runner.device)
+        q = qs["q"].reshape(B * Lq, wl.H, wl.D)[sel].cpu().view(torch.int16).numpy().view(np.uint16)
+        idx = runner.indices.reshape(B * Lq, k)[sel].cpu().numpy()
+        sc = scores[sel].double().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.indexer_kl(rows // Lq, q, kv, idx, sc, wl.scale)
+        return len(rows), time.perf_counter() - t0
+
+    n, dt = sample(max(cores, 4))
+    n_target = int(min(16 * cores, max(n, n * budget_s / max(dt, 1e-3))))
+    if n_target > n * 1.5:
+        n, dt = sample(n_target)
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} query rows spread evenly over the {wl.name} workload (the loss of each row "
+                      f"over its selected positions), {dt:.1f} s on {cores} threads"}
+
+
 # ------------------------------------------------------------------------------------ CPU oracle
 
 def oracle_sample(wl, inp_dev_or_host, n_rows, seed=0):
@@ -544,6 +573,8 @@ def main():
     if not args.no_extra or args.loss:
         kl_line = time_indexer_kl(wl, runner, max(3, args.steps // 2), args.warmup, world, peaks, peak_src)
         if kl_line is not None:
+            if rank == 0 and world == 1 and not args.no_cpu:
+                kl_line["cpu_baseline"] = cpu_baseline_kl(wl, runner)
             extra["indexer_kl_loss"] = kl_line
         line["workloads"] = extra
     if not args.no_extra:
