@@ -104,11 +104,12 @@ def test_kl_vanishes_when_the_scores_reproduce_the_target():
     assert float(kl.abs().max()) <= 2e-5
 
 
-def test_kl_prefill_8k_forward_sampled_rows():
-    # The loss on the forward pass's own outputs at the 8K prefill size: the
-    # indexer scores, the selection and the lse all come from dsa_forward; the
-    # launch is the one the benchmark times for the loss.
-    wl = WORKLOADS["prefill_8k"]
+@pytest.mark.parametrize("name", ["prefill_8k", "prefill_32k"])
+def test_kl_prefill_forward_sampled_rows(name):
+    # The loss on the forward pass's own outputs at the 8K and 32K prefill sizes
+    # (32K is the launch the benchmark times): the indexer scores, the selection
+    # and the lse come from the library's own stages.
+    wl = WORKLOADS[name]
     inp = {k_: v.to(DEV) for k_, v in make_inputs(wl, "cpu", 0).items()}
     scores = dsa.indexer_scores(inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], wl.q_offset)
     idx = dsa.topk(scores, wl.k, wl.q_offset)
