@@ -220,18 +220,22 @@ class Runner:
         self.work = [work_model(wl, chunk, q0) for q0, _ in self.chunks]
 
     def step(self, stream, events=None):
+        self.forward_into(stream, self.chunks, self.keys, self.indices, self.out, self.lse, events)
+
+    def forward_into(self, stream, chunks, keys, indices, out, lse, events=None):
+        """One forward pass over the given device buffers (the runner's own, or another set)."""
         wl, c = self.wl, self.chunk_len
-        for n, (q_offset, qs) in enumerate(self.chunks):
+        for n, (q_offset, qs) in enumerate(chunks):
             Lk = q_offset + c
             sl = slice(n * c, (n + 1) * c) if wl.chunk else slice(None)
-            k_I = self.keys["k_I"][:, :Lk] if wl.chunk else self.keys["k_I"]
-            k_scale = self.keys["k_scale"][:, :Lk] if wl.chunk else self.keys["k_scale"]
-            kv = self.keys["kv"][:, :Lk] if wl.chunk else self.keys["kv"]
+            k_I = keys["k_I"][:, :Lk] if wl.chunk else keys["k_I"]
+            k_scale = keys["k_scale"][:, :Lk] if wl.chunk else keys["k_scale"]
+            kv = keys["kv"][:, :Lk] if wl.chunk else keys["kv"]
             if wl.chunk:   # a chunk's key side is a prefix of the whole sequence (contiguous when B == 1)
                 assert wl.B == 1
             self.dsa.forward(qs["q_I"], qs["q_scale"], qs["w"], k_I.contiguous() if wl.B > 1 else k_I,
                              k_scale, qs["q"], kv, wl.k, wl.Dv, wl.scale, q_offset,
-                             indices=self.indices[:, sl], out=self.out[:, sl], lse=self.lse[:, sl],
+                             indices=indices[:, sl], out=out[:, sl], lse=lse[:, sl],
                              workspace=self.ws, stream=stream,
                              stage_events=None if events is None else events[n])
 
@@ -323,116 +327,77 @@ def traffic_from_profiles(kernel_name, workload):
 
 
 def measure_e2e(wl, runner, steps, warmup, world):
-    """Public API with pinned host buffers: H2D inputs + forward + D2H outputs each step."""
-    stream = torch.cuda.current_stream()
-    host_in = []
-    for q_offset, qs in runner.chunks:
-        host_in.append({k: v.cpu().pin_memory() for k, v in qs.items()})
+    """Public API with pinned host buffers: every step copies its inputs host -> device
+    and its outputs (indices, out, lse) device -> host inside the timed region.
+
+    Steps are pipelined the way a caller of the API would run them: two device
+    buffer sets, the input copies on one stream, the forward on another, the output
+    copies on a third, so step i+1's inputs and step i-1's outputs cross PCIe while
+    step i's kernels run.  The timed region starts before the first input copy and
+    ends after the last output copy.
+    """
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    host_in = [{k: v.cpu().pin_memory() for k, v in qs.items()} for _, qs in runner.chunks]
     host_keys = {k: v.cpu().pin_memory() for k, v in runner.keys.items()}
-    h_idx = torch.empty(runner.indices.shape, dtype=torch.int32).pin_memory()
-    h_out = torch.empty(runner.out.shape, dtype=torch.bfloat16).pin_memory()
-    h_lse = torch.empty(runner.lse.shape, dtype=torch.float32).pin_memory()
+    own = {"chunks": runner.chunks, "keys": runner.keys, "indices": runner.indices, "out": runner.out,
+           "lse": runner.lse}
+    other = {"chunks": [(q0, {k: torch.empty_like(v) for k, v in qs.items()}) for q0, qs in runner.chunks],
+             "keys": {k: torch.empty_like(v) for k, v in runner.keys.items()},
+             "indices": torch.empty_like(runner.indices), "out": torch.empty_like(runner.out),
+             "lse": torch.empty_like(runner.lse)}
+    slots = [own, other]
+    host_out = [{f: torch.empty(getattr(runner, f).shape, dtype=getattr(runner, f).dtype).pin_memory()
+                 for f in ("indices", "out", "lse")} for _ in range(2)]
     bi = sum(v.numel() * v.element_size() for v in host_keys.values())
     bi += sum(v.numel() * v.element_size() for d in host_in for v in d.values())
-    bo = sum(t.numel() * t.element_size() for t in (h_idx, h_out, h_lse))
+    bo = sum(t.numel() * t.element_size() for t in host_out[0].values())
 
-    def one():
-        for k, v in host_keys.items():
-            runner.keys[k].copy_(v, non_blocking=True)
-        for (q_offset, qs), hd in zip(runner.chunks, host_in):
-            for k, v in hd.items():
-                qs[k].copy_(v, non_blocking=True)
-        runner.step(stream)
-        h_idx.copy_(runner.indices, non_blocking=True)
-        h_out.copy_(runner.out, non_blocking=True)
-        h_lse.copy_(runner.lse, non_blocking=True)
+    def run(n_steps, start_event):
+        comp_done, out_done = [], []
+        s_in.wait_event(start_event)
+        for i in range(n_steps):
+            sl, ho = slots[i % 2], host_out[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[i - 2])           # the slot's inputs are free
+                for k, v in host_keys.items():
+                    sl["keys"][k].copy_(v, non_blocking=True)
+                for (_, qs), hd in zip(sl["chunks"], host_in):
+                    for k, v in hd.items():
+                        qs[k].copy_(v, non_blocking=True)
+                in_done = torch.cuda.Event()
+                in_done.record(s_in)
+            comp.wait_event(in_done)
+            if i >= 2:
+                comp.wait_event(out_done[i - 2])                # the slot's outputs were read back
+            runner.forward_into(comp, sl["chunks"], sl["keys"], sl["indices"], sl["out"], sl["lse"])
+            ev = torch.cuda.Event()
+            ev.record(comp)
+            comp_done.append(ev)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev)
+                for f in ("indices", "out", "lse"):
+                    ho[f].copy_(sl[f], non_blocking=True)
+                ev_o = torch.cuda.Event()
+                ev_o.record(s_out)
+                out_done.append(ev_o)
+        comp.wait_event(out_done[-1])
 
-    for _ in range(warmup):
-        one()
+    first = torch.cuda.Event()
+    first.record(comp)
+    run(warmup, first)
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(steps):
-        one()
-    e.record(stream)
+    s.record(comp)
+    run(steps, s)
+    e.record(comp)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e) / steps, world)
+    del other, slots
     return ms, bi, bo
-
-
-def time_indexer_kl(wl, runner, steps, warmup, world, peaks, peak_src):
-    """The indexer's training loss (forward) on the step's own outputs: the scores the
-    forward left in its workspace, its selection and its lse.  One launch per call."""
-    dsa = runner.dsa
-    if wl.chunk or len(runner.chunks) != 1 or wl.q_offset + wl.Lq <= wl.k:
-        return None                       # needs the scores of a single indexer call
-    _, qs = runner.chunks[0]
-    B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
-    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B, Lq, Lk)
-    target = torch.empty(B, Lq, k, dtype=torch.float32, device=runner.device)
-    kl = torch.empty(B, Lq, dtype=torch.float32, device=runner.device)
-    stream = torch.cuda.current_stream()
-
-    def call():
-        dsa.indexer_kl_loss(qs["q"], runner.keys["kv"], runner.indices, runner.lse, scores, wl.Dv, wl.scale,
-                            target=target, kl=kl, stream=stream)
-
-    for _ in range(warmup):
-        call()
-    torch.cuda.synchronize()
-    barrier(world)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(steps):
-        call()
-    e.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    ms = max_over_ranks(s.elapsed_time(e) / steps, world)
-    tot = runner.totals()
-    # S = q . c over every (selected pair, head); gathered latent rows as the bytes
-    flops = 2.0 * tot["selected_pairs"] * wl.H * wl.D
-    achieved = flops / (ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"]
-    return {"workload": wl.name, "value": tot["rows"] * world / (ms * 1e-3), "unit": "tokens/s",
-            "ms_per_step": ms, "steps": steps, "warmup": warmup, "gpu_launches": steps,
-            "roofline": {"kernel": "indexer_kl_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "per_launch_algorithmic": flops,
-                         "peak_source": f"{peak_src} burst bf16 (MEASURED_PEAKS.json)",
-                         "gathered_gb": tot["selected_pairs"] * wl.D * 2 / 1e9,
-                         "traffic": traffic_from_profiles("indexer_kl_kernel", wl.name)},
-            "kl_mean": float(kl.mean())}
-
-
-def cpu_baseline_kl(wl, runner, budget_s=8.0):
-    """The oracle's indexer loss on rows spread evenly over the workload (host cores),
-    on the step's own scores, selection and lse inputs."""
-    import oracle
-    cores = oracle.num_threads()
-    _, qs = runner.chunks[0]
-    B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
-    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B * Lq, Lk)
-    kv = runner.keys["kv"].cpu().view(torch.int16).numpy().view(np.uint16)
-
-    def sample(n):
-        rows = np.unique(np.linspace(0, B * Lq - 1, n).astype(np.int64))
-        sel = torch.as_tensor(rows, device=runner.device)
-        q = qs["q"].reshape(B * Lq, wl.H, wl.D)[sel].cpu().view(torch.int16).numpy().view(np.uint16)
-        idx = runner.indices.reshape(B * Lq, k)[sel].cpu().numpy()
-        sc = scores[sel].double().cpu().numpy()
-        t0 = time.perf_counter()
-        oracle.indexer_kl(rows // Lq, q, kv, idx, sc, wl.scale)
-        return len(rows), time.perf_counter() - t0
-
-    n, dt = sample(max(cores, 4))
-    n_target = int(min(16 * cores, max(n, n * budget_s / max(dt, 1e-3))))
-    if n_target > n * 1.5:
-        n, dt = sample(n_target)
-    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} query rows spread evenly over the {wl.name} workload (the loss of each row "
-                      f"over its selected positions), {dt:.1f} s on {cores} threads"}
 
 
 # ------------------------------------------------------------------------------------ CPU oracle
@@ -566,7 +531,7 @@ def main():
         wl_cpu = wl.with_(Lq=runner.chunk_len, q_offset=q_offset0) if wl.chunk else wl
         line["cpu_baseline"] = cpu_baseline(wl_cpu, inp)
     if not args.no_e2e:
-        e_ms, bi, bo = measure_e2e(wl, runner, max(2, min(args.steps, 5)), 1, world)
+        e_ms, bi, bo = measure_e2e(wl, runner, max(3, args.steps), 1, world)
         line["e2e"] = {"value": tokens / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
                        "d2h_bytes_per_step": bo, "ms_per_step": e_ms}
     extra = {}
