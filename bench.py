@@ -400,6 +400,79 @@ def measure_e2e(wl, runner, steps, warmup, world):
     return ms, bi, bo
 
 
+def time_indexer_kl(wl, runner, steps, warmup, world, peaks, peak_src):
+    """The indexer's training loss (forward) on the step's own outputs: the scores the
+    forward left in its workspace, its selection and its lse.  One launch per call."""
+    dsa = runner.dsa
+    if wl.chunk or len(runner.chunks) != 1 or wl.q_offset + wl.Lq <= wl.k:
+        return None                       # needs the scores of a single indexer call
+    _, qs = runner.chunks[0]
+    B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
+    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B, Lq, Lk)
+    target = torch.empty(B, Lq, k, dtype=torch.float32, device=runner.device)
+    kl = torch.empty(B, Lq, dtype=torch.float32, device=runner.device)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        dsa.indexer_kl_loss(qs["q"], runner.keys["kv"], runner.indices, runner.lse, scores, wl.Dv, wl.scale,
+                            target=target, kl=kl, stream=stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        call()
+    e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world)
+    tot = runner.totals()
+    # S = q . c over every (selected pair, head); gathered latent rows as the bytes
+    flops = 2.0 * tot["selected_pairs"] * wl.H * wl.D
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"workload": wl.name, "value": tot["rows"] * world / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": steps, "warmup": warmup, "gpu_launches": steps,
+            "roofline": {"kernel": "indexer_kl_kernel", "bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "per_launch_algorithmic": flops,
+                         "peak_source": f"{peak_src} burst bf16 (MEASURED_PEAKS.json)",
+                         "gathered_gb": tot["selected_pairs"] * wl.D * 2 / 1e9,
+                         "traffic": traffic_from_profiles("indexer_kl_kernel", wl.name)},
+            "kl_mean": float(kl.mean())}
+
+
+def cpu_baseline_kl(wl, runner, budget_s=8.0):
+    """The oracle's indexer loss on rows spread evenly over the workload (host cores),
+    on the step's own scores, selection and lse inputs."""
+    import oracle
+    cores = oracle.num_threads()
+    _, qs = runner.chunks[0]
+    B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
+    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B * Lq, Lk)
+    kv = runner.keys["kv"].cpu().view(torch.int16).numpy().view(np.uint16)
+
+    def sample(n):
+        rows = np.unique(np.linspace(0, B * Lq - 1, n).astype(np.int64))
+        sel = torch.as_tensor(rows, device=runner.device)
+        q = qs["q"].reshape(B * Lq, wl.H, wl.D)[sel].cpu().view(torch.int16).numpy().view(np.uint16)
+        idx = runner.indices.reshape(B * Lq, k)[sel].cpu().numpy()
+        sc = scores[sel].double().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.indexer_kl(rows // Lq, q, kv, idx, sc, wl.scale)
+        return len(rows), time.perf_counter() - t0
+
+    n, dt = sample(max(cores, 4))
+    n_target = int(min(16 * cores, max(n, n * budget_s / max(dt, 1e-3))))
+    if n_target > n * 1.5:
+        n, dt = sample(n_target)
+    return {"value": n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} query rows spread evenly over the {wl.name} workload (the loss of each row "
+                      f"over its selected positions), {dt:.1f} s on {cores} threads"}
+
+
 # ------------------------------------------------------------------------------------ CPU oracle
 
 def oracle_sample(wl, inp_dev_or_host, n_rows, seed=0):
