@@ -122,3 +122,16 @@ def test_indexer_kl_loss_rejects_bad_arguments(L):
     assert f(ctypes.byref(good), 1, 1, 8, p, 0, p, p, None, p, None) == 2              # k < 1
     assert f(ctypes.byref(good), 1, 1, 8, p, 4096, p, p, None, p, None) == 2           # k > 2048
     assert f(ctypes.byref(dsa.AttnArgs(64, 576, 512, 0.07, 16, 16)), 1, 1, 8, p, 8, p, p, None, p, None) == 2
+
+
+def test_product_code_never_reaches_the_oracle():
+    # The oracle is test infrastructure: the package (binding, build script, kernels,
+    # C ABI) neither imports, loads nor includes anything from it.
+    pkg = os.path.join(ROOT, "sparse_attention_19_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if not f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                continue
+            text = open(os.path.join(dirpath, f)).read()
+            assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
+            assert "liboracle" not in text and "dsa_oracle" not in text, f
