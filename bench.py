@@ -60,6 +60,7 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--loss", action="store_true", help="time the indexer loss even with --no-extra")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-fp8-peak", action="store_true", help="skip measuring the FP8 GEMM peak")
     return ap.parse_args()
 
 
@@ -158,6 +159,53 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def measure_fp8_peak(device="cuda", n=8192, sustain_s=2.0):
+    """Dense FP8 (e4m3 x e4m3, fp32 accumulate) GEMM throughput of this GPU through
+    cuBLASLt (torch._scaled_mm), M = N = K = n, in TFLOP/s.
+
+    burst: the best of 10 single calls after warm-up (for a kernel timed alone);
+    sustained: back-to-back calls for about ``sustain_s`` seconds (for a kernel
+    timed inside a long step, under the power cap).  Both accumulation modes of
+    the library are tried and the faster is kept.  No clock or power setting is
+    touched."""
+    g = torch.Generator(device=device).manual_seed(1234)
+    a = torch.randn(n, n, device=device, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=device, generator=g).to(torch.float8_e4m3fn).t()   # column-major operand
+    one = torch.ones((), device=device, dtype=torch.float32)
+    flops = 2.0 * n ** 3
+    best_ms, mode = float("inf"), None
+    for fast in (False, True):
+        def mm():
+            return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16, use_fast_accum=fast)
+        for _ in range(3):
+            mm()
+        torch.cuda.synchronize()
+        for _ in range(10):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            mm()
+            e.record()
+            e.synchronize()
+            ms = s.elapsed_time(e)
+            if ms < best_ms:
+                best_ms, mode = ms, fast
+    def mm():
+        return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16, use_fast_accum=mode)
+    iters = max(10, int(sustain_s / (best_ms * 1e-3)))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(iters):
+        mm()
+    e.record()
+    e.synchronize()
+    sus_ms = s.elapsed_time(e) / iters
+    del a, b
+    torch.cuda.empty_cache()
+    return {"fp8_tflops": flops / (best_ms * 1e-3) / 1e12, "fp8_tflops_sustained": flops / (sus_ms * 1e-3) / 1e12,
+            "method": f"torch._scaled_mm e4m3 {n}^3 (cuBLASLt), use_fast_accum={mode}; burst = best of 10, "
+                      f"sustained = mean of {iters} back-to-back calls"}
+
+
 # ------------------------------------------------------------------------------------ work model
 
 def work_model(wl, Lq=None, q_offset=None):
@@ -173,11 +221,10 @@ def work_model(wl, Lq=None, q_offset=None):
         "rows": rows,
         "causal_pairs": causal,
         "selected_pairs": selected,
-        # indexer: one FP8 dot of width d_I per (pair, head); bytes: keys + scales read, scores written
+        # indexer with the top-k fused into it: one FP8 dot of width d_I per (pair, head);
+        # bytes: keys + scales and the query side read once, the selected indices written
         "indexer_flops": 2.0 * causal * wl.H_I * wl.d_I,
-        "indexer_bytes": wl.B * (q0 + Lq) * (wl.d_I + 4) + rows * wl.H_I * (wl.d_I + 2) + causal * 4.0,
-        # top-k: causal scores read once, indices written
-        "topk_bytes": causal * 4.0 + rows * wl.k * 4.0,
+        "indexer_bytes": wl.B * (q0 + Lq) * (wl.d_I + 4) + rows * wl.H_I * (wl.d_I + 2) + rows * wl.k * 4.0,
         # attention: S = q.c (d_qk) and O = p.v (d_v) per (selected pair, head)
         "attn_flops": 2.0 * selected * wl.H * (wl.D + wl.Dv),
         "attn_bytes": selected * wl.D * 2.0 + rows * wl.H * (wl.D + wl.Dv) * 2.0,
@@ -213,10 +260,14 @@ class Runner:
         self.out = torch.empty(B, wl.Lq, H, Dv, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(B, wl.Lq, H, dtype=torch.float32, device=device)
         ws = 0
-        for q_offset, _ in self.chunks:
-            ws = max(ws, dsa.workspace_size(dsa.OP_FORWARD, B, chunk, q_offset + chunk, k, H, Dv))
+        for q_offset, qs in self.chunks:
+            ia = dsa._indexer_args(qs["q_I"], qs["q_scale"], qs["w"], keys["k_I"][:, : q_offset + chunk],
+                                   keys["k_scale"][:, : q_offset + chunk], q_offset)
+            ws = max(ws, dsa.workspace_size_args(dsa.OP_FORWARD, ia, k, H, Dv))
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
-        self.launches_per_call = 3 + (1 if dsa.workspace_size(dsa.OP_SPARSE_ATTN, B, chunk, wl.Lk, k, H, Dv) else 0)
+        # per forward call: the fused indexer + top-k (or the index fill of a short
+        # sequence), the attention, and its split-k merge when rows are split
+        self.launches_per_call = 2 + (1 if dsa.workspace_size(dsa.OP_SPARSE_ATTN, B, chunk, wl.Lk, k, H, Dv) else 0)
         self.work = [work_model(wl, chunk, q0) for q0, _ in self.chunks]
 
     def step(self, stream, events=None):
@@ -270,6 +321,8 @@ def time_runner(runner, steps, warmup, world, sample_clocks, local):
         sampler.__exit__()
     barrier(world)
     total_ms = start.elapsed_time(end)
+    # spans: [0] indexer with the fused top-k, [1] the rest of the top-k step (0 when
+    # fused; the index fill of a short sequence), [2] attention + split-k merge
     stage_ms = [0.0, 0.0, 0.0]
     for s in range(steps):
         for c in range(nchunks):
@@ -282,21 +335,23 @@ def time_runner(runner, steps, warmup, world, sample_clocks, local):
 
 def roofline_stages(wl, runner, stage_ms, peaks, peak_src):
     tot = runner.totals()
-    fp8_burst = 2.0 * peaks["bf16_tflops"]
-    fp8_sust = 2.0 * peaks["bf16_tflops_sustained"]
+    if "fp8_tflops_sustained" in peaks:
+        fp8_sust = peaks["fp8_tflops_sustained"]
+        fp8_note = "measured sustained fp8 in this run (" + peaks["fp8_method"] + ")"
+    else:
+        fp8_sust = 2.0 * peaks["bf16_tflops_sustained"]
+        fp8_note = f"fp8 = 2 x {peak_src} sustained bf16 (nominal fp8:bf16 ratio)"
     decode = wl.Lq == 1
     calls = len(runner.chunks)
     out = {}
-    # indexer: FP8 contraction for prefill; streams the key cache for decode
+    # indexer + fused top-k: FP8 contraction for prefill; streams the key cache for decode
     if decode:
-        out["indexer"] = dict(bound="hbm", achieved=tot["indexer_bytes"] / (stage_ms[0] * 1e-3) / 1e9,
-                              peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["indexer_bytes"] / calls)
+        out["indexer_topk"] = dict(bound="hbm", achieved=tot["indexer_bytes"] / (stage_ms[0] * 1e-3) / 1e9,
+                                   peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["indexer_bytes"] / calls)
     else:
-        out["indexer"] = dict(bound="tensor", achieved=tot["indexer_flops"] / (stage_ms[0] * 1e-3) / 1e12,
-                              peak=fp8_sust, unit="TFLOP/s", algorithmic=tot["indexer_flops"] / calls,
-                              peak_note=f"fp8 = 2 x {peak_src} sustained bf16 (nominal fp8:bf16 ratio)")
-    out["topk"] = dict(bound="hbm", achieved=tot["topk_bytes"] / (stage_ms[1] * 1e-3) / 1e9,
-                       peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["topk_bytes"] / calls)
+        out["indexer_topk"] = dict(bound="tensor", achieved=tot["indexer_flops"] / (stage_ms[0] * 1e-3) / 1e12,
+                                   peak=fp8_sust, unit="TFLOP/s", algorithmic=tot["indexer_flops"] / calls,
+                                   peak_note=fp8_note)
     if decode:
         out["sparse_attn"] = dict(bound="hbm", achieved=tot["attn_bytes"] / (stage_ms[2] * 1e-3) / 1e9,
                                   peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["attn_bytes"] / calls,
@@ -305,14 +360,16 @@ def roofline_stages(wl, runner, stage_ms, peaks, peak_src):
         out["sparse_attn"] = dict(bound="tensor", achieved=tot["attn_flops"] / (stage_ms[2] * 1e-3) / 1e12,
                                   peak=peaks["bf16_tflops_sustained"], unit="TFLOP/s",
                                   algorithmic=tot["attn_flops"] / calls)
-    for name, ms in zip(("indexer", "topk", "sparse_attn"), stage_ms):
+    for name, ms in (("indexer_topk", stage_ms[0]), ("sparse_attn", stage_ms[2])):
         d = out[name]
         d["ms_per_step"] = ms
         d["frac"] = d["achieved"] / d["peak"]
         d["launches_per_step"] = calls
     total = sum(stage_ms)
-    for name, ms in zip(("indexer", "topk", "sparse_attn"), stage_ms):
+    for name, ms in (("indexer_topk", stage_ms[0]), ("sparse_attn", stage_ms[2])):
         out[name]["share"] = ms / total if total > 0 else None
+    # what is left of the top-k step once it is fused into the indexer (event gap)
+    out["topk_outside_indexer"] = {"ms_per_step": stage_ms[1], "share": stage_ms[1] / total if total > 0 else None}
     return out
 
 
@@ -400,22 +457,92 @@ def measure_e2e(wl, runner, steps, warmup, world):
     return ms, bi, bo
 
 
-def time_indexer_kl(wl, runner, steps, warmup, world, peaks, peak_src):
-    """The indexer's training loss (forward) on the step's own outputs: the scores the
-    forward left in its workspace, its selection and its lse.  One launch per call."""
+def time_dense_vs_gather(steps, warmup, world, peaks, seed=0):
+    """Short-sequence leg (L = k = 2048): the forward pass in its dense mode (keys
+    0..t read as contiguous tiles, index lists written by the attention kernel)
+    beside the gather path on the same input (dsa_sparse_attn over explicit index
+    lists 0..t, which gathers every key row through TMA gather4)."""
+    import sparse_attention_19_b200 as dsa
+    wl = WORKLOADS["prefill_2k"]
+    inp = make_inputs(wl, "cuda", seed)
+    stream = torch.cuda.current_stream()
+    idx = torch.empty(wl.B, wl.Lq, wl.k, dtype=torch.int32, device="cuda")
+    out = torch.empty(wl.B, wl.Lq, wl.H, wl.Dv, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(wl.B, wl.Lq, wl.H, dtype=torch.float32, device="cuda")
+    ws_f = torch.empty(max(256, dsa.workspace_size(dsa.OP_FORWARD, wl.B, wl.Lq, wl.Lk, wl.k, wl.H, wl.Dv)),
+                       dtype=torch.uint8, device="cuda")
+    ws_a = torch.empty(max(256, dsa.workspace_size(dsa.OP_SPARSE_ATTN, wl.B, wl.Lq, wl.Lk, wl.k, wl.H, wl.Dv)),
+                       dtype=torch.uint8, device="cuda")
+    g_idx = torch.empty_like(idx)
+    g_out, g_lse = torch.empty_like(out), torch.empty_like(lse)
+
+    def dense():
+        dsa.forward(inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], inp["q"], inp["kv"], wl.k,
+                    wl.Dv, wl.scale, 0, indices=idx, out=out, lse=lse, workspace=ws_f, stream=stream)
+
+    dense()
+    torch.cuda.synchronize()
+    g_idx.copy_(idx)                                   # 0..t, -1 padded
+
+    def gather():
+        dsa.sparse_attn(inp["q"], inp["kv"], g_idx, wl.Dv, wl.scale, out=g_out, lse=g_lse, workspace=ws_a,
+                        stream=stream)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(steps):
+            fn()
+        e.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(s.elapsed_time(e) / steps, world)
+
+    ms_d, ms_g = timed(dense), timed(gather)
+    tot = work_model(wl)
+    res = {}
+    for name, ms in (("dense", ms_d), ("gather", ms_g)):
+        tf = tot["attn_flops"] / (ms * 1e-3) / 1e12
+        res[name] = {"value": tot["rows"] * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+                     "attn_tflops": tf, "frac": tf / peaks["bf16_tflops"],
+                     "peak": peaks["bf16_tflops"], "peak_note": "burst bf16 (a kernel timed on its own)"}
+    res["speedup_dense_over_gather"] = ms_g / ms_d
+    res["same_result"] = bool(torch.equal(out, g_out) and torch.equal(lse, g_lse))
+    res["workload"] = wl.name
+    res["steps"] = steps
+    return res
+
+
+def selected_scores(runner):
+    """One more forward pass of the headline step that also returns the indexer
+    score of every selected position (fp32 [B, Lq, k]), for the loss leg."""
+    wl = runner.wl
+    sel = torch.empty(wl.B, wl.Lq, wl.k, dtype=torch.float32, device=runner.device)
+    q_offset, qs = runner.chunks[0]
+    runner.dsa.forward(qs["q_I"], qs["q_scale"], qs["w"], runner.keys["k_I"], runner.keys["k_scale"], qs["q"],
+                       runner.keys["kv"], wl.k, wl.Dv, wl.scale, q_offset, indices=runner.indices, out=runner.out,
+                       lse=runner.lse, workspace=runner.ws, sel_scores=sel)
+    torch.cuda.synchronize()
+    return sel
+
+
+def time_indexer_kl(wl, runner, steps, warmup, world, peaks, peak_src, sel):
+    """The indexer's training loss (forward) on the step's own outputs: its selection,
+    the selected positions' scores and its lse.  One launch per call."""
     dsa = runner.dsa
-    if wl.chunk or len(runner.chunks) != 1 or wl.q_offset + wl.Lq <= wl.k:
-        return None                       # needs the scores of a single indexer call
     _, qs = runner.chunks[0]
-    B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
-    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B, Lq, Lk)
+    B, Lq, k = wl.B, wl.Lq, wl.k
     target = torch.empty(B, Lq, k, dtype=torch.float32, device=runner.device)
     kl = torch.empty(B, Lq, dtype=torch.float32, device=runner.device)
     stream = torch.cuda.current_stream()
 
     def call():
-        dsa.indexer_kl_loss(qs["q"], runner.keys["kv"], runner.indices, runner.lse, scores, wl.Dv, wl.scale,
-                            target=target, kl=kl, stream=stream)
+        dsa.indexer_kl_loss_selected(qs["q"], runner.keys["kv"], runner.indices, runner.lse, sel, wl.Dv, wl.scale,
+                                     target=target, kl=kl, stream=stream)
 
     for _ in range(warmup):
         call()
@@ -444,14 +571,13 @@ def time_indexer_kl(wl, runner, steps, warmup, world, peaks, peak_src):
             "kl_mean": float(kl.mean())}
 
 
-def cpu_baseline_kl(wl, runner, budget_s=8.0):
+def cpu_baseline_kl(wl, runner, sel_scores, budget_s=8.0):
     """The oracle's indexer loss on rows spread evenly over the workload (host cores),
-    on the step's own scores, selection and lse inputs."""
+    on the step's own selection, selected scores and lse inputs."""
     import oracle
     cores = oracle.num_threads()
     _, qs = runner.chunks[0]
     B, Lq, Lk, k = wl.B, wl.Lq, wl.Lk, wl.k
-    scores = runner.ws[: B * Lq * Lk * 4].view(torch.float32).view(B * Lq, Lk)
     kv = runner.keys["kv"].cpu().view(torch.int16).numpy().view(np.uint16)
 
     def sample(n):
@@ -459,7 +585,12 @@ def cpu_baseline_kl(wl, runner, budget_s=8.0):
         sel = torch.as_tensor(rows, device=runner.device)
         q = qs["q"].reshape(B * Lq, wl.H, wl.D)[sel].cpu().view(torch.int16).numpy().view(np.uint16)
         idx = runner.indices.reshape(B * Lq, k)[sel].cpu().numpy()
-        sc = scores[sel].double().cpu().numpy()
+        # the oracle takes a row of scores over all positions; only the selected ones are read
+        ss = sel_scores.reshape(B * Lq, k)[sel].double().cpu().numpy()
+        sc = np.zeros((len(rows), Lk))
+        for j in range(len(rows)):
+            ok = idx[j] >= 0
+            sc[j, idx[j][ok]] = ss[j][ok]
         t0 = time.perf_counter()
         oracle.indexer_kl(rows // Lq, q, kv, idx, sc, wl.scale)
         return len(rows), time.perf_counter() - t0
@@ -542,7 +673,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(wl, "host cores (fp64 oracle)"),
+        "config": config_of(wl),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"each step: {n_rows} query rows spread evenly over {wl_eff.name} "
                                    f"(Lq={wl_eff.Lq}, q_offset={wl_eff.q_offset})"},
@@ -551,7 +682,8 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def config_of(wl, l2_note):
+def config_of(wl):
+    l2_note = "inputs larger than L2 (q alone is %.1f GB)" % (wl.B * wl.Lq * wl.H * wl.D * 2 / 1e9)
     return {"workload": wl.name, "B": wl.B, "Lq": wl.Lq, "Lk": wl.Lk, "q_offset": wl.q_offset,
             "chunk": wl.chunk or None, "k": wl.k, "H_I": wl.H_I, "d_I": wl.d_I, "H": wl.H, "d_qk": wl.D,
             "d_v": wl.Dv, "indexer": "fp8 e4m3, per-token fp32 scales", "attention": "bf16, fp32 accumulate",
@@ -571,6 +703,11 @@ def main():
         return
     import sparse_attention_19_b200 as dsa
     peaks, peak_src = load_peaks()
+    fp8 = None
+    if not args.no_fp8_peak:
+        fp8 = measure_fp8_peak()
+        peaks["fp8_tflops_sustained"] = fp8["fp8_tflops_sustained"]
+        peaks["fp8_method"] = fp8["method"]
     wl = WORKLOADS[args.workload]
     runner = Runner(wl, seed=args.seed + rank)
     ms, stage_ms, clocks = time_runner(runner, args.steps, args.warmup, world, rank == 0, local)
@@ -579,9 +716,9 @@ def main():
     tokens = tot["rows"] * world
     value = tokens / (ms_max * 1e-3)
     stages = roofline_stages(wl, runner, stage_ms, peaks, peak_src)
-    dom = max(stages, key=lambda n: stages[n]["ms_per_step"])
+    dom = max(("indexer_topk", "sparse_attn"), key=lambda n: stages[n]["ms_per_step"])
     d = stages[dom]
-    kernel_names = {"indexer": "indexer_kernel", "topk": "topk_kernel", "sparse_attn": "sparse_attn_kernel"}
+    kernel_names = {"indexer_topk": "indexer_kernel", "sparse_attn": "sparse_attn_kernel"}
     roof = {"kernel": kernel_names[dom], "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
             "unit": d["unit"], "frac": d["frac"],
             "traffic": traffic_from_profiles(kernel_names[dom], wl.name),
@@ -590,13 +727,15 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8+bf16 (fp32 accumulate)", "data": "synthetic",
-        "config": config_of(wl, "inputs larger than L2 (q alone is %.1f GB)" % (
-            wl.B * wl.Lq * wl.H * wl.D * 2 / 1e9)),
+        "config": config_of(wl),
         "roofline": roof,
         "stages": {k: {kk: (round(vv, 6) if isinstance(vv, float) else vv) for kk, vv in v.items()}
                    for k, v in stages.items()},
         "gpu_launches": runner.launches_per_call * len(runner.chunks) * args.steps,
         "clocks": clocks,
+        "peaks": {"source": f"{peak_src} (MEASURED_PEAKS.json)", "hbm_gbs": peaks["hbm_gbs"],
+                  "bf16_tflops": peaks["bf16_tflops"], "bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
+                  "fp8": fp8},
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         q_offset0, qs0 = runner.chunks[-1]
@@ -608,14 +747,16 @@ def main():
         line["e2e"] = {"value": tokens / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": bi,
                        "d2h_bytes_per_step": bo, "ms_per_step": e_ms}
     extra = {}
-    if not args.no_extra or args.loss:
-        kl_line = time_indexer_kl(wl, runner, max(3, args.steps // 2), args.warmup, world, peaks, peak_src)
-        if kl_line is not None:
-            if rank == 0 and world == 1 and not args.no_cpu:
-                kl_line["cpu_baseline"] = cpu_baseline_kl(wl, runner)
-            extra["indexer_kl_loss"] = kl_line
+    if (not args.no_extra or args.loss) and not wl.chunk and len(runner.chunks) == 1:
+        sel = selected_scores(runner)
+        kl_line = time_indexer_kl(wl, runner, max(3, args.steps // 2), args.warmup, world, peaks, peak_src, sel)
+        if rank == 0 and world == 1 and not args.no_cpu:
+            kl_line["cpu_baseline"] = cpu_baseline_kl(wl, runner, sel)
+        extra["indexer_kl_loss"] = kl_line
+        del sel
         line["workloads"] = extra
     if not args.no_extra:
+        extra["prefill_2k_dense_vs_gather"] = time_dense_vs_gather(max(5, args.steps), args.warmup, world, peaks)
         for name in ("decode_128k", "prefill_128k"):
             if name == wl.name:
                 continue

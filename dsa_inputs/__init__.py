@@ -87,6 +87,10 @@ WORKLOADS = {
         "decode_128k", B=64, Lq=1, Lk=131072, q_offset=131071, H_I=64, d_I=128, k=2048,
         H=128, D=576, Dv=512, scale=_SCALE,
         description="decode: 64 sequences x 131072 cached tokens, 1 new query each"),
+    "prefill_2k": Workload(
+        "prefill_2k", B=1, Lq=2048, Lk=2048, q_offset=0, H_I=64, d_I=128, k=2048,
+        H=128, D=576, Dv=512, scale=_SCALE,
+        description="short prefill L=2048 = k: every position selected (dense causal attention)"),
     "prefill_128k": Workload(
         "prefill_128k", B=1, Lq=131072, Lk=131072, q_offset=0, H_I=64, d_I=128, k=2048,
         H=128, D=576, Dv=512, scale=_SCALE, salient_frac=0.05, chunk=4096,

@@ -73,7 +73,8 @@ typedef struct {
 typedef enum {
     DSA_OP_TOPK = 0,
     DSA_OP_SPARSE_ATTN = 1,
-    DSA_OP_FORWARD = 2
+    DSA_OP_FORWARD = 2,
+    DSA_OP_INDEXER_TOPK = 3
 } dsa_op;
 
 /*
@@ -97,6 +98,23 @@ dsa_status dsa_indexer_scores(const dsa_indexer_args *args, float *scores, void 
  */
 dsa_status dsa_topk(const float *scores, int B, int Lq, int Lk, int q_offset, int k,
                     int32_t *indices, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Indexer and top-k fused: the k positions with the largest I[t,s] per row
+ * (equation for I_{t,s} of "Молниеносный индексатор", then the Top-k of the
+ * equation for u_t in "Отбор и основное внимание"), selected on chip as the
+ * scores are produced, so the [B, Lq, Lk] score matrix is never written.
+ *   indices:    int32 [B, Lq, k], exactly as dsa_topk would return for the scores
+ *               of dsa_indexer_scores (ties to the smaller position, -0.0 == +0.0,
+ *               ascending position order, -1 padding after min(k, t+1) slots);
+ *   sel_scores: fp32 [B, Lq, k] or NULL: I[t, indices[...]] for each valid slot,
+ *               -INFINITY on padding slots;
+ *   workspace:  dsa_workspace_size_args(DSA_OP_INDEXER_TOPK, args, k, 0, 0) bytes
+ *               (the per-row candidate lists; a few tens of MB, independent of Lk
+ *               for prefill).  Its contents need not be initialised.
+ */
+dsa_status dsa_indexer_topk(const dsa_indexer_args *args, int k, int32_t *indices, float *sel_scores,
+                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Sparse MQA attention over the selected latent rows (equation for u_t).
@@ -127,9 +145,15 @@ dsa_status dsa_sparse_attn(const dsa_attn_args *args, int B, int Lq, int Lk,
  * call allocates and frees nothing.  A call that needs more returns
  * DSA_ERR_WORKSPACE before launching anything.  Nothing in the array has to
  * start at zero: every partial is written before it is read.
- * The first call on each device looks the array's address up (which may make the
- * CUDA runtime load the library's device code); make that first call before any
- * stream capture begins.
+ * Memory: the array is device memory held by every device on which it has been
+ * looked up, until the process exits.  It sits in a module of its own, so with
+ * the CUDA runtime's default lazy module loading only callers of this entry
+ * point reserve it; with eager loading (CUDA_MODULE_LOADING=EAGER) every
+ * context that loads libdsa.so does.
+ * Set-up: the first call that needs the array in a CUDA context of a device
+ * looks its address up (which may make the CUDA runtime load that module); the
+ * address is reused until the context changes (e.g. after cudaDeviceReset).
+ * Make that first call before any stream capture begins.
  * The array is shared by all calls on a device: calls whose executions overlap
  * (different streams, or host threads with no ordering between them) race on it
  * and produce wrong results.  Order them, e.g. on one stream.
@@ -140,29 +164,37 @@ dsa_status dsa_sparse_attn_noalloc(const dsa_attn_args *args, int B, int Lq, int
                                    void *stream);
 
 /*
- * The whole forward pass: indexer -> top-k -> sparse attention.
- * `iargs` and `aargs` describe the same B, Lq, Lk, q_offset.
+ * The whole forward pass: indexer -> top-k (fused, dsa_indexer_topk) -> sparse
+ * attention.  `iargs` and `aargs` describe the same B, Lq, Lk, q_offset.
  * Short sequences (q_offset + Lq <= k): every row selects all of its positions
- * 0..t whatever the indexer says, so the pass is dense causal MLA attention; the
- * indexer is not run (the short-sequence mode of the DSA report's "Стоимость"
- * section, where attention falls back to the masked dense form).
+ * 0..t whatever the indexer says, so the pass is dense causal MLA attention (the
+ * short-sequence mode of the DSA report's "Стоимость" section, where attention
+ * falls back to the masked dense form): neither the indexer nor a top-k runs; the
+ * attention kernel reads keys 0..t as contiguous tiles (no gathers) and writes
+ * the index lists 0..t itself.
  *   indices: int32 [B, Lq, k] (as dsa_topk); out: bf16 [B, Lq, H, d_v];
  *   lse: fp32 [B, Lq, H] or NULL.
- * The workspace holds the indexer scores of the call ([B, Lq, Lk] fp32) and
- * the split-k partials.
+ * The workspace (dsa_workspace_size_args(DSA_OP_FORWARD, ...)) holds the fused
+ * indexer's candidate lists and the split-k partials; no score matrix.
  */
 dsa_status dsa_forward(const dsa_indexer_args *iargs, const dsa_attn_args *aargs, int k,
                        int32_t *indices, void *out, float *lse,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * dsa_forward with stage timing: when `stage_events` is not NULL it points to
- * four cudaEvent_t handles (created by the caller) that are recorded on
- * `stream` before the indexer, after the indexer, after the top-k and after the
- * attention (including its split-k merge).  Everything else is dsa_forward.
+ * dsa_forward with two extras.
+ *   sel_scores:   fp32 [B, Lq, k] or NULL: the indexer score of every selected
+ *                 position (as dsa_indexer_topk), e.g. for dsa_indexer_kl_loss_selected.
+ *                 When given, the indexer runs even for short sequences.
+ *   stage_events: NULL, or four cudaEvent_t handles (created by the caller)
+ *                 recorded on `stream` before the indexer, after the fused
+ *                 indexer + top-k, after the top-k (the same point: the top-k is
+ *                 part of the indexer) and after the attention (including its
+ *                 split-k merge).  For short sequences without sel_scores the
+ *                 first three coincide (the attention writes the index lists).
  */
 dsa_status dsa_forward_timed(const dsa_indexer_args *iargs, const dsa_attn_args *aargs, int k,
-                             int32_t *indices, void *out, float *lse,
+                             int32_t *indices, float *sel_scores, void *out, float *lse,
                              void *workspace, size_t workspace_bytes, void *stream,
                              void *const *stage_events);
 
@@ -189,8 +221,28 @@ dsa_status dsa_indexer_kl_loss(const dsa_attn_args *args, int B, int Lq, int Lk,
                                const int32_t *indices, int k, const float *lse,
                                const float *scores, float *target, float *kl, void *stream);
 
-/* Bytes of device workspace the entry point `op` needs for these sizes (0 = none). */
+/*
+ * dsa_indexer_kl_loss with the indexer scores given per index slot instead of as
+ * a full matrix: sel_scores fp32 [B, Lq, k], sel_scores[b,i,j] = I[t, indices[b,i,j]]
+ * for every valid slot j (padding slots are not read) -- what dsa_forward_timed
+ * and dsa_indexer_topk return.  Everything else is dsa_indexer_kl_loss.
+ */
+dsa_status dsa_indexer_kl_loss_selected(const dsa_attn_args *args, int B, int Lq, int Lk,
+                                        const int32_t *indices, int k, const float *lse,
+                                        const float *sel_scores, float *target, float *kl, void *stream);
+
+/*
+ * Bytes of device workspace the entry point `op` needs for these sizes (0 = none).
+ * For DSA_OP_FORWARD and DSA_OP_INDEXER_TOPK it assumes H_I = 64, d_I = 128 and
+ * q_offset = Lk - Lq (decode, or a prefill chunk); dsa_workspace_size_args gives
+ * the exact figure for any indexer arguments.
+ */
 size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_v);
+
+/* Exact workspace of `op` for these indexer arguments (pointers are not read; 0 for
+ * invalid arguments).  H and d_v describe the attention (ignored for
+ * DSA_OP_INDEXER_TOPK and DSA_OP_TOPK). */
+size_t dsa_workspace_size_args(dsa_op op, const dsa_indexer_args *iargs, int k, int H, int d_v);
 
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *dsa_status_string(dsa_status status);

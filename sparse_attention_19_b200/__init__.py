@@ -19,16 +19,16 @@ import os
 import torch
 
 __all__ = [
-    "DSAError", "lib", "lib_path", "indexer_scores", "topk", "sparse_attn", "sparse_attn_noalloc", "forward",
-    "indexer_kl_loss",
-    "workspace_size", "status_string", "device_status", "selftest_wait_timeout", "version",
-    "OP_TOPK", "OP_SPARSE_ATTN", "OP_FORWARD",
+    "DSAError", "lib", "lib_path", "indexer_scores", "topk", "indexer_topk", "sparse_attn", "sparse_attn_noalloc",
+    "forward", "indexer_kl_loss", "indexer_kl_loss_selected",
+    "workspace_size", "workspace_size_args", "status_string", "device_status", "selftest_wait_timeout", "version",
+    "OP_TOPK", "OP_SPARSE_ATTN", "OP_FORWARD", "OP_INDEXER_TOPK",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libdsa.so")
 
-OP_TOPK, OP_SPARSE_ATTN, OP_FORWARD = 0, 1, 2
+OP_TOPK, OP_SPARSE_ATTN, OP_FORWARD, OP_INDEXER_TOPK = 0, 1, 2, 3
 _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_WORKSPACE",
            4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT"}
 
@@ -67,17 +67,21 @@ def lib():
         L.dsa_sparse_attn.argtypes = [ctypes.POINTER(AttnArgs), I, I, I, P, I, P, P, P, Z, P]
         L.dsa_sparse_attn_noalloc.argtypes = [ctypes.POINTER(AttnArgs), I, I, I, P, I, P, P, P]
         L.dsa_forward.argtypes = [ctypes.POINTER(IndexerArgs), ctypes.POINTER(AttnArgs), I, P, P, P, P, Z, P]
-        L.dsa_forward_timed.argtypes = [ctypes.POINTER(IndexerArgs), ctypes.POINTER(AttnArgs), I, P, P, P, P, Z, P,
-                                        ctypes.POINTER(ctypes.c_void_p)]
+        L.dsa_forward_timed.argtypes = [ctypes.POINTER(IndexerArgs), ctypes.POINTER(AttnArgs), I, P, P, P, P, P, Z,
+                                        P, ctypes.POINTER(ctypes.c_void_p)]
+        L.dsa_indexer_topk.argtypes = [ctypes.POINTER(IndexerArgs), I, P, P, P, Z, P]
         L.dsa_indexer_kl_loss.argtypes = [ctypes.POINTER(AttnArgs), I, I, I, P, I, P, P, P, P, P]
+        L.dsa_indexer_kl_loss_selected.argtypes = [ctypes.POINTER(AttnArgs), I, I, I, P, I, P, P, P, P, P]
         L.dsa_workspace_size.argtypes = [I, I, I, I, I, I, I]
         L.dsa_workspace_size.restype = ctypes.c_size_t
+        L.dsa_workspace_size_args.argtypes = [I, ctypes.POINTER(IndexerArgs), I, I, I]
+        L.dsa_workspace_size_args.restype = ctypes.c_size_t
         L.dsa_status_string.argtypes = [I]
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_device_status.argtypes = [I]
         L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
-        for f in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_sparse_attn_noalloc", "dsa_forward",
-                  "dsa_forward_timed", "dsa_indexer_kl_loss",
+        for f in ("dsa_indexer_scores", "dsa_topk", "dsa_indexer_topk", "dsa_sparse_attn", "dsa_sparse_attn_noalloc",
+                  "dsa_forward", "dsa_forward_timed", "dsa_indexer_kl_loss", "dsa_indexer_kl_loss_selected",
                   "dsa_device_status",
                   "dsa_selftest_wait_timeout", "dsa_version"):
             getattr(L, f).restype = ctypes.c_int
@@ -152,6 +156,11 @@ def workspace_size(op: int, B: int, Lq: int, Lk: int, k: int, H: int, d_v: int) 
     return int(lib().dsa_workspace_size(int(op), B, Lq, Lk, k, H, d_v))
 
 
+def workspace_size_args(op: int, ia: "IndexerArgs", k: int, H: int = 0, d_v: int = 0) -> int:
+    """Exact workspace bytes of `op` for these indexer arguments (dsa_workspace_size_args)."""
+    return int(lib().dsa_workspace_size_args(int(op), ctypes.byref(ia), int(k), int(H), int(d_v)))
+
+
 def indexer_scores(q_I, q_scale, w, k_I, k_scale, q_offset=0, scores=None, stream=None):
     """fp32 [B, Lq, Lk] indexer scores, -inf above the causal boundary."""
     a = _indexer_args(q_I, q_scale, w, k_I, k_scale, q_offset)
@@ -175,8 +184,32 @@ def topk(scores, k, q_offset=0, indices=None, workspace=None, stream=None):
     return indices
 
 
-def _workspace(op, B, Lq, Lk, k, H, d_v, device, workspace):
-    need = workspace_size(op, B, Lq, Lk, k, H, d_v)
+def indexer_topk(q_I, q_scale, w, k_I, k_scale, k, q_offset=0, indices=None, sel_scores=None,
+                 want_scores=True, workspace=None, stream=None):
+    """Indexer with the top-k fused into it (no score matrix is written).
+
+    Returns (indices int32 [B, Lq, k] ascending, -1 padded; sel_scores fp32 [B, Lq, k]
+    or None: the score of each selected position, -inf on padding)."""
+    a = _indexer_args(q_I, q_scale, w, k_I, k_scale, q_offset)
+    dev = w.device
+    if indices is None:
+        indices = torch.empty(a.B, a.Lq, k, dtype=torch.int32, device=dev)
+    _need(indices, torch.int32, (a.B, a.Lq, k), "indices")
+    if sel_scores is None and want_scores:
+        sel_scores = torch.empty(a.B, a.Lq, k, dtype=torch.float32, device=dev)
+    if sel_scores is not None:
+        _need(sel_scores, torch.float32, (a.B, a.Lq, k), "sel_scores")
+    need = workspace_size_args(OP_INDEXER_TOPK, a, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().dsa_indexer_topk(ctypes.byref(a), int(k), _ptr(indices), _ptr(sel_scores), _ptr(workspace),
+                                  nbytes, _stream(stream)), "dsa_indexer_topk")
+    return indices, sel_scores
+
+
+def _workspace(op, B, Lq, Lk, k, H, d_v, device, workspace, ia=None):
+    need = workspace_size_args(op, ia, k, H, d_v) if ia is not None else workspace_size(op, B, Lq, Lk, k, H, d_v)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -221,11 +254,13 @@ def sparse_attn_noalloc(q, kv, indices, d_v, scale, out, lse=None, stream=None):
 
 
 def forward(q_I, q_scale, w, k_I, k_scale, q, kv, k, d_v, scale, q_offset=0, indices=None, out=None,
-            lse=None, want_lse=True, workspace=None, stream=None, stage_events=None):
-    """Indexer -> top-k -> sparse attention.  Returns (indices, out, lse).
+            lse=None, want_lse=True, workspace=None, stream=None, stage_events=None, sel_scores=None):
+    """Indexer -> top-k (fused into the indexer) -> sparse attention.  Returns (indices, out, lse).
 
     ``stage_events``: optional four torch.cuda.Event objects, recorded on the
-    stream before the indexer, after it, after the top-k and after the attention.
+    stream before the indexer, after the fused indexer + top-k, after the top-k
+    (the same point) and after the attention.  ``sel_scores``: optional fp32
+    [B, Lq, k] tensor that receives the indexer score of every selected position.
     """
     ia = _indexer_args(q_I, q_scale, w, k_I, k_scale, q_offset)
     aa = _attn_args(q, kv, d_v, scale)
@@ -238,7 +273,9 @@ def forward(q_I, q_scale, w, k_I, k_scale, q, kv, k, d_v, scale, q_offset=0, ind
     _need(out, torch.bfloat16, (B, Lq, H, d_v), "out")
     if lse is None and want_lse:
         lse = torch.empty(B, Lq, H, dtype=torch.float32, device=q.device)
-    workspace, nbytes = _workspace(OP_FORWARD, B, Lq, Lk, k, H, d_v, q.device, workspace)
+    if sel_scores is not None:
+        _need(sel_scores, torch.float32, (B, Lq, k), "sel_scores")
+    workspace, nbytes = _workspace(OP_FORWARD, B, Lq, Lk, k, H, d_v, q.device, workspace, ia=ia)
     ev = None
     if stage_events is not None:
         if len(stage_events) != 4:
@@ -247,8 +284,9 @@ def forward(q_I, q_scale, w, k_I, k_scale, q, kv, k, d_v, scale, q_offset=0, ind
             if not e.cuda_event:
                 e.record(stream if stream is not None else torch.cuda.current_stream())
         ev = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in stage_events])
-    _check(lib().dsa_forward_timed(ctypes.byref(ia), ctypes.byref(aa), int(k), _ptr(indices), _ptr(out), _ptr(lse),
-                                   _ptr(workspace), nbytes, _stream(stream), ev), "dsa_forward")
+    _check(lib().dsa_forward_timed(ctypes.byref(ia), ctypes.byref(aa), int(k), _ptr(indices), _ptr(sel_scores),
+                                   _ptr(out), _ptr(lse), _ptr(workspace), nbytes, _stream(stream), ev),
+           "dsa_forward")
     return indices, out, lse
 
 
@@ -277,6 +315,30 @@ def indexer_kl_loss(q, kv, indices, lse, scores, d_v, scale, target=None, want_t
     _need(kl, torch.float32, (B, Lq), "kl")
     _check(lib().dsa_indexer_kl_loss(ctypes.byref(a), B, Lq, Lk, _ptr(indices), k, _ptr(lse), _ptr(scores),
                                      _ptr(target), _ptr(kl), _stream(stream)), "dsa_indexer_kl_loss")
+    return target, kl
+
+
+def indexer_kl_loss_selected(q, kv, indices, lse, sel_scores, d_v, scale, target=None, want_target=True, kl=None,
+                             stream=None):
+    """indexer_kl_loss with the scores given per index slot (fp32 [B, Lq, k], as
+    returned by indexer_topk or forward(sel_scores=...)) instead of a full matrix."""
+    a = _attn_args(q, kv, d_v, scale)
+    B, Lq, H, _ = q.shape
+    Lk = kv.shape[1]
+    k = indices.shape[-1]
+    _need(indices, torch.int32, (B, Lq, k), "indices")
+    _need(lse, torch.float32, (B, Lq, H), "lse")
+    _need(sel_scores, torch.float32, (B, Lq, k), "sel_scores")
+    if target is None and want_target:
+        target = torch.empty(B, Lq, k, dtype=torch.float32, device=q.device)
+    if target is not None:
+        _need(target, torch.float32, (B, Lq, k), "target")
+    if kl is None:
+        kl = torch.empty(B, Lq, dtype=torch.float32, device=q.device)
+    _need(kl, torch.float32, (B, Lq), "kl")
+    _check(lib().dsa_indexer_kl_loss_selected(ctypes.byref(a), B, Lq, Lk, _ptr(indices), k, _ptr(lse),
+                                              _ptr(sel_scores), _ptr(target), _ptr(kl), _stream(stream)),
+           "dsa_indexer_kl_loss_selected")
     return target, kl
 
 

@@ -118,30 +118,37 @@ size_t attn_ws_bytes(int B, int Lq, int k, int H, int d_v) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper, cudaStream_t st) {
+// Launch shape of the indexer for these sizes: query block, sub-blocks, key-tile
+// chunks per block and, in the fused top-k mode, the candidate lists and the
+// staging ring.  The same plan sizes the workspace and drives the launch.
+IndexerParams plan_indexer(const dsa_indexer_args* a, bool fused, int k) {
   IndexerParams p{};
   p.B = a->B; p.Lq = a->Lq; p.Lk = a->Lk; p.q_offset = a->q_offset;
   p.H_I = a->H_I; p.d_I = a->d_I;
   if (a->H_I == 64) {
     p.qb = a->Lq >= 4 ? 4 : a->Lq;
+  } else if (fused) {
+    p.qb = 16;                                   // N = 64: one 64-column accumulator per sub-block
   } else {
     const int r4 = (a->Lq + 3) / 4 * 4;
     p.qb = r4 < 64 ? r4 : 64;
   }
   p.nsub = (a->Lq > p.qb) ? 2 : 1;
   p.queries_per_unit = p.qb * p.nsub;
-  if (p.queries_per_unit * a->H_I > 512) return DSA_ERR_UNSUPPORTED;   // epilogue staging limit
   p.n_qblocks = (a->Lq + p.queries_per_unit - 1) / p.queries_per_unit;
   const int sms = sm_count();
   const long long base_units = (long long)p.n_qblocks * a->B;
   const int max_tiles = (a->q_offset + a->Lq - 1) / 128 + 1;
   // Few query blocks (decode): split each sequence's key tiles over kchunks units.
   // Cost model in key tiles per CTA: waves of units over the SMs, each unit its
-  // tiles plus about two tiles of start-up; keep at least ~8 tiles per unit.
+  // tiles plus about two tiles of start-up; keep at least ~8 tiles per unit.  In
+  // the fused mode the last unit of a row also selects over every chunk's list
+  // (up to k candidates each), so chunks are capped at 16.
   int kch = 1;
   if (base_units < 4LL * sms) {
     constexpr double kUnitOverheadTiles = 2.0;
-    const int cap = (max_tiles + 7) / 8;
+    int cap = (max_tiles + 7) / 8;
+    if (fused && cap > 16) cap = 16;
     double best = 1e300;
     for (int c = 1; c <= cap; ++c) {
       const long long waves = (base_units * c + sms - 1) / sms;
@@ -151,31 +158,104 @@ dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper
   }
   p.kchunks = kch;
   p.n_units = (int)(base_units * kch);
+  p.scale_ring = (a->k_scale && a->Lk % 4 == 0 && p.nsub * p.qb * a->H_I <= 128) ? 1 : 0;
+  if (fused) {
+    const int k32 = (k + 31) / 32 * 32;
+    p.k = k;
+    p.cap = k32 + (k32 > 256 ? k32 : 256);       // room for one tile (128) after every cut to k
+    p.rows_per_unit = p.queries_per_unit;
+    const int deep = p.nsub * p.qb * a->H_I <= 128;
+    const int slot_bytes = p.qb * 128 * 8;
+    int ns = (deep ? 16384 : 32768) / slot_bytes;
+    p.n_stage = ns < 2 ? 2 : (ns > indexer_fused_max_stage() ? indexer_fused_max_stage() : ns);
+  }
+  return p;
+}
+
+int indexer_grid(const IndexerParams& p) {
+  const int sms = sm_count();
+  return p.n_units < sms ? p.n_units : sms;
+}
+
+// Workspace of the fused indexer + top-k: the candidate lists (per CTA, or per
+// unit when rows are split over several units), then the per-(unit, row) list
+// summaries and the per-row chunk counters of split rows.
+struct FusedWs {
+  size_t key_off, pos_off, meta_off, done_off, bytes;
+};
+FusedWs fused_ws_layout(const IndexerParams& p) {
+  FusedWs w{};
+  const size_t slots = p.kchunks == 1 ? (size_t)indexer_grid(p) : (size_t)p.n_units;
+  const size_t list = slots * p.rows_per_unit * (size_t)p.cap * 4;
+  w.key_off = 0;
+  w.pos_off = round_up(list, 256);
+  w.meta_off = w.pos_off + round_up(list, 256);
+  const size_t meta = p.kchunks > 1 ? (size_t)p.n_units * p.rows_per_unit * 16 : 0;
+  w.done_off = w.meta_off + round_up(meta, 256);
+  const size_t done = p.kchunks > 1 ? (size_t)p.B * p.Lq * 4 : 0;
+  w.bytes = w.done_off + round_up(done, 256);
+  return w;
+}
+
+size_t indexer_topk_ws_bytes(const dsa_indexer_args* a, int k) {
+  const IndexerParams p = plan_indexer(a, true, k);
+  if (p.queries_per_unit * a->H_I > 512 || p.rows_per_unit > indexer_fused_max_rows()) return 0;
+  return fused_ws_layout(p).bytes;
+}
+
+bool make_indexer_maps(const dsa_indexer_args* a, const IndexerParams& p, CUtensorMap* tq, CUtensorMap* tk,
+                       CUtensorMap* ts) {
+  const CUtensorMapSwizzle swz = (a->d_I == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_tmap(tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->q_I, (uint64_t)a->B * a->Lq * a->H_I, a->d_I,
+                 a->d_I, (uint32_t)(p.qb * a->H_I), swz))
+    return false;
+  if (!make_tmap(tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 32,
+                 swz))                                     // key tiles arrive as four 32-row boxes
+    return false;
+  *ts = *tk;                                               // unused unless scale_ring
+  if (p.scale_ring && !make_tmap(ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a->k_scale, (uint64_t)a->B, a->Lk,
+                                 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  return true;
+}
+
+dsa_status run_indexer(const dsa_indexer_args* a, float* scores, bool fill_upper, cudaStream_t st) {
+  IndexerParams p = plan_indexer(a, false, 0);
+  if (p.queries_per_unit * a->H_I > 512) return DSA_ERR_UNSUPPORTED;   // epilogue staging limit
   p.fill_upper = fill_upper ? 1 : 0;
   p.q_scale = a->q_scale;
   p.w = reinterpret_cast<const __nv_bfloat16*>(a->w);
   p.k_scale = a->k_scale;
   p.scores = scores;
-  // Decode-like calls (a small query block streaming many keys from HBM) take the
-  // key scales through a TMA-filled shared-memory ring, when the [B, Lk] fp32 array
-  // can be described to TMA (rows of a multiple of 16 bytes); prefill reads them
-  // directly (they stay in L2), one tile ahead.
-  p.scale_ring = (a->k_scale && a->Lk % 4 == 0 && p.nsub * p.qb * a->H_I <= 128) ? 1 : 0;
+  CUtensorMap tq, tk, ts;
+  if (!make_indexer_maps(a, p, &tq, &tk, &ts)) return DSA_ERR_CUDA;
+  return launch_indexer(p, tq, tk, ts, indexer_grid(p), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
 
-  const CUtensorMapSwizzle swz = (a->d_I == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  CUtensorMap tq, tk;
-  if (!make_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->q_I, (uint64_t)a->B * a->Lq * a->H_I, a->d_I,
-                 a->d_I, (uint32_t)(p.qb * a->H_I), swz))
-    return DSA_ERR_CUDA;
-  if (!make_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 32,
-                 swz))                                     // key tiles arrive as four 32-row boxes
-    return DSA_ERR_CUDA;
-  CUtensorMap ts = tk;                                     // unused unless scale_ring
-  if (p.scale_ring && !make_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a->k_scale, (uint64_t)a->B, a->Lk,
-                                 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return DSA_ERR_CUDA;
-  const int grid = p.n_units < sms ? p.n_units : sms;
-  return launch_indexer(p, tq, tk, ts, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+// The indexer with top-k selection fused into it: per row the k positions with the
+// largest scores (ties to the smaller position), ascending, -1 padded, and their
+// scores; no score matrix is written.
+dsa_status run_indexer_topk(const dsa_indexer_args* a, int k, int32_t* indices, float* sel_scores, void* ws,
+                            size_t ws_bytes, cudaStream_t st) {
+  IndexerParams p = plan_indexer(a, true, k);
+  if (p.queries_per_unit * a->H_I > 512 || p.rows_per_unit > indexer_fused_max_rows()) return DSA_ERR_UNSUPPORTED;
+  const FusedWs w = fused_ws_layout(p);
+  if (!ws || ws_bytes < w.bytes || !aligned16(ws)) return DSA_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  p.q_scale = a->q_scale;
+  p.w = reinterpret_cast<const __nv_bfloat16*>(a->w);
+  p.k_scale = a->k_scale;
+  p.scores = nullptr;
+  p.indices = indices;
+  p.sel_scores = sel_scores;
+  p.xkey = reinterpret_cast<uint32_t*>(base + w.key_off);
+  p.xpos = reinterpret_cast<uint32_t*>(base + w.pos_off);
+  p.xmeta = reinterpret_cast<uint4*>(base + w.meta_off);
+  p.done = reinterpret_cast<uint32_t*>(base + w.done_off);
+  if (p.kchunks > 1 && cudaMemsetAsync(p.done, 0, (size_t)p.B * p.Lq * 4, st) != cudaSuccess) return DSA_ERR_CUDA;
+  CUtensorMap tq, tk, ts;
+  if (!make_indexer_maps(a, p, &tq, &tk, &ts)) return DSA_ERR_CUDA;
+  return launch_indexer(p, tq, tk, ts, indexer_grid(p), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, int k, int32_t* idx,
@@ -202,11 +282,17 @@ dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, in
   return launch_topk(p, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// Sparse attention over `idx`; or, when `dense_idx_out` is given (short sequence:
+// q_offset + Lq <= k), dense causal attention over keys 0..t read as contiguous
+// tiles, with the index lists 0..t written to dense_idx_out by the same kernel.
 dsa_status run_attn(const dsa_attn_args* a, int B, int Lq, int Lk, int q_offset, bool compact,
                     const int32_t* idx, int k, void* out, float* lse, void* ws, size_t ws_bytes,
-                    cudaStream_t st) {
+                    cudaStream_t st, int32_t* dense_idx_out = nullptr) {
   AttnParams p{};
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = a->H; p.k = k;
+  p.dense = dense_idx_out ? 1 : 0;
+  p.idx_out = dense_idx_out;
+  if (p.dense) compact = true;
   p.n_tiles = (k + kAttnTile - 1) / kAttnTile;
   const int rows = B * Lq;
   p.splits = attn_splits(rows, p.n_tiles);
@@ -232,15 +318,20 @@ dsa_status run_attn(const dsa_attn_args* a, int B, int Lq, int Lk, int q_offset,
   if (!make_tmap(&tkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->kv, (uint64_t)B * Lk, a->d_qk, 64, 1,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
+  CUtensorMap tkv_tile = tkv;                               // 64 contiguous rows per box (dense mode)
+  if (p.dense && !make_tmap(&tkv_tile, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a->kv, (uint64_t)B * Lk, a->d_qk, 64,
+                            64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
   const int pairs = sm_count() / 2;
   const int grid = p.n_units < pairs ? p.n_units : pairs;
-  if (launch_sparse_attn(p, a->d_qk, a->d_v, tq, tkv, grid, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_sparse_attn(p, a->d_qk, a->d_v, tq, tkv, tkv_tile, grid, st) != cudaSuccess) return DSA_ERR_CUDA;
   if (p.splits > 1 && launch_attn_combine(p, a->d_v, st) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }
 
 dsa_status run_indexer_kl(const dsa_attn_args* a, int B, int Lq, int Lk, const int32_t* indices, int k,
-                          const float* lse, const float* scores, float* target, float* kl, cudaStream_t st) {
+                          const float* lse, const float* scores, const float* sel_scores, float* target, float* kl,
+                          cudaStream_t st) {
   KlParams p{};
   p.B = B; p.Lq = Lq; p.Lk = Lk; p.H = a->H; p.k = k;
   p.n_rows = B * Lq;
@@ -249,6 +340,7 @@ dsa_status run_indexer_kl(const dsa_attn_args* a, int B, int Lq, int Lk, const i
   p.indices = indices;
   p.lse = lse;
   p.scores = scores;
+  p.sel_scores = sel_scores;
   p.target = target;
   p.kl = kl;
   CUtensorMap tq, tkv;
@@ -345,95 +437,104 @@ dsa_status dsa_indexer_kl_loss(const dsa_attn_args* args, int B, int Lq, int Lk,
   if (!aligned16(indices) || !aligned16(lse) || !aligned16(scores) || !aligned16(kl)) return DSA_ERR_INVALID_ARG;
   if (target && !aligned16(target)) return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
-  return run_indexer_kl(args, B, Lq, Lk, indices, k, lse, scores, target, kl, static_cast<cudaStream_t>(stream));
+  return run_indexer_kl(args, B, Lq, Lk, indices, k, lse, scores, nullptr, target, kl,
+                        static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_indexer_kl_loss_selected(const dsa_attn_args* args, int B, int Lq, int Lk, const int32_t* indices,
+                                        int k, const float* lse, const float* sel_scores, float* target, float* kl,
+                                        void* stream) {
+  dsa_status s = check_attn(args, B, Lq, Lk);
+  if (s != DSA_OK) return s;
+  if (!indices || !lse || !sel_scores || !kl) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(indices) || !aligned16(lse) || !aligned16(sel_scores) || !aligned16(kl)) return DSA_ERR_INVALID_ARG;
+  if (target && !aligned16(target)) return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
+  return run_indexer_kl(args, B, Lq, Lk, indices, k, lse, nullptr, sel_scores, target, kl,
+                        static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_workspace_size_args(dsa_op op, const dsa_indexer_args* iargs, int k, int H, int d_v) {
+  if (!iargs || check_indexer(iargs) != DSA_OK || k < 1 || k > kMaxK) return 0;
+  switch (op) {
+    case DSA_OP_TOPK:
+      return 0;
+    case DSA_OP_SPARSE_ATTN:
+      return H > 0 && d_v > 0 ? attn_ws_bytes(iargs->B, iargs->Lq, k, H, d_v) : 0;
+    case DSA_OP_INDEXER_TOPK:
+      return indexer_topk_ws_bytes(iargs, k);
+    case DSA_OP_FORWARD:
+      if (H <= 0 || d_v <= 0) return 0;
+      return round_up(indexer_topk_ws_bytes(iargs, k), 256) + attn_ws_bytes(iargs->B, iargs->Lq, k, H, d_v);
+  }
+  return 0;
 }
 
 size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_v) {
-  if (B <= 0 || Lq <= 0 || Lk <= 0 || k < 1 || k > kMaxK || H <= 0 || d_v <= 0) return 0;
+  if (B <= 0 || Lq <= 0 || Lk <= 0 || Lq > Lk || k < 1 || k > kMaxK || H <= 0 || d_v <= 0) return 0;
   switch (op) {
     case DSA_OP_TOPK:
       return 0;
     case DSA_OP_SPARSE_ATTN:
       return attn_ws_bytes(B, Lq, k, H, d_v);
-    case DSA_OP_FORWARD:
-      return round_up((size_t)B * Lq * (size_t)Lk * 4, 256) + attn_ws_bytes(B, Lq, k, H, d_v);
+    case DSA_OP_INDEXER_TOPK:
+    case DSA_OP_FORWARD: {
+      // The documented convention: H_I = 64, d_I = 128, q_offset = Lk - Lq.
+      alignas(16) static const uint8_t dummy[16] = {};
+      dsa_indexer_args a{B, Lq, Lk, Lk - Lq, 64, 128, dummy, nullptr, dummy, dummy, nullptr};
+      return dsa_workspace_size_args(op, &a, k, H, d_v);
+    }
   }
   return 0;
 }
 
-// Split-k partials of dsa_sparse_attn_noalloc: a fixed array in this module's
-// device image, so that call allocates nothing.  Its address is looked up once
-// per device (with that device current) and cached.
-static __device__ __align__(256) unsigned char g_noalloc_scratch[DSA_NOALLOC_SCRATCH_BYTES];
-static constexpr int kMaxDevices = 64;
-
-static dsa_status noalloc_scratch(void** ptr) {
-  static std::mutex mu;
-  static void* addr[kMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
-    addr[dev] = p;
-  }
-  *ptr = addr[dev];
-  return DSA_OK;
-}
-
-dsa_status dsa_sparse_attn_noalloc(const dsa_attn_args* args, int B, int Lq, int Lk, const int32_t* indices,
-                                   int k, void* out, float* lse, void* stream) {
-  dsa_status s = check_attn(args, B, Lq, Lk);
+dsa_status dsa_indexer_topk(const dsa_indexer_args* args, int k, int32_t* indices, float* sel_scores,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status s = check_indexer(args);
   if (s != DSA_OK) return s;
-  if (!indices || !out || !aligned16(indices) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
-  if (lse && !aligned16(lse)) return DSA_ERR_INVALID_ARG;
+  if (!indices || !aligned16(indices)) return DSA_ERR_INVALID_ARG;
+  if (sel_scores && !aligned16(sel_scores)) return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
-  const size_t need = attn_ws_bytes(B, Lq, k, args->H, args->d_v);
-  if (need > DSA_NOALLOC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
-  void* ws = nullptr;
-  if (need > 0 && (s = noalloc_scratch(&ws)) != DSA_OK) return s;
-  return run_attn(args, B, Lq, Lk, 0, false, indices, k, out, lse, ws, DSA_NOALLOC_SCRATCH_BYTES,
-                  static_cast<cudaStream_t>(stream));
+  return run_indexer_topk(args, k, indices, sel_scores, workspace, workspace_bytes,
+                          static_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_forward_timed(const dsa_indexer_args* iargs, const dsa_attn_args* aargs, int k, int32_t* indices,
-                             void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream,
-                             void* const* stage_events) {
+                             float* sel_scores, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream, void* const* stage_events) {
   dsa_status s = check_indexer(iargs);
   if (s != DSA_OK) return s;
   s = check_attn(aargs, iargs->B, iargs->Lq, iargs->Lk);
   if (s != DSA_OK) return s;
   if (!indices || !out || !aligned16(indices) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
   if (lse && !aligned16(lse)) return DSA_ERR_INVALID_ARG;
+  if (sel_scores && !aligned16(sel_scores)) return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
-  const size_t need = dsa_workspace_size(DSA_OP_FORWARD, iargs->B, iargs->Lq, iargs->Lk, k, aargs->H, aargs->d_v);
+  const size_t sel_bytes = round_up(indexer_topk_ws_bytes(iargs, k), 256);
+  const size_t need = sel_bytes + attn_ws_bytes(iargs->B, iargs->Lq, k, aargs->H, aargs->d_v);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> bool {
     return !stage_events || cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
   };
-  float* scores = static_cast<float*>(workspace);
-  const size_t score_bytes = round_up((size_t)iargs->B * iargs->Lq * (size_t)iargs->Lk * 4, 256);
-  char* attn_ws = static_cast<char*>(workspace) + score_bytes;
-  const size_t attn_ws_size = workspace_bytes - score_bytes;
+  char* attn_ws = static_cast<char*>(workspace) + sel_bytes;
+  const size_t attn_ws_size = workspace_bytes - sel_bytes;
   if (!mark(0)) return DSA_ERR_CUDA;
   // Short sequences: when every row's causal range fits in k (q_offset + Lq <= k),
   // every position is selected whatever the scores, and the pass is dense causal
-  // attention.  The indexer is skipped; the top-k step writes the index lists
-  // 0..t without reading scores.
-  const bool dense = (long long)iargs->q_offset + iargs->Lq <= k;
+  // attention.  Unless the selected scores are asked for, the indexer is skipped
+  // and the top-k step writes the index lists 0..t without reading scores.
+  const bool dense = (long long)iargs->q_offset + iargs->Lq <= k && !sel_scores;
   if (!dense) {
-    s = run_indexer(iargs, scores, false, st);
+    // Indexer with the top-k fused into it: no score matrix is written.
+    s = run_indexer_topk(iargs, k, indices, sel_scores, workspace, sel_bytes, st);
     if (s != DSA_OK) return s;
   }
-  if (!mark(1)) return DSA_ERR_CUDA;
-  s = run_topk(scores, iargs->B, iargs->Lq, iargs->Lk, iargs->q_offset, k, indices, st);
-  if (s != DSA_OK) return s;
-  if (!mark(2)) return DSA_ERR_CUDA;
+  if (!mark(1) || !mark(2)) return DSA_ERR_CUDA;
+  // Dense mode: the attention kernel reads keys 0..t as contiguous tiles and writes
+  // the index lists itself (no top-k launch, no gathers).
   s = run_attn(aargs, iargs->B, iargs->Lq, iargs->Lk, iargs->q_offset, true, indices, k, out, lse, attn_ws,
-               attn_ws_size, st);
+               attn_ws_size, st, dense ? indices : nullptr);
   if (s != DSA_OK) return s;
   if (!mark(3)) return DSA_ERR_CUDA;
   return DSA_OK;
@@ -441,7 +542,8 @@ dsa_status dsa_forward_timed(const dsa_indexer_args* iargs, const dsa_attn_args*
 
 dsa_status dsa_forward(const dsa_indexer_args* iargs, const dsa_attn_args* aargs, int k, int32_t* indices,
                        void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
-  return dsa_forward_timed(iargs, aargs, k, indices, out, lse, workspace, workspace_bytes, stream, nullptr);
+  return dsa_forward_timed(iargs, aargs, k, indices, nullptr, out, lse, workspace, workspace_bytes, stream,
+                           nullptr);
 }
 
 const char* dsa_status_string(dsa_status status) {

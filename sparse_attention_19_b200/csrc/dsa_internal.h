@@ -25,11 +25,29 @@ struct IndexerParams {
   const float* q_scale;   // [B, Lq] or null
   const __nv_bfloat16* w; // [B, Lq, H_I]
   const float* k_scale;   // [B, Lk] or null
-  float* scores;          // [B, Lq, Lk]
+  float* scores;          // [B, Lq, Lk] (scores mode)
+  // ---- fused top-k mode (scores == nullptr): every row's k largest scores are
+  // selected on chip; no score reaches global memory except the selected ones.
+  int k;                  // positions selected per row
+  int cap;                // candidate-list capacity per row (multiple of 32, >= k + 128)
+  int n_stage;            // staging slots (one per accumulator use) in shared memory
+  int rows_per_unit;      // queries_per_unit
+  int32_t* indices;       // [B, Lq, k]
+  float* sel_scores;      // [B, Lq, k] or null
+  uint32_t* xkey;         // candidate lists, keys:      [list slot][rows_per_unit][cap]
+  uint32_t* xpos;         // candidate lists, positions: same layout
+  uint4* xmeta;           // kchunks > 1: per (unit, row) {count, min key, max key, 0}
+  uint32_t* done;         // kchunks > 1: per row, chunks finished (zeroed before the launch)
 };
-size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages);
+// Shared-memory bytes of the indexer kernel for a query block of q_rows (query,
+// head) rows, `stages` key stages and, in the fused mode, the staging and
+// selection areas.
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages, bool fused, int qb,
+                          int n_stage, int rows_per_unit);
 cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& ts, int grid, cudaStream_t stream);
+int indexer_fused_max_rows();    // rows per unit the fused mode supports
+int indexer_fused_max_stage();   // staging slots the fused mode supports
 
 // ---------------------------------------------------------------- top-k
 struct TopkParams {
@@ -55,7 +73,10 @@ struct AttnParams {
   int tiles_per_split;
   int n_units;            // B * Lq * splits
   int compact;            // indices are valid-first (top-k output): skip all-padding tiles
-  int q_offset;           // only used when compact
+  int dense;              // short sequence (q_offset + Lq <= k): row t attends to keys 0..t, read as
+                          // contiguous tiles; the kernel writes those positions to idx_out
+  int q_offset;           // only used when compact or dense
+  int32_t* idx_out;       // dense: [B, Lq, k] receives 0..t then -1
   float scale_log2;       // softmax scale * log2(e)
   const int32_t* indices; // [B, Lq, k]
   __nv_bfloat16* out;     // [B, Lq, H, d_v] (splits == 1)
@@ -65,7 +86,8 @@ struct AttnParams {
 };
 size_t attn_smem_bytes(int d_qk, int d_v);
 cudaError_t launch_sparse_attn(const AttnParams& p, int d_qk, int d_v, const CUtensorMap& tq,
-                               const CUtensorMap& tkv, int grid_clusters, cudaStream_t stream);
+                               const CUtensorMap& tkv, const CUtensorMap& tkv_tile, int grid_clusters,
+                               cudaStream_t stream);
 cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t stream);
 
 // ---------------------------------------------------------------- indexer training loss
@@ -76,7 +98,8 @@ struct KlParams {
   float scale_log2;       // softmax scale * log2(e)
   const int32_t* indices; // [B, Lq, k]
   const float* lse;       // [B, Lq, H], natural log
-  const float* scores;    // [B, Lq, Lk]
+  const float* scores;    // [B, Lq, Lk], or null when sel_scores is given
+  const float* sel_scores;  // [B, Lq, k]: the score of each index slot (or null)
   float* target;          // [B, Lq, k] or null
   float* kl;              // [B, Lq]
 };

@@ -18,10 +18,27 @@
 // uses QB = 1 (N = 64) with a deeper key ring, the key scales staged through a TMA
 // ring, and the two epilogue warp halves taking alternate accumulators.
 //
+// Two modes.  Scores mode writes I[t,s] to a [B, Lq, Lk] array.  Fused mode (the
+// forward pass) selects every row's top-k on chip instead ("Отбор и основное
+// внимание": only the k positions with the largest I[t,s] go on to attention), so
+// no score matrix reaches global memory:
+//   * the epilogue compares each score with its row's current threshold and
+//     ballot-compacts the survivors of each (tile, query) into a shared-memory
+//     staging ring;
+//   * three selector warps append the staged candidates to a per-row list kept
+//     in global memory (L2-resident, in position order) and, when a list fills,
+//     cut it to the row's exact top-k by histogram refinement (warp_select.cuh),
+//     which raises the row's threshold: later scores must beat the k-th best so
+//     far (a tie loses, since every later position is larger);
+//   * at the end of a row the list is cut to its final top-k and written out in
+//     ascending position order, with the selected scores.  A row split over
+//     several units (decode) is finished by whichever unit ends last, over the
+//     units' lists.
 // Warp roles (768 threads): warps 0..15 epilogue (warp w reads TMEM lanes
 // 32(w%4) .. 32(w%4)+31 of the 64-column groups w/4, w/4 + 4, ...), warp 16 TMEM
-// owner + MMA issuer, warps 20..23 TMA loaders.  Four epilogue warps per SM
-// sub-partition hide the latency of the per-element ReLU / weighting / head sum.
+// owner + MMA issuer, warps 17..19 selectors (fused mode), warps 20..23 TMA
+// loaders.  Four epilogue warps per SM sub-partition hide the latency of the
+// per-element ReLU / weighting / head sum.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,6 +47,7 @@
 
 #include "dsa_internal.h"
 #include "ptx.cuh"
+#include "warp_select.cuh"
 
 namespace dsa {
 
@@ -39,7 +57,9 @@ constexpr int kKeysPerTile = 128;
 constexpr int kMaxStages = 12;
 constexpr int kEpiWarps = 16;        // four per TMEM lane quarter ("quads" of four warps)
 constexpr int kQuads = kEpiWarps / 4;
-constexpr int kMmaWarp = kEpiWarps;  // warps 16-19: MMA issuer (+ three idle warps of its warpgroup)
+constexpr int kMmaWarp = kEpiWarps;  // warp 16: MMA issuer
+constexpr int kSelWarp0 = kMmaWarp + 1;   // warps 17-19: selectors (fused mode)
+constexpr int kSelWarps = 3;
 constexpr int kLoaders = 4;          // TMA requests from one warp are served in order, so each
                                      // key tile is loaded as four 32-row boxes from four warps
 constexpr int kLoaderWarp0 = kMmaWarp + 4;
@@ -52,6 +72,34 @@ static_assert(32 * kEpiWarps * kRegsEpi + (kThreads - 32 * kEpiWarps) * kRegsOth
 static_assert(kLoaders * 32 == kKeysPerTile, "one 32-row box per loader");
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 16;      // key-scale ring: 128 fp32 per tile, released by the epilogue
+constexpr int kMaxStage = 32;        // staging slots (fused mode)
+constexpr int kMaxRows = 32;         // rows (queries) per unit in fused mode
+
+// Fused mode: shared-memory areas after the weights, as byte offsets from `base`.
+struct FusedLayout {
+  uint32_t stg_key, stg_pos, stg_cnt;      // [n_stage][qb][128], same, [n_stage][qb][4]
+  uint32_t theta;                          // [kMaxRows] u64: (unit ordinal << 32) | threshold key
+  uint32_t row_n, row_thr, row_min, row_max;   // [kMaxRows] each, selector-owned
+  uint32_t hist, cand;                     // [kSelWarps][kSelBins], [kSelWarps][kSelCandCap + 4]
+  uint32_t end;
+};
+__host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ inline FusedLayout fused_layout(uint32_t base, int qb, int n_stage) {
+  FusedLayout L{};
+  const uint32_t entries = (uint32_t)n_stage * qb * 128u;
+  L.stg_key = align_up(base, 16);
+  L.stg_pos = L.stg_key + entries * 4;
+  L.stg_cnt = L.stg_pos + entries * 4;
+  L.theta = align_up(L.stg_cnt + (uint32_t)n_stage * qb * 16u, 16);
+  L.row_n = L.theta + kMaxRows * 8;
+  L.row_thr = L.row_n + kMaxRows * 4;
+  L.row_min = L.row_thr + kMaxRows * 4;
+  L.row_max = L.row_min + kMaxRows * 4;
+  L.hist = align_up(L.row_max + kMaxRows * 4, 16);
+  L.cand = L.hist + kSelWarps * kSelBins * 4;
+  L.end = L.cand + kSelWarps * (kSelCandCap + 4) * 4;
+  return L;
+}
 
 struct IndexerSmem {
   // Barriers and small per-unit data first; big tiles follow at a 1024-byte boundary.
@@ -59,6 +107,7 @@ struct IndexerSmem {
   uint64_t k_full[kMaxStages], k_empty[kMaxStages];
   uint64_t acc_full[8], acc_empty[8];     // TMEM accumulators: 512 / N of them (at most 8)
   uint64_t sc_full[kScaleSlots], sc_empty[kScaleSlots];
+  uint64_t stg_full[kMaxStage], stg_empty[kMaxStage];   // staging ring (fused mode)
   uint64_t final_bar;
   uint64_t epi_bar;          // rendezvous of the epilogue warps
   uint32_t tmem_base;
@@ -92,7 +141,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const IndexerParams& p, int u) {
   return info;
 }
 
-template <int H_I, int D_I, int kStages>
+template <int H_I, int D_I, int kStages, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_s, const IndexerParams p) {
@@ -116,6 +165,17 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   float* sc_smem = reinterpret_cast<float*>(k_smem + (size_t)kStages * kKeysPerTile * kRowBytes);
   float* w_smem = sc_smem + kScaleSlots * kKeysPerTile;   // 2 x QU * H_I (per unit, double-buffered)
   float* sq_smem = w_smem + 2 * QU * H_I;                  // 2 x QU
+  // fused mode: staging ring, per-row thresholds and selector state
+  const FusedLayout FL = fused_layout((uint32_t)(reinterpret_cast<uint8_t*>(sq_smem + 2 * QU) - tiles), p.qb,
+                                      p.n_stage);
+  uint32_t* stg_key = reinterpret_cast<uint32_t*>(tiles + FL.stg_key);
+  uint32_t* stg_pos = reinterpret_cast<uint32_t*>(tiles + FL.stg_pos);
+  uint32_t* stg_cnt = reinterpret_cast<uint32_t*>(tiles + FL.stg_cnt);
+  volatile unsigned long long* theta = reinterpret_cast<volatile unsigned long long*>(tiles + FL.theta);
+  uint32_t* row_n = reinterpret_cast<uint32_t*>(tiles + FL.row_n);
+  uint32_t* row_thr = reinterpret_cast<uint32_t*>(tiles + FL.row_thr);
+  uint32_t* row_min = reinterpret_cast<uint32_t*>(tiles + FL.row_min);
+  uint32_t* row_max = reinterpret_cast<uint32_t*>(tiles + FL.row_max);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -134,9 +194,21 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       mbar_init(&S.acc_full[s], 1);
       mbar_init(&S.acc_empty[s], N <= 64 ? 4 : kEpiWarps);
     }
+    // A tile's key scales are read by the warps that process its accumulators: all
+    // sixteen when an accumulator spans the quads, else the quads that own one of
+    // its sub-blocks (consecutive accumulators go to consecutive quads).
+    const int sc_readers = N <= 64 ? 4 * min(p.nsub, kQuads) : kEpiWarps;
     for (int s = 0; s < kScaleSlots; ++s) {
       mbar_init(&S.sc_full[s], 1);
-      mbar_init(&S.sc_empty[s], kEpiWarps);
+      mbar_init(&S.sc_empty[s], sc_readers);
+    }
+    if (kFused) {
+      for (int s = 0; s < p.n_stage; ++s) {
+        mbar_init(&S.stg_full[s], N <= 64 ? 4 : kEpiWarps);
+        mbar_init(&S.stg_empty[s], min(kSelWarps, p.rows_per_unit));   // selectors that own a row
+      }
+      // No unit owns a threshold yet (unit ordinals start at 0).
+      for (int r = 0; r < kMaxRows; ++r) theta[r] = 0xffffffff00000000ull;
     }
     mbar_init(&S.final_bar, 1);
     mbar_init(&S.epi_bar, kEpiWarps);
@@ -236,6 +308,178 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       mma_commit(&S.final_bar);
       mbar_wait(&S.final_bar, 0, nullptr);
     }
+  } else if (kFused && warp >= (uint32_t)kSelWarp0 && warp < (uint32_t)(kSelWarp0 + kSelWarps)) {
+    // ------------------------------------------------------------ selectors
+    // Selector `me` owns the unit's rows r with r % kSelWarps == me.  It consumes
+    // every staging slot in order (releasing it for the epilogue) and appends its
+    // rows' staged candidates to their lists.
+    const int me = (int)warp - kSelWarp0;
+    const int RPU = p.rows_per_unit;
+    const bool active = me < RPU;            // a unit with fewer rows than selectors leaves some idle
+    const uint32_t k = (uint32_t)p.k;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(tiles + FL.hist) + me * kSelBins;
+    uint32_t* cand = reinterpret_cast<uint32_t*>(tiles + FL.cand) + me * (kSelCandCap + 4);
+    auto list_key = [&](int slot_id, int r) { return p.xkey + ((size_t)slot_id * RPU + r) * p.cap; };
+    auto list_pos = [&](int slot_id, int r) { return p.xpos + ((size_t)slot_id * RPU + r) * p.cap; };
+    // Top-k threshold of one list of n > k candidates with keys in [lo, hi].
+    auto threshold_of = [&](const uint32_t* xk, uint32_t n, uint32_t lo, uint32_t hi, uint32_t& thr,
+                            uint32_t& gt) {
+      auto visit = [&](auto&& f) {
+        for (uint32_t i = lane; i < n; i += 32) f(__ldcg(xk + i));
+      };
+      warp_find_threshold(hist, cand, visit, k, lo, hi, thr, gt);
+    };
+    // Cut a row's list to its top-k in place and raise the row's threshold.
+    auto cut = [&](int r, uint32_t* xk, uint32_t* xp, uint32_t ucount) {
+      const uint32_t n = row_n[r];
+      uint32_t thr, gt;
+      threshold_of(xk, n, row_min[r], row_max[r], thr, gt);
+      auto seg = [&](int) { return CandSeg{xk, xp, (int)n}; };
+      warp_compact(seg, 1, thr, k - gt, 0, [&](uint32_t at, uint32_t key, uint32_t pos) {
+        __stcg(xk + at, key);
+        __stcg(xp + at, pos);
+      });
+      __syncwarp();
+      if (lane == 0) {
+        row_n[r] = k;
+        row_thr[r] = thr;
+        row_min[r] = thr;
+        theta[r] = ((unsigned long long)ucount << 32) | thr;
+      }
+      __syncwarp();
+    };
+    // Final output of one row from the concatenated segments get_seg(0 .. nseg-1)
+    // (position order), holding `total` candidates with keys in [lo, hi].
+    auto emit_row = [&](size_t row, auto get_seg, int nseg, uint32_t total, uint32_t lo, uint32_t hi) {
+      int32_t* oi = p.indices + row * (size_t)p.k;
+      float* os = p.sel_scores ? p.sel_scores + row * (size_t)p.k : nullptr;
+      auto emit = [&](uint32_t at, uint32_t key, uint32_t pos) {
+        oi[at] = (int32_t)pos;
+        if (os) os[at] = key_to_score(key);
+      };
+      uint32_t m;
+      if (total > k) {
+        uint32_t thr, gt;
+        auto visit = [&](auto&& f) {
+          for (int g = 0; g < nseg; ++g) {
+            const CandSeg sg = get_seg(g);
+            for (int i = (int)lane; i < sg.n; i += 32) f(__ldcg(sg.key + i));
+          }
+        };
+        warp_find_threshold(hist, cand, visit, k, lo, hi, thr, gt);
+        m = warp_compact(get_seg, nseg, thr, k - gt, 0, emit);
+      } else {
+        m = warp_compact(get_seg, nseg, 0u, 0u, 0, emit);   // every candidate (all keys > 0)
+      }
+      for (uint32_t j = m + lane; j < k; j += 32) {
+        oi[j] = -1;
+        if (os) os[j] = -INFINITY;
+      }
+    };
+
+    uint32_t seq = 0, ucount = 0;
+    for (int u = blockIdx.x; active && u < p.n_units; u += gridDim.x, ++ucount) {
+      const UnitInfo U = decode_unit(p, u);
+      const int ls = p.kchunks == 1 ? (int)blockIdx.x : u;      // list slot of this unit
+      if (lane == 0)
+        for (int r = me; r < RPU; r += kSelWarps) {
+          row_n[r] = 0;
+          row_thr[r] = 0;
+          row_min[r] = 0xffffffffu;
+          row_max[r] = 0;
+        }
+      __syncwarp();
+      bool ok = true;
+      for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
+        for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
+          const uint32_t gs = seq % (uint32_t)p.n_stage;
+          if (!mbar_wait_warp(&S.stg_full[gs], (seq / (uint32_t)p.n_stage) & 1u, abort_flag)) { ok = false; break; }
+          for (int qi = 0; qi < p.qb; ++qi) {
+            const int r = sb * p.qb + qi;
+            if (r % kSelWarps != me || U.i0 + r >= p.Lq) continue;
+            uint32_t* xk = list_key(ls, r);
+            uint32_t* xp = list_pos(ls, r);
+            const uint32_t* cnt = stg_cnt + (gs * p.qb + qi) * 4;
+            const uint32_t c0 = cnt[0], c1 = cnt[1], c2 = cnt[2], c3 = cnt[3];
+            if (row_n[r] + c0 + c1 + c2 + c3 > (uint32_t)p.cap) cut(r, xk, xp, ucount);
+            uint32_t n = row_n[r];
+            const uint32_t th = row_thr[r];
+            const uint32_t* sk = stg_key + (gs * p.qb + qi) * 128;
+            const uint32_t* sp = stg_pos + (gs * p.qb + qi) * 128;
+            uint32_t mn = 0xffffffffu, mx = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t cq = q == 0 ? c0 : q == 1 ? c1 : q == 2 ? c2 : c3;
+              uint32_t key = 0, pos = 0;
+              if (lane < cq) {
+                key = sk[q * 32 + lane];
+                pos = sp[q * 32 + lane];
+              }
+              const bool keep = lane < cq && key > th;
+              const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+              if (keep) {
+                const uint32_t at = n + __popc(bal & lt);
+                __stcg(xk + at, key);
+                __stcg(xp + at, pos);
+                mn = min(mn, key);
+                mx = max(mx, key);
+              }
+              n += __popc(bal);
+            }
+            mn = __reduce_min_sync(0xffffffffu, mn);
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            __syncwarp();
+            if (lane == 0) {
+              row_n[r] = n;
+              row_min[r] = min(row_min[r], mn);
+              row_max[r] = max(row_max[r], mx);
+            }
+            __syncwarp();
+          }
+          if (lane == 0) mbar_arrive(&S.stg_empty[gs]);
+        }
+      }
+      if (!ok) break;
+      // ---- the unit's rows are complete: output them, or hand them to the last chunk
+      for (int r = me; r < RPU; r += kSelWarps) {
+        if (U.i0 + r >= p.Lq) continue;
+        const size_t row = (size_t)U.b * p.Lq + U.i0 + r;
+        uint32_t* xk = list_key(ls, r);
+        uint32_t* xp = list_pos(ls, r);
+        if (p.kchunks == 1) {
+          const uint32_t n = row_n[r];
+          auto seg = [&](int) { return CandSeg{xk, xp, (int)n}; };
+          emit_row(row, seg, 1, n, row_min[r], row_max[r]);
+          __syncwarp();
+          continue;
+        }
+        if (row_n[r] > k) cut(r, xk, xp, ucount);
+        if (lane == 0)
+          __stcg(p.xmeta + (size_t)u * RPU + r, make_uint4(row_n[r], row_min[r], row_max[r], 0u));
+        __threadfence();
+        __syncwarp();
+        uint32_t prev = 0;
+        if (lane == 0) prev = atomicAdd(p.done + row, 1u);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev != (uint32_t)p.kchunks - 1) continue;
+        // Last chunk of this row: select over every chunk's list, in chunk (= position) order.
+        __threadfence();
+        const int u0 = u - u % p.kchunks;
+        auto seg = [&](int c) {
+          const uint4 m = __ldcg(p.xmeta + (size_t)(u0 + c) * RPU + r);
+          return CandSeg{list_key(u0 + c, r), list_pos(u0 + c, r), (int)m.x};
+        };
+        uint32_t total = 0, lo = 0xffffffffu, hi = 0;
+        for (int c = 0; c < p.kchunks; ++c) {
+          const uint4 m = __ldcg(p.xmeta + (size_t)(u0 + c) * RPU + r);
+          total += m.x;
+          if (m.x) { lo = min(lo, m.y); hi = max(hi, m.z); }
+        }
+        emit_row(row, seg, p.kchunks, total, lo, hi);
+        __syncwarp();
+      }
+    }
   }
   } else {
     regs_increase<kRegsEpi>();
@@ -294,11 +538,20 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       float sk_next = p.scale_ring ? 0.f : key_scale(U.kt0);
       for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
         const int s = kt * kKeysPerTile + (int)row;
-        float sk;
+        float sk = 0.f;
         const uint32_t ss = sc_use % kScaleSlots;
+        // In narrow mode this warp reads the tile only if its quad owns one of the
+        // tile's accumulators (seq .. seq + nsub - 1).
+        bool reads_tile = true;
+        if (narrow) {
+          reads_tile = false;
+          for (int sb = 0; sb < p.nsub; ++sb) reads_tile |= ((seq + sb) % kQuads == quad);
+        }
         if (p.scale_ring) {
-          if (!mbar_wait_warp(&S.sc_full[ss], (sc_use / kScaleSlots) & 1u, abort_flag)) { ok = false; break; }
-          sk = sc_smem[ss * kKeysPerTile + row];
+          if (reads_tile) {
+            if (!mbar_wait_warp(&S.sc_full[ss], (sc_use / kScaleSlots) & 1u, abort_flag)) { ok = false; break; }
+            sk = sc_smem[ss * kKeysPerTile + row];
+          }
         } else {
           sk = sk_next;
           sk_next = key_scale(kt + 1);
@@ -307,15 +560,38 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           const uint32_t slot = seq % nslot, use = seq / nslot;
           if (narrow && seq % kQuads != quad) continue;
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
+          uint32_t gs = 0;                                   // staging slot (fused mode)
+          if constexpr (kFused) {
+            gs = seq % (uint32_t)p.n_stage;
+            if (!mbar_wait_warp(&S.stg_empty[gs], ((seq / (uint32_t)p.n_stage) & 1u) ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+          }
           tc_fence_after();
           const uint32_t t_base = tmem_base + ((quarter * 32u) << 16) + slot * (uint32_t)N;
           // One query's score for this lane's key: ReLU, weighting and head sum over its
           // H_I columns (two interleaved partial sums, packed FMA), then the scales and
-          // the causal mask.
+          // the causal mask.  Scores mode stores it; fused mode stages it (warp-wide
+          // call) if it beats the row's current threshold.
           auto finish = [&](int qi, float acc) {
             const int qq = sb * p.qb + qi;
             const int i = U.i0 + qq;
-            if (i < p.Lq && s < p.Lk) {
+            if constexpr (kFused) {
+              const bool valid = i < p.Lq && s < p.Lk && s <= p.q_offset + i;
+              const uint32_t key = score_to_key(acc * sqbuf[qq] * sk);
+              const unsigned long long tv = theta[qq];
+              const uint32_t th = (uint32_t)(tv >> 32) == ucount ? (uint32_t)tv : 0u;
+              const bool pass = valid && key > th;
+              const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+              const uint32_t base = (gs * (uint32_t)p.qb + (uint32_t)qi) * 128u + quarter * 32u;
+              if (pass) {
+                const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
+                stg_key[at] = key;
+                stg_pos[at] = (uint32_t)s;
+              }
+              if (lane == 0) stg_cnt[(gs * (uint32_t)p.qb + (uint32_t)qi) * 4u + quarter] = __popc(bal);
+            } else if (i < p.Lq && s < p.Lk) {
               const int t = p.q_offset + i;
               float* dst = p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s;
               if (s <= t)
@@ -373,17 +649,20 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S.acc_empty[slot]);
+          if (lane == 0) {
+            mbar_arrive(&S.acc_empty[slot]);
+            if (kFused) mbar_arrive(&S.stg_full[gs]);
+          }
         }
         if (p.scale_ring) {
           __syncwarp();
-          if (lane == 0) mbar_arrive(&S.sc_empty[ss]);
+          if (reads_tile && lane == 0) mbar_arrive(&S.sc_empty[ss]);
           ++sc_use;
         }
       }
       if (!ok) break;
       // Full-matrix output: positions beyond this unit's causal tiles are -inf.
-      if (p.fill_upper && p.kchunks == 1) {
+      if (!kFused && p.fill_upper && p.kchunks == 1) {
         const int nt_all = (p.Lk + kKeysPerTile - 1) / kKeysPerTile;
         for (int kt = U.kt1; kt < nt_all; ++kt) {
           const int s = kt * kKeysPerTile + (int)row;
@@ -407,13 +686,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   }
 }
 
-template <int H_I, int D_I, int kStages>
+template <int H_I, int D_I, int kStages, bool kFused>
 cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                             const CUtensorMap& ts,
-                             int grid, cudaStream_t stream) {
-  const size_t smem = indexer_smem_bytes(p.nsub * p.qb * H_I, D_I, p.queries_per_unit * H_I,
-                                         p.queries_per_unit, kStages);
-  auto kern = indexer_kernel<H_I, D_I, kStages>;
+                             const CUtensorMap& ts, int grid, cudaStream_t stream) {
+  const size_t smem = indexer_smem_bytes(p.nsub * p.qb * H_I, D_I, p.queries_per_unit * H_I, p.queries_per_unit,
+                                         kStages, kFused, p.qb, p.n_stage, p.rows_per_unit);
+  auto kern = indexer_kernel<H_I, D_I, kStages, kFused>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // The register split must fit in what the CTA launches with, or the increase
@@ -428,25 +706,40 @@ cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, cons
 
 }  // namespace
 
-size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages) {
-  size_t b = sizeof(IndexerSmem) + 1024;                       // barriers + alignment slack
-  b += query_buffers((uint32_t)(q_rows * d_I)) * (size_t)q_rows * d_I;   // query block buffers
-  b += (size_t)stages * kKeysPerTile * d_I;                    // key ring
-  b += (size_t)kScaleSlots * kKeysPerTile * sizeof(float);      // key-scale ring
-  b += 2 * (size_t)(w_floats + sq_floats) * sizeof(float);     // weights / query scales, double-buffered
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages, bool fused, int qb,
+                          int n_stage, int rows_per_unit) {
+  (void)rows_per_unit;
+  size_t t = query_buffers((uint32_t)(q_rows * d_I)) * (size_t)q_rows * d_I;   // query block buffers
+  t += (size_t)stages * kKeysPerTile * d_I;                    // key ring
+  t += (size_t)kScaleSlots * kKeysPerTile * sizeof(float);      // key-scale ring
+  t += 2 * (size_t)(w_floats + sq_floats) * sizeof(float);     // weights / query scales, double-buffered
+  if (fused) t = fused_layout((uint32_t)t, qb, n_stage).end;    // staging ring + selector areas
+  const size_t b = sizeof(IndexerSmem) + 1024 + t;             // barriers + alignment slack
   // At least ~116 KB so that one CTA (and its 512 TMEM columns) owns each SM.
   return b < 118784 ? 118784 : b;
 }
 
+int indexer_fused_max_rows() { return kMaxRows; }
+int indexer_fused_max_stage() { return kMaxStage; }
+
 cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                           const CUtensorMap& ts,
-                           int grid, cudaStream_t stream) {
+                           const CUtensorMap& ts, int grid, cudaStream_t stream) {
   // A small resident query block (decode) leaves room for a deeper key ring.
   const bool deep = p.nsub * p.qb * p.H_I <= 128;
-  if (p.H_I == 64 && p.d_I == 128)
-    return deep ? launch_indexer_t<64, 128, 12>(p, tq, tk, ts, grid, stream)
-                : launch_indexer_t<64, 128, 4>(p, tq, tk, ts, grid, stream);
-  if (p.H_I == 4 && p.d_I == 64) return launch_indexer_t<4, 64, 4>(p, tq, tk, ts, grid, stream);
+  const bool fused = p.scores == nullptr;
+  if (fused && (p.rows_per_unit > kMaxRows || p.n_stage > kMaxStage || p.n_stage < 1 || p.cap < p.k + 128 ||
+                p.cap % 32 != 0))
+    return cudaErrorInvalidValue;
+  if (p.H_I == 64 && p.d_I == 128) {
+    if (fused)
+      return deep ? launch_indexer_t<64, 128, 8, true>(p, tq, tk, ts, grid, stream)
+                  : launch_indexer_t<64, 128, 4, true>(p, tq, tk, ts, grid, stream);
+    return deep ? launch_indexer_t<64, 128, 12, false>(p, tq, tk, ts, grid, stream)
+                : launch_indexer_t<64, 128, 4, false>(p, tq, tk, ts, grid, stream);
+  }
+  if (p.H_I == 4 && p.d_I == 64)
+    return fused ? launch_indexer_t<4, 64, 4, true>(p, tq, tk, ts, grid, stream)
+                 : launch_indexer_t<4, 64, 4, false>(p, tq, tk, ts, grid, stream);
   return cudaErrorInvalidValue;
 }
 

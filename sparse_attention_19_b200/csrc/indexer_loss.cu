@@ -423,16 +423,19 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       const int32_t* idx = idx_sm + ib * kMaxIdx;
       const int nt = row_tiles(S.last_word, ib);
       const int bLk = (row / p.Lq) * p.Lk;
-      const float* srow = p.scores + (size_t)row * p.Lk;
+      const float* srow = p.scores ? p.scores + (size_t)row * p.Lk : nullptr;
       float* trow = p.target ? p.target + (size_t)row * p.k : nullptr;
       RowSums acc{0.f, 0.f, 0.f, -INFINITY, 0.f};
       // The indexer score of this thread's key in tile j (0 for padding or past the
       // row's tiles); fetched four tiles before it is used, so that its DRAM latency
       // stays off the chain.
+      const float* selrow = p.sel_scores ? p.sel_scores + (size_t)row * p.k : nullptr;
       auto fetch = [&](int j) -> float {
         if (j >= nt) return 0.f;
-        const int32_t gr = idx[j * kTileKeys + key];
-        return gr >= 0 ? __ldg(srow + (gr - bLk)) : 0.f;
+        const int slot = j * kTileKeys + key;
+        const int32_t gr = idx[slot];
+        if (gr < 0) return 0.f;
+        return selrow ? __ldg(selrow + slot) : __ldg(srow + (gr - bLk));
       };
       auto consume = [&](int j, float iv) -> bool {
         const int slot_x = j * kTileKeys + key;

@@ -162,7 +162,7 @@ __device__ __forceinline__ int gather_row(const int32_t* rows, int pos) {
 template <int NC, int DV>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
-                   const AttnParams p) {
+                   const __grid_constant__ CUtensorMap tmap_kv_tile, const AttnParams p) {
   using VS = VShape<DV>;
   static_assert(NC <= kMaxChunks, "d_qk");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -232,7 +232,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const int part = pw % kKTeamWarps;
       uint32_t ucount = 0, kc = 0;
       bool ok = true;
-      if (pw == 0 && lane == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_kv); }
+      if (pw == 0 && lane == 0) {
+        prefetch_tmap(&tmap_q);
+        prefetch_tmap(p.dense ? &tmap_kv_tile : &tmap_kv);
+      }
       Unit U;
       for (int u = next_unit(p, cluster_id, n_clusters, U); u < p.n_units && ok;
            u = next_unit(p, u + n_clusters, n_clusters, U)) {
@@ -262,6 +265,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             }
             if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
             const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
+            if (p.dense) {
+              // keys 0..t are contiguous: this CTA's 64 rows of the tile in one box
+              if (part == 0 && lane == 0)
+                tma_load_2d_pair(k_sm + st * kPlane64, &tmap_kv_tile, full_l, c * 64,
+                                 U.b * p.Lk + j * kTileKeys + (int)rank * kHalfKeys);
+              continue;
+            }
             const int g = part + kKTeamWarps * (int)lane;            // 4-key group of this lane
             if (g < kHalfKeys / 4) {
               const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
@@ -295,6 +305,26 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         int32_t* dst = idx_sm + buf * kMaxIdx;
         uint32_t* vmask = S.valid_mask[buf];
         const int x_begin = V.j0 * kTileKeys, nwords = (V.j1 - V.j0) * (kTileKeys / 32);
+        if (p.dense) {
+          // Row t selects every position 0..t (in slot order); the loads need no
+          // staged rows, only the validity words.  The leader also writes the
+          // row's index list, and the first split its tail of -1 slots.
+          int32_t* io = p.idx_out + (size_t)V.row * p.k;
+          for (int w = pw; w < nwords; w += kVWarps) {
+            const int x = x_begin + w * 32 + (int)lane;
+            const bool valid = x <= V.t && x < p.k;
+            const uint32_t bal = __ballot_sync(0xffffffffu, valid);
+            if (lane == 0) vmask[w] = bal;
+            if (leader && x < p.k) io[x] = valid ? x : -1;
+          }
+          if (leader && V.split == 0) {
+            const int nt_row = (min(p.k, V.t + 1) + kTileKeys - 1) / kTileKeys;
+            for (int x = nt_row * kTileKeys + pw * 32 + (int)lane; x < p.k; x += kVWarps * 32) io[x] = -1;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.idx_full[buf]);
+          return;
+        }
         const int32_t* src = p.indices + (size_t)V.row * p.k;
         for (int w0 = pw; w0 < nwords; w0 += kVWarps * kStageBatch) {
           int sidx[kStageBatch];
@@ -344,6 +374,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
               }
               if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
               const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
+              if (p.dense) {
+                // 64 contiguous keys x this CTA's value columns: one box per plane
+                if (part == 0 && lane < (uint32_t)VS::kPlanes) {
+                  const int col = h * VS::kN + (int)rank * (VS::kN / 2) + (int)lane * 64;
+                  tma_load_2d_pair(v_sm + st * VS::kStageBytes + lane * kPlane64, &tmap_kv_tile, full_l, col,
+                                   U.b * p.Lk + j * kTileKeys + kh * kHalfKeys);
+                }
+                continue;
+              }
               const int g = part + kVWarpsPerSlot * (int)lane;
               if (g < 16 * VS::kPlanes) {
                 const int pl = g / 16, kg = g % 16;
@@ -670,8 +709,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
 }
 
 template <int NC, int DV>
-cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkv, int grid_clusters,
-                     cudaStream_t stream) {
+cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tkv,
+                     const CUtensorMap& tkv_tile, int grid_clusters, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes(NC * 64, DV);
   auto kern = sparse_attn_kernel<NC, DV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -682,7 +721,7 @@ cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorM
   e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
   if ((uint32_t)fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
-  kern<<<grid_clusters * 2, kThreads, smem, stream>>>(tq, tkv, p);
+  kern<<<grid_clusters * 2, kThreads, smem, stream>>>(tq, tkv, tkv_tile, p);
   return cudaGetLastError();
 }
 
@@ -702,9 +741,10 @@ size_t attn_smem_bytes(int d_qk, int d_v) {
 }
 
 cudaError_t launch_sparse_attn(const AttnParams& p, int d_qk, int d_v, const CUtensorMap& tq,
-                               const CUtensorMap& tkv, int grid_clusters, cudaStream_t stream) {
-  if (d_qk == 576 && d_v == 512) return launch_t<9, 512>(p, tq, tkv, grid_clusters, stream);
-  if (d_qk == 192 && d_v == 128) return launch_t<3, 128>(p, tq, tkv, grid_clusters, stream);
+                               const CUtensorMap& tkv, const CUtensorMap& tkv_tile, int grid_clusters,
+                               cudaStream_t stream) {
+  if (d_qk == 576 && d_v == 512) return launch_t<9, 512>(p, tq, tkv, tkv_tile, grid_clusters, stream);
+  if (d_qk == 192 && d_v == 128) return launch_t<3, 128>(p, tq, tkv, tkv_tile, grid_clusters, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -1,0 +1,184 @@
+// warp_select.cuh -- exact top-k selection by one warp over candidate lists kept in
+// global memory (L2), for the fused indexer + top-k.
+//
+// A candidate is (key, position): key is the order-preserving 32-bit image of an
+// fp32 indexer score (larger key = larger score, -0.0 folded onto +0.0) and
+// position the key token's index s.  Lists are kept in increasing position order.
+// The selection order is "key descending, then position ascending" (ties go to
+// the smaller position), the reading of the top-k step ("Отбор и основное
+// внимание") that makes index sets unique.
+//
+// The top-m of a list is described by a threshold key thr and a count eq_take:
+// every candidate with key > thr, plus the first eq_take candidates (in position
+// order) with key == thr.  warp_find_threshold() finds (thr, gt = #{key > thr})
+// by histogram refinement over the list's key range; warp_compact() then walks
+// the list once, in order, and keeps exactly those candidates, so the output stays
+// in position order.
+#pragma once
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace dsa {
+
+constexpr int kSelBins = 2048;          // histogram bins per refinement level
+constexpr int kSelBinBits = 11;
+constexpr int kSelCandCap = 512;        // boundary-bin keys gathered into shared memory
+
+__device__ __forceinline__ uint32_t score_to_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if ((u << 1) == 0u) u = 0u;                          // -0.0 -> +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// Right shift mapping a key window of width range+1 onto at most kSelBins bins.
+__device__ __forceinline__ int sel_shift(uint32_t range) {
+  return range == 0u ? 0 : max(0, 32 - __clz(range) - kSelBinBits);
+}
+
+// A run of candidates in global memory (keys[i], pos[i]), i < n.
+struct CandSeg {
+  const uint32_t* key;
+  const uint32_t* pos;
+  int n;
+};
+
+// One refinement level: histogram of the keys in [lo, lo + (kSelBins << shift)) that
+// `visit` produces, then the bin b (from the top) where the running count first
+// reaches `need`, and the count strictly above bin b.  `hist` is this warp's
+// shared-memory histogram.
+template <typename Visit>
+__device__ __forceinline__ void sel_level(uint32_t* hist, Visit visit, uint32_t lo, uint32_t hi, int shift,
+                                          uint32_t need, uint32_t& bin, uint32_t& above) {
+  const uint32_t lane = threadIdx.x & 31u;
+  for (int i = (int)lane; i < kSelBins / 4; i += 32) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0, 0, 0, 0);
+  __syncwarp();
+  visit([&](uint32_t key) {
+    if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) >> shift], 1u);
+  });
+  __syncwarp();
+  // Lane j owns bins [64 j, 64 j + 64).  Counts from the top: suffix sums over lanes.
+  constexpr int kPer = kSelBins / 32;
+  uint32_t mine = 0;
+  const uint4* h4 = reinterpret_cast<const uint4*>(hist + lane * kPer);
+#pragma unroll
+  for (int i = 0; i < kPer / 4; ++i) {
+    const uint4 v = h4[i];
+    mine += v.x + v.y + v.z + v.w;
+  }
+  uint32_t suffix = mine;                              // bins of lanes >= this lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, suffix, o);
+    if (lane + o < 32) suffix += y;
+  }
+  const uint32_t above_lane = suffix - mine;           // bins of lanes > this lane
+  const bool here = above_lane < need && suffix >= need;
+  const uint32_t owner = __ffs(__ballot_sync(0xffffffffu, here)) - 1;
+  uint32_t b = 0, ab = 0;
+  if (lane == owner) {
+    uint32_t acc = above_lane;
+    for (int i = kPer - 1; i >= 0; --i) {
+      const uint32_t c = hist[lane * kPer + i];
+      if (acc + c >= need) { b = lane * kPer + i; ab = acc; break; }
+      acc += c;
+    }
+  }
+  bin = __shfl_sync(0xffffffffu, b, owner);
+  above = __shfl_sync(0xffffffffu, ab, owner);
+  __syncwarp();
+}
+
+// Threshold of the top-`m` of the candidates that `visit` produces, all of whose
+// keys lie in [lo, hi] and of which there are more than m.  Returns thr and
+// gt = #{key > thr} (so m - gt candidates equal to thr are taken, the first ones
+// in position order).  `cand` holds up to kSelCandCap keys of the boundary bin.
+template <typename Visit>
+__device__ void warp_find_threshold(uint32_t* hist, uint32_t* cand, Visit visit, uint32_t m, uint32_t lo,
+                                    uint32_t hi, uint32_t& thr, uint32_t& gt) {
+  const uint32_t lane = threadIdx.x & 31u;
+  uint32_t need = m, got = 0;
+  // Levels over the list itself until the boundary bin is small enough to copy.
+  for (;;) {
+    const int shift = sel_shift(hi - lo);
+    uint32_t b, above;
+    sel_level(hist, visit, lo, hi, shift, need, b, above);
+    got += above;
+    need -= above;
+    if (shift == 0) { thr = lo + b; gt = got; return; }
+    const uint32_t nb = hist[b];
+    lo = lo + (b << shift);
+    const unsigned long long top = (unsigned long long)lo + (1ull << shift) - 1ull;
+    hi = top < (unsigned long long)hi ? (uint32_t)top : hi;
+    __syncwarp();
+    if (nb <= (uint32_t)kSelCandCap) break;
+  }
+  // Copy the boundary bin's keys (at most kSelCandCap) to shared memory and refine there.
+  uint32_t* ncand = cand + kSelCandCap;                // counter word after the keys
+  if (lane == 0) *ncand = 0u;
+  __syncwarp();
+  visit([&](uint32_t key) {
+    if (key >= lo && key <= hi) {
+      const uint32_t at = atomicAdd(ncand, 1u);
+      if (at < (uint32_t)kSelCandCap) cand[at] = key;
+    }
+  });
+  __syncwarp();
+  const int nc = (int)*ncand;
+  auto visit_cand = [&](auto&& f) {
+    for (int i = (int)lane; i < nc; i += 32) f(cand[i]);
+  };
+  for (;;) {
+    const int shift = sel_shift(hi - lo);
+    uint32_t b, above;
+    sel_level(hist, visit_cand, lo, hi, shift, need, b, above);
+    got += above;
+    need -= above;
+    if (shift == 0) { thr = lo + b; gt = got; return; }
+    lo = lo + (b << shift);
+    const unsigned long long top = (unsigned long long)lo + (1ull << shift) - 1ull;
+    hi = top < (unsigned long long)hi ? (uint32_t)top : hi;
+    __syncwarp();
+  }
+}
+
+// Stable selection pass: walks the segments get_seg(0 .. nseg-1) in order, 32
+// candidates at a time, and hands every kept candidate to emit(index, key, pos)
+// with consecutive indices from `base`: all keys > thr and the first eq_take keys
+// == thr.  Returns the count.
+// Each batch of 32 is read completely before any of it is emitted, so emitting
+// into the list being read (at an index not above the one read) is safe.
+template <typename GetSeg, typename Emit>
+__device__ uint32_t warp_compact(GetSeg get_seg, int nseg, uint32_t thr, uint32_t eq_take, uint32_t base,
+                                 Emit emit) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t w = base, eq_seen = 0;
+  for (int g = 0; g < nseg; ++g) {
+    const CandSeg sg = get_seg(g);
+    for (int i0 = 0; i0 < sg.n; i0 += 32) {
+      const int i = i0 + (int)lane;
+      uint32_t key = 0, pos = 0;
+      if (i < sg.n) {
+        key = __ldcg(sg.key + i);
+        pos = __ldcg(sg.pos + i);
+      }
+      __syncwarp();
+      const bool valid = i < sg.n;
+      const uint32_t eq = __ballot_sync(0xffffffffu, valid && key == thr);
+      const bool take_eq = valid && key == thr && eq_seen + __popc(eq & lt) < eq_take;
+      const bool keep = (valid && key > thr) || take_eq;
+      const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+      if (keep) emit(w + __popc(kb & lt), key, pos);
+      w += __popc(kb);
+      eq_seen += __popc(eq);
+      __syncwarp();
+    }
+  }
+  return w - base;
+}
+
+}  // namespace dsa

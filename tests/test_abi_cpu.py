@@ -106,9 +106,48 @@ def test_workspace_sizes():
     assert ws >= 4 * 16 * 128 * 512 * 4
     # 64 rows already occupy most pairs: whole rows per unit, no partials
     assert dsa.workspace_size(dsa.OP_SPARSE_ATTN, 64, 1, 131072, 2048, 128, 512) == 0
+    # The forward's indexer selects on chip: its workspace holds candidate lists
+    # (at most 2k + 256 per row in flight), never the [Lq, Lk] score matrix.
     fwd = dsa.workspace_size(dsa.OP_FORWARD, 1, 4096, 131072, 2048, 128, 512)
-    assert fwd >= 4096 * 131072 * 4
+    assert 0 < fwd < 4096 * 131072 * 4 // 4
+    fwd32 = dsa.workspace_size(dsa.OP_FORWARD, 1, 32768, 32768, 2048, 128, 512)
+    assert 0 < fwd32 < 32768 * 32768 * 4 // 16
     assert dsa.workspace_size(dsa.OP_FORWARD, 0, 1, 1, 1, 1, 1) == 0
+    # the exact query agrees with the convention-based one when q_offset = Lk - Lq
+    ia = _idx_args(B=64, Lq=1, Lk=131072, q_offset=131071)
+    assert dsa.workspace_size_args(dsa.OP_FORWARD, ia, 2048, 128, 512) == \
+        dsa.workspace_size(dsa.OP_FORWARD, 64, 1, 131072, 2048, 128, 512)
+    assert dsa.workspace_size_args(dsa.OP_INDEXER_TOPK, ia, 2048) == \
+        dsa.workspace_size(dsa.OP_INDEXER_TOPK, 64, 1, 131072, 2048, 128, 512) > 0
+    # invalid indexer arguments: no size
+    assert dsa.workspace_size_args(dsa.OP_FORWARD, _idx_args(q_I=None), 2048, 128, 512) == 0
+
+
+def test_indexer_topk_rejects_bad_arguments(L):
+    p = ctypes.c_void_p(16)
+    f = L.dsa_indexer_topk
+    ia = _idx_args(Lq=8, Lk=8)
+    need = dsa.workspace_size_args(dsa.OP_INDEXER_TOPK, ia, 8)
+    assert need > 0
+    assert f(None, 8, p, None, p, need, None) == 1
+    assert f(ctypes.byref(_idx_args(q_I=None)), 8, p, None, p, need, None) == 1
+    assert f(ctypes.byref(ia), 8, None, None, p, need, None) == 1                       # no indices
+    assert f(ctypes.byref(ia), 8, p, ctypes.c_void_p(8), p, need, None) == 1            # misaligned scores
+    assert f(ctypes.byref(ia), 0, p, None, p, need, None) == 2                          # k < 1
+    assert f(ctypes.byref(ia), 4096, p, None, p, need, None) == 2                       # k > 2048
+    assert f(ctypes.byref(_idx_args(H_I=32)), 8, p, None, p, need, None) == 2
+    assert f(ctypes.byref(ia), 8, p, None, p, need - 1, None) == 3                      # workspace too small
+    assert f(ctypes.byref(ia), 8, p, None, None, need, None) == 3
+
+
+def test_indexer_kl_loss_selected_rejects_bad_arguments(L):
+    good = dsa.AttnArgs(128, 576, 512, 0.07, 16, 16)
+    p = ctypes.c_void_p(16)
+    f = L.dsa_indexer_kl_loss_selected
+    assert f(ctypes.byref(good), 1, 1, 8, p, 8, None, p, None, p, None) == 1           # no lse
+    assert f(ctypes.byref(good), 1, 1, 8, p, 8, p, None, None, p, None) == 1           # no selected scores
+    assert f(ctypes.byref(good), 1, 1, 8, p, 8, p, ctypes.c_void_p(8), None, p, None) == 1
+    assert f(ctypes.byref(good), 1, 1, 8, p, 4096, p, p, None, p, None) == 2
 
 
 def test_indexer_kl_loss_rejects_bad_arguments(L):

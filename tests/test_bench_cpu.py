@@ -15,6 +15,8 @@ def test_every_called_name_is_defined():
     for node in ast.walk(tree):
         if isinstance(node, (ast.FunctionDef, ast.ClassDef)):
             defined.add(node.name)
+            if isinstance(node, ast.FunctionDef):      # parameters (callables passed in)
+                defined.update(a.arg for a in node.args.args + node.args.kwonlyargs)
         elif isinstance(node, (ast.Import, ast.ImportFrom)):
             defined.update((a.asname or a.name).split(".")[0] for a in node.names)
         elif isinstance(node, ast.Assign):

@@ -223,8 +223,8 @@ def _forward(inp, wl, q_offset=None, Lq=None):
     return idx, out, lse
 
 
-def _check_forward_rows(inp, wl, idx, out, lse, rows, Lq, q_offset, exact_idx=False):
-    res, keys = P.oracle_forward_rows(inp, rows, Lq, q_offset, wl.k, wl.scale, wl.Dv)
+def _check_forward_rows(inp, wl, idx, out, lse, rows, Lq, q_offset, exact_idx=False, keys=None):
+    res, keys = P.oracle_forward_rows(inp, rows, Lq, q_offset, wl.k, wl.scale, wl.Dv, keys=keys)
     sel = torch.as_tensor(rows, device=DEV)
     gi = idx.reshape(-1, wl.k)[sel].cpu().numpy()
     swaps = P.check_index_sets(gi, res["scores"], res["row_t"], wl.k, exact=exact_idx)
@@ -281,24 +281,53 @@ def test_forward_decode_128k_sampled_sequences():
     _check_forward_rows(inp, wl, idx, out, lse, np.array([0, 17, 40, 63]), 1, wl.q_offset)
 
 
+def _rows_32k(L, k):
+    """512 rows of an L-query prefill: every 64th row of t < k, the last 64 rows,
+    and the rest spread evenly over the middle."""
+    head = np.arange(0, k, 64)
+    tail = np.arange(L - 64, L)
+    mid = np.linspace(k, L - 65, 512 - len(head) - len(tail)).round().astype(np.int64)
+    rows = np.unique(np.r_[head, mid, tail])
+    assert len(rows) == 512
+    return rows
+
+
 def test_forward_prefill_32k_sampled_rows():
     wl = WORKLOADS["prefill_32k"]
     inp = make_inputs(wl, DEV, 0)
     idx, out, lse = _forward(inp, wl)
-    rows = np.r_[0, 5, 2047, 2048, 9000, 16384, 30000, 32766, 32767]
-    _check_forward_rows(inp, wl, idx, out, lse, rows, wl.Lq, 0)
+    _check_forward_rows(inp, wl, idx, out, lse, _rows_32k(wl.Lq, wl.k), wl.Lq, 0)
 
 
-def test_forward_prefill_128k_last_chunk_sampled_rows():
+def test_forward_prefill_128k_chunked_as_benchmarked():
+    # The 32 chunk calls the benchmark times (bench.Runner), 256 rows checked:
+    # eight per chunk, spread over the chunk, in every chunk.
+    from bench import Runner
     wl = WORKLOADS["prefill_128k"]
-    keys = make_key_side(wl, DEV, 0)
-    c = wl.Lq // wl.chunk - 1
-    q_offset = c * wl.chunk
-    qs = make_query_side(wl, DEV, 0, chunk_index=c, Lq=wl.chunk)
-    inp = dict(keys, **qs)
-    cw = wl.with_(Lq=wl.chunk, q_offset=q_offset)
-    idx, out, lse = _forward(inp, cw)
-    _check_forward_rows(inp, cw, idx, out, lse, np.array([0, 2048, 4095]), cw.Lq, q_offset)
+    runner = Runner(wl, seed=0, device=DEV)
+    runner.step(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    keys = oracle.keys_from_inputs(runner.keys)
+    c = runner.chunk_len
+    local = np.linspace(0, c - 1, 8).round().astype(np.int64)
+    for n, (q_offset, qs) in enumerate(runner.chunks):
+        inp = dict(runner.keys, **qs)
+        cw = wl.with_(Lq=c, q_offset=q_offset)
+        sl = slice(n * c, (n + 1) * c)
+        _check_forward_rows(inp, cw, runner.indices[:, sl], runner.out[:, sl], runner.lse[:, sl], local, c,
+                            q_offset, keys=keys)
+    del runner
+    torch.cuda.empty_cache()
+
+
+def test_forward_decode_single_cached_token():
+    # Lk = 1: the one key is selected and every head returns its value row.
+    wl = WORKLOADS["decode_128k"].with_(B=5, Lk=1, q_offset=0)
+    inp = make_inputs(wl, DEV, 4)
+    idx, out, lse = _forward(inp, wl)
+    got = idx.reshape(-1, wl.k).cpu().numpy()
+    assert np.all(got[:, 0] == 0) and np.all(got[:, 1:] == -1)
+    _check_forward_rows(inp, wl, idx, out, lse, np.arange(wl.B), 1, 0, exact_idx=True)
 
 
 def test_wait_timeout_is_reported_not_trapped():
@@ -324,9 +353,15 @@ def test_context_parallel_single_rank_matches_the_whole_sequence():
                for c in mine}
     res = cp.cp_forward(queries, local, 2, chunk, wl.k, wl.Dv, wl.scale, world=1, rank=0)
     torch.cuda.synchronize()
+    keys = oracle.keys_from_inputs(inp)
     for c in mine:
         ci, co, cl = res[c]
         sl = slice(c * chunk, (c + 1) * chunk)
         assert torch.equal(ci, idx[:, sl])
         assert float((co.float() - out[:, sl].float()).abs().max()) <= 1e-2
         assert float((cl - lse[:, sl]).abs().max()) <= 1e-4
+        # each chunk's own result against the oracle, rows spread over the chunk
+        cw = wl.with_(Lq=chunk, q_offset=c * chunk)
+        qin = dict(inp, **queries[c])
+        _check_forward_rows(qin, cw, ci, co, cl, np.r_[0, 1, 700, 1500, chunk - 2, chunk - 1], chunk, c * chunk,
+                            keys=keys)

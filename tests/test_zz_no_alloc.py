@@ -1,19 +1,33 @@
 """dsa_sparse_attn_noalloc (split-k partials in the library's fixed scratch array)
 against dsa_sparse_attn (caller-provided workspace), through the C ABI.
 
+Some callers cannot allocate device memory when they run attention: a serving
+loop that handed all device memory to its own pool at start-up, or code that
+must not risk the device-wide synchronisation that freeing memory brings.
+dsa_sparse_attn_noalloc serves them with a fixed array inside the library.
+
+Both entry points run the same kernels with the same split of each row over
+the key tiles; only the address of the partials differs, so their results must
+be identical bit for bit.  One case is also held against the fp64 oracle.
+
 Collected last on purpose: it must give the same results whether it runs alone
 or after every other test has used the device."""
 import ctypes
+import os
+import re
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 import sparse_attention_19_b200 as dsa
 import parity as P
 
 DEV = "cuda"
 H, D, DV = 128, 576, 512
 SCALE = 192 ** -0.5
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _case(B, Lq, Lk, k, seed, pad_every=0):
@@ -27,14 +41,14 @@ def _case(B, Lq, Lk, k, seed, pad_every=0):
 
 
 def _compare(q, kv, idx):
-    B, Lq, _, _ = q.shape
     ref_out, ref_lse = dsa.sparse_attn(q, kv, idx, DV, SCALE)
     out = torch.full_like(ref_out, float("nan"))
     lse = torch.full_like(ref_lse, float("nan"))
     dsa.sparse_attn_noalloc(q, kv, idx, DV, SCALE, out, lse)
     torch.cuda.synchronize()
-    P.check_attention(out, lse, ref_out.float().cpu().numpy(), ref_lse.cpu().numpy())
-    return out, ref_out
+    assert torch.equal(out, ref_out), "output differs from dsa_sparse_attn"
+    assert torch.equal(lse, ref_lse), "lse differs from dsa_sparse_attn"
+    return out, lse
 
 
 @pytest.mark.gpu
@@ -45,10 +59,16 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
     B, Lq, Lk, k = 4, 1, 8192, 2048
     need = dsa.workspace_size(dsa.OP_SPARSE_ATTN, B, Lq, Lk, k, H, DV)
     assert 0 < need <= dsa.NOALLOC_SCRATCH_BYTES
-    first = _compare(*_case(B, Lq, Lk, k, seed=1))
-    second = _compare(*_case(B, Lq, Lk, k, seed=2, pad_every=3))
+    q, kv, idx = _case(B, Lq, Lk, k, seed=1)
+    first, first_lse = _compare(q, kv, idx)
+    # the first call against the fp64 oracle as well
+    rows = np.arange(B * Lq)
+    oo, ol = oracle.sparse_attn(rows // Lq, P.bf16_bits(q).reshape(B * Lq, H, D), P.bf16_bits(kv),
+                                idx.reshape(B * Lq, k).cpu().numpy(), SCALE, DV)
+    P.check_attention(first.reshape(B * Lq, H, DV), first_lse.reshape(B * Lq, H), oo, ol)
+    second, _ = _compare(*_case(B, Lq, Lk, k, seed=2, pad_every=3))
     # the second call really recomputed (different inputs, same scratch)
-    assert not torch.equal(first[0], second[0])
+    assert not torch.equal(first, second)
     assert dsa.device_status() == 0
 
 
@@ -63,12 +83,21 @@ def test_noalloc_without_split_needs_no_scratch():
 
 
 def test_noalloc_rejects_calls_beyond_the_scratch_size():
-    # 160 single-query rows are split two ways (on 148 SMs): ~80 MiB of partials >
-    # 64 MiB.  The call must refuse on the host before touching CUDA (the pointers
-    # are never used).
+    # The smallest number of single-query rows whose split-k partials exceed the
+    # array, for the SM count this process sees (the workspace query reads it
+    # from the device, or assumes 148 without one).  The call must refuse before
+    # launching anything or reading any pointer: the pointers here are fake.
+    rows = next(r for r in range(1, 4096)
+                if dsa.workspace_size(dsa.OP_SPARSE_ATTN, r, 1, 131072, 2048, H, DV) > dsa.NOALLOC_SCRATCH_BYTES)
     L = dsa.lib()
     a = dsa.AttnArgs(H=H, d_qk=D, d_v=DV, scale=SCALE, q=16, kv=16)
     fake = ctypes.c_void_p(256)
-    assert dsa.workspace_size(dsa.OP_SPARSE_ATTN, 160, 1, 131072, 2048, H, DV) > dsa.NOALLOC_SCRATCH_BYTES
-    rc = L.dsa_sparse_attn_noalloc(ctypes.byref(a), 160, 1, 131072, fake, 2048, fake, None, None)
+    rc = L.dsa_sparse_attn_noalloc(ctypes.byref(a), rows, 1, 131072, fake, 2048, fake, None, None)
     assert rc == 3 and dsa.status_string(rc).startswith("DSA_ERR_WORKSPACE")
+
+
+def test_binding_scratch_size_matches_the_header():
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    m = re.search(r"#define\s+DSA_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
+    assert m, "DSA_NOALLOC_SCRATCH_BYTES not found in include/dsa.h"
+    assert dsa.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
