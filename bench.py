@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--loss", action="store_true", help="time the indexer loss even with --no-extra")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-fp8-peak", action="store_true", help="skip measuring the FP8 GEMM peak")
+    ap.add_argument("--stage", choices=["forward", "indexer_topk"], default="forward",
+                    help="indexer_topk: time only the fused indexer + top-k of the workload (profiling runs); "
+                         "prints its own JSON line")
     return ap.parse_args()
 
 
@@ -692,9 +695,63 @@ def config_of(wl):
 
 # ------------------------------------------------------------------------------------ main
 
+def run_indexer_topk_only(args, world):
+    """The fused indexer + top-k alone on the chosen workload (one call per step and
+    chunk, inputs resident): a small, self-contained command for profilers."""
+    import sparse_attention_19_b200 as dsa
+    wl = WORKLOADS[args.workload]
+    chunk = wl.chunk or wl.Lq
+    keys = make_key_side(wl, "cuda", args.seed)
+    keys.pop("kv")
+    calls = []
+    for c in range(wl.Lq // chunk):
+        qs = make_query_side(wl, "cuda", args.seed, chunk_index=c if wl.chunk else -1, Lq=chunk)
+        qs.pop("q")
+        q0 = wl.q_offset + c * chunk
+        L = q0 + chunk if wl.chunk else wl.Lk
+        calls.append((q0, qs, keys["k_I"][:, :L], keys["k_scale"][:, :L]))
+    torch.cuda.empty_cache()
+    idx = torch.empty(wl.B, chunk, wl.k, dtype=torch.int32, device="cuda")
+    ws = 0
+    for q0, qs, kI, ks in calls:
+        ws = max(ws, dsa.workspace_size_args(dsa.OP_INDEXER_TOPK,
+                                             dsa._indexer_args(qs["q_I"], qs["q_scale"], qs["w"], kI, ks, q0), wl.k))
+    ws = torch.empty(max(ws, 256), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for q0, qs, kI, ks in calls:
+            dsa.indexer_topk(qs["q_I"], qs["q_scale"], qs["w"], kI, ks, wl.k, q0, indices=idx, want_scores=False,
+                             workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e) / args.steps, world)
+    tot = work_model(wl)
+    print(json.dumps({"stage": "indexer_topk", "workload": wl.name, "ms_per_step": ms, "launches_per_step": len(calls),
+                      "tflops": tot["indexer_flops"] / (ms * 1e-3) / 1e12,
+                      "gbs": tot["indexer_bytes"] / (ms * 1e-3) / 1e9,
+                      "allocated_gb": torch.cuda.memory_allocated() / 1e9}), flush=True)
+    assert dsa.device_status() == 0
+
+
 def main():
     args = parse()
     rank, local, world = dist_init(args)
+    if args.stage == "indexer_topk" and args.impl == "ours":
+        run_indexer_topk_only(args, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         if world > 1:

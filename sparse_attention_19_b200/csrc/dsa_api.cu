@@ -209,8 +209,8 @@ bool make_indexer_maps(const dsa_indexer_args* a, const IndexerParams& p, CUtens
   if (!make_tmap(tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->q_I, (uint64_t)a->B * a->Lq * a->H_I, a->d_I,
                  a->d_I, (uint32_t)(p.qb * a->H_I), swz))
     return false;
-  if (!make_tmap(tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 32,
-                 swz))                                     // key tiles arrive as four 32-row boxes
+  if (!make_tmap(tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a->k_I, (uint64_t)a->B * a->Lk, a->d_I, a->d_I, 128,
+                 swz))                                     // one 128-key tile per box
     return false;
   *ts = *tk;                                               // unused unless scale_ring
   if (p.scale_ring && !make_tmap(ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a->k_scale, (uint64_t)a->B, a->Lk,

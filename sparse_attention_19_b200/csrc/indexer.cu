@@ -69,7 +69,7 @@ constexpr int kThreads = 32 * (kLoaderWarp0 + kLoaders);   // 768
 constexpr uint32_t kRegsLaunch = 80, kRegsEpi = 88, kRegsOther = 64;
 static_assert(32 * kEpiWarps * kRegsEpi + (kThreads - 32 * kEpiWarps) * kRegsOther <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
-static_assert(kLoaders * 32 == kKeysPerTile, "one 32-row box per loader");
+
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 16;      // key-scale ring: 128 fp32 per tile, released by the epilogue
 constexpr int kMaxStage = 32;        // staging slots (fused mode)
@@ -146,6 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_s, const IndexerParams p) {
   static_assert(D_I == 64 || D_I == 128, "d_I");
+  static_assert(kStages % kLoaders == 0 && kStages <= kMaxStages, "loaders own whole residues of the ring");
+  static_assert(kScaleSlots % kLoaders == 0, "a scale slot always belongs to the same loader");
   constexpr uint32_t kRowBytes = D_I;                  // one e4m3 row
   constexpr uint32_t kLayout = (D_I == 128) ? LAYOUT_SW128 : LAYOUT_SW64;
   constexpr uint32_t kAtomBytes = 8 * kRowBytes;       // 8-row swizzle atom
@@ -228,8 +230,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     regs_decrease<kRegsOther>();
   if (warp >= kLoaderWarp0) {
     // ------------------------------------------------------------ TMA loaders
-    // Loader 0 also loads the query block; every loader fills rows [32*pw, 32*pw+32)
-    // of each key stage.
+    // Loader 0 also loads the query block.  Loader pw owns the ring stages
+    // congruent to pw (mod kLoaders): it waits only for those, and fills each with
+    // one 128-key box and, when staged, the tile's key scales.
     const int pw = (int)warp - kLoaderWarp0;
     if (elect_one()) {
       if (pw == 0) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_k); if (p.scale_ring) prefetch_tmap(&tmap_s); }
@@ -249,19 +252,21 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
         bool ok = true;
         for (int kt = U.kt0; kt < U.kt1; ++kt) {
-          if (!mbar_wait(&S.k_empty[kstage], kphase ^ 1, abort_flag)) { ok = false; break; }
-          if (pw == 0) mbar_arrive_expect_tx(&S.k_full[kstage], kKeysPerTile * kRowBytes);
-          tma_load_2d(k_smem + (size_t)kstage * kKeysPerTile * kRowBytes + pw * 32 * kRowBytes, &tmap_k,
-                      &S.k_full[kstage], 0, U.b * p.Lk + kt * kKeysPerTile + pw * 32);
-          if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
-          if (pw == 0 && p.scale_ring) {
-            // the tile's 128 key scales (zero-filled past Lk) into the scale ring
-            const uint32_t ss = sc_use % kScaleSlots;
-            if (!mbar_wait(&S.sc_empty[ss], ((sc_use / kScaleSlots) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(&S.sc_full[ss], kKeysPerTile * 4);
-            tma_load_2d(sc_smem + ss * kKeysPerTile, &tmap_s, &S.sc_full[ss], kt * kKeysPerTile, U.b);
-            ++sc_use;
+          if (kstage % kLoaders == (uint32_t)pw) {
+            if (!mbar_wait(&S.k_empty[kstage], kphase ^ 1, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&S.k_full[kstage], kKeysPerTile * kRowBytes);
+            tma_load_2d(k_smem + (size_t)kstage * kKeysPerTile * kRowBytes, &tmap_k, &S.k_full[kstage], 0,
+                        U.b * p.Lk + kt * kKeysPerTile);
+            if (p.scale_ring) {
+              // the tile's 128 key scales (zero-filled past Lk) into the scale ring
+              const uint32_t ss = sc_use % kScaleSlots;
+              if (!mbar_wait(&S.sc_empty[ss], ((sc_use / kScaleSlots) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+              mbar_arrive_expect_tx(&S.sc_full[ss], kKeysPerTile * 4);
+              tma_load_2d(sc_smem + ss * kKeysPerTile, &tmap_s, &S.sc_full[ss], kt * kKeysPerTile, U.b);
+            }
           }
+          if (p.scale_ring) ++sc_use;
+          if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
         }
         if (!ok) break;
       }
