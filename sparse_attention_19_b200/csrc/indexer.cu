@@ -732,8 +732,11 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
   // A small resident query block (decode) leaves room for a deeper key ring.
   const bool deep = p.nsub * p.qb * p.H_I <= 128;
   const bool fused = p.scores == nullptr;
+  // Narrow accumulators (N <= 64) go to the four quads in turn; each staging slot
+  // must stay with one quad (see the staging ring), so n_stage % 4 == 0 there.
+  const bool narrow = p.qb * p.H_I <= 64;
   if (fused && (p.rows_per_unit > kMaxRows || p.n_stage > kMaxStage || p.n_stage < 1 || p.cap < p.k + 128 ||
-                p.cap % 32 != 0))
+                p.cap % 32 != 0 || (narrow && p.n_stage % kQuads != 0)))
     return cudaErrorInvalidValue;
   if (p.H_I == 64 && p.d_I == 128) {
     if (fused)
