@@ -133,7 +133,9 @@ IndexerParams plan_indexer(const dsa_indexer_args* a, bool fused, int k) {
     const int r4 = (a->Lq + 3) / 4 * 4;
     p.qb = r4 < 64 ? r4 : 64;
   }
-  p.nsub = (a->Lq > p.qb) ? 2 : 1;
+  // The fused mode keeps each unit's rows' candidate lists in shared memory, so its
+  // units hold one sub-block (four rows in prefill).
+  p.nsub = (a->Lq > p.qb && !fused) ? 2 : 1;
   p.queries_per_unit = p.qb * p.nsub;
   p.n_qblocks = (a->Lq + p.queries_per_unit - 1) / p.queries_per_unit;
   const int sms = sm_count();
@@ -162,11 +164,13 @@ IndexerParams plan_indexer(const dsa_indexer_args* a, bool fused, int k) {
   if (fused) {
     const int k32 = (k + 31) / 32 * 32;
     p.k = k;
-    p.cap = k32 + (k32 > 256 ? k32 : 256);       // room for one tile (128) after every cut to k
+    // List capacity: k plus room for several tiles' candidates (at least one tile,
+    // 128, must fit after every cut to k); more room means fewer cuts.
+    const int room = k32 < 256 ? 256 : (k32 > 512 ? 512 : k32);
+    p.cap = k32 + room;
     p.rows_per_unit = p.queries_per_unit;
-    const int deep = p.nsub * p.qb * a->H_I <= 128;
     const int slot_bytes = p.qb * 128 * 8;
-    int ns = (deep ? 16384 : 32768) / slot_bytes;
+    int ns = 16384 / slot_bytes;
     ns = ns < 2 ? 2 : (ns > indexer_fused_max_stage() ? indexer_fused_max_stage() : ns);
     // With one 64-column accumulator per sub-block the four epilogue quads take
     // accumulators (and so staging slots) in turn.  A slot must always belong to
@@ -192,7 +196,8 @@ struct FusedWs {
 };
 FusedWs fused_ws_layout(const IndexerParams& p) {
   FusedWs w{};
-  const size_t slots = p.kchunks == 1 ? (size_t)indexer_grid(p) : (size_t)p.n_units;
+  // Lists live in shared memory; only rows split over units leave one per unit here.
+  const size_t slots = p.kchunks == 1 ? 0 : (size_t)p.n_units;
   const size_t list = slots * p.rows_per_unit * (size_t)p.cap * 4;
   w.key_off = 0;
   w.pos_off = round_up(list, 256);
@@ -201,6 +206,7 @@ FusedWs fused_ws_layout(const IndexerParams& p) {
   w.done_off = w.meta_off + round_up(meta, 256);
   const size_t done = p.kchunks > 1 ? (size_t)p.B * p.Lq * 4 : 0;
   w.bytes = w.done_off + round_up(done, 256);
+  if (w.bytes == 0) w.bytes = 256;             // a non-empty workspace keeps the argument checks uniform
   return w;
 }
 

@@ -34,16 +34,16 @@ struct IndexerParams {
   int rows_per_unit;      // queries_per_unit
   int32_t* indices;       // [B, Lq, k]
   float* sel_scores;      // [B, Lq, k] or null
-  uint32_t* xkey;         // candidate lists, keys:      [list slot][rows_per_unit][cap]
-  uint32_t* xpos;         // candidate lists, positions: same layout
+  uint32_t* xkey;         // kchunks > 1: each unit's top-k per row, keys:  [unit][rows_per_unit][cap]
+  uint32_t* xpos;         // kchunks > 1: the same, positions
   uint4* xmeta;           // kchunks > 1: per (unit, row) {count, min key, max key, 0}
   uint32_t* done;         // kchunks > 1: per row, chunks finished (zeroed before the launch)
 };
 // Shared-memory bytes of the indexer kernel for a query block of q_rows (query,
 // head) rows, `stages` key stages and, in the fused mode, the staging and
 // selection areas.
-size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages, bool fused, int qb,
-                          int n_stage, int rows_per_unit);
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages, bool scale_ring,
+                          bool fused, int qb, int n_stage, int rows_per_unit, int cap);
 cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& ts, int grid, cudaStream_t stream);
 int indexer_fused_max_rows();    // rows per unit the fused mode supports

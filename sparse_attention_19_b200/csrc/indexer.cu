@@ -44,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "dsa_internal.h"
 #include "ptx.cuh"
@@ -65,10 +66,12 @@ constexpr int kLoaders = 4;          // TMA requests from one warp are served in
 constexpr int kLoaderWarp0 = kMmaWarp + 4;
 constexpr int kThreads = 32 * (kLoaderWarp0 + kLoaders);   // 768
 // Register split: 80 per thread at launch (6 warps per SM sub-partition); the four
-// epilogue warpgroups take 88, the MMA / loader warpgroups keep 64.
-constexpr uint32_t kRegsLaunch = 80, kRegsEpi = 88, kRegsOther = 64;
-static_assert(32 * kEpiWarps * kRegsEpi + (kThreads - 32 * kEpiWarps) * kRegsOther <= kThreads * kRegsLaunch,
+// epilogue warpgroups take 88, the MMA / selector warpgroup keeps the 80 it
+// launched with, and the loader warpgroup (TMA issue only) gives up to 48.
+constexpr uint32_t kRegsLaunch = 80, kRegsEpi = 88, kRegsLoader = 48;
+static_assert(32 * kEpiWarps * kRegsEpi + 128 * kRegsLaunch + 128 * kRegsLoader <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
+static_assert(kThreads == 32 * kEpiWarps + 256, "one MMA/selector warpgroup and one loader warpgroup");
 
 constexpr int kTmemCols = 512;
 constexpr int kScaleSlots = 16;      // key-scale ring: 128 fp32 per tile, released by the epilogue
@@ -81,10 +84,11 @@ struct FusedLayout {
   uint32_t theta;                          // [kMaxRows] u64: (unit ordinal << 32) | threshold key
   uint32_t row_n, row_thr, row_min, row_max;   // [kMaxRows] each, selector-owned
   uint32_t hist, cand;                     // [kSelWarps][kSelBins], [kSelWarps][kSelCandCap + 4]
+  uint32_t lkey, lpos;                     // candidate lists: [rows][cap] keys, [rows][cap] positions
   uint32_t end;
 };
 __host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
-__host__ __device__ inline FusedLayout fused_layout(uint32_t base, int qb, int n_stage) {
+__host__ __device__ inline FusedLayout fused_layout(uint32_t base, int qb, int n_stage, int rows, int cap) {
   FusedLayout L{};
   const uint32_t entries = (uint32_t)n_stage * qb * 128u;
   L.stg_key = align_up(base, 16);
@@ -97,7 +101,9 @@ __host__ __device__ inline FusedLayout fused_layout(uint32_t base, int qb, int n
   L.row_max = L.row_min + kMaxRows * 4;
   L.hist = align_up(L.row_max + kMaxRows * 4, 16);
   L.cand = L.hist + kSelWarps * kSelBins * 4;
-  L.end = L.cand + kSelWarps * (kSelCandCap + 4) * 4;
+  L.lkey = align_up(L.cand + kSelWarps * (kSelCandCap + 4) * 4, 16);
+  L.lpos = L.lkey + (uint32_t)rows * cap * 4;
+  L.end = L.lpos + (uint32_t)rows * cap * 4;
   return L;
 }
 
@@ -116,7 +122,7 @@ struct IndexerSmem {
 
 // Query-block buffers: two (the next unit's block loads while this one runs) when a
 // block is small, as in decode; one for the large prefill blocks.
-__host__ __device__ constexpr uint32_t query_buffers(uint32_t q_bytes) { return q_bytes <= 32768u ? 2u : 1u; }
+__host__ __device__ constexpr uint32_t query_buffers(uint32_t q_bytes) { return q_bytes < 32768u ? 2u : 1u; }
 
 struct UnitInfo {
   int b, i0, kt0, kt1;  // batch, first query, key-tile range [kt0, kt1)
@@ -165,11 +171,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   uint8_t* q_smem = tiles;                             // n_qbuf x (nsub * N rows)
   uint8_t* k_smem = tiles + n_qbuf * (size_t)q_bytes;
   float* sc_smem = reinterpret_cast<float*>(k_smem + (size_t)kStages * kKeysPerTile * kRowBytes);
-  float* w_smem = sc_smem + kScaleSlots * kKeysPerTile;   // 2 x QU * H_I (per unit, double-buffered)
+  float* w_smem = sc_smem + (p.scale_ring ? kScaleSlots * kKeysPerTile : 0);   // 2 x QU * H_I (double-buffered)
   float* sq_smem = w_smem + 2 * QU * H_I;                  // 2 x QU
-  // fused mode: staging ring, per-row thresholds and selector state
+  // fused mode: staging ring, per-row thresholds, selector state and candidate lists
   const FusedLayout FL = fused_layout((uint32_t)(reinterpret_cast<uint8_t*>(sq_smem + 2 * QU) - tiles), p.qb,
-                                      p.n_stage);
+                                      p.n_stage, p.rows_per_unit, p.cap);
   uint32_t* stg_key = reinterpret_cast<uint32_t*>(tiles + FL.stg_key);
   uint32_t* stg_pos = reinterpret_cast<uint32_t*>(tiles + FL.stg_pos);
   uint32_t* stg_cnt = reinterpret_cast<uint32_t*>(tiles + FL.stg_cnt);
@@ -227,8 +233,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   const uint32_t tmem_base = S.tmem_base;
 
   if (warp >= (uint32_t)kEpiWarps) {
-    regs_decrease<kRegsOther>();
   if (warp >= kLoaderWarp0) {
+    regs_decrease<kRegsLoader>();
     // ------------------------------------------------------------ TMA loaders
     // Loader 0 also loads the query block.  Loader pw owns the ring stages
     // congruent to pw (mod kLoaders): it waits only for those, and fills each with
@@ -317,7 +323,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // ------------------------------------------------------------ selectors
     // Selector `me` owns the unit's rows r with r % kSelWarps == me.  It consumes
     // every staging slot in order (releasing it for the epilogue) and appends its
-    // rows' staged candidates to their lists.
+    // rows' staged candidates to their lists, which live in shared memory.
     const int me = (int)warp - kSelWarp0;
     const int RPU = p.rows_per_unit;
     const bool active = me < RPU;            // a unit with fewer rows than selectors leaves some idle
@@ -325,25 +331,23 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     const uint32_t lt = (1u << lane) - 1u;
     uint32_t* hist = reinterpret_cast<uint32_t*>(tiles + FL.hist) + me * kSelBins;
     uint32_t* cand = reinterpret_cast<uint32_t*>(tiles + FL.cand) + me * (kSelCandCap + 4);
-    auto list_key = [&](int slot_id, int r) { return p.xkey + ((size_t)slot_id * RPU + r) * p.cap; };
-    auto list_pos = [&](int slot_id, int r) { return p.xpos + ((size_t)slot_id * RPU + r) * p.cap; };
-    // Top-k threshold of one list of n > k candidates with keys in [lo, hi].
-    auto threshold_of = [&](const uint32_t* xk, uint32_t n, uint32_t lo, uint32_t hi, uint32_t& thr,
-                            uint32_t& gt) {
-      auto visit = [&](auto&& f) {
-        for (uint32_t i = lane; i < n; i += 32) f(__ldcg(xk + i));
-      };
-      warp_find_threshold(hist, cand, visit, k, lo, hi, thr, gt);
-    };
-    // Cut a row's list to its top-k in place and raise the row's threshold.
-    auto cut = [&](int r, uint32_t* xk, uint32_t* xp, uint32_t ucount) {
+    uint32_t* lkey = reinterpret_cast<uint32_t*>(tiles + FL.lkey);
+    uint32_t* lpos = reinterpret_cast<uint32_t*>(tiles + FL.lpos);
+    // Rows split over units leave their per-unit top-k in global memory.
+    auto glist_key = [&](int unit, int r) { return p.xkey + ((size_t)unit * RPU + r) * p.cap; };
+    auto glist_pos = [&](int unit, int r) { return p.xpos + ((size_t)unit * RPU + r) * p.cap; };
+    // Cut a row's shared-memory list to its top-k in place and raise its threshold.
+    auto cut = [&](int r, uint32_t ucount) {
+      uint32_t* xk = lkey + (size_t)r * p.cap;
+      uint32_t* xp = lpos + (size_t)r * p.cap;
       const uint32_t n = row_n[r];
       uint32_t thr, gt;
-      threshold_of(xk, n, row_min[r], row_max[r], thr, gt);
+      auto visit = [&](auto&& f) { visit_list_keys<false>(xk, (int)n, f); };
+      warp_find_threshold(hist, cand, visit, k, row_min[r], row_max[r], thr, gt);
       auto seg = [&](int) { return CandSeg{xk, xp, (int)n}; };
-      warp_compact(seg, 1, thr, k - gt, 0, [&](uint32_t at, uint32_t key, uint32_t pos) {
-        __stcg(xk + at, key);
-        __stcg(xp + at, pos);
+      warp_compact<false>(seg, 1, thr, k - gt, 0, [&](uint32_t at, uint32_t key, uint32_t pos) {
+        xk[at] = key;
+        xp[at] = pos;
       });
       __syncwarp();
       if (lane == 0) {
@@ -356,7 +360,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     };
     // Final output of one row from the concatenated segments get_seg(0 .. nseg-1)
     // (position order), holding `total` candidates with keys in [lo, hi].
-    auto emit_row = [&](size_t row, auto get_seg, int nseg, uint32_t total, uint32_t lo, uint32_t hi) {
+    auto emit_row = [&](auto global, size_t row, auto get_seg, int nseg, uint32_t total, uint32_t lo,
+                        uint32_t hi) {
+      constexpr bool kG = decltype(global)::value;
       int32_t* oi = p.indices + row * (size_t)p.k;
       float* os = p.sel_scores ? p.sel_scores + row * (size_t)p.k : nullptr;
       auto emit = [&](uint32_t at, uint32_t key, uint32_t pos) {
@@ -369,13 +375,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         auto visit = [&](auto&& f) {
           for (int g = 0; g < nseg; ++g) {
             const CandSeg sg = get_seg(g);
-            for (int i = (int)lane; i < sg.n; i += 32) f(__ldcg(sg.key + i));
+            visit_list_keys<kG>(sg.key, sg.n, f);
           }
         };
         warp_find_threshold(hist, cand, visit, k, lo, hi, thr, gt);
-        m = warp_compact(get_seg, nseg, thr, k - gt, 0, emit);
+        m = warp_compact<kG>(get_seg, nseg, thr, k - gt, 0, emit);
       } else {
-        m = warp_compact(get_seg, nseg, 0u, 0u, 0, emit);   // every candidate (all keys > 0)
+        m = warp_compact<kG>(get_seg, nseg, 0u, 0u, 0, emit);   // every candidate (all keys > 0)
       }
       for (uint32_t j = m + lane; j < k; j += 32) {
         oi[j] = -1;
@@ -386,7 +392,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     uint32_t seq = 0, ucount = 0;
     for (int u = blockIdx.x; active && u < p.n_units; u += gridDim.x, ++ucount) {
       const UnitInfo U = decode_unit(p, u);
-      const int ls = p.kchunks == 1 ? (int)blockIdx.x : u;      // list slot of this unit
       if (lane == 0)
         for (int r = me; r < RPU; r += kSelWarps) {
           row_n[r] = 0;
@@ -403,11 +408,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           for (int qi = 0; qi < p.qb; ++qi) {
             const int r = sb * p.qb + qi;
             if (r % kSelWarps != me || U.i0 + r >= p.Lq) continue;
-            uint32_t* xk = list_key(ls, r);
-            uint32_t* xp = list_pos(ls, r);
             const uint32_t* cnt = stg_cnt + (gs * p.qb + qi) * 4;
             const uint32_t c0 = cnt[0], c1 = cnt[1], c2 = cnt[2], c3 = cnt[3];
-            if (row_n[r] + c0 + c1 + c2 + c3 > (uint32_t)p.cap) cut(r, xk, xp, ucount);
+            if (row_n[r] + c0 + c1 + c2 + c3 > (uint32_t)p.cap) cut(r, ucount);
+            uint32_t* xk = lkey + (size_t)r * p.cap;
+            uint32_t* xp = lpos + (size_t)r * p.cap;
             uint32_t n = row_n[r];
             const uint32_t th = row_thr[r];
             const uint32_t* sk = stg_key + (gs * p.qb + qi) * 128;
@@ -425,8 +430,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
               const uint32_t bal = __ballot_sync(0xffffffffu, keep);
               if (keep) {
                 const uint32_t at = n + __popc(bal & lt);
-                __stcg(xk + at, key);
-                __stcg(xp + at, pos);
+                xk[at] = key;
+                xp[at] = pos;
                 mn = min(mn, key);
                 mx = max(mx, key);
               }
@@ -450,18 +455,25 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       for (int r = me; r < RPU; r += kSelWarps) {
         if (U.i0 + r >= p.Lq) continue;
         const size_t row = (size_t)U.b * p.Lq + U.i0 + r;
-        uint32_t* xk = list_key(ls, r);
-        uint32_t* xp = list_pos(ls, r);
+        uint32_t* xk = lkey + (size_t)r * p.cap;
+        uint32_t* xp = lpos + (size_t)r * p.cap;
         if (p.kchunks == 1) {
           const uint32_t n = row_n[r];
           auto seg = [&](int) { return CandSeg{xk, xp, (int)n}; };
-          emit_row(row, seg, 1, n, row_min[r], row_max[r]);
+          emit_row(std::false_type{}, row, seg, 1, n, row_min[r], row_max[r]);
           __syncwarp();
           continue;
         }
-        if (row_n[r] > k) cut(r, xk, xp, ucount);
-        if (lane == 0)
-          __stcg(p.xmeta + (size_t)u * RPU + r, make_uint4(row_n[r], row_min[r], row_max[r], 0u));
+        if (row_n[r] > k) cut(r, ucount);
+        // this unit's top-k of the row (position order) to global memory
+        const uint32_t n = row_n[r];
+        uint32_t* gk = glist_key(u, r);
+        uint32_t* gp = glist_pos(u, r);
+        for (uint32_t i = lane * 4; i < n; i += 128) {
+          __stcg(reinterpret_cast<uint4*>(gk + i), *reinterpret_cast<const uint4*>(xk + i));
+          __stcg(reinterpret_cast<uint4*>(gp + i), *reinterpret_cast<const uint4*>(xp + i));
+        }
+        if (lane == 0) __stcg(p.xmeta + (size_t)u * RPU + r, make_uint4(n, row_min[r], row_max[r], 0u));
         __threadfence();
         __syncwarp();
         uint32_t prev = 0;
@@ -473,7 +485,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int u0 = u - u % p.kchunks;
         auto seg = [&](int c) {
           const uint4 m = __ldcg(p.xmeta + (size_t)(u0 + c) * RPU + r);
-          return CandSeg{list_key(u0 + c, r), list_pos(u0 + c, r), (int)m.x};
+          return CandSeg{glist_key(u0 + c, r), glist_pos(u0 + c, r), (int)m.x};
         };
         uint32_t total = 0, lo = 0xffffffffu, hi = 0;
         for (int c = 0; c < p.kchunks; ++c) {
@@ -481,7 +493,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           total += m.x;
           if (m.x) { lo = min(lo, m.y); hi = max(hi, m.z); }
         }
-        emit_row(row, seg, p.kchunks, total, lo, hi);
+        emit_row(std::true_type{}, row, seg, p.kchunks, total, lo, hi);
         __syncwarp();
       }
     }
@@ -695,7 +707,8 @@ template <int H_I, int D_I, int kStages, bool kFused>
 cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& ts, int grid, cudaStream_t stream) {
   const size_t smem = indexer_smem_bytes(p.nsub * p.qb * H_I, D_I, p.queries_per_unit * H_I, p.queries_per_unit,
-                                         kStages, kFused, p.qb, p.n_stage, p.rows_per_unit);
+                                         kStages, p.scale_ring != 0, kFused, p.qb, p.n_stage, p.rows_per_unit,
+                                         p.cap);
   auto kern = indexer_kernel<H_I, D_I, kStages, kFused>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -711,14 +724,13 @@ cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, cons
 
 }  // namespace
 
-size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages, bool fused, int qb,
-                          int n_stage, int rows_per_unit) {
-  (void)rows_per_unit;
+size_t indexer_smem_bytes(int q_rows, int d_I, int w_floats, int sq_floats, int stages, bool scale_ring,
+                          bool fused, int qb, int n_stage, int rows_per_unit, int cap) {
   size_t t = query_buffers((uint32_t)(q_rows * d_I)) * (size_t)q_rows * d_I;   // query block buffers
   t += (size_t)stages * kKeysPerTile * d_I;                    // key ring
-  t += (size_t)kScaleSlots * kKeysPerTile * sizeof(float);      // key-scale ring
+  if (scale_ring) t += (size_t)kScaleSlots * kKeysPerTile * sizeof(float);   // key-scale ring
   t += 2 * (size_t)(w_floats + sq_floats) * sizeof(float);     // weights / query scales, double-buffered
-  if (fused) t = fused_layout((uint32_t)t, qb, n_stage).end;    // staging ring + selector areas
+  if (fused) t = fused_layout((uint32_t)t, qb, n_stage, rows_per_unit, cap).end;   // staging, selectors, lists
   const size_t b = sizeof(IndexerSmem) + 1024 + t;             // barriers + alignment slack
   // At least ~116 KB so that one CTA (and its 512 TMEM columns) owns each SM.
   return b < 118784 ? 118784 : b;

@@ -258,6 +258,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           for (int c = 0; c < NC; ++c, ++kc) {
             const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
             if (st / kKTeamSlots != my_team) continue;
+            // Dense mode: one box per chunk from the team's first warp; the others
+            // have nothing to load and must not wait either (a waiter that adds
+            // nothing to a phase can fall two phases behind, where its parity test
+            // would no longer see the phase it waits for).
+            if (p.dense && part != 0) continue;
             bool w_ok = true;
             if (lane == 0) {
               w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
@@ -367,6 +372,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             for (int h = 0; h < VS::kNpv; ++h, ++vc) {
               const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
               if (st != my_slot) continue;
+              if (p.dense && part != 0) continue;         // one issuing warp per slot (see the key loaders)
               bool w_ok = true;
               if (lane == 0) {
                 w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);

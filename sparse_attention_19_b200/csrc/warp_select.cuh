@@ -21,8 +21,8 @@
 
 namespace dsa {
 
-constexpr int kSelBins = 2048;          // histogram bins per refinement level
-constexpr int kSelBinBits = 11;
+constexpr int kSelBins = 1024;          // histogram bins per refinement level
+constexpr int kSelBinBits = 10;
 constexpr int kSelCandCap = 512;        // boundary-bin keys gathered into shared memory
 
 __device__ __forceinline__ uint32_t score_to_key(float f) {
@@ -60,7 +60,7 @@ __device__ __forceinline__ void sel_level(uint32_t* hist, Visit visit, uint32_t 
     if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) >> shift], 1u);
   });
   __syncwarp();
-  // Lane j owns bins [64 j, 64 j + 64).  Counts from the top: suffix sums over lanes.
+  // Lane j owns bins [kPer j, kPer (j + 1)).  Counts from the top: suffix sums over lanes.
   constexpr int kPer = kSelBins / 32;
   uint32_t mine = 0;
   const uint4* h4 = reinterpret_cast<const uint4*>(hist + lane * kPer);
@@ -97,7 +97,7 @@ __device__ __forceinline__ void sel_level(uint32_t* hist, Visit visit, uint32_t 
 // gt = #{key > thr} (so m - gt candidates equal to thr are taken, the first ones
 // in position order).  `cand` holds up to kSelCandCap keys of the boundary bin.
 template <typename Visit>
-__device__ void warp_find_threshold(uint32_t* hist, uint32_t* cand, Visit visit, uint32_t m, uint32_t lo,
+__device__ __forceinline__ void warp_find_threshold(uint32_t* hist, uint32_t* cand, Visit visit, uint32_t m, uint32_t lo,
                                     uint32_t hi, uint32_t& thr, uint32_t& gt) {
   const uint32_t lane = threadIdx.x & 31u;
   uint32_t need = m, got = 0;
@@ -145,36 +145,112 @@ __device__ void warp_find_threshold(uint32_t* hist, uint32_t* cand, Visit visit,
   }
 }
 
-// Stable selection pass: walks the segments get_seg(0 .. nseg-1) in order, 32
-// candidates at a time, and hands every kept candidate to emit(index, key, pos)
-// with consecutive indices from `base`: all keys > thr and the first eq_take keys
-// == thr.  Returns the count.
-// Each batch of 32 is read completely before any of it is emitted, so emitting
-// into the list being read (at an index not above the one read) is safe.
-template <typename GetSeg, typename Emit>
-__device__ uint32_t warp_compact(GetSeg get_seg, int nseg, uint32_t thr, uint32_t eq_take, uint32_t base,
-                                 Emit emit) {
+// Calls f(key) for the keys[0 .. n) of a list, read as 16-byte groups with kVisitU
+// groups in flight per lane.  A list in global memory (kGlobal) is read through L2
+// only (its writers may be other CTAs), where latency rather than bytes would
+// otherwise set the pace; a list in shared memory is read directly.  The list must
+// start 16-byte aligned and be readable up to n rounded up to a multiple of four
+// (list capacities are multiples of 32).  Lanes call f different numbers of
+// times: f must not contain warp-collective operations.
+constexpr int kVisitU = 4;
+constexpr int kCompactU = 2;          // (key, position) group pairs in flight per lane when compacting
+
+template <bool kGlobal>
+__device__ __forceinline__ uint4 load_group(const uint4* p) {
+  if constexpr (kGlobal) return __ldcg(p);
+  else return *p;
+}
+
+template <bool kGlobal, typename F>
+__device__ __forceinline__ void visit_list_keys(const uint32_t* key, int n, F f) {
+  const int lane = (int)(threadIdx.x & 31u);
+  const uint4* k4 = reinterpret_cast<const uint4*>(key);
+  const int n4 = (n + 3) >> 2;
+  for (int g0 = 0; g0 < n4; g0 += 32 * kVisitU) {
+    uint4 v[kVisitU];
+#pragma unroll
+    for (int u = 0; u < kVisitU; ++u) {
+      const int g = g0 + u * 32 + lane;
+      v[u] = g < n4 ? load_group<kGlobal>(k4 + g) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < kVisitU; ++u) {
+      const int i = (g0 + u * 32 + lane) * 4;
+      if (i + 0 < n) f(v[u].x);
+      if (i + 1 < n) f(v[u].y);
+      if (i + 2 < n) f(v[u].z);
+      if (i + 3 < n) f(v[u].w);
+    }
+  }
+}
+
+// Exclusive prefix sum of v over the lanes of the warp; `total` receives the sum.
+__device__ __forceinline__ uint32_t warp_exclusive_sum(uint32_t v, uint32_t& total) {
   const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= (uint32_t)o) x += y;
+  }
+  total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
+}
+
+// Stable selection pass: walks the segments get_seg(0 .. nseg-1) in order and
+// hands every kept candidate to emit(index, key, pos) with consecutive indices from
+// `base`: all keys > thr and the first eq_take keys == thr.  Returns the count.
+// Entries are read as 16-byte groups (lane l holds entries 4l .. 4l+3 of each 128),
+// kCompactU groups per lane in flight; every group of a block is read before any of
+// the block is emitted, so emitting into the list being read (at an index not
+// above the one read) is safe.
+template <bool kGlobal, typename GetSeg, typename Emit>
+__device__ __forceinline__ uint32_t warp_compact(GetSeg get_seg, int nseg, uint32_t thr, uint32_t eq_take,
+                                                 uint32_t base, Emit emit) {
+  const int lane = (int)(threadIdx.x & 31u);
   uint32_t w = base, eq_seen = 0;
   for (int g = 0; g < nseg; ++g) {
     const CandSeg sg = get_seg(g);
-    for (int i0 = 0; i0 < sg.n; i0 += 32) {
-      const int i = i0 + (int)lane;
-      uint32_t key = 0, pos = 0;
-      if (i < sg.n) {
-        key = __ldcg(sg.key + i);
-        pos = __ldcg(sg.pos + i);
+    const uint4* k4 = reinterpret_cast<const uint4*>(sg.key);
+    const uint4* p4 = reinterpret_cast<const uint4*>(sg.pos);
+    const int n4 = (sg.n + 3) >> 2;
+    for (int g0 = 0; g0 < n4; g0 += 32 * kCompactU) {
+      uint4 kv[kCompactU], pv[kCompactU];
+#pragma unroll
+      for (int u = 0; u < kCompactU; ++u) {
+        const int q = g0 + u * 32 + lane;
+        kv[u] = q < n4 ? load_group<kGlobal>(k4 + q) : make_uint4(0u, 0u, 0u, 0u);
+        pv[u] = q < n4 ? load_group<kGlobal>(p4 + q) : make_uint4(0u, 0u, 0u, 0u);
       }
       __syncwarp();
-      const bool valid = i < sg.n;
-      const uint32_t eq = __ballot_sync(0xffffffffu, valid && key == thr);
-      const bool take_eq = valid && key == thr && eq_seen + __popc(eq & lt) < eq_take;
-      const bool keep = (valid && key > thr) || take_eq;
-      const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-      if (keep) emit(w + __popc(kb & lt), key, pos);
-      w += __popc(kb);
-      eq_seen += __popc(eq);
+#pragma unroll
+      for (int u = 0; u < kCompactU; ++u) {
+        const int i = (g0 + u * 32 + lane) * 4;
+        const int nv = min(4, max(0, sg.n - i));          // valid entries of this lane's group
+        const uint32_t vmask = (1u << nv) - 1u;
+        const uint32_t gt = vmask & ((kv[u].x > thr ? 1u : 0u) | (kv[u].y > thr ? 2u : 0u) |
+                                     (kv[u].z > thr ? 4u : 0u) | (kv[u].w > thr ? 8u : 0u));
+        const uint32_t eq = vmask & ((kv[u].x == thr ? 1u : 0u) | (kv[u].y == thr ? 2u : 0u) |
+                                     (kv[u].z == thr ? 4u : 0u) | (kv[u].w == thr ? 8u : 0u));
+        uint32_t eq_total;
+        const uint32_t eq_rank = eq_seen + warp_exclusive_sum(__popc(eq), eq_total);
+        // equal keys are taken in order while fewer than eq_take have been taken
+        const uint32_t room = eq_take > eq_rank ? eq_take - eq_rank : 0u;   // equal keys this lane may take
+        uint32_t take = 0, e = eq;
+        for (uint32_t t = 0; e && t < room; ++t) {
+          take |= e & (0u - e);                             // lowest remaining equal entry
+          e &= e - 1u;
+        }
+        const uint32_t keep = gt | take;
+        uint32_t keep_total;
+        uint32_t at = w + warp_exclusive_sum(__popc(keep), keep_total);
+        if (keep & 1u) emit(at++, kv[u].x, pv[u].x);
+        if (keep & 2u) emit(at++, kv[u].y, pv[u].y);
+        if (keep & 4u) emit(at++, kv[u].z, pv[u].z);
+        if (keep & 8u) emit(at++, kv[u].w, pv[u].w);
+        w += keep_total;
+        eq_seen += eq_total;
+      }
       __syncwarp();
     }
   }
