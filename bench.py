@@ -224,10 +224,12 @@ def work_model(wl, Lq=None, q_offset=None):
         "rows": rows,
         "causal_pairs": causal,
         "selected_pairs": selected,
-        # indexer with the top-k fused into it: one FP8 dot of width d_I per (pair, head);
-        # bytes: keys + scales and the query side read once, the selected indices written
+        # indexer: one FP8 dot of width d_I per (pair, head); bytes: keys + scales and
+        # the query side read once, the causal scores written (staged selection)
         "indexer_flops": 2.0 * causal * wl.H_I * wl.d_I,
-        "indexer_bytes": wl.B * (q0 + Lq) * (wl.d_I + 4) + rows * wl.H_I * (wl.d_I + 2) + rows * wl.k * 4.0,
+        "indexer_bytes": wl.B * (q0 + Lq) * (wl.d_I + 4) + rows * wl.H_I * (wl.d_I + 2) + causal * 4.0,
+        # top-k: the causal scores read once, the selected indices written
+        "topk_bytes": causal * 4.0 + rows * wl.k * 4.0,
         # attention: S = q.c (d_qk) and O = p.v (d_v) per (selected pair, head)
         "attn_flops": 2.0 * selected * wl.H * (wl.D + wl.Dv),
         "attn_bytes": selected * wl.D * 2.0 + rows * wl.H * (wl.D + wl.Dv) * 2.0,
@@ -239,7 +241,7 @@ def work_model(wl, Lq=None, q_offset=None):
 class Runner:
     """Inputs resident on the device, outputs and workspace preallocated."""
 
-    def __init__(self, wl, seed, device="cuda"):
+    def __init__(self, wl, seed, device="cuda", low_memory=False):
         import sparse_attention_19_b200 as dsa
         self.dsa = dsa
         self.wl = wl
@@ -266,11 +268,14 @@ class Runner:
         for q_offset, qs in self.chunks:
             ia = dsa._indexer_args(qs["q_I"], qs["q_scale"], qs["w"], keys["k_I"][:, : q_offset + chunk],
                                    keys["k_scale"][:, : q_offset + chunk], q_offset)
-            ws = max(ws, dsa.workspace_size_args(dsa.OP_FORWARD, ia, k, H, Dv))
+            op = dsa.OP_FORWARD_LOWMEM if low_memory else dsa.OP_FORWARD
+            ws = max(ws, dsa.workspace_size_args(op, ia, k, H, Dv))
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
-        # per forward call: the fused indexer + top-k (or the index fill of a short
-        # sequence), the attention, and its split-k merge when rows are split
-        self.launches_per_call = 2 + (1 if dsa.workspace_size(dsa.OP_SPARSE_ATTN, B, chunk, wl.Lk, k, H, Dv) else 0)
+        self.low_memory = low_memory
+        # per forward call: the indexer and the top-k (one fused launch in low-memory
+        # mode), the attention, and its split-k merge when rows are split
+        self.launches_per_call = (2 if low_memory else 3) + \
+            (1 if dsa.workspace_size(dsa.OP_SPARSE_ATTN, B, chunk, wl.Lk, k, H, Dv) else 0)
         self.work = [work_model(wl, chunk, q0) for q0, _ in self.chunks]
 
     def step(self, stream, events=None):
@@ -290,7 +295,7 @@ class Runner:
             self.dsa.forward(qs["q_I"], qs["q_scale"], qs["w"], k_I.contiguous() if wl.B > 1 else k_I,
                              k_scale, qs["q"], kv, wl.k, wl.Dv, wl.scale, q_offset,
                              indices=indices[:, sl], out=out[:, sl], lse=lse[:, sl],
-                             workspace=self.ws, stream=stream,
+                             workspace=self.ws, stream=stream, low_memory=self.low_memory,
                              stage_events=None if events is None else events[n])
 
     def totals(self):
@@ -324,8 +329,8 @@ def time_runner(runner, steps, warmup, world, sample_clocks, local):
         sampler.__exit__()
     barrier(world)
     total_ms = start.elapsed_time(end)
-    # spans: [0] indexer with the fused top-k, [1] the rest of the top-k step (0 when
-    # fused; the index fill of a short sequence), [2] attention + split-k merge
+    # spans: [0] indexer (with the top-k when fused), [1] top-k (0 when fused),
+    # [2] attention + split-k merge
     stage_ms = [0.0, 0.0, 0.0]
     for s in range(steps):
         for c in range(nchunks):
@@ -347,14 +352,18 @@ def roofline_stages(wl, runner, stage_ms, peaks, peak_src):
     decode = wl.Lq == 1
     calls = len(runner.chunks)
     out = {}
-    # indexer + fused top-k: FP8 contraction for prefill; streams the key cache for decode
+    # indexer: FP8 contraction for prefill; streams the key cache for decode
     if decode:
-        out["indexer_topk"] = dict(bound="hbm", achieved=tot["indexer_bytes"] / (stage_ms[0] * 1e-3) / 1e9,
-                                   peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["indexer_bytes"] / calls)
+        out["indexer"] = dict(bound="hbm", achieved=tot["indexer_bytes"] / (stage_ms[0] * 1e-3) / 1e9,
+                              peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["indexer_bytes"] / calls)
     else:
-        out["indexer_topk"] = dict(bound="tensor", achieved=tot["indexer_flops"] / (stage_ms[0] * 1e-3) / 1e12,
-                                   peak=fp8_sust, unit="TFLOP/s", algorithmic=tot["indexer_flops"] / calls,
-                                   peak_note=fp8_note)
+        out["indexer"] = dict(bound="tensor", achieved=tot["indexer_flops"] / (stage_ms[0] * 1e-3) / 1e12,
+                              peak=fp8_sust, unit="TFLOP/s", algorithmic=tot["indexer_flops"] / calls,
+                              peak_note=fp8_note)
+    if stage_ms[1] > 0:
+        # top-k: a streaming selection over the causal scores
+        out["topk"] = dict(bound="hbm", achieved=tot["topk_bytes"] / (stage_ms[1] * 1e-3) / 1e9,
+                           peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["topk_bytes"] / calls)
     if decode:
         out["sparse_attn"] = dict(bound="hbm", achieved=tot["attn_bytes"] / (stage_ms[2] * 1e-3) / 1e9,
                                   peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["attn_bytes"] / calls,
@@ -363,16 +372,15 @@ def roofline_stages(wl, runner, stage_ms, peaks, peak_src):
         out["sparse_attn"] = dict(bound="tensor", achieved=tot["attn_flops"] / (stage_ms[2] * 1e-3) / 1e12,
                                   peak=peaks["bf16_tflops_sustained"], unit="TFLOP/s",
                                   algorithmic=tot["attn_flops"] / calls)
-    for name, ms in (("indexer_topk", stage_ms[0]), ("sparse_attn", stage_ms[2])):
+    total = sum(stage_ms)
+    for name, ms in (("indexer", stage_ms[0]), ("topk", stage_ms[1]), ("sparse_attn", stage_ms[2])):
+        if name not in out:
+            continue
         d = out[name]
         d["ms_per_step"] = ms
         d["frac"] = d["achieved"] / d["peak"]
         d["launches_per_step"] = calls
-    total = sum(stage_ms)
-    for name, ms in (("indexer_topk", stage_ms[0]), ("sparse_attn", stage_ms[2])):
-        out[name]["share"] = ms / total if total > 0 else None
-    # what is left of the top-k step once it is fused into the indexer (event gap)
-    out["topk_outside_indexer"] = {"ms_per_step": stage_ms[1], "share": stage_ms[1] / total if total > 0 else None}
+        d["share"] = ms / total if total > 0 else None
     return out
 
 
@@ -773,9 +781,10 @@ def main():
     tokens = tot["rows"] * world
     value = tokens / (ms_max * 1e-3)
     stages = roofline_stages(wl, runner, stage_ms, peaks, peak_src)
-    dom = max(("indexer_topk", "sparse_attn"), key=lambda n: stages[n]["ms_per_step"])
+    dom = max((n for n in ("indexer", "topk", "sparse_attn") if n in stages),
+              key=lambda n: stages[n]["ms_per_step"])
     d = stages[dom]
-    kernel_names = {"indexer_topk": "indexer_kernel", "sparse_attn": "sparse_attn_kernel"}
+    kernel_names = {"indexer": "indexer_kernel", "topk": "topk_kernel", "sparse_attn": "sparse_attn_kernel"}
     roof = {"kernel": kernel_names[dom], "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
             "unit": d["unit"], "frac": d["frac"],
             "traffic": traffic_from_profiles(kernel_names[dom], wl.name),
@@ -788,6 +797,7 @@ def main():
         "roofline": roof,
         "stages": {k: {kk: (round(vv, 6) if isinstance(vv, float) else vv) for kk, vv in v.items()}
                    for k, v in stages.items()},
+        "selection": "staged: the indexer writes the causal scores, a top-k kernel selects",
         "gpu_launches": runner.launches_per_call * len(runner.chunks) * args.steps,
         "clocks": clocks,
         "peaks": {"source": f"{peak_src} (MEASURED_PEAKS.json)", "hbm_gbs": peaks["hbm_gbs"],
@@ -811,6 +821,21 @@ def main():
             kl_line["cpu_baseline"] = cpu_baseline_kl(wl, runner, sel)
         extra["indexer_kl_loss"] = kl_line
         del sel
+        line["workloads"] = extra
+    if not args.no_extra and not wl.chunk:
+        # the same forward with the selection fused into the indexer (no score matrix)
+        del runner
+        torch.cuda.empty_cache()
+        runner = Runner(wl, seed=args.seed + rank, low_memory=True)
+        steps3 = max(3, args.steps // 4)
+        ms3, st3, _ = time_runner(runner, steps3, 2, world, False, local)
+        ms3 = max_over_ranks(ms3, world)
+        s3 = roofline_stages(wl, runner, st3, peaks, peak_src)
+        extra["fused_selection"] = {
+            "value": runner.totals()["rows"] * world / (ms3 * 1e-3), "unit": "tokens/s", "ms_per_step": ms3,
+            "steps": steps3, "warmup": 2, "workspace_bytes": runner.ws.numel(),
+            "stages": {k: {kk: (round(vv, 6) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                       for k, v in s3.items()}}
         line["workloads"] = extra
     if not args.no_extra:
         extra["prefill_2k_dense_vs_gather"] = time_dense_vs_gather(max(5, args.steps), args.warmup, world, peaks)

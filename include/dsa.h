@@ -73,8 +73,9 @@ typedef struct {
 typedef enum {
     DSA_OP_TOPK = 0,
     DSA_OP_SPARSE_ATTN = 1,
-    DSA_OP_FORWARD = 2,
-    DSA_OP_INDEXER_TOPK = 3
+    DSA_OP_FORWARD = 2,          /* dsa_forward, staged selection (the faster path) */
+    DSA_OP_INDEXER_TOPK = 3,
+    DSA_OP_FORWARD_LOWMEM = 4    /* dsa_forward, fused selection (no score matrix) */
 } dsa_op;
 
 /*
@@ -164,8 +165,19 @@ dsa_status dsa_sparse_attn_noalloc(const dsa_attn_args *args, int B, int Lq, int
                                    void *stream);
 
 /*
- * The whole forward pass: indexer -> top-k (fused, dsa_indexer_topk) -> sparse
- * attention.  `iargs` and `aargs` describe the same B, Lq, Lk, q_offset.
+ * The whole forward pass: indexer -> top-k -> sparse attention.  `iargs` and
+ * `aargs` describe the same B, Lq, Lk, q_offset.
+ * The selection runs one of two ways, chosen by the workspace the caller gives;
+ * both produce identical indices and selected scores:
+ *   staged (workspace >= dsa_workspace_size_args(DSA_OP_FORWARD, ...)): the
+ *     indexer writes the causal part of the [B, Lq, Lk] fp32 score matrix into
+ *     the workspace and a separate top-k kernel selects from it.  The faster
+ *     path on every measured shape: the selection then runs on all SMs at full
+ *     issue rate instead of competing with the indexer's epilogue.
+ *   fused (workspace >= dsa_workspace_size_args(DSA_OP_FORWARD_LOWMEM, ...) but
+ *     below the staged size): dsa_indexer_topk; no score matrix, a workspace of
+ *     a few tens of MB, slower.
+ * A workspace below both sizes is refused with DSA_ERR_WORKSPACE.
  * Short sequences (q_offset + Lq <= k): every row selects all of its positions
  * 0..t whatever the indexer says, so the pass is dense causal MLA attention (the
  * short-sequence mode of the DSA report's "Стоимость" section, where attention
@@ -174,8 +186,8 @@ dsa_status dsa_sparse_attn_noalloc(const dsa_attn_args *args, int B, int Lq, int
  * the index lists 0..t itself.
  *   indices: int32 [B, Lq, k] (as dsa_topk); out: bf16 [B, Lq, H, d_v];
  *   lse: fp32 [B, Lq, H] or NULL.
- * The workspace (dsa_workspace_size_args(DSA_OP_FORWARD, ...)) holds the fused
- * indexer's candidate lists and the split-k partials; no score matrix.
+ * The workspace holds the score matrix (staged) or the candidate lists (fused),
+ * then the split-k partials; its contents need not be initialised.
  */
 dsa_status dsa_forward(const dsa_indexer_args *iargs, const dsa_attn_args *aargs, int k,
                        int32_t *indices, void *out, float *lse,
@@ -187,11 +199,12 @@ dsa_status dsa_forward(const dsa_indexer_args *iargs, const dsa_attn_args *aargs
  *                 position (as dsa_indexer_topk), e.g. for dsa_indexer_kl_loss_selected.
  *                 When given, the indexer runs even for short sequences.
  *   stage_events: NULL, or four cudaEvent_t handles (created by the caller)
- *                 recorded on `stream` before the indexer, after the fused
- *                 indexer + top-k, after the top-k (the same point: the top-k is
- *                 part of the indexer) and after the attention (including its
- *                 split-k merge).  For short sequences without sel_scores the
- *                 first three coincide (the attention writes the index lists).
+ *                 recorded on `stream` before the indexer, after the indexer,
+ *                 after the top-k (on the fused path the second and third
+ *                 coincide: the top-k is part of the indexer) and after the
+ *                 attention (including its split-k merge).  For short sequences
+ *                 without sel_scores the first three coincide (the attention
+ *                 writes the index lists).
  */
 dsa_status dsa_forward_timed(const dsa_indexer_args *iargs, const dsa_attn_args *aargs, int k,
                              int32_t *indices, float *sel_scores, void *out, float *lse,
@@ -233,9 +246,11 @@ dsa_status dsa_indexer_kl_loss_selected(const dsa_attn_args *args, int B, int Lq
 
 /*
  * Bytes of device workspace the entry point `op` needs for these sizes (0 = none).
- * For DSA_OP_FORWARD and DSA_OP_INDEXER_TOPK it assumes H_I = 64, d_I = 128 and
- * q_offset = Lk - Lq (decode, or a prefill chunk); dsa_workspace_size_args gives
- * the exact figure for any indexer arguments.
+ * For DSA_OP_FORWARD, DSA_OP_FORWARD_LOWMEM and DSA_OP_INDEXER_TOPK it assumes
+ * H_I = 64, d_I = 128 and q_offset = Lk - Lq (decode, or a prefill chunk);
+ * dsa_workspace_size_args gives the exact figure for any indexer arguments.
+ * DSA_OP_FORWARD includes the fp32 score matrix, B * Lq * Lk * 4 bytes (4.3 GB
+ * at Lq = Lk = 32768).
  */
 size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_v);
 

@@ -22,13 +22,13 @@ __all__ = [
     "DSAError", "lib", "lib_path", "indexer_scores", "topk", "indexer_topk", "sparse_attn", "sparse_attn_noalloc",
     "forward", "indexer_kl_loss", "indexer_kl_loss_selected",
     "workspace_size", "workspace_size_args", "status_string", "device_status", "selftest_wait_timeout", "version",
-    "OP_TOPK", "OP_SPARSE_ATTN", "OP_FORWARD", "OP_INDEXER_TOPK",
+    "OP_TOPK", "OP_SPARSE_ATTN", "OP_FORWARD", "OP_INDEXER_TOPK", "OP_FORWARD_LOWMEM",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libdsa.so")
 
-OP_TOPK, OP_SPARSE_ATTN, OP_FORWARD, OP_INDEXER_TOPK = 0, 1, 2, 3
+OP_TOPK, OP_SPARSE_ATTN, OP_FORWARD, OP_INDEXER_TOPK, OP_FORWARD_LOWMEM = 0, 1, 2, 3, 4
 _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_WORKSPACE",
            4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT"}
 
@@ -254,12 +254,17 @@ def sparse_attn_noalloc(q, kv, indices, d_v, scale, out, lse=None, stream=None):
 
 
 def forward(q_I, q_scale, w, k_I, k_scale, q, kv, k, d_v, scale, q_offset=0, indices=None, out=None,
-            lse=None, want_lse=True, workspace=None, stream=None, stage_events=None, sel_scores=None):
-    """Indexer -> top-k (fused into the indexer) -> sparse attention.  Returns (indices, out, lse).
+            lse=None, want_lse=True, workspace=None, stream=None, stage_events=None, sel_scores=None,
+            low_memory=False):
+    """Indexer -> top-k -> sparse attention.  Returns (indices, out, lse).
 
+    The selection is staged (score matrix in the workspace, then the top-k
+    kernel; the faster path) unless ``low_memory`` is set or the given
+    ``workspace`` is too small for the score matrix, in which case it is fused
+    into the indexer (dsa_indexer_topk).  Both give identical results.
     ``stage_events``: optional four torch.cuda.Event objects, recorded on the
-    stream before the indexer, after the fused indexer + top-k, after the top-k
-    (the same point) and after the attention.  ``sel_scores``: optional fp32
+    stream before the indexer, after the indexer, after the top-k (the same
+    point when fused) and after the attention.  ``sel_scores``: optional fp32
     [B, Lq, k] tensor that receives the indexer score of every selected position.
     """
     ia = _indexer_args(q_I, q_scale, w, k_I, k_scale, q_offset)
@@ -275,7 +280,8 @@ def forward(q_I, q_scale, w, k_I, k_scale, q, kv, k, d_v, scale, q_offset=0, ind
         lse = torch.empty(B, Lq, H, dtype=torch.float32, device=q.device)
     if sel_scores is not None:
         _need(sel_scores, torch.float32, (B, Lq, k), "sel_scores")
-    workspace, nbytes = _workspace(OP_FORWARD, B, Lq, Lk, k, H, d_v, q.device, workspace, ia=ia)
+    workspace, nbytes = _workspace(OP_FORWARD_LOWMEM if low_memory else OP_FORWARD, B, Lq, Lk, k, H, d_v,
+                                   q.device, workspace, ia=ia)
     ev = None
     if stage_events is not None:
         if len(stage_events) != 4:

@@ -210,6 +210,11 @@ FusedWs fused_ws_layout(const IndexerParams& p) {
   return w;
 }
 
+// The staged forward's score matrix (fp32 [B, Lq, Lk]; only s <= t is written and read).
+size_t scores_ws_bytes(const dsa_indexer_args* a) {
+  return round_up((size_t)a->B * a->Lq * a->Lk * sizeof(float), 256);
+}
+
 size_t indexer_topk_ws_bytes(const dsa_indexer_args* a, int k) {
   const IndexerParams p = plan_indexer(a, true, k);
   if (p.queries_per_unit * a->H_I > 512 || p.rows_per_unit > indexer_fused_max_rows()) return 0;
@@ -272,9 +277,10 @@ dsa_status run_indexer_topk(const dsa_indexer_args* a, int k, int32_t* indices, 
 }
 
 dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, int k, int32_t* idx,
-                    cudaStream_t st) {
+                    float* sel_scores, cudaStream_t st) {
   TopkParams p{};
   p.scores = scores; p.B = B; p.Lq = Lq; p.Lk = Lk; p.q_offset = q_offset; p.k = k; p.indices = idx;
+  p.sel_scores = sel_scores;
   const long long nmax = (long long)q_offset + Lq < Lk ? (long long)q_offset + Lq : Lk;   // longest row
   // Rows up to kTopkCacheMax scores stay in shared memory between passes; longer
   // ones are re-read from L2 (measured faster at 32K: the small CTA lets more rows
@@ -428,7 +434,7 @@ dsa_status dsa_topk(const float* scores, int B, int Lq, int Lk, int q_offset, in
   if (!aligned16(scores) || !aligned16(indices)) return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
   if ((long long)B * Lq >= (1LL << 31)) return DSA_ERR_UNSUPPORTED;
-  return run_topk(scores, B, Lq, Lk, q_offset, k, indices, static_cast<cudaStream_t>(stream));
+  return run_topk(scores, B, Lq, Lk, q_offset, k, indices, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_sparse_attn(const dsa_attn_args* args, int B, int Lq, int Lk, const int32_t* indices, int k,
@@ -478,7 +484,12 @@ size_t dsa_workspace_size_args(dsa_op op, const dsa_indexer_args* iargs, int k, 
       return indexer_topk_ws_bytes(iargs, k);
     case DSA_OP_FORWARD:
       if (H <= 0 || d_v <= 0) return 0;
-      return round_up(indexer_topk_ws_bytes(iargs, k), 256) + attn_ws_bytes(iargs->B, iargs->Lq, k, H, d_v);
+      return scores_ws_bytes(iargs) + attn_ws_bytes(iargs->B, iargs->Lq, k, H, d_v);
+    case DSA_OP_FORWARD_LOWMEM: {
+      if (H <= 0 || d_v <= 0) return 0;
+      const size_t sel = indexer_topk_ws_bytes(iargs, k);
+      return sel ? round_up(sel, 256) + attn_ws_bytes(iargs->B, iargs->Lq, k, H, d_v) : 0;
+    }
   }
   return 0;
 }
@@ -491,7 +502,8 @@ size_t dsa_workspace_size(dsa_op op, int B, int Lq, int Lk, int k, int H, int d_
     case DSA_OP_SPARSE_ATTN:
       return attn_ws_bytes(B, Lq, k, H, d_v);
     case DSA_OP_INDEXER_TOPK:
-    case DSA_OP_FORWARD: {
+    case DSA_OP_FORWARD:
+    case DSA_OP_FORWARD_LOWMEM: {
       // The documented convention: H_I = 64, d_I = 128, q_offset = Lk - Lq.
       alignas(16) static const uint8_t dummy[16] = {};
       dsa_indexer_args a{B, Lq, Lk, Lk - Lq, 64, 128, dummy, nullptr, dummy, dummy, nullptr};
@@ -523,9 +535,18 @@ dsa_status dsa_forward_timed(const dsa_indexer_args* iargs, const dsa_attn_args*
   if (lse && !aligned16(lse)) return DSA_ERR_INVALID_ARG;
   if (sel_scores && !aligned16(sel_scores)) return DSA_ERR_INVALID_ARG;
   if (k < 1 || k > kMaxK) return DSA_ERR_UNSUPPORTED;
-  const size_t sel_bytes = round_up(indexer_topk_ws_bytes(iargs, k), 256);
-  const size_t need = sel_bytes + attn_ws_bytes(iargs->B, iargs->Lq, k, aargs->H, aargs->d_v);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  const size_t attn_need = attn_ws_bytes(iargs->B, iargs->Lq, k, aargs->H, aargs->d_v);
+  if (!workspace || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  // Staged selection when the workspace holds the score matrix (the faster path),
+  // else the fused indexer + top-k with its candidate lists.
+  const size_t staged_bytes = scores_ws_bytes(iargs);
+  const size_t fused_sel = indexer_topk_ws_bytes(iargs, k);
+  const size_t fused_bytes = fused_sel ? round_up(fused_sel, 256) : 0;
+  bool staged;
+  if (workspace_bytes >= staged_bytes + attn_need) staged = true;
+  else if (fused_bytes && workspace_bytes >= fused_bytes + attn_need) staged = false;
+  else return DSA_ERR_WORKSPACE;
+  const size_t sel_bytes = staged ? staged_bytes : fused_bytes;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> bool {
     return !stage_events || cudaEventRecord(static_cast<cudaEvent_t>(stage_events[i]), st) == cudaSuccess;
@@ -536,14 +557,25 @@ dsa_status dsa_forward_timed(const dsa_indexer_args* iargs, const dsa_attn_args*
   // Short sequences: when every row's causal range fits in k (q_offset + Lq <= k),
   // every position is selected whatever the scores, and the pass is dense causal
   // attention.  Unless the selected scores are asked for, the indexer is skipped
-  // and the top-k step writes the index lists 0..t without reading scores.
+  // and the attention kernel writes the index lists 0..t.
   const bool dense = (long long)iargs->q_offset + iargs->Lq <= k && !sel_scores;
-  if (!dense) {
-    // Indexer with the top-k fused into it: no score matrix is written.
-    s = run_indexer_topk(iargs, k, indices, sel_scores, workspace, sel_bytes, st);
+  if (!dense && staged) {
+    // Scores of s <= t only (the top-k reads no others), then the selection.
+    float* scores = static_cast<float*>(workspace);
+    s = run_indexer(iargs, scores, false, st);
     if (s != DSA_OK) return s;
+    if (!mark(1)) return DSA_ERR_CUDA;
+    s = run_topk(scores, iargs->B, iargs->Lq, iargs->Lk, iargs->q_offset, k, indices, sel_scores, st);
+    if (s != DSA_OK) return s;
+    if (!mark(2)) return DSA_ERR_CUDA;
+  } else {
+    if (!dense) {
+      // Indexer with the top-k fused into it: no score matrix is written.
+      s = run_indexer_topk(iargs, k, indices, sel_scores, workspace, sel_bytes, st);
+      if (s != DSA_OK) return s;
+    }
+    if (!mark(1) || !mark(2)) return DSA_ERR_CUDA;
   }
-  if (!mark(1) || !mark(2)) return DSA_ERR_CUDA;
   // Dense mode: the attention kernel reads keys 0..t as contiguous tiles and writes
   // the index lists itself (no top-k launch, no gathers).
   s = run_attn(aargs, iargs->B, iargs->Lq, iargs->Lk, iargs->q_offset, true, indices, k, out, lse, attn_ws,

@@ -54,6 +54,7 @@ struct TopkParams {
   const float* scores;    // [B, Lq, Lk]
   int B, Lq, Lk, q_offset, k;
   int32_t* indices;       // [B, Lq, k]
+  float* sel_scores;      // [B, Lq, k] or null: score of each selected position (-0.0 as +0.0), -inf padding
   int cache_cap;          // row elements cached in shared memory (0 = re-read from global); multiple of 4
   int bit_words;          // 32-bit words of each position bitmap (>= ceil(row length / 32)); multiple of 4
   int cand_cap;           // candidate (key, position) pairs held in shared memory

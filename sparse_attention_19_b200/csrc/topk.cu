@@ -50,6 +50,12 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The score at a selected position as the selection saw it: -0.0 reads as +0.0.
+__device__ __forceinline__ float selected_score(const float* src, int s) {
+  const float v = __ldg(src + s);
+  return v == 0.f ? 0.f : v;
+}
+
 // Block-wide scratch for scans and reductions.
 struct ScanScratch {
   uint32_t warp_tot[kWarps];
@@ -176,10 +182,14 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
   const int n = (int)((t + 1 < p.Lk) ? t + 1 : p.Lk);
   const int k = p.k;
   int32_t* out = p.indices + (size_t)row * k;
+  float* sel_out = p.sel_scores ? p.sel_scores + (size_t)row * k : nullptr;
   const float* src = p.scores + (size_t)row * p.Lk;
 
   if (n <= k) {                                     // everything up to t is selected
-    for (int x = threadIdx.x; x < k; x += kThreads) out[x] = (x < n) ? x : -1;
+    for (int x = threadIdx.x; x < k; x += kThreads) {
+      out[x] = (x < n) ? x : -1;
+      if (sel_out) sel_out[x] = (x < n) ? selected_score(src, x) : -INFINITY;
+    }
     return;
   }
   const bool cached = n <= p.cache_cap;
@@ -354,10 +364,16 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
       const int s = w * 32 + bit;
       if ((gw >> bit) & 1u) {
         const uint32_t pos = gg + min(ee, eq_take);
-        if (pos < (uint32_t)k) out[pos] = s;
+        if (pos < (uint32_t)k) {
+          out[pos] = s;
+          if (sel_out) sel_out[pos] = selected_score(src, s);
+        }
         ++gg;
       } else {
-        if (ee < eq_take && gg + ee < (uint32_t)k) out[gg + ee] = s;
+        if (ee < eq_take && gg + ee < (uint32_t)k) {
+          out[gg + ee] = s;
+          if (sel_out) sel_out[gg + ee] = selected_score(src, s);
+        }
         ++ee;
       }
     }
@@ -413,11 +429,15 @@ topk_cluster_kernel(const TopkParams p) {
   const int n = (int)((t + 1 < p.Lk) ? t + 1 : p.Lk);
   const int k = p.k;
   int32_t* out = p.indices + (size_t)row * k;
+  float* sel_out = p.sel_scores ? p.sel_scores + (size_t)row * k : nullptr;
   const float* src = p.scores + (size_t)row * p.Lk;
 
   if (n <= k) {                                     // the whole cluster leaves together
     if (r == 0)
-      for (int x = threadIdx.x; x < k; x += kThreads) out[x] = (x < n) ? x : -1;
+      for (int x = threadIdx.x; x < k; x += kThreads) {
+        out[x] = (x < n) ? x : -1;
+        if (sel_out) sel_out[x] = (x < n) ? selected_score(src, x) : -INFINITY;
+      }
     return;
   }
   const int seg = ((n + kClusterCtas - 1) / kClusterCtas + 31) / 32 * 32;
@@ -582,10 +602,16 @@ topk_cluster_kernel(const TopkParams p) {
       const int s = s0 + w * 32 + bit;
       if ((gw >> bit) & 1u) {
         const uint32_t pos = gg + min(ee, eq_take);
-        if (pos < (uint32_t)k) out[pos] = s;
+        if (pos < (uint32_t)k) {
+          out[pos] = s;
+          if (sel_out) sel_out[pos] = selected_score(src, s);
+        }
         ++gg;
       } else {
-        if (ee < eq_take && gg + ee < (uint32_t)k) out[gg + ee] = s;
+        if (ee < eq_take && gg + ee < (uint32_t)k) {
+          out[gg + ee] = s;
+          if (sel_out) sel_out[gg + ee] = selected_score(src, s);
+        }
         ++ee;
       }
     }

@@ -106,17 +106,22 @@ def test_workspace_sizes():
     assert ws >= 4 * 16 * 128 * 512 * 4
     # 64 rows already occupy most pairs: whole rows per unit, no partials
     assert dsa.workspace_size(dsa.OP_SPARSE_ATTN, 64, 1, 131072, 2048, 128, 512) == 0
-    # The forward's indexer selects on chip: its workspace holds candidate lists
-    # (at most 2k + 256 per row in flight), never the [Lq, Lk] score matrix.
+    # The staged forward keeps the fp32 score matrix in its workspace ...
     fwd = dsa.workspace_size(dsa.OP_FORWARD, 1, 4096, 131072, 2048, 128, 512)
-    assert 0 < fwd < 4096 * 131072 * 4 // 4
-    fwd32 = dsa.workspace_size(dsa.OP_FORWARD, 1, 32768, 32768, 2048, 128, 512)
-    assert 0 < fwd32 < 32768 * 32768 * 4 // 16
-    assert dsa.workspace_size(dsa.OP_FORWARD, 0, 1, 1, 1, 1, 1) == 0
+    assert 4096 * 131072 * 4 <= fwd < 4096 * 131072 * 4 + (1 << 20)
+    # ... the low-memory one selects on chip: candidate lists (at most 2k + 512
+    # per row in flight), never the [Lq, Lk] score matrix.
+    low = dsa.workspace_size(dsa.OP_FORWARD_LOWMEM, 1, 4096, 131072, 2048, 128, 512)
+    assert 0 < low < 4096 * 131072 * 4 // 4
+    low32 = dsa.workspace_size(dsa.OP_FORWARD_LOWMEM, 1, 32768, 32768, 2048, 128, 512)
+    assert 0 < low32 < 32768 * 32768 * 4 // 16
+    for op in (dsa.OP_FORWARD, dsa.OP_FORWARD_LOWMEM):
+        assert dsa.workspace_size(op, 0, 1, 1, 1, 1, 1) == 0
     # the exact query agrees with the convention-based one when q_offset = Lk - Lq
     ia = _idx_args(B=64, Lq=1, Lk=131072, q_offset=131071)
-    assert dsa.workspace_size_args(dsa.OP_FORWARD, ia, 2048, 128, 512) == \
-        dsa.workspace_size(dsa.OP_FORWARD, 64, 1, 131072, 2048, 128, 512)
+    for op in (dsa.OP_FORWARD, dsa.OP_FORWARD_LOWMEM):
+        assert dsa.workspace_size_args(op, ia, 2048, 128, 512) == \
+            dsa.workspace_size(op, 64, 1, 131072, 2048, 128, 512)
     assert dsa.workspace_size_args(dsa.OP_INDEXER_TOPK, ia, 2048) == \
         dsa.workspace_size(dsa.OP_INDEXER_TOPK, 64, 1, 131072, 2048, 128, 512) > 0
     # invalid indexer arguments: no size
