@@ -172,12 +172,14 @@ IndexerParams plan_indexer(const dsa_indexer_args* a, bool fused, int k) {
     const int slot_bytes = p.qb * 128 * 8;
     int ns = 16384 / slot_bytes;
     ns = ns < 2 ? 2 : (ns > indexer_fused_max_stage() ? indexer_fused_max_stage() : ns);
-    // With one 64-column accumulator per sub-block the four epilogue quads take
-    // accumulators (and so staging slots) in turn.  A slot must always belong to
-    // the same quad, since an mbarrier's parity only tells its current phase from
-    // the one before: a quad that could run two uses of a slot ahead of the
-    // selector would pass its wait early.  So the slot count is a multiple of four.
-    if (p.qb * a->H_I <= 64) ns = ns < 4 ? 4 : ns / 4 * 4;
+    // The epilogue's quad groups take accumulators (and so staging slots) in turn:
+    // four groups when an accumulator is one 64-column group, else two.  A slot must
+    // always belong to the same group, since an mbarrier's parity only tells its
+    // current phase from the one before: a group that could run two uses of a slot
+    // ahead of the selector would pass its wait early.  So the slot count is a
+    // multiple of the group count.
+    const int ngroups = p.qb * a->H_I <= 64 ? 4 : 2;
+    ns = ns < ngroups ? ngroups : ns / ngroups * ngroups;
     p.n_stage = ns;
   }
   return p;

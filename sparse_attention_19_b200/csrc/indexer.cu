@@ -165,6 +165,15 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   uint8_t* tiles = smem_raw + (((raw_addr + (uint32_t)sizeof(IndexerSmem) + 1023u) & ~1023u) - raw_addr);
   const int N = p.qb * H_I;                            // MMA N (queries x heads)
   const uint32_t nslot = min(8, kTmemCols / N);        // accumulators in flight (more when N is small)
+  // Epilogue quads work on accumulators in groups of `span`: the groups take
+  // accumulators in turn (group g gets seq = g mod ngroups), and within a group quad
+  // q reads the 64-column groups (q mod span) * 64, + span * 64, ...  Two quads per
+  // accumulator (prefill, N = 256): two accumulators are read at once, each warp
+  // reading two queries, so one group's fixed per-accumulator costs overlap the
+  // other group's arithmetic.  One quad per accumulator when N <= 64 (decode).
+  const int span = N <= 64 ? 1 : 2;
+  const uint32_t ngroups = (uint32_t)(kQuads / span);
+  const int warps_per_acc = 4 * span;
   const int QU = p.queries_per_unit;                   // = qb * nsub
   const uint32_t q_bytes = (uint32_t)(p.nsub * N) * kRowBytes;   // one query block
   const uint32_t n_qbuf = query_buffers(q_bytes);
@@ -200,19 +209,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
     for (int s = 0; s < 8; ++s) {
       mbar_init(&S.acc_full[s], 1);
-      mbar_init(&S.acc_empty[s], N <= 64 ? 4 : kEpiWarps);
+      mbar_init(&S.acc_empty[s], warps_per_acc);
     }
-    // A tile's key scales are read by the warps that process its accumulators: all
-    // sixteen when an accumulator spans the quads, else the quads that own one of
-    // its sub-blocks (consecutive accumulators go to consecutive quads).
-    const int sc_readers = N <= 64 ? 4 * min(p.nsub, kQuads) : kEpiWarps;
+    // A tile's key scales are read by the warps of the groups that process one of
+    // its sub-blocks' accumulators (consecutive accumulators go to consecutive groups).
+    const int sc_readers = warps_per_acc * min(p.nsub, (int)ngroups);
     for (int s = 0; s < kScaleSlots; ++s) {
       mbar_init(&S.sc_full[s], 1);
       mbar_init(&S.sc_empty[s], sc_readers);
     }
     if (kFused) {
       for (int s = 0; s < p.n_stage; ++s) {
-        mbar_init(&S.stg_full[s], N <= 64 ? 4 : kEpiWarps);
+        mbar_init(&S.stg_full[s], warps_per_acc);
         mbar_init(&S.stg_empty[s], min(kSelWarps, p.rows_per_unit));   // selectors that own a row
       }
       // No unit owns a threshold yet (unit ordinals start at 0).
@@ -281,7 +289,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       const uint32_t idesc = make_idesc(0, 0, 128, (uint32_t)N, 0, 0);  // e4m3 x e4m3 -> f32
-      uint32_t ucount = 0, kstage = 0, kphase = 0, seq = 0;
+      uint32_t ucount = 0, kstage = 0, kphase = 0, slot = 0, use = 0;
       const uint32_t k_base = smem_u32(k_smem);
       for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++ucount) {
         const UnitInfo U = decode_unit(p, u);
@@ -295,7 +303,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           tc_fence_after();
           const uint32_t a_addr = k_base + kstage * kKeysPerTile * kRowBytes;
           for (int sb = 0; sb < p.nsub; ++sb) {
-            const uint32_t slot = seq % nslot, use = seq / nslot;
             if (!mbar_wait(&S.acc_empty[slot], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + slot * (uint32_t)N;
@@ -307,7 +314,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
               mma_f8_ss(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
             }
             mma_commit(&S.acc_full[slot]);
-            ++seq;
+            if (++slot == nslot) { slot = 0; ++use; }
           }
           mma_commit(&S.k_empty[kstage]);
           if (++kstage == kStages) { kstage = 0; kphase ^= 1; }
@@ -502,13 +509,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     regs_increase<kRegsEpi>();
     // ------------------------------------------------------------ epilogue
     const uint32_t quarter = warp & 3u;              // TMEM lane quarter this warp may read
-    const uint32_t quad = warp >> 2;                 // which 64-column groups: quad, quad + 4, ...
-    // With a single 64-column group (decode: one query per sequence) the quads take
-    // accumulators in turn instead of column groups.
-    const bool narrow = N <= 64;
+    const uint32_t quad = warp >> 2;
+    const uint32_t group = quad / (uint32_t)span;    // reads accumulators seq = group mod ngroups
+    // this warp's 64-column groups of such an accumulator: g_first, g_first + g_step, ...
+    const int g_first = (int)(quad % (uint32_t)span) * 64, g_step = 64 * span;
     const uint32_t row = quarter * 32 + lane;        // key row within the tile
     const int et = threadIdx.x;                      // 0 .. 32 * kEpiWarps - 1
-    uint32_t seq = 0, epi_phase = 0, sc_use = 0, ucount = 0;
+    uint32_t seq = 0, epi_phase = 0, sc_use = 0, ucount = 0, acc_slot = 0, acc_use = 0;
     // A unit's weights and query scales sit in smem buffer (unit ordinal % 2).  The
     // next unit's values are read into registers when a unit starts and stored when
     // it ends, so their memory latency hides under the unit's work.
@@ -557,13 +564,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         const int s = kt * kKeysPerTile + (int)row;
         float sk = 0.f;
         const uint32_t ss = sc_use % kScaleSlots;
-        // In narrow mode this warp reads the tile only if its quad owns one of the
-        // tile's accumulators (seq .. seq + nsub - 1).
-        bool reads_tile = true;
-        if (narrow) {
-          reads_tile = false;
-          for (int sb = 0; sb < p.nsub; ++sb) reads_tile |= ((seq + sb) % kQuads == quad);
-        }
+        // This warp reads the tile only if its group owns one of the tile's
+        // accumulators (seq .. seq + nsub - 1).
+        bool reads_tile = false;
+        for (int sb = 0; sb < p.nsub; ++sb) reads_tile |= ((seq + (uint32_t)sb) & (ngroups - 1u)) == group;
         if (p.scale_ring) {
           if (reads_tile) {
             if (!mbar_wait_warp(&S.sc_full[ss], (sc_use / kScaleSlots) & 1u, abort_flag)) { ok = false; break; }
@@ -574,8 +578,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           sk_next = key_scale(kt + 1);
         }
         for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
-          const uint32_t slot = seq % nslot, use = seq / nslot;
-          if (narrow && seq % kQuads != quad) continue;
+          const uint32_t slot = acc_slot, use = acc_use;
+          if (++acc_slot == nslot) { acc_slot = 0; ++acc_use; }
+          if ((seq & (ngroups - 1u)) != group) continue;
           if (!mbar_wait_warp(&S.acc_full[slot], use & 1u, abort_flag)) { ok = false; break; }
           uint32_t gs = 0;                                   // staging slot (fused mode)
           if constexpr (kFused) {
@@ -630,21 +635,32 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             }
             return fadd2(acc2, acc_b);
           };
-          const int g_first = narrow ? 0 : (int)quad * 64, g_step = narrow ? 64 : 64 * kQuads;
+          // The accumulator is handed back to the MMA issuer as soon as this warp's
+          // last TMEM load of it has completed.
+          auto release = [&]() {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acc_empty[slot]);
+          };
           if constexpr (H_I == 64) {
-            // This warp's 64-column groups (one query each), 32 columns per TMEM load.
+            // This warp's 64-column groups (one query each), 32 columns per TMEM load;
+            // the accumulator goes back to the MMA issuer once the last load is in.
             for (int g0 = g_first; g0 < N; g0 += g_step) {
               const int qi = g0 / 64;                            // query within the sub-block
               const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
               uint32_t v[32];
               tmem_ld32(t_base + (uint32_t)g0, v);
               tmem_ld_wait();
+              tmem_regs_ready(v);
               float2 acc2 = relu_dot(v, wq, 32, make_float2(0.f, 0.f));
               tmem_ld32(t_base + (uint32_t)g0 + 32, v);
               tmem_ld_wait();
+              tmem_regs_ready(v);
+              if (g0 + g_step >= N) release();
               acc2 = relu_dot(v, wq + 8, 32, acc2);
               finish(qi, acc2.x + acc2.y);
             }
+            if (g_first >= N) release();
           } else {
             // Small H_I: each 64-column group holds 64 / H_I queries, 32 / H_I per load.
             constexpr int QPL = 32 / H_I;
@@ -654,6 +670,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                 uint32_t v[32];
                 tmem_ld32(t_base + (uint32_t)(g0 + part * 32), v);
                 tmem_ld_wait();
+                tmem_regs_ready(v);
 #pragma unroll
                 for (int a = 0; a < QPL; ++a) {
                   const int qi = (g0 + part * 32) / H_I + a;
@@ -663,12 +680,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
                 }
               }
             }
+            release();
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&S.acc_empty[slot]);
-            if (kFused) mbar_arrive(&S.stg_full[gs]);
+          if (kFused) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.stg_full[gs]);
           }
         }
         if (p.scale_ring) {
@@ -744,11 +760,12 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
   // A small resident query block (decode) leaves room for a deeper key ring.
   const bool deep = p.nsub * p.qb * p.H_I <= 128;
   const bool fused = p.scores == nullptr;
-  // Narrow accumulators (N <= 64) go to the four quads in turn; each staging slot
-  // must stay with one quad (see the staging ring), so n_stage % 4 == 0 there.
-  const bool narrow = p.qb * p.H_I <= 64;
+  // Accumulators go to the epilogue's quad groups in turn (four groups of one quad
+  // when N <= 64, else two of two); each staging slot must stay with one group (see
+  // the staging ring), so n_stage is a multiple of the group count.
+  const int ngroups = p.qb * p.H_I <= 64 ? kQuads : kQuads / 2;
   if (fused && (p.rows_per_unit > kMaxRows || p.n_stage > kMaxStage || p.n_stage < 1 || p.cap < p.k + 128 ||
-                p.cap % 32 != 0 || (narrow && p.n_stage % kQuads != 0)))
+                p.cap % 32 != 0 || p.n_stage % ngroups != 0))
     return cudaErrorInvalidValue;
   if (p.H_I == 64 && p.d_I == 128) {
     if (fused)

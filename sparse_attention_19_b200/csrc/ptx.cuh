@@ -179,8 +179,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 
 // Warp-uniform bounded wait: every lane polls, and the warp proceeds only if all
 // lanes saw the phase complete (so .sync.aligned instructions never diverge).
+// The first poll is taken by the whole warp and voted on, so the common case (the
+// phase is already complete) stays free of divergence; only a warp that must wait
+// enters the per-lane loop.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
                                                volatile uint32_t* abort_flag, bool cluster_scope = false) {
+  const uint32_t a = smem_u32(bar);
+  const bool first = cluster_scope ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity);
+  if (__all_sync(0xffffffffu, first)) return true;
   const bool ok = mbar_wait(bar, parity, abort_flag, cluster_scope);
   return __all_sync(0xffffffffu, ok);
 }
@@ -424,6 +430,23 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// After tmem_ld_wait: pass the loaded registers through an empty volatile asm, so
+// the compiler cannot move their first use above the wait (the load writes them
+// asynchronously, which the compiler does not know).
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15]));
+}
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                 "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                 "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
