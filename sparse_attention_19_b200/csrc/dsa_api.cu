@@ -300,6 +300,9 @@ dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, in
     p.bit_words = (int)round_up((size_t)(seg / 32), 4);
   }
   p.vec4 = (aligned16(scores) && Lk % 4 == 0) ? 1 : 0;
+  // Many rows (prefill): one warp per row, rows streamed from L2 / HBM with no
+  // block-wide steps; enough of them to give every SM several CTAs of rows.
+  p.warp_rows = (!p.cluster && rows >= 16LL * sm_count()) ? 1 : 0;
   return launch_topk(p, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

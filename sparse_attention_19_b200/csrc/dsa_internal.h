@@ -61,6 +61,7 @@ struct TopkParams {
   int vec4;               // rows start 16-byte aligned (scores aligned, Lk % 4 == 0): 16-byte loads
   int cluster;            // each row spread over a cluster of kTopkClusterCtas CTAs (few long rows);
                           // bit_words then covers one CTA's segment
+  int warp_rows;          // one warp per row (many rows): no block-wide steps, rows streamed from L2
 };
 constexpr int kTopkClusterCtas = 4;
 size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap, bool cluster);

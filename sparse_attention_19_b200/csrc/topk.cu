@@ -31,6 +31,7 @@
 
 #include "dsa_internal.h"
 #include "ptx.cuh"
+#include "warp_select.cuh"
 
 namespace dsa {
 
@@ -620,6 +621,230 @@ topk_cluster_kernel(const TopkParams p) {
   }
 }
 
+// ------------------------------------------------------------------ many rows
+// One warp per row, eight rows per CTA: no block-wide barrier anywhere, so each
+// warp streams its row (from L2 / HBM) at its own pace and an SM keeps many rows
+// in flight.  The same selection as above:
+//   1. a strided sample of 256 scores sets the key range [lo, hi] of a 1024-bin
+//      histogram (keys outside it are counted in the end bins);
+//   2. one pass over the row builds that histogram and gives the bin b holding the
+//      m-th largest key and the count above it;
+//   3. the exact threshold inside bin b's key window: histogram levels over the
+//      window's keys until the boundary bin's keys fit the warp's candidate buffer,
+//      then levels over the candidates (warp_find_threshold);
+//   4. one ordered pass writes every position above the threshold and the first
+//      positions equal to it, in ascending position order.
+constexpr int kWarpRowsPerCta = 8;
+constexpr int kWarpSample = 256;
+
+struct WarpTopkSmem {
+  uint32_t hist[kSelBins];
+  uint32_t cand[kSelCandCap + 4];
+};
+
+// f(key) for every score of src[0 .. n) (16-byte loads when vec4, else 4-byte);
+// lanes call f different numbers of times.
+template <typename F>
+__device__ __forceinline__ void visit_row_keys(const float* src, int n, bool vec4, F f) {
+  const int lane = (int)(threadIdx.x & 31u);
+  if (vec4) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    const int n4 = n >> 2;
+    constexpr int kU = 4;
+    for (int g0 = 0; g0 < n4; g0 += 32 * kU) {
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int g = g0 + u * 32 + lane;
+        v[u] = g < n4 ? __ldg(s4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        if (g0 + u * 32 + lane < n4) {
+          f(score_to_key(v[u].x));
+          f(score_to_key(v[u].y));
+          f(score_to_key(v[u].z));
+          f(score_to_key(v[u].w));
+        }
+      }
+    }
+    for (int s = (n4 << 2) + lane; s < n; s += 32) f(score_to_key(__ldg(src + s)));
+  } else {
+    constexpr int kU = 8;
+    for (int s0 = 0; s0 < n; s0 += 32 * kU) {
+      float v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int s = s0 + u * 32 + lane;
+        v[u] = s < n ? __ldg(src + s) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (s0 + u * 32 + lane < n) f(score_to_key(v[u]));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int lane = (int)(threadIdx.x & 31u), warp = (int)(threadIdx.x >> 5);
+  WarpTopkSmem& sh = reinterpret_cast<WarpTopkSmem*>(smem_raw)[warp];
+  const long long row = (long long)blockIdx.x * kWarpRowsPerCta + warp;   // b * Lq + i
+  if (row >= (long long)p.B * p.Lq) return;                             // whole warp
+  const int i = (int)(row % p.Lq);
+  const long long t = (long long)p.q_offset + i;
+  const int n = (int)((t + 1 < p.Lk) ? t + 1 : p.Lk);
+  const uint32_t k = (uint32_t)p.k;
+  int32_t* out = p.indices + (size_t)row * k;
+  float* sel_out = p.sel_scores ? p.sel_scores + (size_t)row * k : nullptr;
+  const float* src = p.scores + (size_t)row * p.Lk;
+  if ((uint32_t)n <= k) {                           // everything up to t is selected
+    for (uint32_t x = lane; x < k; x += 32) {
+      out[x] = (x < (uint32_t)n) ? (int32_t)x : -1;
+      if (sel_out) sel_out[x] = (x < (uint32_t)n) ? key_to_score(score_to_key(__ldg(src + x))) : -INFINITY;
+    }
+    return;
+  }
+  const bool vec4 = p.vec4 != 0;
+
+  // ---- 1. key range of a strided sample
+  uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+  for (int u = 0; u < kWarpSample / 32; ++u) {
+    const int j = u * 32 + lane;
+    const uint32_t key = score_to_key(__ldg(src + (int)(((long long)j * n) / kWarpSample)));
+    lo = min(lo, key);
+    hi = max(hi, key);
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  const int shift = sel_shift(hi - lo);
+
+  // ---- 2. clamped histogram of the whole row and the boundary bin
+  for (int x = lane; x < kSelBins / 4; x += 32) reinterpret_cast<uint4*>(sh.hist)[x] = make_uint4(0, 0, 0, 0);
+  __syncwarp();
+  visit_row_keys(src, n, vec4, [&](uint32_t key) {
+    const uint32_t d = key < lo ? 0u : min((uint32_t)(kSelBins - 1), (key - lo) >> shift);
+    atomicAdd(&sh.hist[d], 1u);
+  });
+  __syncwarp();
+  constexpr int kPer = kSelBins / 32;                // bins per lane
+  uint32_t mine = 0;
+#pragma unroll
+  for (int x = 0; x < kPer / 4; ++x) {
+    const uint4 v = reinterpret_cast<const uint4*>(sh.hist + lane * kPer)[x];
+    mine += v.x + v.y + v.z + v.w;
+  }
+  uint32_t suffix = mine;                            // bins of lanes >= this lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, suffix, o);
+    if (lane + o < 32) suffix += y;
+  }
+  const uint32_t above_lane = suffix - mine;
+  const uint32_t owner = __ffs(__ballot_sync(0xffffffffu, above_lane < k && suffix >= k)) - 1;
+  uint32_t b = 0, above = 0;
+  if ((uint32_t)lane == owner) {
+    uint32_t acc = above_lane;
+    for (int x = kPer - 1; x >= 0; --x) {
+      const uint32_t c = sh.hist[lane * kPer + x];
+      if (acc + c >= k) { b = lane * kPer + x; above = acc; break; }
+      acc += c;
+    }
+  }
+  b = __shfl_sync(0xffffffffu, b, owner);
+  above = __shfl_sync(0xffffffffu, above, owner);
+  __syncwarp();
+
+  // ---- 3. exact threshold among the keys of bin b's window
+  const uint32_t wlo = b == 0 ? 0u : lo + (b << shift);
+  uint32_t whi = 0xffffffffu;
+  if (b + 1 < (uint32_t)kSelBins) {
+    const unsigned long long top = (unsigned long long)lo + ((unsigned long long)(b + 1) << shift) - 1ull;
+    whi = top < 0xffffffffull ? (uint32_t)top : 0xffffffffu;
+  }
+  uint32_t thr, gt_w;
+  auto visit = [&](auto&& f) { visit_row_keys(src, n, vec4, f); };
+  warp_find_threshold(sh.hist, sh.cand, visit, k - above, wlo, whi, thr, gt_w, sh.hist[b]);
+  const uint32_t eq_take = k - above - gt_w;
+
+  // ---- 4. ordered output: every key above thr and the first eq_take equal to it
+  uint32_t w = 0, eq_seen = 0;
+  // keys[] are positions s .. s + cnt - 1 of this lane (cnt <= 4), lanes in position order
+  auto emit_group = [&](int s, const uint32_t (&key)[4], int cnt) {
+    uint32_t gtm = 0, eqm = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      gtm |= (j < cnt && key[j] > thr) ? (1u << j) : 0u;
+      eqm |= (j < cnt && key[j] == thr) ? (1u << j) : 0u;
+    }
+    uint32_t eq_tot;
+    const uint32_t eq_rank = eq_seen + warp_exclusive_sum(__popc(eqm), eq_tot);
+    uint32_t take = gtm, e = eqm;
+    for (uint32_t r = eq_rank; e && r < eq_take; ++r) {   // equal keys taken in position order
+      take |= e & (0u - e);
+      e &= e - 1u;
+    }
+    uint32_t kept;
+    uint32_t at = w + warp_exclusive_sum(__popc(take), kept);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (take & (1u << j)) {
+        out[at] = s + j;
+        if (sel_out) sel_out[at] = key_to_score(key[j]);
+        ++at;
+      }
+    }
+    w += kept;
+    eq_seen += eq_tot;
+  };
+  if (vec4) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    const int n4 = (n + 3) >> 2;                     // the last group may run past n (masked below)
+    constexpr int kU = 4;
+    for (int g0 = 0; g0 < n4; g0 += 32 * kU) {
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int g = g0 + u * 32 + lane;
+        v[u] = g < (n >> 2) ? __ldg(s4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (g == (n >> 2) && (n & 3)) {               // ragged tail: scalar loads inside the row
+          v[u].x = __ldg(src + 4 * g);
+          if ((n & 3) > 1) v[u].y = __ldg(src + 4 * g + 1);
+          if ((n & 3) > 2) v[u].z = __ldg(src + 4 * g + 2);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        if (g0 + u * 32 < n4) {
+          const int g = g0 + u * 32 + lane;
+          const uint32_t key[4] = {score_to_key(v[u].x), score_to_key(v[u].y), score_to_key(v[u].z),
+                                   score_to_key(v[u].w)};
+          emit_group(4 * g, key, max(0, min(4, n - 4 * g)));
+        }
+      }
+    }
+  } else {
+    constexpr int kU = 8;
+    for (int s0 = 0; s0 < n; s0 += 32 * kU) {
+      float v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int s = s0 + u * 32 + lane;
+        v[u] = s < n ? __ldg(src + s) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int s = s0 + u * 32 + lane;
+        if (s0 + u * 32 < n) {
+          const uint32_t key[4] = {score_to_key(v[u]), 0u, 0u, 0u};
+          emit_group(s, key, s < n ? 1 : 0);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
 size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap, bool cluster) {
@@ -630,8 +855,16 @@ size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap, bool cluster)
 }
 
 cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream) {
-  const size_t smem = topk_smem_bytes(p.cache_cap, p.bit_words, p.cand_cap, p.cluster != 0);
   const int rows = p.B * p.Lq;
+  if (p.warp_rows) {
+    const size_t wsmem = sizeof(WarpTopkSmem) * kWarpRowsPerCta;
+    cudaError_t e = cudaFuncSetAttribute(topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem);
+    if (e != cudaSuccess) return e;
+    if (rows == 0) return cudaSuccess;
+    topk_warp_kernel<<<(rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta, 32 * kWarpRowsPerCta, wsmem, stream>>>(p);
+    return cudaGetLastError();
+  }
+  const size_t smem = topk_smem_bytes(p.cache_cap, p.bit_words, p.cand_cap, p.cluster != 0);
   if (p.cluster) {
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -26,9 +26,10 @@ constexpr int kSelBinBits = 10;
 constexpr int kSelCandCap = 512;        // boundary-bin keys gathered into shared memory
 
 __device__ __forceinline__ uint32_t score_to_key(float f) {
-  uint32_t u = __float_as_uint(f);
-  if ((u << 1) == 0u) u = 0u;                          // -0.0 -> +0.0
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  // f + 0.0f turns -0.0 into +0.0 (round-to-nearest) and leaves every other value
+  // as it is; then negatives are complemented and positives get the top bit set.
+  const uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
 }
 __device__ __forceinline__ float key_to_score(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
@@ -92,17 +93,19 @@ __device__ __forceinline__ void sel_level(uint32_t* hist, Visit visit, uint32_t 
   __syncwarp();
 }
 
-// Threshold of the top-`m` of the candidates that `visit` produces, all of whose
-// keys lie in [lo, hi] and of which there are more than m.  Returns thr and
-// gt = #{key > thr} (so m - gt candidates equal to thr are taken, the first ones
-// in position order).  `cand` holds up to kSelCandCap keys of the boundary bin.
+// Threshold of the top-`m` of the keys in [lo, hi] that `visit` produces (keys
+// outside the window are ignored), of which there are at least m.  Returns thr and
+// gt = #{lo <= key <= hi, key > thr} (so m - gt keys equal to thr are taken, the
+// first ones in position order).  `cand` holds up to kSelCandCap keys of the
+// boundary bin.  `count`, when not 0xffffffff, is the number of keys in the window,
+// known to the caller: at most kSelCandCap of them go straight to the candidates.
 template <typename Visit>
 __device__ __forceinline__ void warp_find_threshold(uint32_t* hist, uint32_t* cand, Visit visit, uint32_t m, uint32_t lo,
-                                    uint32_t hi, uint32_t& thr, uint32_t& gt) {
+                                    uint32_t hi, uint32_t& thr, uint32_t& gt, uint32_t count = 0xffffffffu) {
   const uint32_t lane = threadIdx.x & 31u;
   uint32_t need = m, got = 0;
   // Levels over the list itself until the boundary bin is small enough to copy.
-  for (;;) {
+  for (; count > (uint32_t)kSelCandCap;) {
     const int shift = sel_shift(hi - lo);
     uint32_t b, above;
     sel_level(hist, visit, lo, hi, shift, need, b, above);
