@@ -384,6 +384,16 @@ def roofline_stages(wl, runner, stage_ms, peaks, peak_src):
     return out
 
 
+def topk_kernel_name(wl, chunk):
+    """Which top-k kernel dsa_topk launches for these rows (the library's dispatch rule)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rows = wl.B * chunk
+    nmax = min(wl.q_offset + wl.Lq, wl.Lk) if not wl.chunk else wl.Lk
+    if rows * 4 <= 2 * sms and nmax > 16384:
+        return "topk_cluster_kernel"
+    return "topk_warp_kernel" if rows >= 16 * sms else "topk_kernel"
+
+
 def traffic_from_profiles(kernel_name, workload):
     """ncu DRAM bytes per launch recorded under profiles/ for this kernel + workload, if current."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -784,7 +794,8 @@ def main():
     dom = max((n for n in ("indexer", "topk", "sparse_attn") if n in stages),
               key=lambda n: stages[n]["ms_per_step"])
     d = stages[dom]
-    kernel_names = {"indexer": "indexer_kernel", "topk": "topk_kernel", "sparse_attn": "sparse_attn_kernel"}
+    kernel_names = {"indexer": "indexer_kernel", "topk": topk_kernel_name(wl, runner.chunk_len),
+                    "sparse_attn": "sparse_attn_kernel"}
     roof = {"kernel": kernel_names[dom], "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
             "unit": d["unit"], "frac": d["frac"],
             "traffic": traffic_from_profiles(kernel_names[dom], wl.name),

@@ -1,0 +1,88 @@
+"""Top-k over many rows (prefill-sized row counts), the shape that runs one warp
+per row: a sampled key range, one histogram pass, the exact threshold inside the
+boundary bin (its keys straight to a 512-entry buffer when they fit, else
+histogram levels over the row), and an ordered output pass.
+
+Every row is held against the fp64 oracle's top-k ("Отбор и основное внимание":
+the k positions with the largest I[t, s]; ties to the smaller position, -0.0
+equal to +0.0), bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_19_b200 as dsa
+from dsa_inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+ROWS = 2600          # above the many-rows threshold (16 rows per SM on a 148-SM part)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    dsa.lib()
+    yield
+    assert dsa.device_status() == 0
+
+
+def _check(scores, q_offset, k):
+    B, Lq, Lk = scores.shape
+    idx = dsa.topk(scores, k, q_offset)
+    torch.cuda.synchronize()
+    sc = scores.double().cpu().numpy().reshape(B * Lq, Lk)
+    row_t = q_offset + np.arange(B * Lq) % Lq
+    exp = oracle.topk(sc, row_t, k)
+    got = idx.cpu().numpy().reshape(B * Lq, k)
+    bad = np.nonzero(~np.all(got == exp, axis=1))[0]
+    assert bad.size == 0, f"{bad.size} rows differ, first {bad[:5]}"
+    return got
+
+
+def test_many_rows_random_scores_aligned_rows():
+    g = torch.Generator().manual_seed(21)
+    s = torch.randn(1, ROWS, 6000, generator=g)       # 16-byte aligned rows
+    _check(s.to(DEV), 6000 - ROWS, 2048)
+
+
+def test_many_rows_ragged_length_and_heavy_ties():
+    # Lk not a multiple of four (4-byte loads); scores on a 0.1 grid: many ties
+    g = torch.Generator().manual_seed(22)
+    s = torch.round(torch.randn(1, ROWS, 5003, generator=g) * 10) / 10
+    _check(s.to(DEV), 5003 - ROWS, 2048)
+
+
+def test_many_rows_boundary_bin_overflows_the_buffer():
+    # a block of 3000 equal scores straddles the threshold in every row: the
+    # boundary bin holds more than 512 keys, so the threshold comes from
+    # histogram levels over the row
+    g = torch.Generator().manual_seed(23)
+    s = torch.randn(1, ROWS, 8000, generator=g)
+    s[:, :, 2000:5000] = 1.25
+    _check(s.to(DEV), 8000 - ROWS, 2048)
+
+
+def test_many_rows_all_equal_and_signed_zero():
+    s = torch.full((2, ROWS // 2, 4100), 0.75)
+    s[0, ::2] = 0.0
+    s[0, ::2, ::3] = -0.0
+    got = _check(s.to(DEV), 4100 - ROWS // 2, 1024)
+    assert np.array_equal(got[0], np.arange(1024))
+
+
+def test_forward_selected_scores_from_the_many_rows_kernel():
+    # dsa_forward's staged selection returns I[t, s] at every selected position
+    wl = WORKLOADS["prefill_8k"].with_(Lq=ROWS, Lk=6000, q_offset=6000 - ROWS)
+    inp = make_inputs(wl, DEV, 7)
+    sel = torch.empty(wl.B, wl.Lq, wl.k, dtype=torch.float32, device=DEV)
+    idx, _, _ = dsa.forward(inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], inp["q"],
+                            inp["kv"], wl.k, wl.Dv, wl.scale, wl.q_offset, sel_scores=sel)
+    scores = dsa.indexer_scores(inp["q_I"], inp["q_scale"], inp["w"], inp["k_I"], inp["k_scale"], wl.q_offset)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, dsa.topk(scores, wl.k, wl.q_offset))
+    valid = idx >= 0
+    want = torch.gather(scores, 2, idx.clamp_min(0).long())
+    assert torch.equal(sel[valid], want[valid])
+    assert torch.all(torch.isneginf(sel[~valid]))
