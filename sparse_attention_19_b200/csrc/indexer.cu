@@ -643,8 +643,30 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             if (lane == 0) mbar_arrive(&S.acc_empty[slot]);
           };
           if constexpr (H_I == 64) {
-            // This warp's 64-column groups (one query each), 32 columns per TMEM load;
-            // the accumulator goes back to the MMA issuer once the last load is in.
+            // This warp's 64-column groups (one query each).  Two of them (prefill:
+            // each warp holds two queries of the accumulator) are read together, 16
+            // columns of each per TMEM load, so the two reductions interleave; the
+            // accumulator goes back to the MMA issuer once the last load is in.
+            if (g_first + g_step < N) {
+              const int qa = g_first / 64, qb2 = (g_first + g_step) / 64;   // queries within the sub-block
+              const float4* wa = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qa) * H_I);
+              const float4* wb = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qb2) * H_I);
+              float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                uint32_t va[16], vb[16];
+                tmem_ld16(t_base + (uint32_t)(g_first + c * 16), va);
+                tmem_ld16(t_base + (uint32_t)(g_first + g_step + c * 16), vb);
+                tmem_ld_wait();
+                tmem_regs_ready(va);
+                tmem_regs_ready(vb);
+                if (c == 3) release();
+                acc_a = relu_dot(va, wa + c * 4, 16, acc_a);
+                acc_b = relu_dot(vb, wb + c * 4, 16, acc_b);
+              }
+              finish(qa, acc_a.x + acc_a.y);
+              finish(qb2, acc_b.x + acc_b.y);
+            } else
             for (int g0 = g_first; g0 < N; g0 += g_step) {
               const int qi = g0 / 64;                            // query within the sub-block
               const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
