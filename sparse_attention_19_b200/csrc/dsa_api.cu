@@ -300,9 +300,17 @@ dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, in
     p.bit_words = (int)round_up((size_t)(seg / 32), 4);
   }
   p.vec4 = (aligned16(scores) && Lk % 4 == 0) ? 1 : 0;
-  // Many rows (prefill): one warp per row, rows streamed from L2 / HBM with no
-  // block-wide steps; enough of them to give every SM several CTAs of rows.
-  p.warp_rows = (!p.cluster && rows >= 16LL * sm_count()) ? 1 : 0;
+  // Many rows of moderate length (prefill up to 32K): one warp per row, rows
+  // streamed from L2 / HBM with no block-wide steps; enough of them to give every
+  // SM several CTAs of rows.
+  p.warp_rows = (!p.cluster && rows >= 16LL * sm_count() && nmax <= 32768) ? 1 : 0;
+  // Longer rows (a 128K prefill's chunks) are read once: a sampled threshold keeps
+  // the few thousand keys that can be in the top-k (the candidate buffer grows to
+  // 8192 entries for them), with the two-pass selection as the fallback.
+  if (!p.cluster && !p.warp_rows && p.cache_cap == 0) {
+    p.sampled = 1;
+    p.cand_cap = 8192;
+  }
   return launch_topk(p, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

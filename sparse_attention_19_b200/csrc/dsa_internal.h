@@ -62,6 +62,7 @@ struct TopkParams {
   int cluster;            // each row spread over a cluster of kTopkClusterCtas CTAs (few long rows);
                           // bit_words then covers one CTA's segment
   int warp_rows;          // one warp per row (many rows): no block-wide steps, rows streamed from L2
+  int sampled;            // long rows: try the single-pass selection above a sampled threshold first
 };
 constexpr int kTopkClusterCtas = 4;
 size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap, bool cluster);

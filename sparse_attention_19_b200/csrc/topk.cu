@@ -197,22 +197,92 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
   auto key_at = [&](int s) -> uint32_t { return cached ? cache[s] : score_key(__ldg(src + s)); };
   auto load_key = [&](int s) -> uint32_t { return score_key(__ldg(src + s)); };
 
-  // ---- 1. key range of a strided sample
+  // ---- 1. key range of a strided sample (kept in the candidate buffer for step 1b)
   const int ns = n < kSample ? n : kSample;
+  const bool try_single = p.sampled && !cached && p.cand_cap >= kSample;
   uint32_t smin = 0xffffffffu, smax = 0u;
   for (int j = threadIdx.x; j < ns; j += kThreads) {
     const uint32_t key = load_key((int)(((long long)j * n) / ns));
+    if (try_single) cand[j].x = key;
     smin = min(smin, key);
     smax = max(smax, key);
   }
   block_min_max(sh.x, smin, smax);
-
-  // ---- 2. histogram over the sampled range (outliers clamped into the end bins)
   const uint32_t lo = smin;
   const int shift = bin_shift(smax - smin);
   auto bin_of = [lo, shift](uint32_t key) -> uint32_t {
     return key < lo ? 0u : min((uint32_t)(kBins - 1), (key - lo) >> shift);
   };
+
+  // ---- 1b. long rows, one pass: a threshold theta at the sample's j-th largest key
+  // (its bin's lower edge), j six standard deviations above the count the sample
+  // is expected to hold above the k-th largest key of the row.  Every key >= theta
+  // is kept with its position; if at least k and at most cand_cap of them are
+  // found, the row's top-k is among them (each key below theta has k keys above
+  // it), and the threshold is resolved on the candidates alone.  Otherwise the
+  // row takes the two-pass route below (a rare event by construction, or rows of
+  // many equal keys).
+  bool single = false;
+  uint32_t nsingle = 0;
+  if (try_single) {
+    const float mu = (float)ns * (float)k / (float)n;
+    const float sig = sqrtf(mu * (1.f - (float)k / (float)n));
+    const uint32_t j = (uint32_t)ceilf(mu + 6.f * sig + 2.f);
+    if (j < (uint32_t)ns) {
+      clear_hist(sh.hist);
+      for (int x = threadIdx.x; x < ns; x += kThreads) atomicAdd(&sh.hist[bin_of(cand[x].x)], 1u);
+      __syncthreads();
+      find_bin(sh.hist, sh.x, j);
+      const uint32_t tb = sh.x.bin;
+      const uint32_t theta = tb == 0 ? 0u : lo + (tb << shift);
+      const int W = (n + 31) >> 5;
+      for (int x = threadIdx.x; x < W; x += kThreads) { gt_bits[x] = 0u; eq_bits[x] = 0u; }
+      if (threadIdx.x == 0) sh.x.ncand = 0u;
+      __syncthreads();
+      auto keep = [&](int s, uint32_t key) {
+        if (key >= theta) {
+          const uint32_t at = atomicAdd(&sh.x.ncand, 1u);
+          if (at < (uint32_t)p.cand_cap) cand[at] = make_uint2(key, (uint32_t)s);
+        }
+      };
+      if (p.vec4) {
+        const float4* src4 = reinterpret_cast<const float4*>(src);
+        const int nq = n >> 2;
+        for (int q0 = threadIdx.x; q0 < nq; q0 += kThreads * kUnroll4) {
+          float4 f[kUnroll4];
+#pragma unroll
+          for (int u = 0; u < kUnroll4; ++u) {
+            const int q = q0 + u * kThreads;
+            f[u] = (q < nq) ? __ldg(src4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < kUnroll4; ++u) {
+            const int q = q0 + u * kThreads;
+            if (q >= nq) break;
+            keep(4 * q, score_key(f[u].x));
+            keep(4 * q + 1, score_key(f[u].y));
+            keep(4 * q + 2, score_key(f[u].z));
+            keep(4 * q + 3, score_key(f[u].w));
+          }
+        }
+        for (int s = (nq << 2) + (int)threadIdx.x; s < n; s += kThreads) keep(s, load_key(s));
+      } else {
+        row_pass(n, load_key, [&](int s, bool valid, uint32_t key) {
+          if (valid) keep(s, key);
+        });
+      }
+      __syncthreads();
+      nsingle = sh.x.ncand;
+      single = nsingle >= (uint32_t)k && nsingle <= (uint32_t)p.cand_cap;
+      __syncthreads();
+    }
+  }
+
+  uint32_t need = (uint32_t)k;                       // n > k, so m = k
+  uint32_t b = 0, cnt_b = nsingle;
+  bool fits = true;
+  if (!single) {
+  // ---- 2. histogram over the sampled range (outliers clamped into the end bins)
   clear_hist(sh.hist);
   if (p.vec4) {
     // 16-byte loads (rows start 16-byte aligned): four scores per thread per step.
@@ -250,11 +320,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
     });
   }
   __syncthreads();
-  uint32_t need = (uint32_t)k;                       // n > k, so m = k
   find_bin(sh.hist, sh.x, need);
-  const uint32_t b = sh.x.bin;
+  b = sh.x.bin;
   need -= sh.x.above;
-  const uint32_t cnt_b = sh.hist[b];
+  cnt_b = sh.hist[b];
 
   // ---- 3. bins above b are selected; bin b becomes the candidate list
   if (threadIdx.x == 0) sh.x.ncand = 0u;
@@ -269,9 +338,11 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
     }
   });
   __syncthreads();
-  const bool fits = cnt_b <= (uint32_t)p.cand_cap;
+  fits = cnt_b <= (uint32_t)p.cand_cap;
+  }   // two-pass route
 
-  // Exact threshold: the need-th largest key among the elements of bin b, found
+  // Exact threshold: the need-th largest key among the elements of bin b (or of
+  // the single-pass candidates), found
   // by 2048-bin histograms over a shrinking key window [wlo, whi] (inclusive).
   uint32_t wlo, whi;
   if (fits) {

@@ -86,3 +86,34 @@ def test_forward_selected_scores_from_the_many_rows_kernel():
     want = torch.gather(scores, 2, idx.clamp_min(0).long())
     assert torch.equal(sel[valid], want[valid])
     assert torch.all(torch.isneginf(sel[~valid]))
+
+
+# Long rows (more than 32768 scores, or fewer rows than the one-warp kernel
+# wants): one CTA per row reads the row once, keeping every key at or above a
+# threshold taken from a strided sample, and falls back to two passes when the
+# kept keys number fewer than k or more than the 8192-entry buffer.
+
+def test_long_rows_single_pass_random_scores():
+    g = torch.Generator().manual_seed(31)
+    s = torch.randn(1, 300, 40000, generator=g)
+    _check(s.to(DEV), 40000 - 300, 2048)
+
+
+def test_long_rows_ragged_length_with_planted_block():
+    # Lk not a multiple of four; a block of high scores at the start of every row
+    # (the strided sample sees few of them) and a band of ties
+    g = torch.Generator().manual_seed(32)
+    s = torch.randn(1, 200, 50001, generator=g)
+    s[:, :, :1500] += 6.0
+    s[:, :, 30000:30100] = 2.0
+    _check(s.to(DEV), 50001 - 200, 2048)
+
+
+def test_long_rows_fall_back_when_too_many_keys_pass():
+    # half of every row equal to one value above the sample's threshold: far more
+    # than 8192 keys pass, so the row takes the two-pass route
+    g = torch.Generator().manual_seed(33)
+    s = torch.randn(2, 100, 36000, generator=g)
+    s[:, :, ::2] = 1.5
+    s[1, :, 1::3] = -0.0
+    _check(s.to(DEV), 36000 - 100, 2048)
