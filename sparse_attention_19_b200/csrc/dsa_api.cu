@@ -85,8 +85,6 @@ dsa_status check_attn(const dsa_attn_args* a, int B, int Lq, int Lk) {
   return DSA_OK;
 }
 
-// Split-k factor for the attention: enough (row, split) units to cover the SM
-// pairs several times over; 1 for prefill-sized batches.
 // Split-k factor for the attention: each row's key tiles are spread over s units
 // (s a power of two).  Cost model in units of one tile's pipelined time on a CTA
 // pair (measured ~2.5 us): a unit costs its tiles plus about 1.8 tiles of fill,
