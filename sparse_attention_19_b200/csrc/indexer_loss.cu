@@ -19,17 +19,19 @@
 //     16 chunks of 64 gathered latent rows x 64 columns per CTA (TMA
 //     tile::gather4, 128-byte swizzle).  One warp issues its TMA requests in
 //     order, so each chunk's 16 gathers are split over a team of four warps.
-//   * Keys come in tiles of 128 selected positions; S = Q K^T is one pair-MMA
-//     chain (M = 128 heads, N = 128 keys, K = 16 per instruction) issued by one
-//     thread of the leader CTA, into four S buffers in TMEM.  Each CTA's TMEM holds
-//     its 64 heads: lanes 0-63 keys 0-63 of the tile, lanes 64-127 keys 64-127.
+//   * Keys come in tiles of 128 selected positions; S^T = K Q^T is one pair-MMA
+//     chain (M = 128 keys, 64 per CTA: the CTA's own gathered rows; N = 128 heads,
+//     64 per CTA: its own Q rows; K = 16 per instruction) issued by one thread of
+//     the leader CTA, into four S buffers in TMEM.  Each CTA's TMEM holds its 64
+//     keys against all 128 heads: lane l holds key l % 64 and heads
+//     64 (l / 64) .. 64 (l / 64) + 63 in its 64 columns.  So a key's head sum is
+//     a per-thread sum over columns, with no exchange between threads.
 //   * Eight reduction warps per CTA read S: warp w holds TMEM lane quarter w % 4
-//     (32 heads, one key half) for 32 of the half's 64 keys.  Each lane turns its
-//     logits into probabilities with its head's lse, then the warp sums them over
-//     its 32 heads by a butterfly transpose-reduction (31 shuffles leave lane i
-//     holding key i's sum) and posts the sums to a 4-tile ring in the leader's
-//     shared memory: the leader's warps with plain stores and an arrive, the
-//     other CTA's with st.async, whose bytes complete the same barrier.
+//     (32 keys, one head half) and 32 of the half's 64 heads.  Each thread turns
+//     its key's 32 logits into probabilities with the heads' lse and sums them,
+//     then posts the sum to a 3-tile ring in the leader's shared memory: the
+//     leader's warps with plain stores and an arrive, the other CTA's with
+//     st.async, whose bytes complete the same barrier.
 //   * Four loss warps of the leader own one key each: per tile they add the four
 //     head-quarter sums into P, fold it into the row's running sums (sum P,
 //     sum P log P, sum P (I - m), and the indexer log-sum-exp with a running
@@ -69,7 +71,7 @@ constexpr int kTeamWarps = 4;          // loader warps sharing each chunk's 16 g
 constexpr int kTeamSlots = 4;          // consecutive ring slots a team owns
 constexpr int kLoadWarps = kStages / kTeamSlots * kTeamWarps;   // 16
 constexpr int kThreads = 32 * (kLoadWarp0 + kLoadWarps);   // 1024
-constexpr int kRedSlots = 4;           // tiles of head sums in flight to the loss warps
+constexpr int kRedSlots = 3;           // tiles of head sums in flight to the loss warps
 constexpr uint32_t kPeerBytes = kRedWarps * 32 * 4;       // the other CTA's sums per tile
 constexpr int kStageBatch = 8;         // index words in flight per staging warp
 constexpr int kMaxIdx = 2048;
@@ -92,7 +94,8 @@ struct KlShared {
   uint32_t abort_flag;
   uint32_t valid_mask[2][kMaxIdx / 32];  // per 32 staged slots: bit set = valid position
   int32_t last_word[2][kStageWarps];     // per staging warp: last 32-slot word with a valid position
-  float red[kRedSlots][4][kTileKeys];    // leader: per tile, 32-head sums (rank * 2 + quarter), per key
+  float red[kRedSlots][4][kTileKeys];    // leader: per tile, 32-head sums (head quarter), per key
+  alignas(16) float nl[kRedWarps][32];   // per reduction warp: -lse * log2 e of its 32 heads (row)
   float fin[kLossWarps][5];              // leader: per loss warp (Z, A, Bs, m, s) of the row
 };
 
@@ -284,8 +287,8 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    // S = Q K^T for each tile into TMEM buffer (tile ordinal % 2): per key chunk,
-    // 4 pair-MMAs of K = 16 (descriptor start addresses advance 32 B, encoded 2).
+    // S^T = K Q^T for each tile into TMEM buffer (tile ordinal % kSBufs): per key
+    // chunk, 4 pair-MMAs of K = 16 (descriptor start addresses advance 32 B, encoded 2).
     if (leader && elect_one()) {
       constexpr uint32_t idesc = make_idesc(1, 1, 128, kTileKeys, 0, 0);   // bf16, K-major x K-major
       const uint64_t q_desc = make_smem_desc(smem_u32(q_sm), 16, 1024, LAYOUT_SW128);
@@ -307,8 +310,9 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
             const uint32_t st = kc % kStages, ph = (kc / kStages) & 1u;
             if (!mbar_wait(&S.k_full[st], ph, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t ad = q_desc + (uint64_t)(c * (kPlane >> 4));
-            const uint64_t bd = k_desc + (uint64_t)(st * (kPlane >> 4));
+            // A = this tile's key chunk (keys on M), B = the Q plane (heads on N)
+            const uint64_t ad = k_desc + (uint64_t)(st * (kPlane >> 4));
+            const uint64_t bd = q_desc + (uint64_t)(c * (kPlane >> 4));
             mma_bf16_ss_pair(d, ad + 0, bd + 0, idesc, c ? 1u : 0u);
             mma_bf16_ss_pair(d, ad + 2, bd + 2, idesc, 1u);
             mma_bf16_ss_pair(d, ad + 4, bd + 4, idesc, 1u);
@@ -329,26 +333,31 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
   } else if (warp < (uint32_t)kRedWarps) {
     // ------------------------------------------------------------------ reduction warps
     const uint32_t quarter = warp & 3u;            // TMEM lane quarter
-    const int hq = (int)(quarter & 1u);            // head quarter within this CTA's 64 heads
-    const int kh = (int)(quarter >> 1);            // key half of the tile held by these lanes
-    const int c0 = (int)(warp >> 2) * 32;          // this warp's 32 of the half's 64 keys
-    const int kk0 = kh * kHalfKeys + c0;           // first key of the tile this warp reduces
-    const int head = (int)rank * 64 + hq * 32 + (int)lane;
-    const bool head_ok = head < p.H;
+    const int hh = (int)(quarter >> 1);            // head half held by these lanes
+    const int key_c = (int)(quarter & 1u) * 32 + (int)lane;   // this thread's key among the CTA's 64
+    const int key = (int)rank * kHalfKeys + key_c; // and within the tile
+    const int c0 = (int)(warp >> 2) * 32;          // this warp's 32 of the half's 64 heads (columns)
+    const int hq = hh * 2 + (int)(warp >> 2);      // head quarter: heads 32 hq .. 32 hq + 31
     const uint32_t lane_addr = (quarter * 32u) << 16;
     const float2 scl = make_float2(p.scale_log2, p.scale_log2);
-    // where this warp's 32 sums go in the leader's ring, and the barrier that counts them
-    const uint32_t red_dst = mapa_shared(smem_u32(&S.red[0][(int)rank * 2 + hq][kk0 + (int)lane]), 0);
+    // where this thread's sum goes in the leader's ring, and the barrier that counts them
+    const uint32_t red_dst = mapa_shared(smem_u32(&S.red[0][hq][key]), 0);
     const uint32_t red_full0 = mapa_shared(smem_u32(&S.red_full[0]), 0);
+    const float4* nl4 = reinterpret_cast<const float4*>(S.nl[warp]);
     uint32_t ucount = 0, sc = 0;
     for (int row = cluster_id; row < p.n_rows && ok; row += n_clusters, ++ucount) {
       const uint32_t ib = ucount & 1u, uph = (ucount >> 1) & 1u;
       ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
       if (!ok) break;
       const int nt = row_tiles(S.last_word, ib);
-      // exponent offset: a_h[s] = 2^(z * scale * log2 e - lse * log2 e)
-      const float nl = (head_ok && nt > 0) ? -p.lse[(size_t)row * p.H + head] * kLog2e : 0.f;
-      const float2 nl2 = make_float2(nl, nl);
+      // exponent offsets of this warp's 32 heads: a_h[s] = 2^(z * scale * log2 e - lse_h * log2 e);
+      // heads past H get -inf (probability 0)
+      {
+        const int head = hq * 32 + (int)lane;
+        __syncwarp();                                // the previous row's reads are done
+        S.nl[warp][lane] = (head < p.H && nt > 0) ? -p.lse[(size_t)row * p.H + head] * kLog2e : -INFINITY;
+        __syncwarp();
+      }
       for (int j = 0; j < nt && ok; ++j, ++sc) {
         const uint32_t sb = sc % kSBufs;
         ok = mbar_wait_warp(&S.s_full[sb], (sc / kSBufs) & 1u, abort_flag);
@@ -357,54 +366,39 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
         uint32_t v[32];
         tmem_ld32(tmem_base + lane_addr + sb * kHalfKeys + c0, v);
         tmem_ld_wait();
+        tmem_regs_ready(v);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&S.s_empty[sb]), 0));
-        const uint32_t vm = head_ok ? S.valid_mask[ib][(j * kTileKeys + kk0) >> 5] : 0u;
-        float pr[32];
-        if (vm == 0xffffffffu) {                       // warp-uniform: every key valid
+        const bool kvalid = (S.valid_mask[ib][(j * kTileKeys + key) >> 5] >> (key & 31)) & 1u;
+        // sum over the 32 heads of 2^(z * scale * log2 e + nl_h)
+        float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scl, nl2);
-            pr[e] = ex2_approx(x.x);
-            pr[e + 1] = ex2_approx(x.y);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scl, nl2);
-            pr[e] = ((vm >> e) & 1u) ? ex2_approx(x.x) : 0.f;
-            pr[e + 1] = ((vm >> (e + 1)) & 1u) ? ex2_approx(x.y) : 0.f;
-          }
+        for (int e = 0; e < 32; e += 4) {
+          const float4 n4 = nl4[e / 4];
+          const float2 xa = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scl,
+                                  make_float2(n4.x, n4.y));
+          const float2 xb = ffma2(make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])), scl,
+                                  make_float2(n4.z, n4.w));
+          acc_a = fadd2(acc_a, make_float2(ex2_approx(xa.x), ex2_approx(xa.y)));
+          acc_b = fadd2(acc_b, make_float2(ex2_approx(xb.x), ex2_approx(xb.y)));
         }
-        // Butterfly transpose-reduction over the warp's 32 heads: at each step a lane
-        // keeps the half of its columns selected by one bit of its lane number and
-        // adds the partner's copy of that half.  Lane i ends with key kk0 + i.
-#pragma unroll
-        for (int half = 16; half >= 1; half >>= 1) {
-          const bool up = (lane & (uint32_t)half) != 0u;
-#pragma unroll
-          for (int e = 0; e < half; ++e) {
-            const float lo = pr[e], hi = pr[e + half];
-            const float send = up ? lo : hi;
-            const float keep = up ? hi : lo;
-            pr[e] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-          }
-        }
+        const float2 t2 = fadd2(acc_a, acc_b);
+        const float psum = kvalid ? t2.x + t2.y : 0.f;
         // Post to ring slot sc % kRedSlots once the loss warps are done with it.
         const uint32_t slot = sc % kRedSlots, rph = (sc / kRedSlots) & 1u;
         ok = mbar_wait_warp(&S.red_empty[slot], rph ^ 1u, abort_flag, true);
         if (!ok) break;
         const uint32_t off = slot * (uint32_t)sizeof(S.red[0]);
         if (leader) {
-          S.red[slot][hq][kk0 + (int)lane] = pr[0];
+          S.red[slot][hq][key] = psum;
           __syncwarp();
           if (lane == 0) {
             if (warp == 0) mbar_arrive_expect_tx(&S.red_full[slot], kPeerBytes);
             else mbar_arrive(&S.red_full[slot]);
           }
         } else {
-          st_async_f32(red_dst + off, pr[0], red_full0 + slot * 8u);
+          st_async_f32(red_dst + off, psum, red_full0 + slot * 8u);
         }
       }
       if (!ok) break;
