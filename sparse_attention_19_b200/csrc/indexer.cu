@@ -559,8 +559,22 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         if (kt >= U.kt1 || s >= p.Lk) return 0.f;
         return p.k_scale ? __ldg(p.k_scale + (size_t)U.b * p.Lk + s) : 1.f;
       };
-      float sk_next = p.scale_ring ? 0.f : key_scale(U.kt0);
-      for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
+      // With one sub-block per tile (decode, fused mode) a group owns every
+      // ngroups-th tile: the warp visits only those, stepping the tile, accumulator
+      // and scale-slot counters over the others instead of looping through them
+      // (each skipped pass cost as much as a few hundred instructions of issue).
+      const bool stride = p.nsub == 1;
+      const uint32_t seq_u = seq, sc_u = sc_use;
+      const int kt_first = stride ? U.kt0 + (int)((group - seq_u) & (ngroups - 1u)) : U.kt0;
+      const int kt_step = stride ? (int)ngroups : 1;
+      float sk_next = p.scale_ring ? 0.f : key_scale(kt_first);
+      for (int kt = kt_first; kt < U.kt1 && ok; kt += kt_step) {
+        if (stride) {
+          seq = seq_u + (uint32_t)(kt - U.kt0);
+          sc_use = sc_u + (uint32_t)(kt - U.kt0);
+          acc_slot = seq % nslot;
+          acc_use = seq / nslot;
+        }
         const int s = kt * kKeysPerTile + (int)row;
         float sk = 0.f;
         const uint32_t ss = sc_use % kScaleSlots;
@@ -575,7 +589,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           }
         } else {
           sk = sk_next;
-          sk_next = key_scale(kt + 1);
+          sk_next = key_scale(kt + kt_step);
         }
         for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
           const uint32_t slot = acc_slot, use = acc_use;
@@ -716,6 +730,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         }
       }
       if (!ok) break;
+      if (stride) {
+        // counters past the unit's last tile, whichever tile this warp saw last
+        const uint32_t nt = (uint32_t)(U.kt1 - U.kt0);
+        seq = seq_u + nt;
+        if (p.scale_ring) sc_use = sc_u + nt;
+        acc_slot = seq % nslot;
+        acc_use = seq / nslot;
+      }
       // Full-matrix output: positions beyond this unit's causal tiles are -inf.
       if (!kFused && p.fill_upper && p.kchunks == 1) {
         const int nt_all = (p.Lk + kKeysPerTile - 1) / kKeysPerTile;
