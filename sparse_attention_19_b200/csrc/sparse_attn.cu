@@ -254,38 +254,47 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
         if (!ok) break;
         const int32_t* idx = idx_sm + ib * kMaxIdx;
-        for (int j = U.j0; j < U.j1 && ok; ++j) {
-          for (int c = 0; c < NC; ++c, ++kc) {
-            const uint32_t st = kc % kKStages, ph = (kc / kKStages) & 1u;
-            if (st / kKTeamSlots != my_team) continue;
-            // Dense mode: one box per chunk from the team's first warp; the others
-            // have nothing to load and must not wait either (a waiter that adds
-            // nothing to a phase can fall two phases behind, where its parity test
-            // would no longer see the phase it waits for).
-            if (p.dense && part != 0) continue;
-            bool w_ok = true;
-            if (lane == 0) {
-              w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
-              if (w_ok && leader && part == 0) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
-            }
-            if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-            const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
-            if (p.dense) {
-              // keys 0..t are contiguous: this CTA's 64 rows of the tile in one box
-              if (part == 0 && lane == 0)
-                tma_load_2d_pair(k_sm + st * kPlane64, &tmap_kv_tile, full_l, c * 64,
-                                 U.b * p.Lk + j * kTileKeys + (int)rank * kHalfKeys);
-              continue;
-            }
-            const int g = part + kKTeamWarps * (int)lane;            // 4-key group of this lane
-            if (g < kHalfKeys / 4) {
-              const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
-              tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
-                               gather_row(idx, base + 0), gather_row(idx, base + 1),
-                               gather_row(idx, base + 2), gather_row(idx, base + 3));
-            }
+        // The unit's chunks are kc_u .. kc_u + nk - 1; chunk x goes to slot x % kKStages.
+        // The team visits only the chunks of its own slots (lo .. lo + kKTeamSlots - 1)
+        // rather than stepping through all of them.
+        const uint32_t kc_u = kc, nk = (uint32_t)(U.j1 - U.j0) * NC, lo = my_team * kKTeamSlots;
+        uint32_t x = kc_u;
+        {
+          const uint32_t r = x % kKStages;
+          if (r < lo) x += lo - r;
+          else if (r >= lo + kKTeamSlots) x += kKStages - r + lo;
+        }
+        for (; x < kc_u + nk && ok; x += (x % kKStages + 1 < lo + kKTeamSlots) ? 1u : kKStages - kKTeamSlots + 1u) {
+          const uint32_t st = x % kKStages, ph = (x / kKStages) & 1u;
+          const int j = U.j0 + (int)((x - kc_u) / NC), c = (int)((x - kc_u) % NC);
+          // Dense mode: one box per chunk from the team's first warp; the others
+          // have nothing to load and must not wait either (a waiter that adds
+          // nothing to a phase can fall two phases behind, where its parity test
+          // would no longer see the phase it waits for).
+          if (p.dense && part != 0) continue;
+          bool w_ok = true;
+          if (lane == 0) {
+            w_ok = mbar_wait(&S.k_empty[st], ph ^ 1u, abort_flag);
+            if (w_ok && leader && part == 0) mbar_arrive_expect_tx(&S.k_full[st], 2u * kPlane64);
+          }
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+          const uint32_t full_l = mapa_shared(smem_u32(&S.k_full[st]), 0);
+          if (p.dense) {
+            // keys 0..t are contiguous: this CTA's 64 rows of the tile in one box
+            if (part == 0 && lane == 0)
+              tma_load_2d_pair(k_sm + st * kPlane64, &tmap_kv_tile, full_l, c * 64,
+                               U.b * p.Lk + j * kTileKeys + (int)rank * kHalfKeys);
+            continue;
+          }
+          const int g = part + kKTeamWarps * (int)lane;            // 4-key group of this lane
+          if (g < kHalfKeys / 4) {
+            const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
+            tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
+                             gather_row(idx, base + 0), gather_row(idx, base + 1),
+                             gather_row(idx, base + 2), gather_row(idx, base + 3));
           }
         }
+        kc = kc_u + nk;
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
         ++ucount;
@@ -367,40 +376,44 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         ok = mbar_wait_warp(&S.idx_full[ib], uph, abort_flag);
         if (!ok) break;
         const int32_t* idx = idx_sm + ib * kMaxIdx;
-        for (int j = U.j0; j < U.j1 && ok; ++j) {
-          for (int kh = 0; kh < 2 && ok; ++kh) {
-            for (int h = 0; h < VS::kNpv; ++h, ++vc) {
-              const uint32_t st = vc % kVStages, ph = (vc / kVStages) & 1u;
-              if (st != my_slot) continue;
-              if (p.dense && part != 0) continue;         // one issuing warp per slot (see the key loaders)
-              bool w_ok = true;
-              if (lane == 0) {
-                w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
-                if (w_ok && leader && part == 0) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
-              }
-              if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
-              const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
-              if (p.dense) {
-                // 64 contiguous keys x this CTA's value columns: one box per plane
-                if (part == 0 && lane < (uint32_t)VS::kPlanes) {
-                  const int col = h * VS::kN + (int)rank * (VS::kN / 2) + (int)lane * 64;
-                  tma_load_2d_pair(v_sm + st * VS::kStageBytes + lane * kPlane64, &tmap_kv_tile, full_l, col,
-                                   U.b * p.Lk + j * kTileKeys + kh * kHalfKeys);
-                }
-                continue;
-              }
-              const int g = part + kVWarpsPerSlot * (int)lane;
-              if (g < 16 * VS::kPlanes) {
-                const int pl = g / 16, kg = g % 16;
-                const int base = (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4;
-                const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
-                tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
-                                 gather_row(idx, base + 0), gather_row(idx, base + 1),
-                                 gather_row(idx, base + 2), gather_row(idx, base + 3));
-              }
+        // The unit's value stages are vc_u .. vc_u + nv - 1 (per tile: key half kh,
+        // then value block h); stage x goes to slot x % kVStages, and this warp visits
+        // only its own slot's stages.
+        constexpr uint32_t kPerTile = 2u * VS::kNpv;
+        const uint32_t vc_u = vc, nv = (uint32_t)(U.j1 - U.j0) * kPerTile;
+        for (uint32_t x = vc_u + (my_slot + kVStages - vc_u % kVStages) % kVStages; x < vc_u + nv && ok;
+             x += kVStages) {
+          const uint32_t st = my_slot, ph = (x / kVStages) & 1u;
+          const uint32_t rem = (x - vc_u) % kPerTile;
+          const int j = U.j0 + (int)((x - vc_u) / kPerTile), kh = (int)(rem / VS::kNpv), h = (int)(rem % VS::kNpv);
+          if (p.dense && part != 0) continue;         // one issuing warp per slot (see the key loaders)
+          bool w_ok = true;
+          if (lane == 0) {
+            w_ok = mbar_wait(&S.v_empty[st], ph ^ 1u, abort_flag);
+            if (w_ok && leader && part == 0) mbar_arrive_expect_tx(&S.v_full[st], 2u * VS::kStageBytes);
+          }
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+          const uint32_t full_l = mapa_shared(smem_u32(&S.v_full[st]), 0);
+          if (p.dense) {
+            // 64 contiguous keys x this CTA's value columns: one box per plane
+            if (part == 0 && lane < (uint32_t)VS::kPlanes) {
+              const int col = h * VS::kN + (int)rank * (VS::kN / 2) + (int)lane * 64;
+              tma_load_2d_pair(v_sm + st * VS::kStageBytes + lane * kPlane64, &tmap_kv_tile, full_l, col,
+                               U.b * p.Lk + j * kTileKeys + kh * kHalfKeys);
             }
+            continue;
+          }
+          const int g = part + kVWarpsPerSlot * (int)lane;
+          if (g < 16 * VS::kPlanes) {
+            const int pl = g / 16, kg = g % 16;
+            const int base = (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4;
+            const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
+            tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
+                             gather_row(idx, base + 0), gather_row(idx, base + 1),
+                             gather_row(idx, base + 2), gather_row(idx, base + 3));
           }
         }
+        vc = vc_u + nv;
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.idx_empty[ib]);
         ++ucount;
