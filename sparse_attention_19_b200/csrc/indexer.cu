@@ -158,6 +158,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   constexpr uint32_t kLayout = (D_I == 128) ? LAYOUT_SW128 : LAYOUT_SW64;
   constexpr uint32_t kAtomBytes = 8 * kRowBytes;       // 8-row swizzle atom
   constexpr int kKSteps = D_I / 32;                    // MMA K = 32 bytes of e4m3
+  // Units of one query sub-block: every fused launch, and the deep-ring launch,
+  // which serves decode-sized query blocks (the launcher checks p.nsub == 1).
+  constexpr bool kOneSubBlock = kFused || kStages == kMaxStages;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IndexerSmem& S = *reinterpret_cast<IndexerSmem*>(smem_raw);
@@ -563,7 +566,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       // ngroups-th tile: the warp visits only those, stepping the tile, accumulator
       // and scale-slot counters over the others instead of looping through them
       // (each skipped pass cost as much as a few hundred instructions of issue).
-      const bool stride = p.nsub == 1;
+      constexpr bool stride = kOneSubBlock;
       const uint32_t seq_u = seq, sc_u = sc_use;
       const int kt_first = stride ? U.kt0 + (int)((group - seq_u) & (ngroups - 1u)) : U.kt0;
       const int kt_step = stride ? (int)ngroups : 1;
@@ -808,6 +811,7 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
   // when N <= 64, else two of two); each staging slot must stay with one group (see
   // the staging ring), so n_stage is a multiple of the group count.
   const int ngroups = p.qb * p.H_I <= 64 ? kQuads : kQuads / 2;
+  if (fused && p.nsub != 1) return cudaErrorInvalidValue;   // fused units hold one sub-block
   if (fused && (p.rows_per_unit > kMaxRows || p.n_stage > kMaxStage || p.n_stage < 1 || p.cap < p.k + 128 ||
                 p.cap % 32 != 0 || p.n_stage % ngroups != 0))
     return cudaErrorInvalidValue;
@@ -815,6 +819,7 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
     if (fused)
       return deep ? launch_indexer_t<64, 128, 8, true>(p, tq, tk, ts, grid, stream)
                   : launch_indexer_t<64, 128, 4, true>(p, tq, tk, ts, grid, stream);
+    if (deep && p.nsub != 1) return cudaErrorInvalidValue;   // the deep-ring build visits tiles by group
     return deep ? launch_indexer_t<64, 128, 12, false>(p, tq, tk, ts, grid, stream)
                 : launch_indexer_t<64, 128, 4, false>(p, tq, tk, ts, grid, stream);
   }
