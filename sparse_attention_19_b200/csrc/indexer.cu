@@ -147,7 +147,7 @@ __device__ __forceinline__ UnitInfo decode_unit(const IndexerParams& p, int u) {
   return info;
 }
 
-template <int H_I, int D_I, int kStages, bool kFused>
+template <int H_I, int D_I, int kStages, bool kFused, int kQB, int kNSub>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                const __grid_constant__ CUtensorMap tmap_s, const IndexerParams p) {
@@ -159,14 +159,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   constexpr uint32_t kAtomBytes = 8 * kRowBytes;       // 8-row swizzle atom
   constexpr int kKSteps = D_I / 32;                    // MMA K = 32 bytes of e4m3
   // Units of one query sub-block: every fused launch, and the deep-ring launch,
-  // which serves decode-sized query blocks (the launcher checks p.nsub == 1).
+  // which serves decode-sized query blocks (the launcher checks nsub == 1).
   constexpr bool kOneSubBlock = kFused || kStages == kMaxStages;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IndexerSmem& S = *reinterpret_cast<IndexerSmem*>(smem_raw);
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* tiles = smem_raw + (((raw_addr + (uint32_t)sizeof(IndexerSmem) + 1023u) & ~1023u) - raw_addr);
-  const int N = p.qb * H_I;                            // MMA N (queries x heads)
+  // Query-block shape: compile-time in the builds specialised for the common
+  // prefill and decode shapes (kQB, kNSub > 0), else the launch's values.
+  const int qb = kQB > 0 ? kQB : p.qb;
+  const int nsub = kNSub > 0 ? kNSub : p.nsub;
+  const int N = qb * H_I;                              // MMA N (queries x heads)
   const uint32_t nslot = min(8, kTmemCols / N);        // accumulators in flight (more when N is small)
   // Epilogue quads work on accumulators in groups of `span`: the groups take
   // accumulators in turn (group g gets seq = g mod ngroups), and within a group quad
@@ -178,7 +182,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   const uint32_t ngroups = (uint32_t)(kQuads / span);
   const int warps_per_acc = 4 * span;
   const int QU = p.queries_per_unit;                   // = qb * nsub
-  const uint32_t q_bytes = (uint32_t)(p.nsub * N) * kRowBytes;   // one query block
+  const uint32_t q_bytes = (uint32_t)(nsub * N) * kRowBytes;   // one query block
   const uint32_t n_qbuf = query_buffers(q_bytes);
   uint8_t* q_smem = tiles;                             // n_qbuf x (nsub * N rows)
   uint8_t* k_smem = tiles + n_qbuf * (size_t)q_bytes;
@@ -186,7 +190,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   float* w_smem = sc_smem + (p.scale_ring ? kScaleSlots * kKeysPerTile : 0);   // 2 x QU * H_I (double-buffered)
   float* sq_smem = w_smem + 2 * QU * H_I;                  // 2 x QU
   // fused mode: staging ring, per-row thresholds, selector state and candidate lists
-  const FusedLayout FL = fused_layout((uint32_t)(reinterpret_cast<uint8_t*>(sq_smem + 2 * QU) - tiles), p.qb,
+  const FusedLayout FL = fused_layout((uint32_t)(reinterpret_cast<uint8_t*>(sq_smem + 2 * QU) - tiles), qb,
                                       p.n_stage, p.rows_per_unit, p.cap);
   uint32_t* stg_key = reinterpret_cast<uint32_t*>(tiles + FL.stg_key);
   uint32_t* stg_pos = reinterpret_cast<uint32_t*>(tiles + FL.stg_pos);
@@ -216,7 +220,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
     }
     // A tile's key scales are read by the warps of the groups that process one of
     // its sub-blocks' accumulators (consecutive accumulators go to consecutive groups).
-    const int sc_readers = warps_per_acc * min(p.nsub, (int)ngroups);
+    const int sc_readers = warps_per_acc * min(nsub, (int)ngroups);
     for (int s = 0; s < kScaleSlots; ++s) {
       mbar_init(&S.sc_full[s], 1);
       mbar_init(&S.sc_empty[s], sc_readers);
@@ -262,8 +266,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           const uint32_t qb_i = ucount % n_qbuf;
           if (!mbar_wait(&S.q_empty[qb_i], ((ucount / n_qbuf) & 1u) ^ 1u, abort_flag)) break;
           mbar_arrive_expect_tx(&S.q_full[qb_i], q_bytes);
-          for (int sb = 0; sb < p.nsub; ++sb) {
-            const int row = ((U.b * p.Lq) + U.i0 + sb * p.qb) * H_I;
+          for (int sb = 0; sb < nsub; ++sb) {
+            const int row = ((U.b * p.Lq) + U.i0 + sb * qb) * H_I;
             tma_load_2d(q_smem + qb_i * q_bytes + (size_t)sb * N * kRowBytes, &tmap_q, &S.q_full[qb_i], 0, row);
           }
         }
@@ -305,7 +309,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           if (!mbar_wait(&S.k_full[kstage], kphase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = k_base + kstage * kKeysPerTile * kRowBytes;
-          for (int sb = 0; sb < p.nsub; ++sb) {
+          for (int sb = 0; sb < nsub; ++sb) {
             if (!mbar_wait(&S.acc_empty[slot], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + slot * (uint32_t)N;
@@ -412,21 +416,21 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
       __syncwarp();
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt1 && ok; ++kt) {
-        for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
+        for (int sb = 0; sb < nsub; ++sb, ++seq) {
           const uint32_t gs = seq % (uint32_t)p.n_stage;
           if (!mbar_wait_warp(&S.stg_full[gs], (seq / (uint32_t)p.n_stage) & 1u, abort_flag)) { ok = false; break; }
-          for (int qi = 0; qi < p.qb; ++qi) {
-            const int r = sb * p.qb + qi;
+          for (int qi = 0; qi < qb; ++qi) {
+            const int r = sb * qb + qi;
             if (r % kSelWarps != me || U.i0 + r >= p.Lq) continue;
-            const uint32_t* cnt = stg_cnt + (gs * p.qb + qi) * 4;
+            const uint32_t* cnt = stg_cnt + (gs * qb + qi) * 4;
             const uint32_t c0 = cnt[0], c1 = cnt[1], c2 = cnt[2], c3 = cnt[3];
             if (row_n[r] + c0 + c1 + c2 + c3 > (uint32_t)p.cap) cut(r, ucount);
             uint32_t* xk = lkey + (size_t)r * p.cap;
             uint32_t* xp = lpos + (size_t)r * p.cap;
             uint32_t n = row_n[r];
             const uint32_t th = row_thr[r];
-            const uint32_t* sk = stg_key + (gs * p.qb + qi) * 128;
-            const uint32_t* sp = stg_pos + (gs * p.qb + qi) * 128;
+            const uint32_t* sk = stg_key + (gs * qb + qi) * 128;
+            const uint32_t* sp = stg_pos + (gs * qb + qi) * 128;
             uint32_t mn = 0xffffffffu, mx = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -584,7 +588,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
         // This warp reads the tile only if its group owns one of the tile's
         // accumulators (seq .. seq + nsub - 1).
         bool reads_tile = false;
-        for (int sb = 0; sb < p.nsub; ++sb) reads_tile |= ((seq + (uint32_t)sb) & (ngroups - 1u)) == group;
+        for (int sb = 0; sb < nsub; ++sb) reads_tile |= ((seq + (uint32_t)sb) & (ngroups - 1u)) == group;
         if (p.scale_ring) {
           if (reads_tile) {
             if (!mbar_wait_warp(&S.sc_full[ss], (sc_use / kScaleSlots) & 1u, abort_flag)) { ok = false; break; }
@@ -594,7 +598,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           sk = sk_next;
           sk_next = key_scale(kt + kt_step);
         }
-        for (int sb = 0; sb < p.nsub; ++sb, ++seq) {
+        for (int sb = 0; sb < nsub; ++sb, ++seq) {
           const uint32_t slot = acc_slot, use = acc_use;
           if (++acc_slot == nslot) { acc_slot = 0; ++acc_use; }
           if ((seq & (ngroups - 1u)) != group) continue;
@@ -614,7 +618,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
           // the causal mask.  Scores mode stores it; fused mode stages it (warp-wide
           // call) if it beats the row's current threshold.
           auto finish = [&](int qi, float acc) {
-            const int qq = sb * p.qb + qi;
+            const int qq = sb * qb + qi;
             const int i = U.i0 + qq;
             if constexpr (kFused) {
               const bool valid = i < p.Lq && s < p.Lk && s <= p.q_offset + i;
@@ -623,13 +627,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
               const uint32_t th = (uint32_t)(tv >> 32) == ucount ? (uint32_t)tv : 0u;
               const bool pass = valid && key > th;
               const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-              const uint32_t base = (gs * (uint32_t)p.qb + (uint32_t)qi) * 128u + quarter * 32u;
+              const uint32_t base = (gs * (uint32_t)qb + (uint32_t)qi) * 128u + quarter * 32u;
               if (pass) {
                 const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
                 stg_key[at] = key;
                 stg_pos[at] = (uint32_t)s;
               }
-              if (lane == 0) stg_cnt[(gs * (uint32_t)p.qb + (uint32_t)qi) * 4u + quarter] = __popc(bal);
+              if (lane == 0) stg_cnt[(gs * (uint32_t)qb + (uint32_t)qi) * 4u + quarter] = __popc(bal);
             } else if (i < p.Lq && s < p.Lk) {
               const int t = p.q_offset + i;
               float* dst = p.scores + ((size_t)U.b * p.Lq + i) * (size_t)p.Lk + s;
@@ -666,8 +670,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             // accumulator goes back to the MMA issuer once the last load is in.
             if (g_first + g_step < N) {
               const int qa = g_first / 64, qb2 = (g_first + g_step) / 64;   // queries within the sub-block
-              const float4* wa = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qa) * H_I);
-              const float4* wb = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qb2) * H_I);
+              const float4* wa = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * qb + qa) * H_I);
+              const float4* wb = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * qb + qb2) * H_I);
               float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
@@ -686,7 +690,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
             } else
             for (int g0 = g_first; g0 < N; g0 += g_step) {
               const int qi = g0 / 64;                            // query within the sub-block
-              const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
+              const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * qb + qi) * H_I);
               uint32_t v[32];
               tmem_ld32(t_base + (uint32_t)g0, v);
               tmem_ld_wait();
@@ -713,7 +717,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
 #pragma unroll
                 for (int a = 0; a < QPL; ++a) {
                   const int qi = (g0 + part * 32) / H_I + a;
-                  const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * p.qb + qi) * H_I);
+                  const float4* wq = reinterpret_cast<const float4*>(wbuf + (size_t)(sb * qb + qi) * H_I);
                   const float2 acc2 = relu_dot(v + a * H_I, wq, H_I, make_float2(0.f, 0.f));
                   finish(qi, acc2.x + acc2.y);
                 }
@@ -766,13 +770,14 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   }
 }
 
-template <int H_I, int D_I, int kStages, bool kFused>
+template <int H_I, int D_I, int kStages, bool kFused, int kQB = 0, int kNSub = 0>
 cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& ts, int grid, cudaStream_t stream) {
+  if ((kQB > 0 && p.qb != kQB) || (kNSub > 0 && p.nsub != kNSub)) return cudaErrorInvalidValue;
   const size_t smem = indexer_smem_bytes(p.nsub * p.qb * H_I, D_I, p.queries_per_unit * H_I, p.queries_per_unit,
                                          kStages, p.scale_ring != 0, kFused, p.qb, p.n_stage, p.rows_per_unit,
                                          p.cap);
-  auto kern = indexer_kernel<H_I, D_I, kStages, kFused>;
+  auto kern = indexer_kernel<H_I, D_I, kStages, kFused, kQB, kNSub>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // The register split must fit in what the CTA launches with, or the increase
@@ -820,6 +825,10 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
       return deep ? launch_indexer_t<64, 128, 8, true>(p, tq, tk, ts, grid, stream)
                   : launch_indexer_t<64, 128, 4, true>(p, tq, tk, ts, grid, stream);
     if (deep && p.nsub != 1) return cudaErrorInvalidValue;   // the deep-ring build visits tiles by group
+    // Builds specialised for the prefill block (4 queries x 2 sub-blocks) and the
+    // decode block (one query).
+    if (!deep && p.qb == 4 && p.nsub == 2) return launch_indexer_t<64, 128, 4, false, 4, 2>(p, tq, tk, ts, grid, stream);
+    if (deep && p.qb == 1) return launch_indexer_t<64, 128, 12, false, 1, 1>(p, tq, tk, ts, grid, stream);
     return deep ? launch_indexer_t<64, 128, 12, false>(p, tq, tk, ts, grid, stream)
                 : launch_indexer_t<64, 128, 4, false>(p, tq, tk, ts, grid, stream);
   }
