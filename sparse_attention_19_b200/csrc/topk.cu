@@ -233,8 +233,27 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
       for (int x = threadIdx.x; x < ns; x += kThreads) atomicAdd(&sh.hist[bin_of(cand[x].x)], 1u);
       __syncthreads();
       find_bin(sh.hist, sh.x, j);
-      const uint32_t tb = sh.x.bin;
-      const uint32_t theta = tb == 0 ? 0u : lo + (tb << shift);
+      // The first histogram's bins are coarse when the sample spans both signs (its
+      // key range then covers half the key space), and the lower edge of the bin
+      // alone can let through more keys than the buffer holds; a second histogram
+      // of the sample keys inside that bin places theta just below the sample's
+      // j-th largest key.  (Any theta is safe: the count check below decides.)
+      uint32_t theta;
+      {
+        const uint32_t tb = sh.x.bin, need2 = j - sh.x.above;
+        const uint32_t wlo = lo + (tb << shift);
+        const unsigned long long top = (unsigned long long)wlo + (1ull << shift) - 1ull;
+        const uint32_t whi = (tb == (uint32_t)(kBins - 1) || top > smax) ? smax : (uint32_t)top;
+        const int sh2 = bin_shift(whi - wlo);
+        clear_hist(sh.hist);
+        for (int x = threadIdx.x; x < ns; x += kThreads) {
+          const uint32_t key = cand[x].x;
+          if (key >= wlo && key <= whi) atomicAdd(&sh.hist[(key - wlo) >> sh2], 1u);
+        }
+        __syncthreads();
+        find_bin(sh.hist, sh.x, need2);
+        theta = wlo + (sh.x.bin << sh2);
+      }
       const int W = (n + 31) >> 5;
       for (int x = threadIdx.x; x < W; x += kThreads) { gt_bits[x] = 0u; eq_bits[x] = 0u; }
       if (threadIdx.x == 0) sh.x.ncand = 0u;
