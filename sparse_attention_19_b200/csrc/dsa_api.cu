@@ -296,6 +296,7 @@ dsa_status run_topk(const float* scores, int B, int Lq, int Lk, int q_offset, in
     p.cluster = 1;
     p.cache_cap = 0;
     p.bit_words = (int)round_up((size_t)(seg / 32), 4);
+    p.sampled = 1;            // one pass with a sampled threshold first (see the cluster kernel)
   }
   p.vec4 = (aligned16(scores) && Lk % 4 == 0) ? 1 : 0;
   // Many rows of moderate length (prefill up to 32K): one warp per row, rows

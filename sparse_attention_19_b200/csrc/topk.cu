@@ -537,11 +537,14 @@ topk_cluster_kernel(const TopkParams p) {
   // row passes over this CTA's segment: positions s0 + (0 .. s1 - s0)
   auto seg_key = [&](int s) -> uint32_t { return load_key(s0 + s); };
 
-  // ---- 1. sampled key range (the same in every CTA)
+  // ---- 1. sampled key range (the same in every CTA; kept in the candidate buffer
+  // for step 1b)
   const int ns = n < kSample ? n : kSample;
+  const bool try_single = p.sampled && p.cand_cap >= kSample;
   uint32_t smin = 0xffffffffu, smax = 0u;
   for (int j = threadIdx.x; j < ns; j += kThreads) {
     const uint32_t key = load_key((int)(((long long)j * n) / ns));
+    if (try_single) cand[j].x = key;
     smin = min(smin, key);
     smax = max(smax, key);
   }
@@ -552,6 +555,68 @@ topk_cluster_kernel(const TopkParams p) {
     return key < lo ? 0u : min((uint32_t)(kBins - 1), (key - lo) >> shift);
   };
 
+  // ---- 1b. one pass, as in the one-CTA kernel: every key of the segment at or
+  // above theta (just below the sample's j-th largest key, the same in every CTA)
+  // is kept with its position.  The cluster takes this route when at least k keys
+  // pass over the whole row and every segment's share fits its buffer; the
+  // decision is taken from cluster-wide counts, so every CTA reaches the same
+  // barriers.  Otherwise the two passes below.
+  bool single = false;
+  if (try_single) {
+    const float mu = (float)ns * (float)k / (float)n;
+    const float sig = sqrtf(mu * (1.f - (float)k / (float)n));
+    const uint32_t j = (uint32_t)ceilf(mu + 6.f * sig + 2.f);
+    if (j < (uint32_t)ns) {
+      clear_hist(sh.hist);
+      for (int x = threadIdx.x; x < ns; x += kThreads) atomicAdd(&sh.hist[bin_of(cand[x].x)], 1u);
+      __syncthreads();
+      find_bin(sh.hist, sh.x, j);
+      uint32_t theta;
+      {
+        const uint32_t tb = sh.x.bin, need2 = j - sh.x.above;
+        const uint32_t wlo = lo + (tb << shift);
+        const unsigned long long top = (unsigned long long)wlo + (1ull << shift) - 1ull;
+        const uint32_t whi = (tb == (uint32_t)(kBins - 1) || top > smax) ? smax : (uint32_t)top;
+        const int sh2 = bin_shift(whi - wlo);
+        clear_hist(sh.hist);
+        for (int x = threadIdx.x; x < ns; x += kThreads) {
+          const uint32_t key = cand[x].x;
+          if (key >= wlo && key <= whi) atomicAdd(&sh.hist[(key - wlo) >> sh2], 1u);
+        }
+        __syncthreads();
+        find_bin(sh.hist, sh.x, need2);
+        theta = wlo + (sh.x.bin << sh2);
+      }
+      const int W = (s1 - s0 + 31) >> 5;
+      for (int x = threadIdx.x; x < W; x += kThreads) { gt_bits[x] = 0u; eq_bits[x] = 0u; }
+      if (threadIdx.x == 0) sh.x.ncand = 0u;
+      __syncthreads();
+      row_pass(s1 - s0, seg_key, [&](int s, bool valid, uint32_t key) {
+        if (valid && key >= theta) {
+          const uint32_t at = atomicAdd(&sh.x.ncand, 1u);
+          if (at < (uint32_t)p.cand_cap) cand[at] = make_uint2(key, (uint32_t)s);
+        }
+      });
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        sh.pub_a = sh.x.ncand;
+        sh.pub_b = sh.x.ncand > (uint32_t)p.cand_cap ? 1u : 0u;
+      }
+      cluster_sync();
+      uint32_t total = 0, over = 0;
+#pragma unroll
+      for (int c = 0; c < kClusterCtas; ++c) {
+        total += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c));
+        over |= ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_b), c));
+      }
+      cluster_sync();                               // pub_a / pub_b are not rewritten before all have read them
+      single = over == 0u && total >= (uint32_t)k;
+    }
+  }
+
+  uint32_t need = (uint32_t)k;
+  uint32_t b = 0, cnt_b = 0;
+  if (!single) {
   // ---- 2. segment histogram, summed over the cluster
   clear_hist(sh.hist);
   row_pass(s1 - s0, seg_key, [&](int, bool valid, uint32_t key) {
@@ -559,11 +624,10 @@ topk_cluster_kernel(const TopkParams p) {
   });
   __syncthreads();
   cluster_sum_hist(sh);
-  uint32_t need = (uint32_t)k;
   find_bin(sh.tot, sh.x, need);
-  const uint32_t b = sh.x.bin;
+  b = sh.x.bin;
   need -= sh.x.above;
-  const uint32_t cnt_b = sh.tot[b];
+  cnt_b = sh.tot[b];
 
   // ---- 3. this segment's bins above b into the bitmap; its bin-b elements as candidates
   if (threadIdx.x == 0) sh.x.ncand = 0u;
@@ -578,7 +642,10 @@ topk_cluster_kernel(const TopkParams p) {
     }
   });
   __syncthreads();
-  const bool fits = cnt_b <= (uint32_t)p.cand_cap;  // then every CTA's share fits as well
+  }   // two-pass route
+  // After one pass every CTA's share fits its buffer; after two, the bin's whole
+  // count must fit (then every CTA's share fits as well).
+  const bool fits = single || cnt_b <= (uint32_t)p.cand_cap;
   const int own = (int)sh.x.ncand;
 
   // Exact threshold, refined over the window [wlo, whi] with cluster-summed histograms

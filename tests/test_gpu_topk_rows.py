@@ -117,3 +117,19 @@ def test_long_rows_fall_back_when_too_many_keys_pass():
     s[:, :, ::2] = 1.5
     s[1, :, 1::3] = -0.0
     _check(s.to(DEV), 36000 - 100, 2048)
+
+
+# Few long rows (decode): each row spread over a cluster of CTAs, one pass over the
+# row first (keys at or above a sampled threshold, per CTA segment), the two-pass
+# route when the keys that pass are fewer than k over the row or overflow any
+# segment's buffer.
+
+def test_cluster_rows_one_pass_and_segment_overflow():
+    g = torch.Generator().manual_seed(41)
+    Lk = 131072
+    s = torch.randn(1, 4, Lk, generator=g)
+    s[0, 1, 1000:5500] = 5.0                         # one segment holds more than its buffer
+    s[0, 2, ::87] = 4.0                              # 1507 planted ties, spread over all segments
+    s[0, 2] = torch.where(s[0, 2] == 4.0, s[0, 2], torch.round(s[0, 2] * 8) / 8)
+    s[0, 3] = 0.5                                    # every key passes: the two-pass route
+    _check(s.to(DEV), Lk - 4, 2048)
