@@ -246,6 +246,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
+  griddep_launch_dependents();
+  griddep_wait();                                      // the previous kernel's writes are visible
 
   if (warp >= (uint32_t)kEpiWarps) {
   if (warp >= kLoaderWarp0) {
@@ -786,8 +788,7 @@ cudaError_t launch_indexer_t(const IndexerParams& p, const CUtensorMap& tq, cons
   e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
   if ((uint32_t)fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
-  kern<<<grid, kThreads, smem, stream>>>(tq, tk, ts, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, tq, tk, ts, p);
 }
 
 }  // namespace

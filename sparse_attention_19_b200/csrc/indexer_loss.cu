@@ -186,6 +186,8 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
   const uint16_t kBoth = 0x3;
+  griddep_launch_dependents();
+  griddep_wait();                                      // the previous kernel's writes are visible
   bool ok = true;
 
   if (warp >= kLoadWarp0) {
@@ -536,8 +538,7 @@ cudaError_t launch_t(const KlParams& p, const CUtensorMap& tq, const CUtensorMap
   auto kern = indexer_kl_kernel<NC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid_clusters * 2, kThreads, smem, stream>>>(tq, tkv, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid_clusters * 2), dim3(kThreads), smem, stream, tq, tkv, p);
 }
 
 }  // namespace

@@ -247,6 +247,19 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream serialization,
+// so it may be scheduled while the kernel before it in the stream is finishing.
+// griddep_wait() returns once that kernel has completed and its memory operations
+// are visible; each kernel calls it before its first global-memory access (its
+// prologue -- barriers, TMEM, tensor-map prefetch -- may run earlier).
+// griddep_launch_dependents() lets the next kernel's CTAs be scheduled once every
+// CTA of this grid has called it, i.e. once all of them are resident.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");

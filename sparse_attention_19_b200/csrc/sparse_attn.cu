@@ -218,6 +218,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
   const uint16_t kBoth = 0x3;
+  griddep_launch_dependents();
+  griddep_wait();                                      // the previous kernel's writes are visible
 
   if (warp >= 4) {
     regs_decrease<kRegsOther>();
@@ -697,6 +699,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
 // Merge split-k partials: lse = log sum_i exp(lse_i); out = sum_i exp(lse_i - lse) o_i.
 template <int DV>
 __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
+  griddep_launch_dependents();
+  griddep_wait();                                      // the partials are complete
   const int warps = blockDim.x / 32;
   const int gw = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -740,8 +744,7 @@ cudaError_t launch_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorM
   e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
   if ((uint32_t)fa.numRegs < kRegsLaunch) return cudaErrorInvalidConfiguration;
-  kern<<<grid_clusters * 2, kThreads, smem, stream>>>(tq, tkv, tkv_tile, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid_clusters * 2), dim3(kThreads), smem, stream, tq, tkv, tkv_tile, p);
 }
 
 }  // namespace
@@ -770,10 +773,9 @@ cudaError_t launch_sparse_attn(const AttnParams& p, int d_qk, int d_v, const CUt
 cudaError_t launch_attn_combine(const AttnParams& p, int d_v, cudaStream_t stream) {
   const int n = p.B * p.Lq * p.H;
   const int grid = (n + 3) / 4;
-  if (d_v == 512) attn_combine_kernel<512><<<grid, 128, 0, stream>>>(p);
-  else if (d_v == 128) attn_combine_kernel<128><<<grid, 128, 0, stream>>>(p);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (d_v == 512) return launch_pdl(attn_combine_kernel<512>, dim3(grid), dim3(128), 0, stream, p);
+  if (d_v == 128) return launch_pdl(attn_combine_kernel<128>, dim3(grid), dim3(128), 0, stream, p);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t read_attn_error(uint32_t* value, bool clear) { return read_unit_error(value, clear); }

@@ -169,6 +169,8 @@ __device__ __forceinline__ void row_pass(int n, KeyAt key_at, F f) {
 }
 
 __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
+  griddep_launch_dependents();
+  griddep_wait();                                   // the scores are complete
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
   uint32_t* cache = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
@@ -506,6 +508,8 @@ __device__ void cluster_sum_hist(TopkClusterShared& sh) {
 
 __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kThreads, 2)
 topk_cluster_kernel(const TopkParams p) {
+  griddep_launch_dependents();
+  griddep_wait();                                   // the scores are complete
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkClusterShared& sh = *reinterpret_cast<TopkClusterShared*>(smem_raw);
   uint32_t* gt_bits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkClusterShared));   // segment words
@@ -843,6 +847,8 @@ __device__ __forceinline__ void visit_row_keys(const float* src, int n, bool vec
 }
 
 __global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(const TopkParams p) {
+  griddep_launch_dependents();
+  griddep_wait();                                   // the scores are complete
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int lane = (int)(threadIdx.x & 31u), warp = (int)(threadIdx.x >> 5);
   WarpTopkSmem& sh = reinterpret_cast<WarpTopkSmem*>(smem_raw)[warp];
@@ -1018,22 +1024,20 @@ cudaError_t launch_topk(const TopkParams& p, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(topk_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)wsmem);
     if (e != cudaSuccess) return e;
     if (rows == 0) return cudaSuccess;
-    topk_warp_kernel<<<(rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta, 32 * kWarpRowsPerCta, wsmem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(topk_warp_kernel, dim3((rows + kWarpRowsPerCta - 1) / kWarpRowsPerCta),
+                      dim3(32 * kWarpRowsPerCta), wsmem, stream, p);
   }
   const size_t smem = topk_smem_bytes(p.cache_cap, p.bit_words, p.cand_cap, p.cluster != 0);
   if (p.cluster) {
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (rows == 0) return cudaSuccess;
-    topk_cluster_kernel<<<rows * kClusterCtas, kThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(topk_cluster_kernel, dim3(rows * kClusterCtas), dim3(kThreads), smem, stream, p);
   }
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (rows == 0) return cudaSuccess;
-  topk_kernel<<<rows, kThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(rows), dim3(kThreads), smem, stream, p);
 }
 
 cudaError_t read_topk_error(uint32_t* value, bool clear) { return read_unit_error(value, clear); }
