@@ -99,9 +99,11 @@ struct KlShared {
   float fin[kLossWarps][5];              // leader: per loss warp (Z, A, Bs, m, s) of the row
 };
 
-// Row of kv (in the [B*Lk, d_qk] view) staged for a slot; bit 31 marks padding,
-// which gathers row b*Lk (a valid row) and is masked.
-__device__ __forceinline__ int gather_row(const int32_t* rows, int pos) { return rows[pos] & 0x7fffffff; }
+// Rows of kv (in the [B*Lk, d_qk] view) staged for four consecutive slots; padding
+// was staged as row b*Lk (a valid row) and is masked through valid_mask.
+__device__ __forceinline__ int4 gather_rows4(const int32_t* rows, int pos) {
+  return *reinterpret_cast<const int4*>(rows + pos);   // four consecutive slots, pos a multiple of 4
+}
 
 // Tiles of the staged row in buffer `buf`: up to the last one that holds a valid
 // position (top-k output is valid-first, so this skips its all-padding tail).
@@ -237,10 +239,9 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
           if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
           const int g = part + kTeamWarps * (int)lane;             // 4-key group of this lane
           if (g < kHalfKeys / 4) {
-            const int base = j * kTileKeys + (int)rank * kHalfKeys + g * 4;
+            const int4 r4 = gather_rows4(idx, j * kTileKeys + (int)rank * kHalfKeys + g * 4);
             tma_gather4_pair(k_sm + st * kPlane + g * 512, &tmap_kv, mapa_shared(smem_u32(&S.k_full[st]), 0),
-                             c * 64, gather_row(idx, base + 0), gather_row(idx, base + 1),
-                             gather_row(idx, base + 2), gather_row(idx, base + 3));
+                             c * 64, r4.x, r4.y, r4.z, r4.w);
           }
         }
       }
@@ -250,9 +251,9 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
     }
   } else if (warp >= kStageWarp0 && warp < kStageWarp0 + kStageWarps) {
     // ------------------------------------------------------------------ index staging
-    // Row ordinal n goes to buffer n % 2 as kv rows to gather (batch offset applied,
-    // bit 31 on padding and out-of-range entries) plus one validity ballot per 32
-    // slots.  Slots past k are padding.  Both CTAs stage the whole row.
+    // Row ordinal n goes to buffer n % 2 as kv rows to gather (batch offset applied;
+    // padding and out-of-range entries gather row b*Lk) plus one validity ballot
+    // per 32 slots.  Slots past k are padding.  Both CTAs stage the whole row.
     const int sw = (int)warp - kStageWarp0;
     const int nwords = p.n_tiles * (kTileKeys / 32);
     uint32_t ucount = 0;
@@ -277,7 +278,7 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
           if (w >= nwords) break;                     // warp-uniform
           const bool valid = sidx[e] >= 0 && sidx[e] < p.Lk;
           const int grow = b * p.Lk + (valid ? sidx[e] : 0);
-          dst[w * 32 + (int)lane] = valid ? grow : (int)((uint32_t)grow | 0x80000000u);
+          dst[w * 32 + (int)lane] = grow;              // validity: the ballot below
           const uint32_t bal = __ballot_sync(0xffffffffu, valid);
           if (lane == 0) S.valid_mask[buf][w] = bal;
           if (bal) last = w;                          // words are visited in increasing order
@@ -429,13 +430,12 @@ indexer_kl_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_const
       auto fetch = [&](int j) -> float {
         if (j >= nt) return 0.f;
         const int slot = j * kTileKeys + key;
-        const int32_t gr = idx[slot];
-        if (gr < 0) return 0.f;
-        return selrow ? __ldg(selrow + slot) : __ldg(srow + (gr - bLk));
+        if (!((S.valid_mask[ib][slot >> 5] >> (slot & 31)) & 1u)) return 0.f;
+        return selrow ? __ldg(selrow + slot) : __ldg(srow + (idx[slot] - bLk));
       };
       auto consume = [&](int j, float iv) -> bool {
         const int slot_x = j * kTileKeys + key;
-        const bool kvalid = idx[slot_x] >= 0;
+        const bool kvalid = (S.valid_mask[ib][slot_x >> 5] >> (slot_x & 31)) & 1u;
         const uint32_t slot = sc % kRedSlots, rph = (sc / kRedSlots) & 1u;
         ++sc;
         if (!mbar_wait_warp(&S.red_full[slot], rph, abort_flag, true)) return false;

@@ -153,10 +153,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Row of kv (in the [B*Lk, d_qk] view) for a staged position; padding and
-// out-of-range entries were staged as row b*Lk (a valid row), masked in the softmax.
-__device__ __forceinline__ int gather_row(const int32_t* rows, int pos) {
-  return rows[pos] & 0x7fffffff;
+// Rows of kv (in the [B*Lk, d_qk] view) of four consecutive staged positions
+// (pos a multiple of 4), one 16-byte shared-memory load; padding and out-of-range
+// entries were staged as row b*Lk (a valid row), masked in the softmax.
+__device__ __forceinline__ int4 gather_rows4(const int32_t* rows, int pos) {
+  return *reinterpret_cast<const int4*>(rows + pos);
 }
 
 template <int NC, int DV>
@@ -290,10 +291,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           }
           const int g = part + kKTeamWarps * (int)lane;            // 4-key group of this lane
           if (g < kHalfKeys / 4) {
-            const int base = (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4;
-            tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64,
-                             gather_row(idx, base + 0), gather_row(idx, base + 1),
-                             gather_row(idx, base + 2), gather_row(idx, base + 3));
+            const int4 r4 = gather_rows4(idx, (j - U.j0) * kTileKeys + (int)rank * kHalfKeys + g * 4);
+            tma_gather4_pair(k_sm + st * kPlane64 + g * 512, &tmap_kv, full_l, c * 64, r4.x, r4.y, r4.z, r4.w);
           }
         }
         kc = kc_u + nk;
@@ -305,9 +304,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       // ------------------------------------------------------------------ value loaders
       // Index staging: the value loaders also stage each unit's selected positions
       // [j0*128, j1*128) into buffer (unit ordinal % 2), one unit ahead, as the kv
-      // row to gather -- batch offset applied, bit 31 set for padding and
-      // out-of-range entries, which gather row b*Lk and are masked -- plus one
-      // validity ballot per 32 positions for the softmax.  Warp pw stages the
+      // row to gather -- batch offset applied; padding and out-of-range entries
+      // gather row b*Lk and are masked -- plus one validity ballot per 32
+      // positions for the softmax.  Warp pw stages the
       // 32-position words pw, pw + kVWarps, ...  A buffer is free again once the
       // loaders and the softmax warps are done with the unit two back.
       // Value stages: per tile, 2 x kNpv stages of 64 keys (kh) x this CTA's kN/2
@@ -354,8 +353,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
             const int w = w0 + e * kVWarps;
             if (w >= nwords) break;                       // warp-uniform
             const bool valid = (sidx[e] >= 0) && (sidx[e] < p.Lk);
-            const int row = V.b * p.Lk + (valid ? sidx[e] : 0);
-            dst[w * 32 + (int)lane] = valid ? row : (int)((uint32_t)row | 0x80000000u);
+            dst[w * 32 + (int)lane] = V.b * p.Lk + (valid ? sidx[e] : 0);   // validity: the ballot below
             const uint32_t bal = __ballot_sync(0xffffffffu, valid);
             if (lane == 0) vmask[w] = bal;
           }
@@ -408,11 +406,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           const int g = part + kVWarpsPerSlot * (int)lane;
           if (g < 16 * VS::kPlanes) {
             const int pl = g / 16, kg = g % 16;
-            const int base = (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4;
+            const int4 r4 = gather_rows4(idx, (j - U.j0) * kTileKeys + kh * kHalfKeys + kg * 4);
             const int col = h * VS::kN + (int)rank * (VS::kN / 2) + pl * 64;
             tma_gather4_pair(v_sm + st * VS::kStageBytes + pl * kPlane64 + kg * 512, &tmap_kv, full_l, col,
-                             gather_row(idx, base + 0), gather_row(idx, base + 1),
-                             gather_row(idx, base + 2), gather_row(idx, base + 3));
+                             r4.x, r4.y, r4.z, r4.w);
           }
         }
         vc = vc_u + nv;
