@@ -834,6 +834,8 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
     // decode block (one query).
     if (!deep && p.qb == 4 && p.nsub == 2) return launch_indexer_t<64, 128, 4, false, 4, 2>(p, tq, tk, ts, grid, stream);
     if (deep && p.qb == 1) return launch_indexer_t<64, 128, 12, false, 1, 1>(p, tq, tk, ts, grid, stream);
+    // Two queries per block: two 16 KB query buffers leave room for 8 key stages, not 12.
+    if (deep && p.qb == 2) return launch_indexer_t<64, 128, 8, false>(p, tq, tk, ts, grid, stream);
     return deep ? launch_indexer_t<64, 128, 12, false>(p, tq, tk, ts, grid, stream)
                 : launch_indexer_t<64, 128, 4, false>(p, tq, tk, ts, grid, stream);
   }

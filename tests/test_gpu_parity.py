@@ -77,6 +77,17 @@ def test_indexer_decode_batches_split_keys():
     P.check_scores(gpu, ora, r["row_t"])
 
 
+@pytest.mark.parametrize("Lq", [2, 3, 4])
+def test_indexer_few_query_blocks_generic_builds(Lq):
+    # 2-4 new tokens per sequence (speculative or multi-token decode): query blocks
+    # the specialised prefill (4 x 2) and decode (1 x 1) builds do not take -- the
+    # deep-ring build with two queries per block, and the generic prefill build with
+    # one sub-block of three or four queries.
+    wl = WORKLOADS["decode_128k"].with_(B=2, Lq=Lq, Lk=5003, q_offset=5003 - Lq)
+    gpu, ora, r = _indexer_case(wl, 40 + Lq)
+    P.check_scores(gpu, ora, r["row_t"])
+
+
 # ------------------------------------------------------------------ top-k
 
 def _topk_case(scores_f32, q_offset, k, exact=True):
@@ -328,6 +339,15 @@ def test_forward_decode_single_cached_token():
     got = idx.reshape(-1, wl.k).cpu().numpy()
     assert np.all(got[:, 0] == 0) and np.all(got[:, 1:] == -1)
     _check_forward_rows(inp, wl, idx, out, lse, np.arange(wl.B), 1, 0, exact_idx=True)
+
+
+def test_forward_multi_token_decode():
+    # three new tokens per sequence over a 6000-token cache: the generic indexer
+    # build, the one-CTA top-k with rows kept in shared memory, attention unsplit
+    wl = WORKLOADS["decode_128k"].with_(B=4, Lq=3, Lk=6000, q_offset=5997)
+    inp = make_inputs(wl, DEV, 6)
+    idx, out, lse = _forward(inp, wl)
+    _check_forward_rows(inp, wl, idx, out, lse, np.arange(wl.B * wl.Lq), wl.Lq, wl.q_offset)
 
 
 def test_wait_timeout_is_reported_not_trapped():
