@@ -826,8 +826,9 @@ cudaError_t launch_indexer(const IndexerParams& p, const CUtensorMap& tq, const 
       // Specialised for the prefill (4 queries) and decode (one query) blocks.
       if (!deep && p.qb == 4) return launch_indexer_t<64, 128, 4, true, 4, 1>(p, tq, tk, ts, grid, stream);
       if (deep && p.qb == 1) return launch_indexer_t<64, 128, 8, true, 1, 1>(p, tq, tk, ts, grid, stream);
-      return deep ? launch_indexer_t<64, 128, 8, true>(p, tq, tk, ts, grid, stream)
-                  : launch_indexer_t<64, 128, 4, true>(p, tq, tk, ts, grid, stream);
+      // Any other block (two queries: the deeper ring and the lists of two rows do
+      // not fit together) takes the 4-stage ring.
+      return launch_indexer_t<64, 128, 4, true>(p, tq, tk, ts, grid, stream);
     }
     if (deep && p.nsub != 1) return cudaErrorInvalidValue;   // the deep-ring build visits tiles by group
     // Builds specialised for the prefill block (4 queries x 2 sub-blocks) and the

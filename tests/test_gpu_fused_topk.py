@@ -81,6 +81,15 @@ def test_fused_decode_rows_split_over_units_equal_staged():
     _same_as_staged(inp, wl.q_offset, wl.k)
 
 
+@pytest.mark.parametrize("Lq", [2, 3, 4])
+def test_fused_few_query_blocks_equal_staged(Lq):
+    # 2-4 new tokens per sequence: query blocks of two (the deep-ring sizes, whose
+    # candidate lists and staging need the shorter key ring), three and four
+    wl = WORKLOADS["decode_128k"].with_(B=3, Lq=Lq, Lk=9000, q_offset=9000 - Lq)
+    inp = make_inputs(wl, DEV, 10 + Lq)
+    _same_as_staged(inp, wl.q_offset, wl.k)
+
+
 def test_fused_decode_full_size_sampled_against_the_oracle():
     wl = WORKLOADS["decode_128k"]
     inp = make_key_side(wl, DEV, 0)
