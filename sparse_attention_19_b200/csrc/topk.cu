@@ -941,12 +941,14 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(cons
       gtm |= (j < cnt && key[j] > thr) ? (1u << j) : 0u;
       eqm |= (j < cnt && key[j] == thr) ? (1u << j) : 0u;
     }
-    uint32_t eq_tot;
-    const uint32_t eq_rank = eq_seen + warp_exclusive_sum(__popc(eqm), eq_tot);
-    uint32_t take = gtm, e = eqm;
-    for (uint32_t r = eq_rank; e && r < eq_take; ++r) {   // equal keys taken in position order
-      take |= e & (0u - e);
-      e &= e - 1u;
+    uint32_t eq_tot = 0, take = gtm;
+    if (__any_sync(0xffffffffu, eqm != 0u)) {           // most groups hold no key equal to thr
+      const uint32_t eq_rank = eq_seen + warp_exclusive_sum(__popc(eqm), eq_tot);
+      uint32_t e = eqm;
+      for (uint32_t r = eq_rank; e && r < eq_take; ++r) {   // equal keys taken in position order
+        take |= e & (0u - e);
+        e &= e - 1u;
+      }
     }
     uint32_t kept;
     uint32_t at = w + warp_exclusive_sum(__popc(take), kept);
