@@ -367,7 +367,11 @@ def roofline_stages(wl, runner, stage_ms, peaks, peak_src):
         out["indexer"] = dict(bound="tensor", achieved=tot["indexer_flops"] / (stage_ms[0] * 1e-3) / 1e12,
                               peak=fp8_sust, unit="TFLOP/s", algorithmic=tot["indexer_flops"] / calls,
                               peak_note=fp8_note)
-    if stage_ms[1] > 0:
+    if runner.low_memory:
+        # the selection runs inside the indexer kernel: no top-k launch to time (the
+        # span between its events holds no kernel), and the indexer's span covers both
+        out["indexer"]["note"] = "indexer with the top-k selection fused into its epilogue"
+    elif stage_ms[1] > 0:
         # top-k: a streaming selection over the causal scores
         out["topk"] = dict(bound="hbm", achieved=tot["topk_bytes"] / (stage_ms[1] * 1e-3) / 1e9,
                            peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=tot["topk_bytes"] / calls)

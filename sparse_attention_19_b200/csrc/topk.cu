@@ -490,7 +490,7 @@ struct alignas(16) TopkClusterShared {
   uint32_t tot[kBins];         // the cluster's
   ScanScratch x;
   uint32_t pub_a, pub_b;       // values this CTA publishes to the cluster
-  uint32_t pad[2];
+  uint32_t pub_c, pub_d;
 };
 
 // tot = sum over the cluster's CTAs of hist.
@@ -566,6 +566,7 @@ topk_cluster_kernel(const TopkParams p) {
   // decision is taken from cluster-wide counts, so every CTA reaches the same
   // barriers.  Otherwise the two passes below.
   bool single = false;
+  uint32_t single_lo = 0xffffffffu, single_hi = 0u;   // the cluster's kept-key range
   if (try_single) {
     const float mu = (float)ns * (float)k / (float)n;
     const float sig = sqrtf(mu * (1.f - (float)k / (float)n));
@@ -595,16 +596,57 @@ topk_cluster_kernel(const TopkParams p) {
       for (int x = threadIdx.x; x < W; x += kThreads) { gt_bits[x] = 0u; eq_bits[x] = 0u; }
       if (threadIdx.x == 0) sh.x.ncand = 0u;
       __syncthreads();
-      row_pass(s1 - s0, seg_key, [&](int s, bool valid, uint32_t key) {
-        if (valid && key >= theta) {
+      auto keep = [&](int s, uint32_t key) {        // s relative to s0
+        if (key >= theta) {
           const uint32_t at = atomicAdd(&sh.x.ncand, 1u);
           if (at < (uint32_t)p.cand_cap) cand[at] = make_uint2(key, (uint32_t)s);
         }
-      });
+      };
+      if (p.vec4) {
+        // s0 is a multiple of 32 scores, so the segment starts 16-byte aligned
+        // whenever the rows do: 16-byte loads, four in flight per thread (twice the
+        // bytes in flight of the 4-byte row pass, which matters with one row per
+        // four CTAs and nothing else on the GPU).
+        const float4* src4 = reinterpret_cast<const float4*>(src + s0);
+        const int nq = (s1 - s0) >> 2;
+        for (int q0 = threadIdx.x; q0 < nq; q0 += kThreads * kUnroll4) {
+          float4 f[kUnroll4];
+#pragma unroll
+          for (int u = 0; u < kUnroll4; ++u) {
+            const int q = q0 + u * kThreads;
+            f[u] = (q < nq) ? __ldg(src4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < kUnroll4; ++u) {
+            const int q = q0 + u * kThreads;
+            if (q >= nq) break;
+            keep(4 * q, score_key(f[u].x));
+            keep(4 * q + 1, score_key(f[u].y));
+            keep(4 * q + 2, score_key(f[u].z));
+            keep(4 * q + 3, score_key(f[u].w));
+          }
+        }
+        for (int s = (nq << 2) + (int)threadIdx.x; s < s1 - s0; s += kThreads) keep(s, seg_key(s));
+      } else {
+        row_pass(s1 - s0, seg_key, [&](int s, bool valid, uint32_t key) {
+          if (valid) keep(s, key);
+        });
+      }
       __syncthreads();
+      // The kept keys' range goes out with the counts, so the single route needs no
+      // second exchange to open its refinement window.
+      const uint32_t kept = min(sh.x.ncand, (uint32_t)p.cand_cap);
+      uint32_t cmin = 0xffffffffu, cmax = 0u;
+      for (int x = threadIdx.x; x < (int)kept; x += kThreads) {
+        cmin = min(cmin, cand[x].x);
+        cmax = max(cmax, cand[x].x);
+      }
+      block_min_max(sh.x, cmin, cmax);
       if (threadIdx.x == 0) {
         sh.pub_a = sh.x.ncand;
         sh.pub_b = sh.x.ncand > (uint32_t)p.cand_cap ? 1u : 0u;
+        sh.pub_c = cmin;
+        sh.pub_d = cmax;
       }
       cluster_sync();
       uint32_t total = 0, over = 0;
@@ -612,8 +654,10 @@ topk_cluster_kernel(const TopkParams p) {
       for (int c = 0; c < kClusterCtas; ++c) {
         total += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c));
         over |= ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_b), c));
+        single_lo = min(single_lo, ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_c), c)));
+        single_hi = max(single_hi, ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_d), c)));
       }
-      cluster_sync();                               // pub_a / pub_b are not rewritten before all have read them
+      cluster_sync();                               // the pub_* words are not rewritten before all have read them
       single = over == 0u && total >= (uint32_t)k;
     }
   }
@@ -655,7 +699,10 @@ topk_cluster_kernel(const TopkParams p) {
   // Exact threshold, refined over the window [wlo, whi] with cluster-summed histograms
   // of the candidates (or of the segments when the candidates do not fit).
   uint32_t wlo, whi;
-  if (fits) {
+  if (single) {
+    wlo = single_lo;
+    whi = single_hi;
+  } else if (fits) {
     uint32_t cmin = 0xffffffffu, cmax = 0u;
     for (int x = threadIdx.x; x < own; x += kThreads) {
       cmin = min(cmin, cand[x].x);
