@@ -51,6 +51,13 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The float whose key is `key` (inverse of score_key; +0.0 for the key of zero).
+// For non-NaN f, score_key(f) >= key exactly when f >= key_score(key): the key
+// order is the float order with -0.0 equal to +0.0, as in float comparison.
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
 // The score at a selected position as the selection saw it: -0.0 reads as +0.0.
 __device__ __forceinline__ float selected_score(const float* src, int s) {
   const float v = __ldg(src + s);
@@ -62,6 +69,7 @@ struct ScanScratch {
   uint32_t warp_tot[kWarps];
   uint32_t warp_a[kWarps], warp_b[kWarps];
   uint32_t bin, above, ncand;
+  uint32_t bcount;             // keys in bin (find_bin)
 };
 
 // 16-byte multiple, so the arrays that follow it in dynamic shared memory stay aligned.
@@ -114,6 +122,7 @@ __device__ void find_bin(const uint32_t* hist, ScanScratch& x, uint32_t need) {
     if (acc < need && acc + c >= need) {
       x.bin = (uint32_t)(lo + i);
       x.above = acc;
+      x.bcount = c;
     }
     acc += c;
   }
@@ -484,6 +493,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
 // threshold; each CTA marks its own segment's bitmaps and candidates, and writes
 // its selected positions after those of the lower-ranked CTAs.
 constexpr int kClusterCtas = kTopkClusterCtas;
+constexpr int kClusterGatherCap = 8192;   // kept keys a CTA copies from the whole cluster (gathered route)
+constexpr int kSmallSelect = 64;
+constexpr int kPassUnroll = 8;           // 16-byte loads in flight per thread in the cluster's single pass          // boundary-bin keys ranked directly by one warp (gathered route)
 
 struct alignas(16) TopkClusterShared {
   uint32_t hist[kBins];        // this CTA's histogram
@@ -491,6 +503,9 @@ struct alignas(16) TopkClusterShared {
   ScanScratch x;
   uint32_t pub_a, pub_b;       // values this CTA publishes to the cluster
   uint32_t pub_c, pub_d;
+  uint32_t lower_gt, lower_eq;  // gathered route: keys above / equal to the threshold in lower-ranked CTAs
+  uint32_t small_n, small_thr, small_need;
+  uint32_t small[kSmallSelect];  // gathered route: the boundary bin's keys, ranked by one warp
 };
 
 // tot = sum over the cluster's CTAs of hist.
@@ -515,6 +530,7 @@ topk_cluster_kernel(const TopkParams p) {
   uint32_t* gt_bits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkClusterShared));   // segment words
   uint32_t* eq_bits = gt_bits + p.bit_words;
   uint2* cand = reinterpret_cast<uint2*>(eq_bits + p.bit_words);
+  uint32_t* allk = reinterpret_cast<uint32_t*>(cand + p.cand_cap);   // kClusterGatherCap keys
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t r = cluster_ctarank();
@@ -542,15 +558,28 @@ topk_cluster_kernel(const TopkParams p) {
   auto seg_key = [&](int s) -> uint32_t { return load_key(s0 + s); };
 
   // ---- 1. sampled key range (the same in every CTA; kept in the candidate buffer
-  // for step 1b)
+  // for step 1b): positions j * (n / ns), every load of a thread in flight at once
   const int ns = n < kSample ? n : kSample;
+  const int stride = n / ns;
   const bool try_single = p.sampled && p.cand_cap >= kSample;
   uint32_t smin = 0xffffffffu, smax = 0u;
-  for (int j = threadIdx.x; j < ns; j += kThreads) {
-    const uint32_t key = load_key((int)(((long long)j * n) / ns));
-    if (try_single) cand[j].x = key;
-    smin = min(smin, key);
-    smax = max(smax, key);
+  {
+    constexpr int kPer = (kSample + kThreads - 1) / kThreads;
+    uint32_t sk[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int j = (int)threadIdx.x + u * kThreads;
+      sk[u] = j < ns ? load_key(j * stride) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int j = (int)threadIdx.x + u * kThreads;
+      if (j < ns) {
+        if (try_single) cand[j].x = sk[u];
+        smin = min(smin, sk[u]);
+        smax = max(smax, sk[u]);
+      }
+    }
   }
   block_min_max(sh.x, smin, smax);
   const uint32_t lo = smin;
@@ -567,6 +596,8 @@ topk_cluster_kernel(const TopkParams p) {
   // barriers.  Otherwise the two passes below.
   bool single = false;
   uint32_t single_lo = 0xffffffffu, single_hi = 0u;   // the cluster's kept-key range
+  uint32_t total = 0;                                  // keys kept over the cluster
+  uint32_t cnt_c[kClusterCtas] = {};                   // ... by each CTA
   if (try_single) {
     const float mu = (float)ns * (float)k / (float)n;
     const float sig = sqrtf(mu * (1.f - (float)k / (float)n));
@@ -606,24 +637,57 @@ topk_cluster_kernel(const TopkParams p) {
         // s0 is a multiple of 32 scores, so the segment starts 16-byte aligned
         // whenever the rows do: 16-byte loads, four in flight per thread (twice the
         // bytes in flight of the 4-byte row pass, which matters with one row per
-        // four CTAs and nothing else on the GPU).
+        // four CTAs and nothing else on the GPU).  A warp appends its kept keys of
+        // a step with one shared atomic (per-key atomics on the one counter
+        // serialised the pass).
         const float4* src4 = reinterpret_cast<const float4*>(src + s0);
         const int nq = (s1 - s0) >> 2;
-        for (int q0 = threadIdx.x; q0 < nq; q0 += kThreads * kUnroll4) {
-          float4 f[kUnroll4];
+        const float theta_f = key_score(theta);
+        for (int q00 = warp * 32; q00 < nq; q00 += kThreads * kPassUnroll) {   // warp-uniform bound
+          const int q0 = q00 + lane;
+          float4 f[kPassUnroll];
 #pragma unroll
-          for (int u = 0; u < kUnroll4; ++u) {
+          for (int u = 0; u < kPassUnroll; ++u) {
             const int q = q0 + u * kThreads;
             f[u] = (q < nq) ? __ldg(src4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+          uint32_t mine = 0;                          // kept keys of this lane in this step
 #pragma unroll
-          for (int u = 0; u < kUnroll4; ++u) {
+          for (int u = 0; u < kPassUnroll; ++u) {
             const int q = q0 + u * kThreads;
-            if (q >= nq) break;
-            keep(4 * q, score_key(f[u].x));
-            keep(4 * q + 1, score_key(f[u].y));
-            keep(4 * q + 2, score_key(f[u].z));
-            keep(4 * q + 3, score_key(f[u].w));
+            if (q < nq) {                              // float compares: no key conversion per score
+              mine += f[u].x >= theta_f ? 1u : 0u;
+              mine += f[u].y >= theta_f ? 1u : 0u;
+              mine += f[u].z >= theta_f ? 1u : 0u;
+              mine += f[u].w >= theta_f ? 1u : 0u;
+            }
+          }
+          uint32_t incl = mine;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+          if (wtot == 0u) continue;
+          uint32_t at = 0;
+          if (lane == 31) at = atomicAdd(&sh.x.ncand, wtot);
+          at = __shfl_sync(0xffffffffu, at, 31) + incl - mine;
+          if (mine != 0u) {
+#pragma unroll
+            for (int u = 0; u < kPassUnroll; ++u) {
+              const int q = q0 + u * kThreads;
+              if (q < nq) {
+                const float fx[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                  if (fx[c] >= theta_f) {                // the predicate the count used
+                    if (at < (uint32_t)p.cand_cap) cand[at] = make_uint2(score_key(fx[c]), (uint32_t)(4 * q + c));
+                    ++at;
+                  }
+                }
+              }
+            }
           }
         }
         for (int s = (nq << 2) + (int)threadIdx.x; s < s1 - s0; s += kThreads) keep(s, seg_key(s));
@@ -649,10 +713,11 @@ topk_cluster_kernel(const TopkParams p) {
         sh.pub_d = cmax;
       }
       cluster_sync();
-      uint32_t total = 0, over = 0;
+      uint32_t over = 0;
 #pragma unroll
       for (int c = 0; c < kClusterCtas; ++c) {
-        total += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c));
+        cnt_c[c] = ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c));
+        total += cnt_c[c];
         over |= ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_b), c));
         single_lo = min(single_lo, ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_c), c)));
         single_hi = max(single_hi, ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_d), c)));
@@ -696,6 +761,29 @@ topk_cluster_kernel(const TopkParams p) {
   const bool fits = single || cnt_b <= (uint32_t)p.cand_cap;
   const int own = (int)sh.x.ncand;
 
+  // Single route with few kept keys (decode rows keep ~5 K): every CTA gets a copy
+  // of the cluster's kept keys, in CTA order (each CTA stores its own keys into
+  // every CTA's copy), and refines the threshold on it alone, with no cluster
+  // barrier per level; the keys that lower-ranked CTAs hold above and at the
+  // threshold then give this CTA's output offsets.
+  const bool gathered = single && total <= (uint32_t)kClusterGatherCap;
+  uint32_t lower = 0;                               // keys kept by lower-ranked CTAs
+  if (gathered) {
+#pragma unroll
+    for (int c = 0; c < kClusterCtas; ++c) {
+      if ((uint32_t)c < r) lower += cnt_c[c];
+    }
+    // each CTA stores its own keys into every CTA's copy, at its offset
+    const uint32_t base = smem_u32(allk + lower);
+    for (int x = threadIdx.x; x < own; x += kThreads) {
+      const uint32_t key = cand[x].x;
+#pragma unroll
+      for (int c = 0; c < kClusterCtas; ++c) st_shared_cluster_u32(mapa_shared(base + 4u * (uint32_t)x, (uint32_t)c), key);
+    }
+    if (threadIdx.x == 0) { sh.lower_gt = 0u; sh.lower_eq = 0u; }
+    cluster_sync();                                 // every copy is complete; no shared memory of a peer is touched after this
+  }
+
   // Exact threshold, refined over the window [wlo, whi] with cluster-summed histograms
   // of the candidates (or of the segments when the candidates do not fit).
   uint32_t wlo, whi;
@@ -728,7 +816,12 @@ topk_cluster_kernel(const TopkParams p) {
     const int wsh = bin_shift(whi - wlo);
     const uint32_t l0 = wlo, h0 = whi;
     clear_hist(sh.hist);
-    if (fits) {
+    if (gathered) {
+      for (int x = threadIdx.x; x < (int)total; x += kThreads) {
+        const uint32_t key = allk[x];
+        if (key >= l0 && key <= h0) atomicAdd(&sh.hist[(key - l0) >> wsh], 1u);
+      }
+    } else if (fits) {
       for (int x = threadIdx.x; x < own; x += kThreads) {
         const uint32_t key = cand[x].x;
         if (key >= l0 && key <= h0) atomicAdd(&sh.hist[(key - l0) >> wsh], 1u);
@@ -739,20 +832,69 @@ topk_cluster_kernel(const TopkParams p) {
       });
     }
     __syncthreads();
-    cluster_sum_hist(sh);
-    find_bin(sh.tot, sh.x, need);
+    if (!gathered) cluster_sum_hist(sh);
+    find_bin(gathered ? sh.hist : sh.tot, sh.x, need);
     const uint32_t bw = sh.x.bin;
     need -= sh.x.above;
     if (wsh == 0) { thr = wlo + bw; break; }
     wlo = l0 + (bw << wsh);
     const unsigned long long top = (unsigned long long)wlo + (1ull << wsh) - 1ull;
     whi = top < (unsigned long long)h0 ? (uint32_t)top : h0;
+    // Gathered route: once the boundary bin [wlo, whi] holds few keys, one warp
+    // ranks them directly (the key with fewer than `need` keys above it and at least
+    // `need` at or above it) instead of further histogram levels.
+    if (gathered && sh.x.bcount <= (uint32_t)kSmallSelect) {
+      if (threadIdx.x == 0) sh.small_n = 0u;
+      __syncthreads();
+      for (int x = threadIdx.x; x < (int)total; x += kThreads) {
+        const uint32_t key = allk[x];
+        if (key >= wlo && key <= whi) {
+          const uint32_t a = atomicAdd(&sh.small_n, 1u);
+          if (a < (uint32_t)kSmallSelect) sh.small[a] = key;
+        }
+      }
+      __syncthreads();
+      const int m = (int)min(sh.small_n, (uint32_t)kSmallSelect);
+      if (warp == 0) {
+        for (int a = lane; a < m; a += 32) {
+          const uint32_t key = sh.small[a];
+          uint32_t gt = 0, eq = 0;
+          for (int b2 = 0; b2 < m; ++b2) {
+            const uint32_t v = sh.small[b2];
+            gt += v > key ? 1u : 0u;
+            eq += v == key ? 1u : 0u;
+          }
+          if (gt < need && need <= gt + eq) {       // equal keys write the same values
+            sh.small_thr = key;
+            sh.small_need = need - gt;
+          }
+        }
+      }
+      __syncthreads();
+      thr = sh.small_thr;
+      need = sh.small_need;
+      break;
+    }
   }
   if (fits) {
     for (int x = threadIdx.x; x < own; x += kThreads) {
       const uint2 c = cand[x];
       if (c.x > thr) atomicOr(&gt_bits[c.y >> 5], 1u << (c.y & 31u));
       else if (c.x == thr) atomicOr(&eq_bits[c.y >> 5], 1u << (c.y & 31u));
+    }
+    if (gathered) {                                 // the lower-ranked CTAs' keys come first in allk
+      uint32_t lg = 0, le = 0;
+      for (int x = threadIdx.x; x < (int)lower; x += kThreads) {
+        const uint32_t key = allk[x];
+        lg += key > thr ? 1u : 0u;
+        le += key == thr ? 1u : 0u;
+      }
+      lg = __reduce_add_sync(0xffffffffu, lg);
+      le = __reduce_add_sync(0xffffffffu, le);
+      if (lane == 0 && (lg | le) != 0u) {
+        atomicAdd(&sh.lower_gt, lg);
+        atomicAdd(&sh.lower_eq, le);
+      }
     }
   } else {
     row_pass(s1 - s0, seg_key, [&](int s, bool valid, uint32_t key) {
@@ -783,13 +925,18 @@ topk_cluster_kernel(const TopkParams p) {
     seg_g += sh.x.warp_a[w];
     seg_e += sh.x.warp_b[w];
   }
-  if (threadIdx.x == 0) { sh.pub_a = seg_g; sh.pub_b = seg_e; }
-  cluster_sync();
-  for (uint32_t c = 0; c < r; ++c) {
-    g += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c));
-    e += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_b), c));
+  if (gathered) {
+    g += sh.lower_gt;
+    e += sh.lower_eq;
+  } else {
+    if (threadIdx.x == 0) { sh.pub_a = seg_g; sh.pub_b = seg_e; }
+    cluster_sync();
+    for (uint32_t c = 0; c < r; ++c) {
+      g += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_a), c));
+      e += ld_shared_cluster_u32(mapa_shared(smem_u32(&sh.pub_b), c));
+    }
+    cluster_sync();                                 // peers' shared memory is no longer read
   }
-  cluster_sync();                                   // peers' shared memory is no longer read
   for (int w0 = w_begin; w0 < w_end; w0 += 32) {
     const int w = w0 + lane;
     const uint32_t gw = (w < w_end) ? gt_bits[w] : 0u;
@@ -1062,7 +1209,8 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(cons
 size_t topk_smem_bytes(int cache_cap, int bit_words, int cand_cap, bool cluster) {
   static_assert(sizeof(TopkShared) % 16 == 0, "arrays that follow must stay 16-byte aligned");
   static_assert(sizeof(TopkClusterShared) % 16 == 0, "arrays that follow must stay 16-byte aligned");
-  if (cluster) return sizeof(TopkClusterShared) + 2 * (size_t)bit_words * 4 + (size_t)cand_cap * 8;
+  if (cluster)
+    return sizeof(TopkClusterShared) + 2 * (size_t)bit_words * 4 + (size_t)cand_cap * 8 + (size_t)kClusterGatherCap * 4;
   return sizeof(TopkShared) + ((size_t)cache_cap + 2 * (size_t)bit_words) * 4 + (size_t)cand_cap * 8;
 }
 

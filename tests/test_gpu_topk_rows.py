@@ -127,9 +127,13 @@ def test_long_rows_fall_back_when_too_many_keys_pass():
 def test_cluster_rows_one_pass_and_segment_overflow():
     g = torch.Generator().manual_seed(41)
     Lk = 131072
-    s = torch.randn(1, 4, Lk, generator=g)
+    s = torch.randn(1, 6, Lk, generator=g)
     s[0, 1, 1000:5500] = 5.0                         # one segment holds more than its buffer
     s[0, 2, ::87] = 4.0                              # 1507 planted ties, spread over all segments
     s[0, 2] = torch.where(s[0, 2] == 4.0, s[0, 2], torch.round(s[0, 2] * 8) / 8)
     s[0, 3] = 0.5                                    # every key passes: the two-pass route
-    _check(s.to(DEV), Lk - 4, 2048)
+    s[0, 4, ::13] = 5.0                              # ~10 K kept keys: one pass, refined over the cluster
+    s[0, 5] *= 0.5                                   # ~5 K kept keys, refined by each CTA on a copy of all
+    s[0, 5, ::67] = 5.0                              # of them; the threshold's ties (4.5) straddle the
+    s[0, 5, 32700:32800] = 4.5                       # first two segments
+    _check(s.to(DEV), Lk - 6, 2048)
