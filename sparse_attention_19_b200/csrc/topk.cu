@@ -276,23 +276,55 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
         }
       };
       if (p.vec4) {
+        // Float compares against theta's float value (no key conversion per score)
+        // and one shared atomic per warp and step for the kept keys' slots.
         const float4* src4 = reinterpret_cast<const float4*>(src);
         const int nq = n >> 2;
-        for (int q0 = threadIdx.x; q0 < nq; q0 += kThreads * kUnroll4) {
+        const float theta_f = key_score(theta);
+        for (int q00 = warp * 32; q00 < nq; q00 += kThreads * kUnroll4) {   // warp-uniform bound
+          const int q0 = q00 + lane;
           float4 f[kUnroll4];
 #pragma unroll
           for (int u = 0; u < kUnroll4; ++u) {
             const int q = q0 + u * kThreads;
             f[u] = (q < nq) ? __ldg(src4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+          uint32_t mine = 0;
 #pragma unroll
           for (int u = 0; u < kUnroll4; ++u) {
-            const int q = q0 + u * kThreads;
-            if (q >= nq) break;
-            keep(4 * q, score_key(f[u].x));
-            keep(4 * q + 1, score_key(f[u].y));
-            keep(4 * q + 2, score_key(f[u].z));
-            keep(4 * q + 3, score_key(f[u].w));
+            if (q0 + u * kThreads < nq) {
+              mine += f[u].x >= theta_f ? 1u : 0u;
+              mine += f[u].y >= theta_f ? 1u : 0u;
+              mine += f[u].z >= theta_f ? 1u : 0u;
+              mine += f[u].w >= theta_f ? 1u : 0u;
+            }
+          }
+          uint32_t incl = mine;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+          if (wtot == 0u) continue;
+          uint32_t at = 0;
+          if (lane == 31) at = atomicAdd(&sh.x.ncand, wtot);
+          at = __shfl_sync(0xffffffffu, at, 31) + incl - mine;
+          if (mine != 0u) {
+#pragma unroll
+            for (int u = 0; u < kUnroll4; ++u) {
+              const int q = q0 + u * kThreads;
+              if (q < nq) {
+                const float fx[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                  if (fx[c] >= theta_f) {                // the predicate the count used
+                    if (at < (uint32_t)p.cand_cap) cand[at] = make_uint2(score_key(fx[c]), (uint32_t)(4 * q + c));
+                    ++at;
+                  }
+                }
+              }
+            }
           }
         }
         for (int s = (nq << 2) + (int)threadIdx.x; s < n; s += kThreads) keep(s, load_key(s));
