@@ -86,12 +86,6 @@ __device__ __forceinline__ void st_async_f32(uint32_t cluster_addr, float v, uin
 __device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
-// Asynchronous prefetch of [addr, addr + bytes) from global memory into L2; addr
-// and bytes are multiples of 16.  Nothing waits for it: it only warms L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* addr, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(addr)), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
