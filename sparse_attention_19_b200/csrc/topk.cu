@@ -44,6 +44,7 @@ constexpr int kBins = 1 << kBinBits;
 constexpr int kUnroll = 8;           // 4-byte loads in flight per thread in the row passes
 constexpr int kUnroll4 = 4;          // 16-byte loads in flight per thread in the histogram pass
 constexpr int kSample = 1024;        // strided sample that sets the first histogram's range
+constexpr int kSmallSelect = 64;     // a boundary bin this small is ranked directly by one warp
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -72,10 +73,17 @@ struct ScanScratch {
   uint32_t bcount;             // keys in bin (find_bin)
 };
 
+// The keys of a small boundary bin, ranked by one warp (small_select).
+struct SmallSel {
+  uint32_t key[kSmallSelect];
+  uint32_t n, thr, need;
+};
+
 // 16-byte multiple, so the arrays that follow it in dynamic shared memory stay aligned.
 struct alignas(16) TopkShared {
   uint32_t hist[kBins];
   ScanScratch x;
+  SmallSel small;
 };
 
 // Block-wide inclusive scan of one value per thread (thread order).
@@ -127,6 +135,45 @@ __device__ void find_bin(const uint32_t* hist, ScanScratch& x, uint32_t need) {
     acc += c;
   }
   __syncthreads();
+}
+
+// The exact threshold inside a boundary bin [wlo, whi] that holds at most
+// kSmallSelect keys (of key_of(0 .. count)): warp 0 ranks them directly and the
+// block receives the need-th largest key (thr) and how many keys equal to it are
+// still to be taken (need).  Replaces the remaining histogram levels.  Every
+// thread of the block calls it.
+template <typename KeyOf>
+__device__ __forceinline__ void small_select(SmallSel& ss, int count, KeyOf key_of, uint32_t wlo, uint32_t whi,
+                                             uint32_t& thr, uint32_t& need) {
+  if (threadIdx.x == 0) ss.n = 0u;
+  __syncthreads();
+  for (int x = threadIdx.x; x < count; x += kThreads) {
+    const uint32_t key = key_of(x);
+    if (key >= wlo && key <= whi) {
+      const uint32_t a = atomicAdd(&ss.n, 1u);
+      if (a < (uint32_t)kSmallSelect) ss.key[a] = key;
+    }
+  }
+  __syncthreads();
+  const int m = (int)min(ss.n, (uint32_t)kSmallSelect);
+  if (threadIdx.x < 32) {
+    for (int a = (int)threadIdx.x; a < m; a += 32) {
+      const uint32_t key = ss.key[a];
+      uint32_t gt = 0, eq = 0;
+      for (int b = 0; b < m; ++b) {
+        const uint32_t v = ss.key[b];
+        gt += v > key ? 1u : 0u;
+        eq += v == key ? 1u : 0u;
+      }
+      if (gt < need && need <= gt + eq) {           // equal keys write the same values
+        ss.thr = key;
+        ss.need = need - gt;
+      }
+    }
+  }
+  __syncthreads();
+  thr = ss.thr;
+  need = ss.need;
 }
 
 // Right shift that maps a key range of width range+1 onto at most kBins bins.
@@ -443,6 +490,10 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
     wlo = l0 + (bw << wsh);
     const unsigned long long top = (unsigned long long)wlo + (1ull << wsh) - 1ull;
     whi = top < (unsigned long long)h0 ? (uint32_t)top : h0;
+    if (fits && sh.x.bcount <= (uint32_t)kSmallSelect) {
+      small_select(sh.small, (int)cnt_b, [&](int x) { return cand[x].x; }, wlo, whi, thr, need);
+      break;
+    }
   }
   if (fits) {
     for (int x = threadIdx.x; x < (int)cnt_b; x += kThreads) {
@@ -526,8 +577,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
 // its selected positions after those of the lower-ranked CTAs.
 constexpr int kClusterCtas = kTopkClusterCtas;
 constexpr int kClusterGatherCap = 8192;   // kept keys a CTA copies from the whole cluster (gathered route)
-constexpr int kSmallSelect = 64;
-constexpr int kPassUnroll = 8;           // 16-byte loads in flight per thread in the cluster's single pass          // boundary-bin keys ranked directly by one warp (gathered route)
+constexpr int kPassUnroll = 8;           // 16-byte loads in flight per thread in the cluster's single pass
 
 struct alignas(16) TopkClusterShared {
   uint32_t hist[kBins];        // this CTA's histogram
@@ -536,8 +586,7 @@ struct alignas(16) TopkClusterShared {
   uint32_t pub_a, pub_b;       // values this CTA publishes to the cluster
   uint32_t pub_c, pub_d;
   uint32_t lower_gt, lower_eq;  // gathered route: keys above / equal to the threshold in lower-ranked CTAs
-  uint32_t small_n, small_thr, small_need;
-  uint32_t small[kSmallSelect];  // gathered route: the boundary bin's keys, ranked by one warp
+  SmallSel small;               // gathered route: a small boundary bin's keys
 };
 
 // tot = sum over the cluster's CTAs of hist.
@@ -873,38 +922,9 @@ topk_cluster_kernel(const TopkParams p) {
     const unsigned long long top = (unsigned long long)wlo + (1ull << wsh) - 1ull;
     whi = top < (unsigned long long)h0 ? (uint32_t)top : h0;
     // Gathered route: once the boundary bin [wlo, whi] holds few keys, one warp
-    // ranks them directly (the key with fewer than `need` keys above it and at least
-    // `need` at or above it) instead of further histogram levels.
+    // ranks them directly instead of further histogram levels.
     if (gathered && sh.x.bcount <= (uint32_t)kSmallSelect) {
-      if (threadIdx.x == 0) sh.small_n = 0u;
-      __syncthreads();
-      for (int x = threadIdx.x; x < (int)total; x += kThreads) {
-        const uint32_t key = allk[x];
-        if (key >= wlo && key <= whi) {
-          const uint32_t a = atomicAdd(&sh.small_n, 1u);
-          if (a < (uint32_t)kSmallSelect) sh.small[a] = key;
-        }
-      }
-      __syncthreads();
-      const int m = (int)min(sh.small_n, (uint32_t)kSmallSelect);
-      if (warp == 0) {
-        for (int a = lane; a < m; a += 32) {
-          const uint32_t key = sh.small[a];
-          uint32_t gt = 0, eq = 0;
-          for (int b2 = 0; b2 < m; ++b2) {
-            const uint32_t v = sh.small[b2];
-            gt += v > key ? 1u : 0u;
-            eq += v == key ? 1u : 0u;
-          }
-          if (gt < need && need <= gt + eq) {       // equal keys write the same values
-            sh.small_thr = key;
-            sh.small_need = need - gt;
-          }
-        }
-      }
-      __syncthreads();
-      thr = sh.small_thr;
-      need = sh.small_need;
+      small_select(sh.small, (int)total, [&](int x) { return allk[x]; }, wlo, whi, thr, need);
       break;
     }
   }
