@@ -45,6 +45,7 @@ constexpr int kUnroll = 8;           // 4-byte loads in flight per thread in the
 constexpr int kUnroll4 = 4;          // 16-byte loads in flight per thread in the histogram pass
 constexpr int kSample = 1024;        // strided sample that sets the first histogram's range
 constexpr int kSmallSelect = 64;     // a boundary bin this small is ranked directly by one warp
+constexpr int kPassUnroll = 8;       // 16-byte loads in flight per thread in the single passes
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -328,17 +329,17 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
         const float4* src4 = reinterpret_cast<const float4*>(src);
         const int nq = n >> 2;
         const float theta_f = key_score(theta);
-        for (int q00 = warp * 32; q00 < nq; q00 += kThreads * kUnroll4) {   // warp-uniform bound
+        for (int q00 = warp * 32; q00 < nq; q00 += kThreads * kPassUnroll) {   // warp-uniform bound
           const int q0 = q00 + lane;
-          float4 f[kUnroll4];
+          float4 f[kPassUnroll];
 #pragma unroll
-          for (int u = 0; u < kUnroll4; ++u) {
+          for (int u = 0; u < kPassUnroll; ++u) {
             const int q = q0 + u * kThreads;
             f[u] = (q < nq) ? __ldg(src4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
           uint32_t mine = 0;
 #pragma unroll
-          for (int u = 0; u < kUnroll4; ++u) {
+          for (int u = 0; u < kPassUnroll; ++u) {
             if (q0 + u * kThreads < nq) {
               mine += f[u].x >= theta_f ? 1u : 0u;
               mine += f[u].y >= theta_f ? 1u : 0u;
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
           at = __shfl_sync(0xffffffffu, at, 31) + incl - mine;
           if (mine != 0u) {
 #pragma unroll
-            for (int u = 0; u < kUnroll4; ++u) {
+            for (int u = 0; u < kPassUnroll; ++u) {
               const int q = q0 + u * kThreads;
               if (q < nq) {
                 const float fx[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
@@ -577,7 +578,6 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(const TopkParams p) {
 // its selected positions after those of the lower-ranked CTAs.
 constexpr int kClusterCtas = kTopkClusterCtas;
 constexpr int kClusterGatherCap = 8192;   // kept keys a CTA copies from the whole cluster (gathered route)
-constexpr int kPassUnroll = 8;           // 16-byte loads in flight per thread in the cluster's single pass
 
 struct alignas(16) TopkClusterShared {
   uint32_t hist[kBins];        // this CTA's histogram
