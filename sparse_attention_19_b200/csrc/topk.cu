@@ -1177,15 +1177,18 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(cons
   warp_find_threshold(sh.hist, sh.cand, visit, k - above, wlo, whi, thr, gt_w, sh.hist[b]);
   const uint32_t eq_take = k - above - gt_w;
 
-  // ---- 4. ordered output: every key above thr and the first eq_take equal to it
+  // ---- 4. ordered output: every key above thr and the first eq_take equal to it.
+  // Scores are compared as floats with thr's float value: the key order is the
+  // float order with -0.0 equal to +0.0, so no key is formed per score.
+  const float thr_f = key_to_score(thr);
   uint32_t w = 0, eq_seen = 0;
-  // keys[] are positions s .. s + cnt - 1 of this lane (cnt <= 4), lanes in position order
-  auto emit_group = [&](int s, const uint32_t (&key)[4], int cnt) {
+  // v[] are the scores at positions s .. s + cnt - 1 of this lane (cnt <= 4), lanes in position order
+  auto emit_group = [&](int s, const float (&v)[4], int cnt) {
     uint32_t gtm = 0, eqm = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      gtm |= (j < cnt && key[j] > thr) ? (1u << j) : 0u;
-      eqm |= (j < cnt && key[j] == thr) ? (1u << j) : 0u;
+      gtm |= (j < cnt && v[j] > thr_f) ? (1u << j) : 0u;
+      eqm |= (j < cnt && v[j] == thr_f) ? (1u << j) : 0u;
     }
     uint32_t eq_tot = 0, take = gtm;
     if (__any_sync(0xffffffffu, eqm != 0u)) {           // most groups hold no key equal to thr
@@ -1202,7 +1205,7 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(cons
     for (int j = 0; j < 4; ++j) {
       if (take & (1u << j)) {
         out[at] = s + j;
-        if (sel_out) sel_out[at] = key_to_score(key[j]);
+        if (sel_out) sel_out[at] = v[j] == 0.f ? 0.f : v[j];   // -0.0 as +0.0, as the selection saw it
         ++at;
       }
     }
@@ -1229,9 +1232,8 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(cons
       for (int u = 0; u < kU; ++u) {
         if (g0 + u * 32 < n4) {
           const int g = g0 + u * 32 + lane;
-          const uint32_t key[4] = {score_to_key(v[u].x), score_to_key(v[u].y), score_to_key(v[u].z),
-                                   score_to_key(v[u].w)};
-          emit_group(4 * g, key, max(0, min(4, n - 4 * g)));
+          const float sv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          emit_group(4 * g, sv, max(0, min(4, n - 4 * g)));
         }
       }
     }
@@ -1248,8 +1250,8 @@ __global__ void __launch_bounds__(32 * kWarpRowsPerCta, 4) topk_warp_kernel(cons
       for (int u = 0; u < kU; ++u) {
         const int s = s0 + u * 32 + lane;
         if (s0 + u * 32 < n) {
-          const uint32_t key[4] = {score_to_key(v[u]), 0u, 0u, 0u};
-          emit_group(s, key, s < n ? 1 : 0);
+          const float sv[4] = {v[u], 0.f, 0.f, 0.f};
+          emit_group(s, sv, s < n ? 1 : 0);
         }
       }
     }
