@@ -136,4 +136,12 @@ def test_cluster_rows_one_pass_and_segment_overflow():
     s[0, 5] *= 0.5                                   # ~5 K kept keys, refined by each CTA on a copy of all
     s[0, 5, ::67] = 5.0                              # of them; the threshold's ties (4.5) straddle the
     s[0, 5, 32700:32800] = 4.5                       # first two segments
-    _check(s.to(DEV), Lk - 6, 2048)
+    # ~7.6 K kept keys, none of them in the last segment and ~3 K in the third: a
+    # CTA with nothing to share and one holding most of the copy
+    g2 = torch.Generator().manual_seed(43)
+    r6 = torch.randn(Lk, generator=g2)
+    high = torch.randperm(32768, generator=g2)[:800] + 65536
+    r6[high] = torch.randn(800, generator=g2) + 5.0
+    r6[98304:] -= 10.0
+    s = torch.cat([s, r6.view(1, 1, Lk)], dim=1)
+    _check(s.to(DEV), Lk - 7, 2048)
