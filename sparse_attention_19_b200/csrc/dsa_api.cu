@@ -139,21 +139,42 @@ IndexerParams plan_indexer(const dsa_indexer_args* a, bool fused, int k) {
   const int sms = sm_count();
   const long long base_units = (long long)p.n_qblocks * a->B;
   const int max_tiles = (a->q_offset + a->Lq - 1) / 128 + 1;
-  // Few query blocks (decode): split each sequence's key tiles over kchunks units.
-  // Cost model in key tiles per CTA: waves of units over the SMs, each unit its
-  // tiles plus about two tiles of start-up; keep at least ~8 tiles per unit.  In
-  // the fused mode the last unit of a row also selects over every chunk's list
-  // (up to k candidates each), so chunks are capped at 16.
+  // Few query blocks (decode): split each sequence's key tiles over kchunks units
+  // (at least ~8 tiles each).
   int kch = 1;
   if (base_units < 4LL * sms) {
-    constexpr double kUnitOverheadTiles = 2.0;
     int cap = (max_tiles + 7) / 8;
-    if (fused && cap > 16) cap = 16;
-    double best = 1e300;
-    for (int c = 1; c <= cap; ++c) {
-      const long long waves = (base_units * c + sms - 1) / sms;
-      const double cost = (double)waves * ((double)(max_tiles + c - 1) / c + kUnitOverheadTiles);
-      if (cost < best) { best = cost; kch = c; }
+    if (fused) {
+      // The last unit of a row also selects over every chunk's list (up to k
+      // candidates each), so chunks are capped at 16.  Cost in key tiles per CTA:
+      // waves of units over the SMs, each unit its tiles plus ~two of start-up.
+      constexpr double kUnitOverheadTiles = 2.0;
+      if (cap > 16) cap = 16;
+      double best = 1e300;
+      for (int c = 1; c <= cap; ++c) {
+        const long long waves = (base_units * c + sms - 1) / sms;
+        const double cost = (double)waves * ((double)(max_tiles + c - 1) / c + kUnitOverheadTiles);
+        if (cost < best) { best = cost; kch = c; }
+      }
+    } else {
+      // Key tiles of the busiest CTA: waves of units over the SMs times the tiles
+      // of a unit.  Many splits come within a few percent of the fewest; among
+      // those, units nearest 32 tiles (4096 keys) measured fastest on B200 (decode,
+      // 64 x 131072 keys: 9 units a sequence 194 us, 16: 196, 23: 187, 32: 183,
+      // 37: 182, 48: 184, 64: 183, 74: 186).
+      constexpr int kPreferTiles = 32;
+      auto cost = [&](int c) {
+        return ((base_units * c + sms - 1) / sms) * (long long)((max_tiles + c - 1) / c);
+      };
+      long long best = cost(1);
+      for (int c = 2; c <= cap; ++c) best = cost(c) < best ? cost(c) : best;
+      int best_gap = 1 << 30;
+      for (int c = 1; c <= cap; ++c) {
+        if (cost(c) * 50 > best * 51) continue;           // more than 2 % above the fewest
+        const int tiles = (max_tiles + c - 1) / c;
+        const int gap = tiles > kPreferTiles ? tiles - kPreferTiles : kPreferTiles - tiles;
+        if (gap <= best_gap) { best_gap = gap; kch = c; }   // ties: the finer split
+      }
     }
   }
   p.kchunks = kch;
