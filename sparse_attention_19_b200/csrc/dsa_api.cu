@@ -144,12 +144,13 @@ IndexerParams plan_indexer(const dsa_indexer_args* a, bool fused, int k) {
   int kch = 1;
   if (base_units < 4LL * sms) {
     int cap = (max_tiles + 7) / 8;
-    if (fused) {
-      // The last unit of a row also selects over every chunk's list (up to k
-      // candidates each), so chunks are capped at 16.  Cost in key tiles per CTA:
-      // waves of units over the SMs, each unit its tiles plus ~two of start-up.
+    if (fused || p.n_qblocks > 1) {
+      // Cost in key tiles per CTA: waves of units over the SMs, each unit its tiles
+      // plus ~two of start-up (the causal query blocks of a long prefill chunk, and
+      // the fused mode, whose last unit of a row also selects over every chunk's
+      // list of up to k candidates, so its chunks are capped at 16).
       constexpr double kUnitOverheadTiles = 2.0;
-      if (cap > 16) cap = 16;
+      if (fused && cap > 16) cap = 16;
       double best = 1e300;
       for (int c = 1; c <= cap; ++c) {
         const long long waves = (base_units * c + sms - 1) / sms;
@@ -157,11 +158,12 @@ IndexerParams plan_indexer(const dsa_indexer_args* a, bool fused, int k) {
         if (cost < best) { best = cost; kch = c; }
       }
     } else {
-      // Key tiles of the busiest CTA: waves of units over the SMs times the tiles
-      // of a unit.  Many splits come within a few percent of the fewest; among
-      // those, units nearest 32 tiles (4096 keys) measured fastest on B200 (decode,
-      // 64 x 131072 keys: 9 units a sequence 194 us, 16: 196, 23: 187, 32: 183,
-      // 37: 182, 48: 184, 64: 183, 74: 186).
+      // One query block per sequence (decode).  Key tiles of the busiest CTA:
+      // waves of units over the SMs times the tiles of a unit.  Many splits come
+      // within a few percent of the fewest; among those, units nearest 32 tiles
+      // (4096 keys) measured fastest on B200 (decode, 64 x 131072 keys: 9 units a
+      // sequence 194 us, 16: 196, 23: 187, 32: 183, 37: 182, 48: 184, 64: 183,
+      // 74: 186).
       constexpr int kPreferTiles = 32;
       auto cost = [&](int c) {
         return ((base_units * c + sms - 1) / sms) * (long long)((max_tiles + c - 1) / c);
