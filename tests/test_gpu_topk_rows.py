@@ -145,3 +145,19 @@ def test_cluster_rows_one_pass_and_segment_overflow():
     r6[98304:] -= 10.0
     s = torch.cat([s, r6.view(1, 1, Lk)], dim=1)
     _check(s.to(DEV), Lk - 7, 2048)
+
+
+def test_rows_not_16_byte_aligned_take_the_4_byte_passes():
+    # Rows whose length is not a multiple of four start at addresses that are not
+    # 16-byte aligned, so the single passes read 4-byte scores: a few long rows
+    # spread over clusters (one with a block of planted ties), and ~100 rows of
+    # 40 K scores, one CTA per row.
+    g = torch.Generator().manual_seed(47)
+    Lk = 131069
+    s = torch.randn(1, 3, Lk, generator=g)
+    s[0, 1, 50000:50600] = 4.0
+    _check(s.to(DEV), Lk - 3, 2048)
+    Lk = 40001
+    s = torch.randn(1, 100, Lk, generator=g)
+    s[0, 7, ::5] = 3.5
+    _check(s.to(DEV), Lk - 100, 2048)
